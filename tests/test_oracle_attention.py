@@ -1,0 +1,201 @@
+"""Pins for oracle/attention.py: lossless special cases against exact fp64
+attention, invariants, mask/causal/GQA identities, brute-force integer
+QK^T, and the pages' shape contracts (no GPU)."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from lossless_cases import LN2, i8f8_case, nvfp4_case
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "page_examples.json")))
+
+
+# ------------------------------------------------------------ exact attention
+def test_exact_attention_rows_sum_to_one_and_shift_invariance():
+    q, k, v = W.make_qkv(W.TINY.scaled(Hq=2, Hkv=1, N=200))
+    ones = torch.ones_like(v, dtype=torch.float64)
+    out1, _ = O.exact_attention(q, k, ones, sm_scale=0.3)
+    np.testing.assert_allclose(out1, 1.0, rtol=0, atol=1e-12)
+    c = torch.randn(1, 1, 1, 64, dtype=torch.float64) * 5
+    outa, lsea = O.exact_attention(q, k, v, sm_scale=0.3)
+    outb, lseb = O.exact_attention(q, k.double() + c, v, sm_scale=0.3)
+    np.testing.assert_allclose(outa, outb, rtol=1e-10, atol=1e-12)
+    qc = np.einsum("bhnc,c->bhn", q.double().numpy(), c[0, 0, 0].numpy())
+    np.testing.assert_allclose(lseb - lsea, 0.3 * qc, atol=1e-9)
+
+
+def test_exact_attention_matches_torch_sdpa():
+    q, k, v = W.make_qkv(W.TINY.scaled(N=130))
+    for causal in (False, True):
+        out, lse = O.exact_attention(q, k, v, causal=causal, sm_scale=0.2)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q.double(), k.double(), v.double(), is_causal=causal, scale=0.2)
+        np.testing.assert_allclose(out, ref.numpy(), atol=1e-12)
+        s = 0.2 * q.double() @ k.double().transpose(-1, -2)
+        if causal:
+            s = s.masked_fill(torch.ones(130, 130, dtype=torch.bool).triu(1), -math.inf)
+        np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), atol=1e-12)
+
+
+# ------------------------------------------------------------ lossless INT8/FP8
+@pytest.mark.parametrize("N,Hq,Hkv,causal", [(256, 2, 2, False), (256, 2, 2, True),
+                                             (300, 4, 2, False), (200, 4, 1, True),
+                                             (384, 2, 1, False)])
+def test_i8f8_oracle_equals_exact_attention_when_lossless(N, Hq, Hkv, causal):
+    q, k, v = i8f8_case(B=1, Hq=Hq, Hkv=Hkv, N=N, D=64, seed=N + Hq)
+    qz = O.quantize_qkv_i8f8(q, k, v)
+    # the construction really is lossless
+    assert np.all(qz["q_scale"] == 1) and np.all(qz["k_scale"] == 1) and np.all(qz["v_scale"] == 1)
+    assert np.all(qz["k_mean"] == 0)
+    np.testing.assert_array_equal(qz["q"][:, :, :N], q.double().numpy())
+    r = O.attention_i8f8(qz, causal=causal, sm_scale=LN2)
+    ex, lse = O.exact_attention(q, k, v, causal=causal, sm_scale=LN2)
+    np.testing.assert_allclose(r["out_f64"], ex, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(r["lse"], lse, rtol=1e-12, atol=1e-12)
+
+
+def test_i8f8_lossless_with_mask():
+    q, k, v = i8f8_case(B=1, Hq=2, Hkv=2, N=256, D=64, seed=9)
+    g = torch.Generator().manual_seed(9)
+    mask = torch.rand(1, 1, 256, 256, generator=g) < 0.7
+    mask[..., 0] = True
+    qz = O.quantize_qkv_i8f8(q, k, v)
+    r = O.attention_i8f8(qz, sm_scale=LN2, mask=mask.numpy())
+    ex, lse = O.exact_attention(q, k, v, sm_scale=LN2, mask=mask.numpy())
+    np.testing.assert_allclose(r["out_f64"], ex, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(r["lse"], lse, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------ identities on random data
+def _random_qz(N=300, Hq=4, Hkv=2, D=64, seed=0):
+    q, k, v = W.make_qkv(W.TINY.scaled(N=N, Hq=Hq, Hkv=Hkv, D=D, seed=seed))
+    return q, k, v, O.quantize_qkv_i8f8(q, k, v)
+
+
+def test_mask_second_half_equals_truncated_keys():
+    mcase = GOLDEN["mask_second_half"]
+    assert mcase["visible_keys"] == "first half"
+    q, k, v, qz = _random_qz(N=256, Hq=2, Hkv=2)
+    mask = np.ones((1, 1, 256, 256), bool)
+    mask[..., 128:] = False                     # mask[:, :, :, N // 2:] = False
+    rm = O.attention_i8f8(qz, mask=mask)
+    cut = dict(qz, Nk=128)                      # same codes and scales, keys 0..127 only
+    rt = O.attention_i8f8(cut)
+    np.testing.assert_array_equal(rm["out"], rt["out"])
+    np.testing.assert_array_equal(rm["lse"], rt["lse"])
+
+
+def test_causal_row_equals_truncated_keys():
+    q, k, v, qz = _random_qz(N=300, Hq=2, Hkv=1)
+    rows = [0, 5, 127, 128, 200, 299]
+    rc = O.attention_i8f8(qz, causal=True, rows=rows)
+    for i, r in enumerate(rows):
+        rt = O.attention_i8f8(dict(qz, Nk=r + 1), rows=[r])
+        np.testing.assert_array_equal(rc["out"][:, :, i], rt["out"][:, :, 0])
+        np.testing.assert_array_equal(rc["lse"][:, :, i], rt["lse"][:, :, 0])
+
+
+def test_gqa_equals_repeated_kv_heads():
+    """16 Q heads over 4 KV heads: Q head h uses KV head h // 4."""
+    q, k, v = W.make_qkv(W.TINY.scaled(Hq=8, Hkv=2, N=130))
+    r = O.attention_i8f8(O.quantize_qkv_i8f8(q, k, v))
+    k4, v4 = k.repeat_interleave(4, dim=1), v.repeat_interleave(4, dim=1)
+    r4 = O.attention_i8f8(O.quantize_qkv_i8f8(q, k4, v4))
+    np.testing.assert_array_equal(r["out"], r4["out"])
+    np.testing.assert_array_equal(r["lse"], r4["lse"])
+
+
+def test_fully_masked_row_gives_zero_and_minus_inf():
+    q, k, v, qz = _random_qz(N=128, Hq=2, Hkv=2)
+    mask = np.ones((1, 1, 128, 128), bool)
+    mask[0, 0, 3, :] = False
+    r = O.attention_i8f8(qz, mask=mask)
+    assert np.all(r["out"][0, :, 3] == 0) and np.all(r["lse"][0, :, 3] == -np.inf)
+    assert np.all(np.isfinite(r["lse"][0, :, 4]))
+
+
+def test_sm_scale_default_is_inverse_sqrt_d():
+    assert O.default_sm_scale(128) == pytest.approx(GOLDEN["nvfp4_layout"]["sm_scale_default"], rel=1e-15)
+    q, k, v, qz = _random_qz(N=128, Hq=2, Hkv=2, D=64)
+    np.testing.assert_array_equal(O.attention_i8f8(qz)["out"], O.attention_i8f8(qz, sm_scale=0.125)["out"])
+
+
+def test_qk_int32_tile_brute_force():
+    q, k, v, qz = _random_qz(N=256, Hq=2, Hkv=1, D=64)
+    t = O.qk_int32_tile(qz, 0, 1, 1, 0)
+    qc = qz["q"][0, 1, 128:256].tolist()
+    kc = qz["k"][0, 0, 0:128].tolist()
+    for i in range(0, 128, 7):
+        for j in range(0, 128, 5):
+            assert t[i, j] == sum(a * b for a, b in zip(qc[i], kc[j]))
+
+
+def test_oracle_close_to_exact_attention_on_tiny_workload():
+    """Sanity floor (the pages print no accuracy number): the INT8/FP8
+    oracle is within cosine 0.999 of fp64 attention on the tiny workload,
+    NVFP4 within 0.97."""
+    w = W.TINY
+    q, k, v = W.make_qkv(w)
+    ex, lse = O.exact_attention(q, k, v, sm_scale=w.sm_scale)
+    r = O.attention_i8f8(O.quantize_qkv_i8f8(q, k, v), sm_scale=w.sm_scale)
+    assert O.cosine(r["out"], ex) > 0.999
+    assert np.abs(r["lse"] - lse).max() < 0.05
+    rn = O.attention_nvfp4(O.quantize_qkv_nvfp4(q, k, v), sm_scale=w.sm_scale)
+    assert O.cosine(rn["out"], ex) > 0.97
+
+
+# ------------------------------------------------------------ NVFP4
+@pytest.mark.parametrize("per_block_mean,L,causal", [(True, 256, False), (False, 224, False),
+                                                     (True, 192, True)])
+def test_nvfp4_oracle_equals_exact_attention_when_lossless(per_block_mean, L, causal):
+    q, k, v = nvfp4_case(B=1, Hq=2, Hkv=1, N=256, D=64, L=L, seed=L)
+    qz = O.quantize_qkv_nvfp4(q, k, v, per_block_mean=per_block_mean, unpadded_k_len=L)
+    assert np.all(qz["qk_correction"] == 0) and np.all(qz["k_mean"] == 0)
+    assert np.all(O.e4m3_decode(qz["q_sf"]) == 1)
+    r = O.attention_nvfp4(qz, causal=causal, sm_scale=LN2)
+    ex, lse = O.exact_attention(q, k, v, causal=causal, sm_scale=LN2, kv_len=L)
+    np.testing.assert_allclose(r["out_f64"], ex, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(r["lse"], lse, rtol=1e-12, atol=1e-12)
+
+
+def test_nvfp4_layout_contract():
+    lay = GOLDEN["nvfp4_layout"]
+    q, k, v = W.make_qkv(W.NVFP4.scaled(Hq=2, Hkv=2, N=256, unpadded_k_len=200))
+    qz = O.quantize_qkv_nvfp4(q, k, v, unpadded_k_len=200)
+    D = 128
+    assert qz["q_packed"].shape == (1, 2, 256, D // 2)                   # [B, Hqo, M_pad, D/2]
+    assert qz["k_packed"].shape == (1, 2, 256, D // 2)                   # [B, Hkv, N_pad, D/2]
+    assert qz["qk_correction"].shape[2] == 256 // 128                    # one row per Q block
+    assert lay["q_fp4"][-1] == lay["head_dim"] // 2
+    assert lay["qk_correction_rows_per_head"] == lay["M"] // 128
+    # keys at and beyond unpadded_k_len are masked: changing them changes nothing
+    r1 = O.attention_nvfp4(qz, rows=[0, 100, 255])
+    qz2 = dict(qz)
+    qz2["k"] = qz["k"].copy()
+    qz2["k"][:, :, 200:] = 7
+    qz2["k_sf"] = qz["k_sf"].copy()
+    qz2["k_sf"][:, :, 200:] = 0x38
+    r2 = O.attention_nvfp4(qz2, rows=[0, 100, 255])
+    np.testing.assert_array_equal(r1["out"], r2["out"])
+
+
+@pytest.mark.parametrize("case", GOLDEN["shape_cases"], ids=lambda c: c["cite"][-40:])
+def test_page_shape_contracts(case):
+    """out has q's shape and lse is [B, H, N] (N shortened to 128: the
+    contract holds at any length)."""
+    B, Hq, _, D = case["q"]
+    Hkv = case["kv"][1]
+    N = 128
+    w = W.TINY.scaled(B=B, Hq=Hq, Hkv=Hkv, N=N, D=D)
+    q, k, v = W.make_qkv(w)
+    heads = [(0, 0), (B - 1, Hq - 1)]
+    r = O.attention_i8f8(O.quantize_qkv_i8f8(q, k, v), causal=case.get("causal", False), heads=heads)
+    assert r["out"].shape == (B, Hq, N, D) and tuple(case["out"][:2]) == (B, Hq)
+    assert r["lse"].shape == (B, Hq, N) and tuple(case["lse"][:2]) == (B, Hq)
+    assert case["out"][3] == D and case["lse"][2] == case["q"][2]
