@@ -1,0 +1,212 @@
+/*
+ * sage_b200.h -- C ABI of the B200 (sm_100a) SageAttention-style quantised
+ * attention forward.
+ *
+ * The operation (thu-ml/sageattention llms.txt):
+ *   "sageattn_qk_int8_pv_fp16_triton": per-block INT8 quantisation of Q and
+ *     K, optional K smoothing ("smooth_k"), boolean attention mask
+ *     broadcastable to [batch, heads, q_len, k_len] (True = attend), LSE.
+ *   "sageattn_qk_int8_pv_fp8_cuda" / "sageattn_qk_int8_pv_fp8_cuda_sm90":
+ *     INT8 Q/K with per-channel FP8 V, PV accumulated in FP32, causal mask,
+ *     LSE of shape [batch, heads, seq].
+ *   "sageattn -- Auto-selecting attention kernel": FP16/BF16 inputs in HND
+ *     or NHD layout, group-query attention (several Q heads per KV head),
+ *     sm_scale defaulting to 1/sqrt(head_dim).
+ *
+ * What each call computes, precisely:
+ *   quantise:  kmean[b,g,c] = mean over tokens of K (exact, rounded once to
+ *              fp32; zero when smooth_k == 0); Ks = fp32(K - kmean);
+ *              per 128-token block of Q (resp. Ks), a = max|x|,
+ *              scale = fp32(a/127), code = clamp(rint(fp32(x * fp32(127/a))), +-127);
+ *              per V channel over all tokens, a = max|v|, vscale = fp32(a/448),
+ *              code = e4m3_rn_satfinite(fp32(v * fp32(448/a))), stored transposed;
+ *              q_dot_kmean[b,h,n] = sum_c q[b,h,n,c] * kmean[b,h/G,c].
+ *   attention: s = S_int * q_scale * k_scale * sm_scale with S_int the exact
+ *              int32 dot product of the codes; online softmax over 128-key
+ *              tiles; P8 = e4m3(448 * exp(s - running_max)); O += P8 . V8 in
+ *              FP32; out = O * vscale / (448 * l), l the sum of the
+ *              unquantised probabilities; lse = natural-log LSE of the
+ *              unsmoothed scores (smoothed LSE + sm_scale * q_dot_kmean).
+ *   A query row with no visible key gives out = 0 and lse = -inf.
+ *
+ * Conventions (all entry points):
+ *   - Every pointer argument named as device memory must point to memory
+ *     of the device that is current on the calling thread; host pointers
+ *     are only the descriptor structs themselves.  The library never
+ *     allocates device memory: the caller owns every buffer, including the
+ *     workspace, whose size the matching *_workspace_bytes query returns.
+ *   - Work is enqueued asynchronously on `stream` (NULL = legacy default
+ *     stream); the call returns after enqueueing.  Argument errors are
+ *     detected on the host before anything is enqueued.
+ *   - Errors: SAGE_ERR_INVALID_ARG (malformed argument), SAGE_ERR_UNSUPPORTED
+ *     (valid but outside what the kernels handle, e.g. head_dim not in
+ *     {64,128}), SAGE_ERR_WORKSPACE (workspace too small), SAGE_ERR_CUDA (a
+ *     CUDA call failed at launch).  Device-side failures (a bounded wait that
+ *     ran out) set a device status word read by sage_get_device_status.
+ *   - The calls are thread-safe.  Calls that share a workspace or outputs
+ *     must be ordered by the caller (same stream or events).
+ */
+#ifndef SAGE_B200_H
+#define SAGE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sage_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARG = 1,
+  SAGE_ERR_UNSUPPORTED = 2,
+  SAGE_ERR_WORKSPACE = 3,
+  SAGE_ERR_CUDA = 4,
+  SAGE_ERR_TIMEOUT = 5
+} sage_status;
+
+/* Input element types: the pages take FP16/BF16 Q/K/V ("SageAttention
+ * Usage" notes). */
+typedef enum { SAGE_BF16 = 0, SAGE_FP16 = 1 } sage_dtype;
+
+/* A strided 4-D input tensor of logical shape [B, H, N, D].
+ * ptr: device pointer to element [0,0,0,0], 16-byte aligned.
+ * sb, sh, sn: element strides of the batch, head and token dimensions; the
+ * channel stride is 1.  HND layout has sn = D, sh = N*D; NHD layout has
+ * sn = H*D, sh = D ("tensor_layout" of the sageattn API).  sn must be a
+ * multiple of 8 elements (16-byte rows). */
+typedef struct {
+  const void* ptr;
+  int32_t dtype; /* sage_dtype */
+  int64_t B, H, N, D;
+  int64_t sb, sh, sn;
+} sage_tensor;
+
+/* Boolean attention mask, one byte per element, nonzero = attend
+ * ("mask[..., seq_len // 2:] = False  # mask out second half of keys").
+ * Logical shape [B, H, Nq, Nk] broadcast over batch and heads: B is 1 or the
+ * attention's batch, H is 1 or the number of Q heads.  sb, sh, sq: byte
+ * strides (ignored for a broadcast dimension of size 1); the key stride is 1.
+ * Device memory, owned by the caller, read-only. */
+typedef struct {
+  const uint8_t* ptr;
+  int64_t B, H, Nq, Nk;
+  int64_t sb, sh, sq;
+} sage_mask;
+
+/* Quantised Q/K/V of the INT8/FP8 path, all device memory owned by the
+ * caller.  Nq_pad = ceil(Nq/128)*128, Nk_pad = ceil(Nk/128)*128; every
+ * array is dense in the order given.
+ *   q        int8  [B, Hq,  Nq_pad, D]   codes; rows >= Nq are 0
+ *   q_scale  fp32  [B, Hq,  Nq_pad/128]  one scale per 128-token block
+ *   k        int8  [B, Hkv, Nk_pad, D]   codes of K - kmean; rows >= Nk are 0
+ *   k_scale  fp32  [B, Hkv, Nk_pad/128]
+ *   k_mean   fp32  [B, Hkv, D]
+ *   v_t      e4m3  [B, Hkv, D, Nk_pad]   V codes, transposed; tokens >= Nk are 0
+ *   v_scale  fp32  [B, Hkv, D]
+ *   q_dot_kmean fp32 [B, Hq, Nq]  (may be NULL when no LSE is wanted)
+ * The base pointers of q, k and v_t must be 16-byte aligned. */
+typedef struct {
+  int8_t* q;
+  float* q_scale;
+  int8_t* k;
+  float* k_scale;
+  float* k_mean;
+  uint8_t* v_t;
+  float* v_scale;
+  float* q_dot_kmean;
+  int64_t B, Hq, Hkv, Nq, Nk, D;
+} sage_qkv_i8f8;
+
+/* ------------------------------------------------------------------ info */
+const char* sage_status_str(sage_status status);
+const char* sage_version(void);
+
+/* Device status word: synchronises `stream`, returns SAGE_ERR_TIMEOUT if a
+ * kernel of this library gave up a bounded wait since the last call (the
+ * wait site is written to *site when site != NULL), SAGE_ERR_CUDA if the
+ * stream reports an error, SAGE_OK otherwise, and clears the word. */
+sage_status sage_get_device_status(sage_stream_t stream, uint32_t* site);
+
+/* ----------------------------------------------------------- quantisation */
+/* Workspace bytes sage_quantize_qkv needs for these sizes (per-split K sums
+ * and V maxima of the reduction pass). */
+size_t sage_quantize_workspace_bytes(int64_t B, int64_t Hkv, int64_t Nk, int64_t D);
+
+/* Quantisation stage: smooth_k + per-block INT8 Q/K, per-channel FP8 V
+ * (north-star "sage_quantize_qkv"; pages: "smooth_k", per-block INT8 QK,
+ * per-channel FP8 V).  q: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D] (same dtype,
+ * Hq % Hkv == 0, D in {64, 128}).  Writes every array of *out (whose shape
+ * fields must match the inputs).  ws: device workspace of at least
+ * sage_quantize_workspace_bytes(B, Hkv, Nk, D) bytes, 256-byte aligned. */
+sage_status sage_quantize_qkv(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                              int smooth_k, const sage_qkv_i8f8* out, void* ws, size_t ws_bytes,
+                              sage_stream_t stream);
+
+/* --------------------------------------------------------------- attention */
+/* Workspace bytes of sage_attn_fwd_quantized: the per-tile mask
+ * classification (zero when mask == NULL). */
+size_t sage_attn_quantized_workspace_bytes(const sage_qkv_i8f8* qkv, const sage_mask* mask);
+
+/* Fused attention on quantised inputs (north-star "sage_attn_fwd" second
+ * stage: INT8 QK^T, dequantise, online softmax, P -> FP8, FP8 PV with FP32
+ * accumulation).
+ *   causal:   keep key j for query i when j <= i + Nk - Nq.
+ *   sm_scale: softmax scale; <= 0 selects 1/sqrt(D).
+ *   mask:     NULL or a boolean mask (see sage_mask).
+ *   out:      device, q's logical shape [B, Hq, Nq, D], element type
+ *             out_dtype (sage_dtype), element strides out_sb/out_sh/out_sn
+ *             (channel stride 1; 16-byte aligned rows).
+ *   lse:      device fp32 [B, Hq, Nq], written iff return_lse (then
+ *             q_dot_kmean must be non-NULL); NULL otherwise.
+ *   ws:       device workspace of sage_attn_quantized_workspace_bytes bytes. */
+sage_status sage_attn_fwd_quantized(const sage_qkv_i8f8* qkv, int causal, float sm_scale,
+                                    int return_lse, const sage_mask* mask, void* out,
+                                    int32_t out_dtype, int64_t out_sb, int64_t out_sh,
+                                    int64_t out_sn, float* lse, void* ws, size_t ws_bytes,
+                                    sage_stream_t stream);
+
+/* Workspace bytes of sage_attn_fwd: the quantised Q/K/V plus the two
+ * workspaces above. */
+size_t sage_attn_fwd_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
+                                     int64_t Nk, int64_t D, const sage_mask* mask);
+
+/* The whole path on FP16/BF16 inputs (north-star "sage_attn_fwd (q, k, v,
+ * causal, sm_scale, num_kv_heads, return_lse)"; pages: "sageattn").
+ * num_kv_heads must equal k->H.  smooth_k as in sage_quantize_qkv (the
+ * pages' default is on).  out has q's dtype; the other arguments are those
+ * of sage_attn_fwd_quantized.  Quantises into the workspace, then attends. */
+sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                          int causal, float sm_scale, int num_kv_heads, int return_lse,
+                          int smooth_k, const sage_mask* mask, void* out, int64_t out_sb,
+                          int64_t out_sh, int64_t out_sn, float* lse, void* ws,
+                          size_t ws_bytes, sage_stream_t stream);
+
+/* ------------------------------------------------------------ test exports */
+/* Exact int32 QK^T of one 128x128 tile of codes: rows qblk*128.. of Q head
+ * h, keys kblk*128.. of KV head h / (Hq/Hkv), batch b, computed by one
+ * tcgen05 kind::i8 MMA chain exactly as the attention kernel does.
+ * tile: device int32 [128, 128] (row-major). */
+sage_status sage_debug_qk_int32(const sage_qkv_i8f8* qkv, int64_t b, int64_t h, int64_t qblk,
+                                int64_t kblk, int32_t* tile, sage_stream_t stream);
+
+/* FP8 PV product of one tile as the attention kernel computes it: p is a
+ * device e4m3 [128, 128] row-major matrix (written to shared memory by
+ * threads in the kernel's swizzled layout), times the transposed V codes of
+ * keys kblk*128.. of KV head h_kv, batch b.  acc: device fp32 [128, D]. */
+sage_status sage_debug_pv_fp32(const sage_qkv_i8f8* qkv, const uint8_t* p, int64_t b,
+                               int64_t h_kv, int64_t kblk, float* acc, sage_stream_t stream);
+
+/* Launches one thread that waits on a shared-memory barrier nothing
+ * arrives on, bounded by timeout_us microseconds; the wait gives up, sets
+ * the device status word and the kernel returns.  Used to test the
+ * bounded-wait path without hanging the GPU. */
+sage_status sage_debug_wait_timeout(uint32_t timeout_us, sage_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_B200_H */

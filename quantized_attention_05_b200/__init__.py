@@ -1,0 +1,301 @@
+"""Python binding of libsage_b200.so (include/sage_b200.h).
+
+Argument marshalling only: torch provides device memory and the current
+stream, and every step of the computation runs in the library's CUDA
+kernels.  There is no fallback: if the library cannot be loaded, every call
+raises.
+
+Functions keep the C names: ``sage_quantize_qkv``, ``sage_attn_fwd_quantized``,
+``sage_attn_fwd``, ``sage_debug_qk_int32``, ``sage_debug_pv_fp32``,
+``sage_debug_wait_timeout``, ``sage_get_device_status``.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsage_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "sage_b200.h")
+
+SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_WORKSPACE, SAGE_ERR_CUDA, \
+    SAGE_ERR_TIMEOUT = range(6)
+SAGE_BF16, SAGE_FP16 = 0, 1
+
+_i64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+
+
+class SageError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{msg}: status {status}")
+        self.status = status
+
+
+class SageTensor(ctypes.Structure):
+    _fields_ = [("ptr", _vp), ("dtype", ctypes.c_int32), ("B", _i64), ("H", _i64), ("N", _i64),
+                ("D", _i64), ("sb", _i64), ("sh", _i64), ("sn", _i64)]
+
+
+class SageMask(ctypes.Structure):
+    _fields_ = [("ptr", _vp), ("B", _i64), ("H", _i64), ("Nq", _i64), ("Nk", _i64),
+                ("sb", _i64), ("sh", _i64), ("sq", _i64)]
+
+
+class SageQkvI8F8(ctypes.Structure):
+    _fields_ = [("q", _vp), ("q_scale", _vp), ("k", _vp), ("k_scale", _vp), ("k_mean", _vp),
+                ("v_t", _vp), ("v_scale", _vp), ("q_dot_kmean", _vp),
+                ("B", _i64), ("Hq", _i64), ("Hkv", _i64), ("Nq", _i64), ("Nk", _i64), ("D", _i64)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libsage_b200.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with "
+                          "`python -m quantized_attention_05_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER
+    sig = {
+        "sage_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+        "sage_version": (ctypes.c_char_p, []),
+        "sage_get_device_status": (ctypes.c_int, [_vp, P(ctypes.c_uint32)]),
+        "sage_quantize_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, _i64]),
+        "sage_quantize_qkv": (ctypes.c_int, [P(SageTensor), P(SageTensor), P(SageTensor), ctypes.c_int,
+                                             P(SageQkvI8F8), _vp, ctypes.c_size_t, _vp]),
+        "sage_attn_quantized_workspace_bytes": (ctypes.c_size_t, [P(SageQkvI8F8), P(SageMask)]),
+        "sage_attn_fwd_quantized": (ctypes.c_int, [P(SageQkvI8F8), ctypes.c_int, ctypes.c_float,
+                                                   ctypes.c_int, P(SageMask), _vp, ctypes.c_int32,
+                                                   _i64, _i64, _i64, _vp, _vp, ctypes.c_size_t, _vp]),
+        "sage_attn_fwd_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, _i64, _i64, _i64,
+                                                            P(SageMask)]),
+        "sage_attn_fwd": (ctypes.c_int, [P(SageTensor), P(SageTensor), P(SageTensor), ctypes.c_int,
+                                         ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         P(SageMask), _vp, _i64, _i64, _i64, _vp, _vp,
+                                         ctypes.c_size_t, _vp]),
+        "sage_debug_qk_int32": (ctypes.c_int, [P(SageQkvI8F8), _i64, _i64, _i64, _i64, _vp, _vp]),
+        "sage_debug_pv_fp32": (ctypes.c_int, [P(SageQkvI8F8), _vp, _i64, _i64, _i64, _vp, _vp]),
+        "sage_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, _vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(status, what):
+    if status != SAGE_OK:
+        msg = lib().sage_status_str(status).decode()
+        raise SageError(status, f"{what} failed ({msg})")
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return SAGE_BF16
+    if t.dtype == torch.float16:
+        return SAGE_FP16
+    raise TypeError(f"q/k/v must be bf16 or fp16, got {t.dtype}")
+
+
+def _as_tensor(t: torch.Tensor, layout: str = "HND") -> SageTensor:
+    """Describe a 4-D tensor.  layout "HND": logical (B, H, N, D);
+    "NHD": logical (B, N, H, D).  Strides are passed as they are."""
+    if t.dim() != 4:
+        raise ValueError("expected a 4-D tensor")
+    if layout == "NHD":
+        t = t.transpose(1, 2)
+    elif layout != "HND":
+        raise ValueError(layout)
+    if t.stride(3) != 1:
+        raise ValueError("the channel dimension must be contiguous")
+    B, H, N, D = t.shape
+    sb, sh, sn, _ = t.stride()
+    return SageTensor(t.data_ptr(), _dtype_code(t), B, H, N, D, sb, sh, sn)
+
+
+def _as_mask(mask: Optional[torch.Tensor], B, Hq, Nq, Nk):
+    if mask is None:
+        return None
+    if mask.dtype != torch.bool and mask.dtype != torch.uint8:
+        raise TypeError("mask must be bool or uint8 (nonzero = attend)")
+    m = mask
+    while m.dim() < 4:
+        m = m.unsqueeze(0)
+    m = m.expand(m.shape[0], m.shape[1], Nq, Nk) if (m.shape[2] == 1 or m.shape[3] == 1) else m
+    if m.stride(3) != 1:
+        m = m.contiguous()
+    mb, mh = m.shape[0], m.shape[1]
+    return SageMask(m.data_ptr(), mb, mh, Nq, Nk, m.stride(0) if mb > 1 else 0,
+                    m.stride(1) if mh > 1 else 0, m.stride(2)), m
+
+
+def pad128(n):
+    return (n + 127) // 128 * 128
+
+
+@dataclasses.dataclass
+class QuantizedQKV:
+    """Quantised Q/K/V (device tensors) with the layouts of sage_qkv_i8f8."""
+    q: torch.Tensor            # int8  [B, Hq, Nq_pad, D]
+    q_scale: torch.Tensor      # fp32  [B, Hq, Nq_pad/128]
+    k: torch.Tensor            # int8  [B, Hkv, Nk_pad, D]
+    k_scale: torch.Tensor      # fp32  [B, Hkv, Nk_pad/128]
+    k_mean: torch.Tensor       # fp32  [B, Hkv, D]
+    v_t: torch.Tensor          # uint8 (E4M3) [B, Hkv, D, Nk_pad]
+    v_scale: torch.Tensor      # fp32  [B, Hkv, D]
+    q_dot_kmean: Optional[torch.Tensor]  # fp32 [B, Hq, Nq]
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    D: int
+
+    @classmethod
+    def empty(cls, B, Hq, Hkv, Nq, Nk, D, device, with_qdk=True):
+        Nqp, Nkp = pad128(Nq), pad128(Nk)
+        kw = dict(device=device)
+        return cls(torch.empty(B, Hq, Nqp, D, dtype=torch.int8, **kw),
+                   torch.empty(B, Hq, Nqp // 128, dtype=torch.float32, **kw),
+                   torch.empty(B, Hkv, Nkp, D, dtype=torch.int8, **kw),
+                   torch.empty(B, Hkv, Nkp // 128, dtype=torch.float32, **kw),
+                   torch.empty(B, Hkv, D, dtype=torch.float32, **kw),
+                   torch.empty(B, Hkv, D, Nkp, dtype=torch.uint8, **kw),
+                   torch.empty(B, Hkv, D, dtype=torch.float32, **kw),
+                   torch.empty(B, Hq, Nq, dtype=torch.float32, **kw) if with_qdk else None,
+                   B, Hq, Hkv, Nq, Nk, D)
+
+    def struct(self) -> SageQkvI8F8:
+        p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        return SageQkvI8F8(p(self.q), p(self.q_scale), p(self.k), p(self.k_scale), p(self.k_mean),
+                           p(self.v_t), p(self.v_scale), p(self.q_dot_kmean),
+                           self.B, self.Hq, self.Hkv, self.Nq, self.Nk, self.D)
+
+
+def _ws(nbytes, device):
+    # 256-byte aligned: torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def sage_quantize_qkv(q, k, v, smooth_k=True, layout="HND", with_qdk=True,
+                      out: Optional[QuantizedQKV] = None, ws: Optional[torch.Tensor] = None):
+    """smooth_k + per-block INT8 Q/K + per-channel FP8 V (sage_quantize_qkv)."""
+    L = lib()
+    tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
+    if out is None:
+        out = QuantizedQKV.empty(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D, q.device, with_qdk)
+    nbytes = L.sage_quantize_workspace_bytes(tk.B, tk.H, tk.N, tk.D)
+    if ws is None:
+        ws = _ws(nbytes, q.device)
+    s = out.struct()
+    _check(L.sage_quantize_qkv(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                               int(bool(smooth_k)), ctypes.byref(s), ws.data_ptr(), ws.numel(),
+                               _stream(q.device)), "sage_quantize_qkv")
+    return out
+
+
+def sage_attn_fwd_quantized(qkv: QuantizedQKV, causal=False, sm_scale=None, return_lse=False,
+                            mask=None, out=None, out_dtype=torch.bfloat16, lse=None, ws=None):
+    """Fused INT8-QK / FP8-PV attention on quantised inputs."""
+    L = lib()
+    dev = qkv.q.device
+    if out is None:
+        out = torch.empty(qkv.B, qkv.Hq, qkv.Nq, qkv.D, dtype=out_dtype, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty(qkv.B, qkv.Hq, qkv.Nq, dtype=torch.float32, device=dev)
+    mk = _as_mask(mask, qkv.B, qkv.Hq, qkv.Nq, qkv.Nk)
+    mstruct = ctypes.byref(mk[0]) if mk else None
+    s = qkv.struct()
+    if ws is None:
+        ws = _ws(L.sage_attn_quantized_workspace_bytes(ctypes.byref(s), mstruct), dev)
+    sb, sh, sn, _ = out.stride()
+    _check(L.sage_attn_fwd_quantized(ctypes.byref(s), int(bool(causal)),
+                                     float(sm_scale) if sm_scale else 0.0, int(bool(return_lse)),
+                                     mstruct, out.data_ptr(), _dtype_code(out), sb, sh, sn,
+                                     lse.data_ptr() if return_lse else None, ws.data_ptr(),
+                                     ws.numel(), _stream(dev)), "sage_attn_fwd_quantized")
+    return (out, lse) if return_lse else out
+
+
+def sage_attn_fwd_workspace_bytes(B, Hq, Hkv, Nq, Nk, D, mask_shape=None):
+    m = None
+    if mask_shape is not None:
+        m = SageMask(None, mask_shape[0], mask_shape[1], Nq, Nk, 0, 0, Nk)
+    return lib().sage_attn_fwd_workspace_bytes(B, Hq, Hkv, Nq, Nk, D,
+                                              ctypes.byref(m) if m else None)
+
+
+def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, num_kv_heads=None, return_lse=False,
+                  smooth_k=True, mask=None, layout="HND", out=None, lse=None, ws=None):
+    """The whole path on bf16/fp16 Q/K/V (sage_attn_fwd): quantise, then attend.
+
+    Returns out (same shape/layout/dtype as q) and, with return_lse, lse
+    [B, Hq, Nq] fp32."""
+    L = lib()
+    tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
+    if num_kv_heads is None:
+        num_kv_heads = tk.H
+    if out is None:
+        out = torch.empty_like(q)
+    to = _as_tensor(out, layout)
+    if return_lse and lse is None:
+        lse = torch.empty(tq.B, tq.H, tq.N, dtype=torch.float32, device=q.device)
+    mk = _as_mask(mask, tq.B, tq.H, tq.N, tk.N)
+    mstruct = ctypes.byref(mk[0]) if mk else None
+    nbytes = L.sage_attn_fwd_workspace_bytes(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D, mstruct)
+    if ws is None or ws.numel() < nbytes:
+        ws = _ws(nbytes, q.device)
+    _check(L.sage_attn_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), int(bool(causal)),
+                           float(sm_scale) if sm_scale else 0.0, int(num_kv_heads),
+                           int(bool(return_lse)), int(bool(smooth_k)), mstruct, to.ptr, to.sb,
+                           to.sh, to.sn, lse.data_ptr() if return_lse else None, ws.data_ptr(),
+                           ws.numel(), _stream(q.device)), "sage_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def sage_debug_qk_int32(qkv: QuantizedQKV, b, h, qblk, kblk):
+    tile = torch.empty(128, 128, dtype=torch.int32, device=qkv.q.device)
+    s = qkv.struct()
+    _check(lib().sage_debug_qk_int32(ctypes.byref(s), b, h, qblk, kblk, tile.data_ptr(),
+                                     _stream(qkv.q.device)), "sage_debug_qk_int32")
+    return tile
+
+
+def sage_debug_pv_fp32(qkv: QuantizedQKV, p_e4m3: torch.Tensor, b, h_kv, kblk):
+    p = p_e4m3.contiguous().view(torch.uint8)
+    acc = torch.empty(128, qkv.D, dtype=torch.float32, device=qkv.q.device)
+    s = qkv.struct()
+    _check(lib().sage_debug_pv_fp32(ctypes.byref(s), p.data_ptr(), b, h_kv, kblk, acc.data_ptr(),
+                                    _stream(qkv.q.device)), "sage_debug_pv_fp32")
+    return acc
+
+
+def sage_debug_wait_timeout(timeout_us=1000):
+    _check(lib().sage_debug_wait_timeout(int(timeout_us), _stream()), "sage_debug_wait_timeout")
+
+
+def sage_get_device_status():
+    """(status, site): SAGE_OK or SAGE_ERR_TIMEOUT with the wait site."""
+    site = ctypes.c_uint32(0)
+    st = lib().sage_get_device_status(_stream(), ctypes.byref(site))
+    return st, site.value
+
+
+def default_sm_scale(D):
+    return 1.0 / math.sqrt(D)

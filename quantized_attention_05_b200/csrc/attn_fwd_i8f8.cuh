@@ -1,0 +1,677 @@
+// attn_fwd_i8f8.cuh -- fused INT8-QK / FP8-PV attention forward for sm_100a
+// (thu-ml/sageattention llms.txt: "sageattn_qk_int8_pv_fp8_cuda",
+// "sageattn_qk_int8_pv_fp8_cuda_sm90": INT8 Q/K with per-block scales,
+// per-channel FP8 V, PV accumulated in FP32, causal mask, LSE; "sageattn":
+// GQA and sm_scale; the Triton kernel's boolean mask).
+//
+// One CTA owns two 128-row Q tiles of one (batch, Q head) and streams the
+// 128-key K/V tiles of its KV head:
+//   warp 8      TMA producer: Q tiles once, then K and V^T tiles into a
+//               3-stage ring;
+//   warp 9      MMA issuer (one thread): S_i = Q_i K^T with tcgen05
+//               kind::i8 into TMEM (int32, exact), O_i += P_i V with
+//               kind::f8f6f4 (E4M3 x E4M3 -> FP32 in TMEM); it issues the
+//               next tile's QK^T of a Q tile as soon as that tile's S has
+//               been read, so the tensor pipe runs while softmax works;
+//   warps 0..7  two softmax warpgroups, one per Q tile, one thread per row:
+//               tcgen05.ld of the int32 scores, dequantisation by
+//               q_scale*k_scale*sm_scale*log2(e), masking, online softmax
+//               with exp2, P -> E4M3 (pre-scaled by 448) into shared
+//               memory in the 128-byte-swizzled K-major layout of the MMA,
+//               O rescaled in TMEM when the running max moves, and the
+//               epilogue (O * vscale / l -> bf16/fp16, LSE).
+// TMEM: 512 columns = 2 x (S 128 columns + O D columns, padded to 256).
+// Every wait on a barrier is bounded (sage_ptx.cuh).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "sage_ptx.cuh"
+
+namespace sage {
+
+constexpr int ATT_BM = 128, ATT_BN = 128;
+constexpr int ATT_STAGES = 3;
+constexpr int ATT_THREADS = 320;
+constexpr int ATT_MAX_NKT = 2048;   // keys <= 262144
+constexpr float LOG2_448 = 8.807354922057604f;
+constexpr float LN2_F = 0.6931471805599453f;
+
+struct AttnArgs {
+  const float* q_scale;
+  const float* k_scale;
+  const float* v_scale;
+  const float* qdk;
+  void* out;
+  int64_t out_sb, out_sh, out_sn;
+  int out_fp16;
+  float* lse;
+  const uint8_t* tile_class;       // [Bm, Hm, nqt, nkt] or null
+  const uint8_t* mask;
+  int64_t m_sb, m_sh, m_sq;
+  int m_bcast_b, m_bcast_h, mask_vec16;
+  int B, Hq, Hkv, G, Nq, Nk, Nqp, Nkp, nqt, nkt, nqp;
+  int causal, return_lse, causal_off;
+  float c0;                        // sm_scale * log2(e)
+  float sm_scale;
+};
+
+template <int D>
+struct AttnLayout {
+  static constexpr int Q_BYTES = ATT_BM * D;
+  static constexpr int K_BYTES = ATT_BN * D;
+  static constexpr int V_BYTES = D * ATT_BN;
+  static constexpr int P_BYTES = ATT_BM * ATT_BN;
+  static constexpr int QK_SWIZZLE = D;            // bytes per Q/K row: 128 or 64
+  static constexpr int QK_SBO = 8 * D;            // 8-row group stride
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + ATT_STAGES * K_BYTES;
+  static constexpr int OFF_P = OFF_V + ATT_STAGES * V_BYTES;
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int NBAR = 1 + 2 * ATT_STAGES + 8 + 1;
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_VS = (OFF_TMEM + 16 + 15) / 16 * 16;
+  static constexpr int OFF_NLIST = OFF_VS + D * 4;
+  static constexpr int OFF_LIST = OFF_NLIST + 16;
+  static size_t bytes(int nkt) { return 1024 + OFF_LIST + (size_t)nkt * 4; }
+};
+
+// Write one thread's row of 128 E4M3 probabilities (32 packed words) into a
+// 128x128-byte K-major tile with the 128-byte swizzle: 16-byte chunk c of
+// row r lives at r*128 + ((c ^ (r % 8)) * 16).  Tile base 1024-aligned.
+__device__ __forceinline__ void store_p_row(uint8_t* tile, int r, const uint32_t* pk) {
+  uint8_t* row = tile + r * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) =
+        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+}
+
+// Flags of key tile kt for Q tile qt (0 if nothing in it is visible):
+// bit 0 visible, bit 2 needs per-element masking, bit 4 reads the boolean
+// mask; shifted left by `wg` (0 or 1).
+__device__ __forceinline__ uint32_t tile_flags(const AttnArgs& a, int b, int h, int qt, int wg,
+                                               int kt) {
+  const int row_lo = qt * ATT_BM;
+  if (row_lo >= a.Nq) return 0;
+  const int row_hi = min(row_lo + ATT_BM - 1, a.Nq - 1);
+  const int key_lo = kt * ATT_BN, key_hi = key_lo + ATT_BN - 1;
+  if (key_lo >= a.Nk) return 0;
+  if (a.causal && key_lo > row_hi + a.causal_off) return 0;
+  bool need = key_hi >= a.Nk || (a.causal && key_hi > row_lo + a.causal_off);
+  bool part = false;
+  if (a.tile_class) {
+    const int bm = a.m_bcast_b ? 0 : b, hm = a.m_bcast_h ? 0 : h;
+    const int Hm = a.m_bcast_h ? 1 : a.Hq;
+    const uint8_t cls = a.tile_class[(((int64_t)bm * Hm + hm) * a.nqt + qt) * a.nkt + kt];
+    if (cls == 0) return 0;
+    part = cls == 2;
+  }
+  const uint32_t f = 1u | ((need || part) ? 4u : 0u) | (part ? 16u : 0u);
+  return f << wg;
+}
+
+__device__ __forceinline__ void decode_work(const AttnArgs& a, int bid, int& qp, int& b, int& h) {
+  if (a.causal) {  // longest rows first
+    const int per = a.B * a.Hq;
+    qp = a.nqp - 1 - bid / per;
+    const int r = bid % per;
+    b = r / a.Hq;
+    h = r % a.Hq;
+  } else {         // Q heads sharing a KV head run side by side (K/V reuse in L2)
+    const int j = bid % a.G;
+    int t = bid / a.G;
+    qp = t % a.nqp;
+    t /= a.nqp;
+    const int g = t % a.Hkv;
+    b = t / a.Hkv;
+    h = g * a.G + j;
+  }
+}
+
+template <typename OutT>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <>
+__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int D, typename OutT>
+__device__ __forceinline__ void store_out_chunk(const AttnArgs& a, OutT* orow, int cb,
+                                                const uint32_t* o, const float* s_vs, float inv_l) {
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float x0 = __uint_as_float(o[2 * i]) * s_vs[cb + 2 * i] * inv_l;
+    const float x1 = __uint_as_float(o[2 * i + 1]) * s_vs[cb + 2 * i + 1] * inv_l;
+    w[i] = pack2<OutT>(x0, x1);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(orow + cb);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+}
+
+template <int D>
+__global__ void __launch_bounds__(ATT_THREADS, 1)
+    attn_fwd_i8f8_kernel(const __grid_constant__ CUtensorMap tmQ,
+                         const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
+  using L = AttnLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sQ = smem + L::OFF_Q;
+  uint8_t* sK = smem + L::OFF_K;
+  uint8_t* sV = smem + L::OFF_V;
+  uint8_t* sP = smem + L::OFF_P;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + ATT_STAGES;
+  uint64_t* s_full = kv_empty + ATT_STAGES;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* o_ready = p_full + 2;
+  uint64_t* mma_done = o_ready + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
+  float* s_vs = reinterpret_cast<float*>(smem + L::OFF_VS);
+  int* s_nlist = reinterpret_cast<int*>(smem + L::OFF_NLIST);
+  uint32_t* s_list = reinterpret_cast<uint32_t*>(smem + L::OFF_LIST);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int qp, b, h;
+  decode_work(a, blockIdx.x, qp, b, h);
+  const int g = h / a.G;
+  const int bhq = b * a.Hq + h, bhk = b * a.Hkv + g;
+  const int qt0 = 2 * qp;
+  const bool has1 = qt0 + 1 < a.nqt;
+
+  // ------------------------------------------------------------ setup
+  if (warp == 0) {
+    int count = 0;
+    uint32_t orf = 0;
+    for (int base = 0; base < a.nkt; base += 32) {
+      const int kt = base + lane;
+      uint32_t f = 0;
+      if (kt < a.nkt) {
+        f = tile_flags(a, b, h, qt0, 0, kt);
+        if (has1) f |= tile_flags(a, b, h, qt0 + 1, 1, kt);
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, (f & 3u) != 0);
+      if (f & 3u) s_list[count + __popc(bal & ((1u << lane) - 1u))] = ((uint32_t)kt << 8) | f;
+      count += __popc(bal);
+      orf |= f;
+    }
+    orf = __reduce_or_sync(0xffffffffu, orf);
+    if (lane == 0) {
+      s_nlist[0] = count;
+      s_nlist[1] = (int)orf;
+    }
+  } else if (warp == 1 && lane == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < ATT_STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_ready[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  } else if (warp == 9) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  } else if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  for (int c = threadIdx.x; c < D; c += blockDim.x) s_vs[c] = a.v_scale[(int64_t)bhk * D + c];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int ntile = s_nlist[0];
+  const uint32_t orf = (uint32_t)s_nlist[1];
+
+  if (warp == 8) {
+    // ---------------------------------------------------------- TMA producer
+    // The whole warp runs the loop and waits; lane 0 issues the copies.
+    const bool act0 = orf & 1u, act1 = (orf >> 1) & 1u;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, (uint32_t)((act0 ? L::Q_BYTES : 0) + (act1 ? L::Q_BYTES : 0)));
+      if (act0) tma_load_2d(sQ, &tmQ, q_full, 0, bhq * a.Nqp + qt0 * ATT_BM);
+      if (act1) tma_load_2d(sQ + L::Q_BYTES, &tmQ, q_full, 0, bhq * a.Nqp + (qt0 + 1) * ATT_BM);
+    }
+    __syncwarp();
+    for (int idx = 0; idx < ntile; ++idx) {
+      const int st = idx % ATT_STAGES, rd = idx / ATT_STAGES;
+      if (idx >= ATT_STAGES &&
+          !__all_sync(0xffffffffu, mbar_wait(&kv_empty[st], (rd - 1) & 1, SITE_KV_EMPTY)))
+        break;
+      if (lane == 0) {
+        const int kt = (int)(s_list[idx] >> 8);
+        mbar_arrive_expect_tx(&kv_full[st], (uint32_t)(L::K_BYTES + L::V_BYTES));
+        tma_load_2d(sK + st * L::K_BYTES, &tmK, &kv_full[st], 0, bhk * a.Nkp + kt * ATT_BN);
+        tma_load_2d(sV + st * L::V_BYTES, &tmV, &kv_full[st], kt * ATT_BN, bhk * D);
+      }
+      __syncwarp();
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issuer
+    // The whole warp runs the schedule and waits; lane 0 issues MMAs/commits.
+    constexpr uint32_t IDESC_QK = instr_desc(kDS32, kS8, kS8, ATT_BM, ATT_BN);
+    constexpr uint32_t IDESC_PV = instr_desc(kDF32, kE4M3, kE4M3, ATT_BM, D);
+    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+    auto issue_qk = [&](int i, int st) {
+      const uint32_t tS = tmem + (uint32_t)(i * 256);
+      const uint32_t qa = aQ + i * L::Q_BYTES, ka = aK + st * L::K_BYTES;
+#pragma unroll
+      for (int k = 0; k < D / 32; ++k)
+        mma_i8(tS, smem_desc(qa + 32 * k, L::QK_SBO, L::QK_SWIZZLE),
+               smem_desc(ka + 32 * k, L::QK_SBO, L::QK_SWIZZLE), IDESC_QK, k > 0 ? 1u : 0u);
+    };
+    auto issue_pv = [&](int i, int st, bool acc) {
+      const uint32_t tO = tmem + (uint32_t)(i * 256 + 128);
+      const uint32_t pa = aP + i * L::P_BYTES, va = aV + st * L::V_BYTES;
+#pragma unroll
+      for (int k = 0; k < ATT_BN / 32; ++k)
+        mma_f8f6f4(tO, smem_desc(pa + 32 * k, 1024, 128), smem_desc(va + 32 * k, 1024, 128),
+                   IDESC_PV, (acc || k > 0) ? 1u : 0u);
+    };
+    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, SITE_Q_FULL));
+    tc_fence_after();
+    uint32_t qk_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
+    if (ok && ntile > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[0], 0, SITE_KV_FULL));
+      tc_fence_after();
+      const uint32_t f = s_list[0];
+      for (int i = 0; ok && i < 2; ++i)
+        if ((f >> i) & 1u) {
+          if (lane == 0) {
+            issue_qk(i, 0);
+            tc_commit(&s_full[i]);
+          }
+          __syncwarp();
+          ++qk_cnt[i];
+        }
+    }
+    for (int idx = 0; ok && idx < ntile; ++idx) {
+      const int st = idx % ATT_STAGES;
+      const uint32_t f = s_list[idx];
+      const int nx = idx + 1;
+      const uint32_t fn = nx < ntile ? s_list[nx] : 0u;
+      bool next_ready = false;
+      for (int i = 0; ok && i < 2; ++i) {
+        if ((fn >> i) & 1u) {
+          if (!next_ready) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[nx % ATT_STAGES],
+                                                   (nx / ATT_STAGES) & 1, SITE_KV_FULL));
+            next_ready = true;
+          }
+          if (ok && qk_cnt[i] > 0)
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(&s_free[i], (qk_cnt[i] - 1) & 1, SITE_S_FREE));
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            issue_qk(i, nx % ATT_STAGES);
+            tc_commit(&s_full[i]);
+          }
+          __syncwarp();
+          ++qk_cnt[i];
+        }
+        if ((f >> i) & 1u) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&p_full[i], pv_cnt[i] & 1, SITE_P_FULL));
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            issue_pv(i, st, pv_cnt[i] > 0);
+            tc_commit(&o_ready[i]);
+          }
+          __syncwarp();
+          ++pv_cnt[i];
+        }
+      }
+      if (lane == 0) tc_commit(&kv_empty[st]);
+      __syncwarp();
+    }
+    // every MMA issued above completes before the CTA tears down TMEM
+    if (lane == 0) tc_commit(mma_done);
+    __syncwarp();
+    mbar_wait(mma_done, 0, SITE_MMA_DONE);
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- softmax WGs
+    const int wg = warp >> 2;
+    const int rt = threadIdx.x & 127;
+    const int qt = qt0 + wg;
+    const int row = qt * ATT_BM + rt;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (uint32_t)(wg * 256);
+    const uint32_t tO = tS + 128;
+    uint8_t* sPw = sP + wg * L::P_BYTES;
+    const bool tile_exists = qt < a.nqt;
+    const float cq = tile_exists ? a.q_scale[(int64_t)bhq * a.nqt + qt] * a.c0 : 0.f;
+    const uint8_t* mrow = nullptr;
+    if (a.mask && row < a.Nq) {
+      const int bm = a.m_bcast_b ? 0 : b, hm = a.m_bcast_h ? 0 : h;
+      mrow = a.mask + bm * a.m_sb + hm * a.m_sh + (int64_t)row * a.m_sq;
+    }
+    float m = -INFINITY, l = 0.f;
+    uint32_t n = 0;
+    bool ok = true;
+    for (int idx = 0; idx < ntile; ++idx) {
+      const uint32_t e = s_list[idx];
+      if (!((e >> wg) & 1u)) continue;
+      const int kt = (int)(e >> 8);
+      const bool need = (e >> (2 + wg)) & 1u;
+      const bool part = (e >> (4 + wg)) & 1u;
+      const float c = cq * a.k_scale[(int64_t)bhk * a.nkt + kt];
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], n & 1, SITE_S_FULL));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[128];
+      SAGE_TMEM_LD32(tS + 0, (sr + 0));
+      SAGE_TMEM_LD32(tS + 32, (sr + 32));
+      SAGE_TMEM_LD32(tS + 64, (sr + 64));
+      SAGE_TMEM_LD32(tS + 96, (sr + 96));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&s_free[wg]);
+
+      // visibility of the 128 keys of this tile for this row (bit j of vis[j/32])
+      uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
+      if (need) {
+        const int key0 = kt * ATT_BN;
+        int jmax = min(ATT_BN - 1, a.Nk - 1 - key0);
+        if (a.causal) jmax = min(jmax, row + a.causal_off - key0);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int hi = jmax - 32 * w;  // keep bits 0..hi
+          vis[w] = hi >= 31 ? ~0u : (hi < 0 ? 0u : ((2u << hi) - 1u));
+        }
+        if (part && mrow) {
+          const uint8_t* mk = mrow + key0;
+          if (a.mask_vec16 && key0 + ATT_BN <= a.Nk) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint4 mv = __ldg(reinterpret_cast<const uint4*>(mk) + q);
+              const uint32_t wds[4] = {mv.x, mv.y, mv.z, mv.w};
+              uint32_t bits = 0;
+#pragma unroll
+              for (int t = 0; t < 16; ++t) bits |= (((wds[t >> 2] >> (8 * (t & 3))) & 0xFFu) ? 1u : 0u) << t;
+              vis[q >> 1] &= ~(((~bits) & 0xFFFFu) << (16 * (q & 1)));
+            }
+          } else {
+            for (int j = 0; j < ATT_BN; ++j)
+              if (key0 + j < a.Nk && mk[j] == 0) vis[j >> 5] &= ~(1u << (j & 31));
+          }
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 128; ++j) {
+        const float x = (float)(int)sr[j];
+        const bool v = (vis[j >> 5] >> (j & 31)) & 1u;
+        mx = v ? fmaxf(mx, x) : mx;
+      }
+      const float mt = mx == -INFINITY ? -INFINITY : mx * c;
+      const float m_new = fmaxf(m, mt);
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = ex2_approx(m - m_use);
+      const float bias = LOG2_448 - m_use;
+      float rs = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int j = 0; j < 128; j += 4) {
+        float p[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const bool v = (vis[(j + t) >> 5] >> ((j + t) & 31)) & 1u;
+          p[t] = v ? ex2_approx(fmaf((float)(int)sr[j + t], c, bias)) : 0.f;
+          rs += p[t];
+        }
+        pk[j >> 2] = (uint32_t)cvt_e4m3x2(p[0], p[1]) | ((uint32_t)cvt_e4m3x2(p[2], p[3]) << 16);
+      }
+      l = l * alpha + rs;
+
+      if (n > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[wg], (n - 1) & 1, SITE_O_READY));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int cb = 0; cb < D; cb += 32) {
+            uint32_t o[32];
+            SAGE_TMEM_LD32(tO + cb, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            SAGE_TMEM_ST32(tO + cb, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      store_p_row(sPw, rt, pk);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[wg]);
+      m = m_new;
+      ++n;
+    }
+    if (ok && n > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[wg], (n - 1) & 1, SITE_O_READY));
+      tc_fence_after();
+    }
+    if (tile_exists) {
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const bool live = ok && n > 0;
+      char* obase = reinterpret_cast<char*>(a.out) +
+                    ((int64_t)b * a.out_sb + (int64_t)h * a.out_sh + (int64_t)row * a.out_sn) * 2;
+#pragma unroll
+      for (int cb = 0; cb < D; cb += 32) {
+        uint32_t o[32];
+        if (live) {
+          SAGE_TMEM_LD32(tO + cb, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        if (row < a.Nq) {
+          if (a.out_fp16)
+            store_out_chunk<D, __half>(a, reinterpret_cast<__half*>(obase), cb, o, s_vs, inv_l);
+          else
+            store_out_chunk<D, __nv_bfloat16>(a, reinterpret_cast<__nv_bfloat16*>(obase), cb, o,
+                                              s_vs, inv_l);
+        }
+      }
+      if (a.return_lse && row < a.Nq) {
+        float v = -INFINITY;
+        if (l > 0.f) v = (m + log2f(l) - LOG2_448) * LN2_F + a.sm_scale * a.qdk[(int64_t)bhq * a.Nq + row];
+        a.lse[(int64_t)bhq * a.Nq + row] = v;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------ mask classes
+// One CTA per (mask batch/head, q tile, k tile): 0 = nothing visible,
+// 1 = everything visible, 2 = mixed.  Only rows < Nq and keys < Nk count.
+__global__ void __launch_bounds__(256) mask_classify_kernel(const uint8_t* __restrict__ mask,
+                                                            int64_t sb, int64_t sh, int64_t sq,
+                                                            int Hm, int Nq, int Nk, int nqt,
+                                                            int nkt, uint8_t* __restrict__ cls) {
+  const int kt = blockIdx.x, qt = blockIdx.y, bhm = blockIdx.z;
+  const int bm = bhm / Hm, hm = bhm % Hm;
+  const uint8_t* base = mask + bm * sb + hm * sh;
+  int any = 0, all = 1;
+  for (int idx = threadIdx.x; idx < ATT_BM * ATT_BN; idx += blockDim.x) {
+    const int r = qt * ATT_BM + idx / ATT_BN, c = kt * ATT_BN + idx % ATT_BN;
+    if (r < Nq && c < Nk) {
+      const int v = base[(int64_t)r * sq + c] != 0;
+      any |= v;
+      all &= v;
+    }
+  }
+  any = __syncthreads_or(any);
+  all = __syncthreads_and(all);
+  if (threadIdx.x == 0) cls[((int64_t)bhm * nqt + qt) * nkt + kt] = any ? (all ? 1 : 2) : 0;
+}
+
+// ------------------------------------------------------------ test kernels
+// One 128x128 int32 tile of Q K^T through the same TMA maps, descriptors
+// and kind::i8 MMA chain as the attention kernel.
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+    debug_qk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    int qrow, int krow, int32_t* __restrict__ tile) {
+  using L = AttnLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + L::Q_BYTES;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::Q_BYTES + L::K_BYTES);
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 2);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 32) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bar[0], L::Q_BYTES + L::K_BYTES);
+    tma_load_2d(sQ, &tmQ, &bar[0], 0, qrow);
+    tma_load_2d(sK, &tmK, &bar[0], 0, krow);
+    if (mbar_wait(&bar[0], 0, SITE_DEBUG)) {
+      tc_fence_after();
+      constexpr uint32_t IDESC = instr_desc(kDS32, kS8, kS8, ATT_BM, ATT_BN);
+#pragma unroll
+      for (int k = 0; k < D / 32; ++k)
+        mma_i8(tmem, smem_desc(smem_u32(sQ) + 32 * k, L::QK_SBO, L::QK_SWIZZLE),
+               smem_desc(smem_u32(sK) + 32 * k, L::QK_SBO, L::QK_SWIZZLE), IDESC, k > 0 ? 1u : 0u);
+    }
+    tc_commit(&bar[1]);
+  }
+  __syncwarp();
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar[1], 0, SITE_DEBUG));
+  tc_fence_after();
+  const int r = threadIdx.x;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+#pragma unroll
+  for (int cb = 0; cb < 128; cb += 32) {
+    uint32_t v[32];
+    SAGE_TMEM_LD32(tmem + lane_base + cb, v);
+    tmem_wait_ld();
+    if (ok)
+      for (int i = 0; i < 32; ++i) tile[r * 128 + cb + i] = (int32_t)v[i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// One P (threads -> swizzled smem) times V^T (TMA) tile, FP32 result.
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+    debug_pv_kernel(const __grid_constant__ CUtensorMap tmV, int vrow, int vcol,
+                    const uint8_t* __restrict__ p, float* __restrict__ acc) {
+  using L = AttnLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sP = smem;
+  uint8_t* sV = smem + L::P_BYTES;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::P_BYTES + L::V_BYTES);
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 2);
+  const int warp = threadIdx.x >> 5;
+  const int r = threadIdx.x;
+  if (threadIdx.x == 32) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(slot, 128);
+    tmem_relinquish();
+  }
+  uint32_t pk[32];
+  for (int i = 0; i < 32; ++i) pk[i] = __ldg(reinterpret_cast<const uint32_t*>(p + r * 128) + i);
+  store_p_row(sP, r, pk);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bar[0], L::V_BYTES);
+    tma_load_2d(sV, &tmV, &bar[0], vcol, vrow);
+    if (mbar_wait(&bar[0], 0, SITE_DEBUG)) {
+      tc_fence_after();
+      constexpr uint32_t IDESC = instr_desc(kDF32, kE4M3, kE4M3, ATT_BM, D);
+#pragma unroll
+      for (int k = 0; k < ATT_BN / 32; ++k)
+        mma_f8f6f4(tmem, smem_desc(smem_u32(sP) + 32 * k, 1024, 128),
+                   smem_desc(smem_u32(sV) + 32 * k, 1024, 128), IDESC, k > 0 ? 1u : 0u);
+    }
+    tc_commit(&bar[1]);
+  }
+  __syncwarp();
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar[1], 0, SITE_DEBUG));
+  tc_fence_after();
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+#pragma unroll
+  for (int cb = 0; cb < D; cb += 32) {
+    uint32_t v[32];
+    SAGE_TMEM_LD32(tmem + lane_base + cb, v);
+    tmem_wait_ld();
+    if (ok)
+      for (int i = 0; i < 32; ++i) acc[r * D + cb + i] = __uint_as_float(v[i]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// A single thread waits on a barrier that nothing arrives on.
+__global__ void debug_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0, SITE_DEBUG, limit_ns);
+  }
+}
+
+}  // namespace sage

@@ -1,0 +1,343 @@
+// quantize_i8f8.cuh -- quantisation stage of the INT8-QK / FP8-PV attention
+// (thu-ml/sageattention llms.txt: "smooth_k", per-block INT8 Q/K in
+// "sageattn_qk_int8_pv_fp16_triton", per-channel FP8 V in
+// "sageattn_qk_int8_pv_fp8_cuda").
+//
+// Two launches, both HBM-bound, 128-bit coalesced loads and stores:
+//   pass A  per (batch, KV head, token split): exact-in-practice K channel
+//           sums (double-double accumulation, fixed reduction order) and V
+//           channel maxima into the workspace;
+//   pass B  one CTA per 128-token block of Q, K or V: the block's amax,
+//           scale and INT8 codes (Q, K - kmean) or the E4M3 codes of V,
+//           transposed through shared memory.
+// Every arithmetic step that decides a code uses an explicitly rounded
+// IEEE operation (__fsub_rn, __fmul_rn, __fdiv_rn, cvt.rn), so the codes and
+// scales are reproducible bit for bit.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "sage_ptx.cuh"
+
+namespace sage {
+
+constexpr int QB = 128;           // tokens per quantisation block
+constexpr int QUANT_THREADS = 256;
+
+struct QuantArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int64_t q_sb, q_sh, q_sn, k_sb, k_sh, k_sn, v_sb, v_sh, v_sn;
+  int B, Hq, Hkv, G, Nq, Nk, Nqp, Nkp, nqt, nkt;
+  int smooth_k;
+  int splits, split_tokens;       // pass A token splits
+  double* part_hi;                // [B*Hkv, splits, D]
+  double* part_lo;
+  float* part_amax;
+  int8_t* q8;
+  float* q_scale;
+  int8_t* k8;
+  float* k_scale;
+  float* k_mean;
+  uint8_t* v8t;
+  float* v_scale;
+  float* qdk;                     // may be null
+  int kv_limit;                   // tokens of K/V used for the mean / codes (Nk)
+};
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half x) {
+  return __half2float(x);
+}
+
+// 8 consecutive elements (one 16-byte load) as fp32.
+template <typename T>
+__device__ __forceinline__ void unpack8(const uint4& raw, float* f) {
+  const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = to_f32<T>(e[i]);
+}
+
+__device__ __forceinline__ uint4 ldg16(const void* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// ------------------------------------------------------------ double-double
+struct DD {
+  double hi, lo;
+};
+// hi + lo += x without rounding error in hi + x (error-free transformation).
+__device__ __forceinline__ void dd_add(DD& acc, double x) {
+  const double s = __dadd_rn(acc.hi, x);
+  const double bb = __dsub_rn(s, acc.hi);
+  const double err = __dadd_rn(__dsub_rn(acc.hi, __dsub_rn(s, bb)), __dsub_rn(x, bb));
+  acc.hi = s;
+  acc.lo = __dadd_rn(acc.lo, err);
+}
+__device__ __forceinline__ void dd_add(DD& acc, const DD& y) {
+  dd_add(acc, y.hi);
+  acc.lo = __dadd_rn(acc.lo, y.lo);
+}
+// fp32 value of (hi + lo) / n rounded once (see DESIGN notes on exactness).
+__device__ __forceinline__ float dd_mean_f32(const DD& s, double n) {
+  const double q1 = __ddiv_rn(s.hi, n);
+  const double r = __fma_rn(-q1, n, s.hi);  // exact remainder of the division
+  const double q2 = __ddiv_rn(__dadd_rn(r, s.lo), n);
+  return __double2float_rn(__dadd_rn(q1, q2));
+}
+
+// ------------------------------------------------------------ pass A
+// grid (splits, B*Hkv), 256 threads.  Thread layout: D/8 threads per token
+// row (one 16-byte load each), 256/(D/8) rows per step.
+template <typename T, int D>
+__global__ void __launch_bounds__(QUANT_THREADS) kmean_vamax_partial_kernel(QuantArgs a) {
+  constexpr int TPR = D / 8;
+  constexpr int RPP = QUANT_THREADS / TPR;
+  __shared__ double s_hi[RPP][D];
+  __shared__ double s_lo[RPP][D];
+  __shared__ float s_am[RPP][D];
+
+  const int split = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / a.Hkv, h = bh % a.Hkv;
+  const int cg = threadIdx.x % TPR, rs = threadIdx.x / TPR;
+  const int n0 = split * a.split_tokens;
+  const int n1 = min(a.kv_limit, n0 + a.split_tokens);
+
+  DD acc[8];
+  float am[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    acc[i] = {0.0, 0.0};
+    am[i] = 0.f;
+  }
+  const char* kb = reinterpret_cast<const char*>(a.k) +
+                   (b * a.k_sb + h * a.k_sh + cg * 8) * (int64_t)sizeof(T);
+  const char* vb = reinterpret_cast<const char*>(a.v) +
+                   (b * a.v_sb + h * a.v_sh + cg * 8) * (int64_t)sizeof(T);
+  for (int n = n0 + rs; n < n1; n += RPP) {
+    float f[8];
+    if (a.smooth_k) {
+      unpack8<T>(ldg16(kb + (int64_t)n * a.k_sn * sizeof(T)), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dd_add(acc[i], (double)f[i]);
+    }
+    unpack8<T>(ldg16(vb + (int64_t)n * a.v_sn * sizeof(T)), f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) am[i] = fmaxf(am[i], fabsf(f[i]));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    s_hi[rs][cg * 8 + i] = acc[i].hi;
+    s_lo[rs][cg * 8 + i] = acc[i].lo;
+    s_am[rs][cg * 8 + i] = am[i];
+  }
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    DD s = {0.0, 0.0};
+    float m = 0.f;
+    for (int r = 0; r < RPP; ++r) {  // fixed order: deterministic
+      dd_add(s, DD{s_hi[r][c], s_lo[r][c]});
+      m = fmaxf(m, s_am[r][c]);
+    }
+    const int64_t o = ((int64_t)bh * a.splits + split) * D + c;
+    a.part_hi[o] = s.hi;
+    a.part_lo[o] = s.lo;
+    a.part_amax[o] = m;
+  }
+}
+
+// Combine the splits of KV head (b, h) in fixed order: kmean and V amax.
+template <int D>
+__device__ __forceinline__ void combine_splits(const QuantArgs& a, int bh, float* s_km,
+                                               float* s_va) {
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    DD s = {0.0, 0.0};
+    float m = 0.f;
+    for (int sp = 0; sp < a.splits; ++sp) {
+      const int64_t o = ((int64_t)bh * a.splits + sp) * D + c;
+      dd_add(s, DD{a.part_hi[o], a.part_lo[o]});
+      m = fmaxf(m, a.part_amax[o]);
+    }
+    if (s_km) s_km[c] = a.smooth_k ? dd_mean_f32(s, (double)a.kv_limit) : 0.f;
+    if (s_va) s_va[c] = m;
+  }
+}
+
+__device__ __forceinline__ float block_max(float v, float* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) s_red[w] = v;
+  __syncthreads();
+  float r = s_red[0];
+#pragma unroll
+  for (int i = 1; i < QUANT_THREADS / 32; ++i) r = fmaxf(r, s_red[i]);
+  return r;
+}
+
+__device__ __forceinline__ int8_t int8_code(float x, float inv) {
+  int c = __float2int_rn(__fmul_rn(x, inv));
+  c = max(-127, min(127, c));
+  return (int8_t)c;
+}
+
+// ------------------------------------------------------------ pass B
+// One CTA per 128-token block: [0, nQb) Q blocks, [nQb, nQb+nKb) K blocks,
+// then V blocks.
+template <typename T, int D>
+__global__ void __launch_bounds__(QUANT_THREADS) quant_blocks_kernel(QuantArgs a) {
+  constexpr int TPR = D / 8;
+  constexpr int RPP = QUANT_THREADS / TPR;
+  constexpr int ITERS = QB / RPP;
+  __shared__ float s_km[D];
+  __shared__ float s_va[D];
+  __shared__ float s_red[QUANT_THREADS / 32];
+  __shared__ __align__(16) uint8_t s_vt[D][QB + 16];
+
+  const int nQb = a.B * a.Hq * a.nqt;
+  const int nKb = a.B * a.Hkv * a.nkt;
+  int job = blockIdx.x;
+  const int cg = threadIdx.x % TPR, rs = threadIdx.x / TPR;
+
+  if (job < nQb) {
+    // ---------------- Q block
+    const int bh = job / a.nqt, qt = job % a.nqt;
+    const int b = bh / a.Hq, h = bh % a.Hq;
+    const int g = h / a.G;
+    if (a.qdk) combine_splits<D>(a, b * a.Hkv + g, s_km, nullptr);
+    const char* base = reinterpret_cast<const char*>(a.q) +
+                       (b * a.q_sb + h * a.q_sh + cg * 8) * (int64_t)sizeof(T);
+    uint4 raw[ITERS];
+    float am = 0.f;
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int n = qt * QB + rs + it * RPP;
+      raw[it] = n < a.Nq ? ldg16(base + (int64_t)n * a.q_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
+      float f[8];
+      unpack8<T>(raw[it], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(f[i]));
+    }
+    const float amax = block_max(am, s_red);  // also orders s_km
+    const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int n = qt * QB + rs + it * RPP;
+      float f[8];
+      unpack8<T>(raw[it], f);
+      uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w0 |= (uint32_t)(uint8_t)int8_code(f[i], inv) << (8 * i);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w1 |= (uint32_t)(uint8_t)int8_code(f[4 + i], inv) << (8 * i);
+      *reinterpret_cast<uint2*>(a.q8 + ((int64_t)bh * a.Nqp + n) * D + cg * 8) = make_uint2(w0, w1);
+      if (a.qdk) {
+        float d = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d = fmaf(f[i], s_km[cg * 8 + i], d);
+#pragma unroll
+        for (int o = TPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        if (cg == 0 && n < a.Nq) a.qdk[(int64_t)bh * a.Nq + n] = d;
+      }
+    }
+    if (threadIdx.x == 0) a.q_scale[(int64_t)bh * a.nqt + qt] = __fdiv_rn(amax, 127.f);
+    return;
+  }
+  job -= nQb;
+  if (job < nKb) {
+    // ---------------- K block: codes of K - kmean
+    const int bh = job / a.nkt, kt = job % a.nkt;
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    combine_splits<D>(a, bh, s_km, nullptr);
+    __syncthreads();
+    const char* base = reinterpret_cast<const char*>(a.k) +
+                       (b * a.k_sb + h * a.k_sh + cg * 8) * (int64_t)sizeof(T);
+    float x[ITERS][8];
+    float am = 0.f;
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int n = kt * QB + rs + it * RPP;
+      if (n < a.kv_limit) {
+        float f[8];
+        unpack8<T>(ldg16(base + (int64_t)n * a.k_sn * sizeof(T)), f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[it][i] = __fsub_rn(f[i], s_km[cg * 8 + i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[it][i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(x[it][i]));
+    }
+    const float amax = block_max(am, s_red);
+    const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int n = kt * QB + rs + it * RPP;
+      uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w0 |= (uint32_t)(uint8_t)int8_code(x[it][i], inv) << (8 * i);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w1 |= (uint32_t)(uint8_t)int8_code(x[it][4 + i], inv) << (8 * i);
+      *reinterpret_cast<uint2*>(a.k8 + ((int64_t)bh * a.Nkp + n) * D + cg * 8) = make_uint2(w0, w1);
+    }
+    if (threadIdx.x == 0) a.k_scale[(int64_t)bh * a.nkt + kt] = __fdiv_rn(amax, 127.f);
+    if (kt == 0)
+      for (int c = threadIdx.x; c < D; c += blockDim.x) a.k_mean[(int64_t)bh * D + c] = s_km[c];
+    return;
+  }
+  job -= nKb;
+  {
+    // ---------------- V block: E4M3 codes, transposed
+    const int bh = job / a.nkt, vt = job % a.nkt;
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    combine_splits<D>(a, bh, nullptr, s_va);
+    __syncthreads();
+    const char* base = reinterpret_cast<const char*>(a.v) +
+                       (b * a.v_sb + h * a.v_sh + cg * 8) * (int64_t)sizeof(T);
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int nl = rs + it * RPP;
+      const int n = vt * QB + nl;
+      float f[8];
+      if (n < a.kv_limit) {
+        unpack8<T>(ldg16(base + (int64_t)n * a.v_sn * sizeof(T)), f);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        const float va0 = s_va[cg * 8 + i], va1 = s_va[cg * 8 + i + 1];
+        const float y0 = va0 > 0.f ? __fmul_rn(f[i], __fdiv_rn(448.f, va0)) : 0.f;
+        const float y1 = va1 > 0.f ? __fmul_rn(f[i + 1], __fdiv_rn(448.f, va1)) : 0.f;
+        uint16_t two = cvt_e4m3x2(y0, y1);
+        if (n >= a.kv_limit) two = 0;
+        s_vt[cg * 8 + i][nl] = (uint8_t)(two & 0xFF);
+        s_vt[cg * 8 + i + 1][nl] = (uint8_t)(two >> 8);
+      }
+    }
+    __syncthreads();
+    // write D rows of 128 bytes: 8 threads x 16 bytes per channel row
+    for (int idx = threadIdx.x; idx < D * 8; idx += blockDim.x) {
+      const int c = idx >> 3, ch = idx & 7;
+      const uint4 val = *reinterpret_cast<const uint4*>(&s_vt[c][ch * 16]);
+      *reinterpret_cast<uint4*>(a.v8t + ((int64_t)bh * D + c) * a.Nkp + vt * QB + ch * 16) = val;
+    }
+    if (vt == 0)
+      for (int c = threadIdx.x; c < D; c += blockDim.x)
+        a.v_scale[(int64_t)bh * D + c] = __fdiv_rn(s_va[c], 448.f);
+  }
+}
+
+}  // namespace sage

@@ -1,0 +1,479 @@
+// sage_b200.cu -- the C ABI of include/sage_b200.h: argument validation,
+// workspace layout, TMA descriptors and kernel launches.  Built as one
+// translation unit with the kernel headers (device state such as the status
+// word lives here once).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "sage_b200.h"
+#include "sage_ptx.cuh"
+#include "quantize_i8f8.cuh"
+#include "attn_fwd_i8f8.cuh"
+
+using namespace sage;
+
+namespace {
+
+constexpr int kSMs = 148;
+
+int64_t pad128(int64_t n) { return (n + 127) / 128 * 128; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool log_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("SAGE_LOG");
+    return e && e[0] == '1';
+  }();
+  return on;
+}
+
+// ---------------------------------------------------------------- checks
+bool valid_dims(int64_t B, int64_t H, int64_t N, int64_t D) {
+  return B >= 1 && H >= 1 && N >= 1 && D >= 1 && B <= (1 << 16) && H <= (1 << 12);
+}
+
+sage_status check_tensor(const sage_tensor* t) {
+  if (!t || !t->ptr) return SAGE_ERR_INVALID_ARG;
+  if (t->dtype != SAGE_BF16 && t->dtype != SAGE_FP16) return SAGE_ERR_INVALID_ARG;
+  if (!valid_dims(t->B, t->H, t->N, t->D)) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(t->ptr)) return SAGE_ERR_INVALID_ARG;
+  if (t->sn < t->D || t->sn % 8 || t->sh % 8 || t->sb % 8 || t->sh < 0 || t->sb < 0)
+    return SAGE_ERR_INVALID_ARG;
+  if (t->D != 64 && t->D != 128) return SAGE_ERR_UNSUPPORTED;
+  if (t->N > 128 * ATT_MAX_NKT) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+sage_status check_qkv_shapes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk,
+                             int64_t D) {
+  if (!valid_dims(B, Hq, Nq, D) || !valid_dims(B, Hkv, Nk, D)) return SAGE_ERR_INVALID_ARG;
+  if (Hq % Hkv) return SAGE_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+  if (Nq > 128 * ATT_MAX_NKT || Nk > 128 * ATT_MAX_NKT) return SAGE_ERR_UNSUPPORTED;
+  // TMA row coordinates are int32
+  if (B * Hq * pad128(Nq) >= (int64_t(1) << 31) || B * Hkv * pad128(Nk) >= (int64_t(1) << 31) ||
+      B * Hkv * D >= (int64_t(1) << 31))
+    return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+sage_status check_qkv(const sage_qkv_i8f8* z, bool need_qdk) {
+  if (!z) return SAGE_ERR_INVALID_ARG;
+  sage_status st = check_qkv_shapes(z->B, z->Hq, z->Hkv, z->Nq, z->Nk, z->D);
+  if (st != SAGE_OK) return st;
+  if (!z->q || !z->q_scale || !z->k || !z->k_scale || !z->k_mean || !z->v_t || !z->v_scale)
+    return SAGE_ERR_INVALID_ARG;
+  if (need_qdk && !z->q_dot_kmean) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(z->q) || !aligned16(z->k) || !aligned16(z->v_t)) return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
+}
+
+sage_status check_mask(const sage_mask* m, int64_t B, int64_t Hq, int64_t Nq, int64_t Nk) {
+  if (!m) return SAGE_OK;
+  if (!m->ptr) return SAGE_ERR_INVALID_ARG;
+  if (!(m->B == 1 || m->B == B) || !(m->H == 1 || m->H == Hq)) return SAGE_ERR_INVALID_ARG;
+  if (m->Nq != Nq || m->Nk != Nk) return SAGE_ERR_INVALID_ARG;
+  if (m->sq < Nk || (m->B > 1 && m->sb < 0) || (m->H > 1 && m->sh < 0)) return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
+}
+
+size_t mask_class_bytes(const sage_mask* m, int64_t Nq, int64_t Nk) {
+  if (!m) return 0;
+  return align256((size_t)m->B * m->H * (pad128(Nq) / 128) * (pad128(Nk) / 128));
+}
+
+// ---------------------------------------------------------------- pass A plan
+struct QuantPlan {
+  int splits, split_tokens;
+  size_t part_bytes;  // hi + lo + amax
+};
+
+QuantPlan quant_plan(int64_t B, int64_t Hkv, int64_t Nk, int64_t D) {
+  const int64_t bh = B * Hkv;
+  const int64_t max_split = std::max<int64_t>(1, (Nk + 255) / 256);
+  const int64_t want = std::max<int64_t>(1, (2 * kSMs + bh - 1) / bh);
+  int64_t s = std::min(want, max_split);
+  int64_t t = ((Nk + s - 1) / s + 31) / 32 * 32;
+  s = (Nk + t - 1) / t;
+  QuantPlan p;
+  p.splits = (int)s;
+  p.split_tokens = (int)t;
+  const size_t n = (size_t)bh * s * D;
+  p.part_bytes = align256(n * 8) * 2 + align256(n * 4);
+  return p;
+}
+
+// ---------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D byte tensor [outer][inner] with rows `row_bytes` apart, box
+// [box_outer][box_inner].
+bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                  CUtensorMapSwizzle sw) {
+  auto enc = tmap_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+CUtensorMapSwizzle qk_swizzle(int64_t D) {
+  return D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+}
+
+bool make_qkv_tmaps(const sage_qkv_i8f8* z, CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv) {
+  const int64_t Nqp = pad128(z->Nq), Nkp = pad128(z->Nk), D = z->D;
+  return make_tmap_u8(tq, z->q, D, z->B * z->Hq * Nqp, D, (uint32_t)D, 128, qk_swizzle(D)) &&
+         make_tmap_u8(tk, z->k, D, z->B * z->Hkv * Nkp, D, (uint32_t)D, 128, qk_swizzle(D)) &&
+         make_tmap_u8(tv, z->v_t, Nkp, z->B * z->Hkv * D, Nkp, 128, (uint32_t)D,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Dynamic shared memory opt-in, once per device and kernel.
+template <typename K>
+bool ensure_smem(K kernel, size_t bytes, std::atomic<uint32_t>* flags) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 32) return false;
+  const uint32_t bit = 1u << dev;
+  if (flags->load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess)
+    return false;
+  flags->fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+
+sage_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- quantise
+sage_status run_quantize(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                         int smooth_k, const sage_qkv_i8f8* out, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+  sage_status st;
+  if ((st = check_tensor(q)) || (st = check_tensor(k)) || (st = check_tensor(v))) return st;
+  if (!out) return SAGE_ERR_INVALID_ARG;
+  if (q->dtype != k->dtype || q->dtype != v->dtype) return SAGE_ERR_INVALID_ARG;
+  if (k->B != q->B || v->B != q->B || k->H != v->H || k->N != v->N || k->D != q->D ||
+      v->D != q->D)
+    return SAGE_ERR_INVALID_ARG;
+  if ((st = check_qkv(out, false))) return st;
+  if (out->B != q->B || out->Hq != q->H || out->Hkv != k->H || out->Nq != q->N ||
+      out->Nk != k->N || out->D != q->D)
+    return SAGE_ERR_INVALID_ARG;
+  const QuantPlan plan = quant_plan(k->B, k->H, k->N, k->D);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < plan.part_bytes) return SAGE_ERR_WORKSPACE;
+
+  QuantArgs a{};
+  a.q = q->ptr;
+  a.k = k->ptr;
+  a.v = v->ptr;
+  a.q_sb = q->sb; a.q_sh = q->sh; a.q_sn = q->sn;
+  a.k_sb = k->sb; a.k_sh = k->sh; a.k_sn = k->sn;
+  a.v_sb = v->sb; a.v_sh = v->sh; a.v_sn = v->sn;
+  a.B = (int)q->B; a.Hq = (int)q->H; a.Hkv = (int)k->H; a.G = a.Hq / a.Hkv;
+  a.Nq = (int)q->N; a.Nk = (int)k->N;
+  a.Nqp = (int)pad128(q->N); a.Nkp = (int)pad128(k->N);
+  a.nqt = a.Nqp / 128; a.nkt = a.Nkp / 128;
+  a.smooth_k = smooth_k ? 1 : 0;
+  a.splits = plan.splits;
+  a.split_tokens = plan.split_tokens;
+  const size_t n = (size_t)a.B * a.Hkv * plan.splits * q->D;
+  char* w = static_cast<char*>(ws);
+  a.part_hi = reinterpret_cast<double*>(w);
+  a.part_lo = reinterpret_cast<double*>(w + align256(n * 8));
+  a.part_amax = reinterpret_cast<float*>(w + 2 * align256(n * 8));
+  a.q8 = out->q; a.q_scale = out->q_scale; a.k8 = out->k; a.k_scale = out->k_scale;
+  a.k_mean = out->k_mean; a.v8t = out->v_t; a.v_scale = out->v_scale; a.qdk = out->q_dot_kmean;
+  a.kv_limit = a.Nk;
+
+  const dim3 gridA(plan.splits, a.B * a.Hkv);
+  const int nblocks = a.B * a.Hq * a.nqt + 2 * a.B * a.Hkv * a.nkt;
+  if (log_enabled())
+    std::fprintf(stderr, "[sage] quantize B=%d Hq=%d Hkv=%d Nq=%d Nk=%d D=%lld splits=%d x %d, blocks=%d\n",
+                 a.B, a.Hq, a.Hkv, a.Nq, a.Nk, (long long)q->D, plan.splits, plan.split_tokens, nblocks);
+  const bool fp16 = q->dtype == SAGE_FP16;
+  if (q->D == 128) {
+    if (fp16) {
+      kmean_vamax_partial_kernel<__half, 128><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      quant_blocks_kernel<__half, 128><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
+    } else {
+      kmean_vamax_partial_kernel<__nv_bfloat16, 128><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      quant_blocks_kernel<__nv_bfloat16, 128><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
+    }
+  } else {
+    if (fp16) {
+      kmean_vamax_partial_kernel<__half, 64><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      quant_blocks_kernel<__half, 64><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
+    } else {
+      kmean_vamax_partial_kernel<__nv_bfloat16, 64><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      quant_blocks_kernel<__nv_bfloat16, 64><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
+    }
+  }
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- attention
+std::atomic<uint32_t> g_smem_set_64{0}, g_smem_set_128{0};
+
+sage_status run_attention(const sage_qkv_i8f8* z, int causal, float sm_scale, int return_lse,
+                          const sage_mask* mask, void* out, int32_t out_dtype, int64_t out_sb,
+                          int64_t out_sh, int64_t out_sn, float* lse, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+  sage_status st;
+  if ((st = check_qkv(z, return_lse != 0))) return st;
+  if (!out || !aligned16(out)) return SAGE_ERR_INVALID_ARG;
+  if (out_dtype != SAGE_BF16 && out_dtype != SAGE_FP16) return SAGE_ERR_INVALID_ARG;
+  if (out_sn < z->D || out_sn % 8 || out_sh % 8 || out_sb % 8 || out_sh < 0 || out_sb < 0)
+    return SAGE_ERR_INVALID_ARG;
+  if ((return_lse != 0) != (lse != nullptr)) return SAGE_ERR_INVALID_ARG;
+  if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_mask(mask, z->B, z->Hq, z->Nq, z->Nk))) return st;
+  const size_t need = mask_class_bytes(mask, z->Nq, z->Nk);
+  if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))) return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < need) return SAGE_ERR_WORKSPACE;
+
+  AttnArgs a{};
+  a.q_scale = z->q_scale; a.k_scale = z->k_scale; a.v_scale = z->v_scale; a.qdk = z->q_dot_kmean;
+  a.out = out; a.out_sb = out_sb; a.out_sh = out_sh; a.out_sn = out_sn;
+  a.out_fp16 = out_dtype == SAGE_FP16;
+  a.lse = lse;
+  a.B = (int)z->B; a.Hq = (int)z->Hq; a.Hkv = (int)z->Hkv; a.G = a.Hq / a.Hkv;
+  a.Nq = (int)z->Nq; a.Nk = (int)z->Nk;
+  a.Nqp = (int)pad128(z->Nq); a.Nkp = (int)pad128(z->Nk);
+  a.nqt = a.Nqp / 128; a.nkt = a.Nkp / 128; a.nqp = (a.nqt + 1) / 2;
+  a.causal = causal ? 1 : 0;
+  a.return_lse = return_lse ? 1 : 0;
+  a.causal_off = a.Nk - a.Nq;
+  const float s = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)z->D);
+  a.sm_scale = s;
+  a.c0 = (float)((double)s * 1.4426950408889634);
+  if (mask) {
+    a.mask = mask->ptr;
+    a.m_sb = mask->sb; a.m_sh = mask->sh; a.m_sq = mask->sq;
+    a.m_bcast_b = mask->B == 1; a.m_bcast_h = mask->H == 1;
+    a.mask_vec16 = aligned16(mask->ptr) && mask->sq % 16 == 0 &&
+                   (mask->B == 1 || mask->sb % 16 == 0) && (mask->H == 1 || mask->sh % 16 == 0);
+    uint8_t* cls = static_cast<uint8_t*>(ws);
+    a.tile_class = cls;
+    const int Hm = (int)mask->H;
+    mask_classify_kernel<<<dim3(a.nkt, a.nqt, (unsigned)(mask->B * mask->H)), 256, 0, stream>>>(
+        mask->ptr, mask->B == 1 ? 0 : mask->sb, mask->H == 1 ? 0 : mask->sh, mask->sq, Hm, a.Nq,
+        a.Nk, a.nqt, a.nkt, cls);
+    if ((st = launch_status())) return st;
+  }
+  CUtensorMap tq, tk, tv;
+  if (!make_qkv_tmaps(z, &tq, &tk, &tv)) return SAGE_ERR_CUDA;
+  const int grid = a.nqp * a.B * a.Hq;
+  if (log_enabled())
+    std::fprintf(stderr, "[sage] attn B=%d Hq=%d Hkv=%d Nq=%d Nk=%d D=%lld causal=%d grid=%d\n", a.B,
+                 a.Hq, a.Hkv, a.Nq, a.Nk, (long long)z->D, a.causal, grid);
+  if (z->D == 128) {
+    const size_t smem = AttnLayout<128>::bytes(a.nkt);
+    if (!ensure_smem(attn_fwd_i8f8_kernel<128>, AttnLayout<128>::bytes(ATT_MAX_NKT), &g_smem_set_128))
+      return SAGE_ERR_CUDA;
+    attn_fwd_i8f8_kernel<128><<<grid, ATT_THREADS, smem, stream>>>(tq, tk, tv, a);
+  } else {
+    const size_t smem = AttnLayout<64>::bytes(a.nkt);
+    if (!ensure_smem(attn_fwd_i8f8_kernel<64>, AttnLayout<64>::bytes(ATT_MAX_NKT), &g_smem_set_64))
+      return SAGE_ERR_CUDA;
+    attn_fwd_i8f8_kernel<64><<<grid, ATT_THREADS, smem, stream>>>(tq, tk, tv, a);
+  }
+  return launch_status();
+}
+
+// Carve the fused call's workspace: quantised Q/K/V, then the quantiser's
+// partials, then the mask classes.
+struct FusedLayout {
+  size_t q8, qs, k8, ks, km, v8, vs, qdk, part, cls, total;
+};
+FusedLayout fused_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
+                         const sage_mask* mask) {
+  const int64_t Nqp = pad128(Nq), Nkp = pad128(Nk);
+  FusedLayout f{};
+  size_t o = 0;
+  f.q8 = o; o += align256((size_t)B * Hq * Nqp * D);
+  f.qs = o; o += align256((size_t)B * Hq * (Nqp / 128) * 4);
+  f.k8 = o; o += align256((size_t)B * Hkv * Nkp * D);
+  f.ks = o; o += align256((size_t)B * Hkv * (Nkp / 128) * 4);
+  f.km = o; o += align256((size_t)B * Hkv * D * 4);
+  f.v8 = o; o += align256((size_t)B * Hkv * D * Nkp);
+  f.vs = o; o += align256((size_t)B * Hkv * D * 4);
+  f.qdk = o; o += align256((size_t)B * Hq * Nq * 4);
+  f.part = o; o += quant_plan(B, Hkv, Nk, D).part_bytes;
+  f.cls = o; o += mask_class_bytes(mask, Nq, Nk);
+  f.total = o;
+  return f;
+}
+
+std::atomic<uint32_t> g_smem_dbg_qk{0}, g_smem_dbg_pv{0};
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* sage_status_str(sage_status s) {
+  switch (s) {
+    case SAGE_OK: return "ok";
+    case SAGE_ERR_INVALID_ARG: return "invalid argument";
+    case SAGE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SAGE_ERR_WORKSPACE: return "workspace too small";
+    case SAGE_ERR_CUDA: return "CUDA error";
+    case SAGE_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* sage_version(void) { return "sage_b200 0.1 (sm_100a)"; }
+
+sage_status sage_get_device_status(sage_stream_t stream, uint32_t* site) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SAGE_ERR_CUDA;
+  uint32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (v && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (site) *site = v;
+  return v ? SAGE_ERR_TIMEOUT : SAGE_OK;
+}
+
+size_t sage_quantize_workspace_bytes(int64_t B, int64_t Hkv, int64_t Nk, int64_t D) {
+  if (!valid_dims(B, Hkv, Nk, D)) return 0;
+  return quant_plan(B, Hkv, Nk, D).part_bytes;
+}
+
+sage_status sage_quantize_qkv(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                              int smooth_k, const sage_qkv_i8f8* out, void* ws, size_t ws_bytes,
+                              sage_stream_t stream) {
+  return run_quantize(q, k, v, smooth_k, out, ws, ws_bytes, stream);
+}
+
+size_t sage_attn_quantized_workspace_bytes(const sage_qkv_i8f8* z, const sage_mask* mask) {
+  if (!z) return 0;
+  return mask_class_bytes(mask, z->Nq, z->Nk);
+}
+
+sage_status sage_attn_fwd_quantized(const sage_qkv_i8f8* qkv, int causal, float sm_scale,
+                                    int return_lse, const sage_mask* mask, void* out,
+                                    int32_t out_dtype, int64_t out_sb, int64_t out_sh,
+                                    int64_t out_sn, float* lse, void* ws, size_t ws_bytes,
+                                    sage_stream_t stream) {
+  return run_attention(qkv, causal, sm_scale, return_lse, mask, out, out_dtype, out_sb, out_sh,
+                       out_sn, lse, ws, ws_bytes, stream);
+}
+
+size_t sage_attn_fwd_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk,
+                                     int64_t D, const sage_mask* mask) {
+  if (!valid_dims(B, Hq, Nq, D) || !valid_dims(B, Hkv, Nk, D)) return 0;
+  return fused_layout(B, Hq, Hkv, Nq, Nk, D, mask).total;
+}
+
+sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                          int causal, float sm_scale, int num_kv_heads, int return_lse,
+                          int smooth_k, const sage_mask* mask, void* out, int64_t out_sb,
+                          int64_t out_sh, int64_t out_sn, float* lse, void* ws, size_t ws_bytes,
+                          sage_stream_t stream) {
+  sage_status st;
+  if ((st = check_tensor(q)) || (st = check_tensor(k)) || (st = check_tensor(v))) return st;
+  if (num_kv_heads != k->H) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_qkv_shapes(q->B, q->H, k->H, q->N, k->N, q->D))) return st;
+  if ((st = check_mask(mask, q->B, q->H, q->N, k->N))) return st;
+  const FusedLayout f = fused_layout(q->B, q->H, k->H, q->N, k->N, q->D, mask);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < f.total) return SAGE_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  sage_qkv_i8f8 z{};
+  z.q = reinterpret_cast<int8_t*>(w + f.q8);
+  z.q_scale = reinterpret_cast<float*>(w + f.qs);
+  z.k = reinterpret_cast<int8_t*>(w + f.k8);
+  z.k_scale = reinterpret_cast<float*>(w + f.ks);
+  z.k_mean = reinterpret_cast<float*>(w + f.km);
+  z.v_t = reinterpret_cast<uint8_t*>(w + f.v8);
+  z.v_scale = reinterpret_cast<float*>(w + f.vs);
+  z.q_dot_kmean = return_lse ? reinterpret_cast<float*>(w + f.qdk) : nullptr;
+  z.B = q->B; z.Hq = q->H; z.Hkv = k->H; z.Nq = q->N; z.Nk = k->N; z.D = q->D;
+  if ((st = run_quantize(q, k, v, smooth_k, &z, w + f.part, f.cls - f.part, stream))) return st;
+  return run_attention(&z, causal, sm_scale, return_lse, mask, out, q->dtype, out_sb, out_sh,
+                       out_sn, lse, w + f.cls, f.total - f.cls, stream);
+}
+
+sage_status sage_debug_qk_int32(const sage_qkv_i8f8* z, int64_t b, int64_t h, int64_t qblk,
+                                int64_t kblk, int32_t* tile, sage_stream_t stream) {
+  sage_status st;
+  if ((st = check_qkv(z, false))) return st;
+  if (!tile || b < 0 || b >= z->B || h < 0 || h >= z->Hq || qblk < 0 ||
+      qblk >= pad128(z->Nq) / 128 || kblk < 0 || kblk >= pad128(z->Nk) / 128)
+    return SAGE_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv;
+  if (!make_qkv_tmaps(z, &tq, &tk, &tv)) return SAGE_ERR_CUDA;
+  const int64_t g = h / (z->Hq / z->Hkv);
+  const int qrow = (int)((b * z->Hq + h) * pad128(z->Nq) + qblk * 128);
+  const int krow = (int)((b * z->Hkv + g) * pad128(z->Nk) + kblk * 128);
+  if (z->D == 128) {
+    const size_t smem = 1024 + AttnLayout<128>::Q_BYTES + AttnLayout<128>::K_BYTES + 64;
+    if (!ensure_smem(debug_qk_kernel<128>, smem, &g_smem_dbg_qk)) return SAGE_ERR_CUDA;
+    debug_qk_kernel<128><<<1, 128, smem, stream>>>(tq, tk, qrow, krow, tile);
+  } else {
+    const size_t smem = 1024 + AttnLayout<64>::Q_BYTES + AttnLayout<64>::K_BYTES + 64;
+    debug_qk_kernel<64><<<1, 128, smem, stream>>>(tq, tk, qrow, krow, tile);
+  }
+  return launch_status();
+}
+
+sage_status sage_debug_pv_fp32(const sage_qkv_i8f8* z, const uint8_t* p, int64_t b, int64_t h_kv,
+                               int64_t kblk, float* acc, sage_stream_t stream) {
+  sage_status st;
+  if ((st = check_qkv(z, false))) return st;
+  if (!p || !acc || !aligned16(p) || b < 0 || b >= z->B || h_kv < 0 || h_kv >= z->Hkv ||
+      kblk < 0 || kblk >= pad128(z->Nk) / 128)
+    return SAGE_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv;
+  if (!make_qkv_tmaps(z, &tq, &tk, &tv)) return SAGE_ERR_CUDA;
+  const int vrow = (int)((b * z->Hkv + h_kv) * z->D);
+  const int vcol = (int)(kblk * 128);
+  if (z->D == 128) {
+    const size_t smem = 1024 + AttnLayout<128>::P_BYTES + AttnLayout<128>::V_BYTES + 64;
+    if (!ensure_smem(debug_pv_kernel<128>, smem, &g_smem_dbg_pv)) return SAGE_ERR_CUDA;
+    debug_pv_kernel<128><<<1, 128, smem, stream>>>(tv, vrow, vcol, p, acc);
+  } else {
+    const size_t smem = 1024 + AttnLayout<64>::P_BYTES + AttnLayout<64>::V_BYTES + 64;
+    debug_pv_kernel<64><<<1, 128, smem, stream>>>(tv, vrow, vcol, p, acc);
+  }
+  return launch_status();
+}
+
+sage_status sage_debug_wait_timeout(uint32_t timeout_us, sage_stream_t stream) {
+  if (timeout_us == 0 || timeout_us > 10000000u) return SAGE_ERR_INVALID_ARG;
+  debug_wait_kernel<<<1, 32, 0, stream>>>((uint64_t)timeout_us * 1000ull);
+  return launch_status();
+}
+
+}  // extern "C"

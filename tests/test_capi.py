@@ -1,0 +1,142 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, the ctypes structs match the C layout, and host-side
+validation rejects bad arguments before anything touches CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import quantized_attention_05_b200 as S
+from quantized_attention_05_b200 import build as B
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return S.lib()
+
+
+def declared_functions():
+    text = open(S.HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sage_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 12
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+    out = subprocess.run(["nm", "-D", "--defined-only", S.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (sage_[a-z0-9_]+)$", out, flags=re.M))
+    assert set(names) <= exported
+
+
+def test_library_has_no_driver_dependency_at_load():
+    out = subprocess.run(["ldd", S.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libcudart" not in out
+
+
+def test_ctypes_layout_matches_header(tmp_path):
+    src = tmp_path / "probe.c"
+    src.write_text("""
+#include <stdio.h>
+#include <stddef.h>
+#include "sage_b200.h"
+int main(void) {
+  printf("%zu %zu %zu\\n", sizeof(sage_tensor), sizeof(sage_mask), sizeof(sage_qkv_i8f8));
+  printf("%zu %zu %zu\\n", offsetof(sage_tensor, B), offsetof(sage_mask, sq), offsetof(sage_qkv_i8f8, D));
+  return 0;
+}""")
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(S.HEADER_PATH), str(src), "-o", str(exe)],
+                   check=True)
+    lines = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    sizes = list(map(int, lines[0].split()))
+    offs = list(map(int, lines[1].split()))
+    assert sizes == [ctypes.sizeof(S.SageTensor), ctypes.sizeof(S.SageMask), ctypes.sizeof(S.SageQkvI8F8)]
+    assert offs == [S.SageTensor.B.offset, S.SageMask.sq.offset, S.SageQkvI8F8.D.offset]
+
+
+def test_status_strings_and_version(L):
+    assert L.sage_status_str(0) == b"ok"
+    assert b"workspace" in L.sage_status_str(3)
+    assert b"sm_100a" in L.sage_version()
+
+
+def _t(ptr=16, dtype=0, B=1, H=2, N=256, D=64, sb=None, sh=None, sn=None):
+    sn = D if sn is None else sn
+    sh = N * sn if sh is None else sh
+    sb = H * sh if sb is None else sb
+    return S.SageTensor(ptr, dtype, B, H, N, D, sb, sh, sn)
+
+
+def _q(ptr=256, B=1, Hq=2, Hkv=2, Nq=256, Nk=256, D=64):
+    return S.SageQkvI8F8(ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, B, Hq, Hkv, Nq, Nk, D)
+
+
+def test_quantize_rejects_bad_arguments_on_host(L):
+    byref = ctypes.byref
+    out = _q()
+    call = lambda q, k, v, o=out, ws=256, nb=1 << 20: L.sage_quantize_qkv(  # noqa: E731
+        byref(q), byref(k), byref(v), 1, byref(o), ws, nb, None)
+    assert call(_t(ptr=0), _t(), _t()) == S.SAGE_ERR_INVALID_ARG          # null pointer
+    assert call(_t(ptr=8), _t(), _t()) == S.SAGE_ERR_INVALID_ARG          # misaligned
+    assert call(_t(D=96), _t(D=96), _t(D=96)) == S.SAGE_ERR_UNSUPPORTED   # head_dim 96
+    assert call(_t(dtype=7), _t(), _t()) == S.SAGE_ERR_INVALID_ARG        # dtype
+    assert call(_t(), _t(dtype=1), _t()) == S.SAGE_ERR_INVALID_ARG        # mixed dtypes
+    assert call(_t(H=3), _t(H=2), _t(H=2), _q(Hq=3)) == S.SAGE_ERR_INVALID_ARG   # Hq % Hkv
+    assert call(_t(sn=60), _t(), _t()) == S.SAGE_ERR_INVALID_ARG          # stride not 16-byte rows
+    assert call(_t(), _t(), _t(), _q(Nk=300)) == S.SAGE_ERR_INVALID_ARG   # out shape mismatch
+    assert call(_t(), _t(), _t(), ws=0) == S.SAGE_ERR_INVALID_ARG         # no workspace
+    assert call(_t(), _t(), _t(), nb=16) == S.SAGE_ERR_WORKSPACE          # workspace too small
+
+
+def test_attention_rejects_bad_arguments_on_host(L):
+    byref = ctypes.byref
+    z = _q()
+    f = L.sage_attn_fwd_quantized
+    assert f(byref(z), 0, 0.0, 1, None, 256, 0, 2 * 256 * 64, 256 * 64, 64, None, None, 0, None) \
+        == S.SAGE_ERR_INVALID_ARG                                   # return_lse without lse
+    zz = _q()
+    zz.q_dot_kmean = None
+    assert f(byref(zz), 0, 0.0, 1, None, 256, 0, 0, 256 * 64, 64, 512, None, 0, None) \
+        == S.SAGE_ERR_INVALID_ARG                                   # LSE needs q_dot_kmean
+    assert f(byref(z), 0, 0.0, 0, None, 8, 0, 0, 256 * 64, 64, None, None, 0, None) \
+        == S.SAGE_ERR_INVALID_ARG                                   # misaligned out
+    assert f(byref(z), 0, 0.0, 0, None, 256, 5, 0, 256 * 64, 64, None, None, 0, None) \
+        == S.SAGE_ERR_INVALID_ARG                                   # out dtype
+    assert f(byref(z), 0, float("nan"), 0, None, 256, 0, 0, 256 * 64, 64, None, None, 0, None) \
+        == S.SAGE_ERR_INVALID_ARG                                   # sm_scale
+    m = S.SageMask(256, 1, 1, 256, 128, 0, 0, 256)                  # wrong key length
+    assert f(byref(z), 0, 0.0, 0, byref(m), 256, 0, 0, 256 * 64, 64, None, 256, 1 << 20, None) \
+        == S.SAGE_ERR_INVALID_ARG
+    m = S.SageMask(256, 1, 1, 256, 256, 0, 0, 256)
+    assert f(byref(z), 0, 0.0, 0, byref(m), 256, 0, 0, 256 * 64, 64, None, 256, 1, None) \
+        == S.SAGE_ERR_WORKSPACE
+    zbig = _q(Nq=128 * 4096, Nk=128 * 4096)
+    assert f(byref(zbig), 0, 0.0, 0, None, 256, 0, 0, 256 * 64, 64, None, None, 0, None) \
+        == S.SAGE_ERR_UNSUPPORTED
+
+
+def test_fused_call_checks_num_kv_heads_and_workspace(L):
+    byref = ctypes.byref
+    q, k, v = _t(H=4), _t(H=2), _t(H=2)
+    f = L.sage_attn_fwd
+    assert f(byref(q), byref(k), byref(v), 0, 0.0, 3, 0, 1, None, 256, 0, 0, 64, None, 256, 1 << 30,
+             None) == S.SAGE_ERR_INVALID_ARG                        # num_kv_heads != k.H
+    need = L.sage_attn_fwd_workspace_bytes(1, 4, 2, 256, 256, 64, None)
+    assert f(byref(q), byref(k), byref(v), 0, 0.0, 2, 0, 1, None, 256, 0, 0, 64, None, 256, need - 1,
+             None) == S.SAGE_ERR_WORKSPACE
+
+
+def test_workspace_sizes_cover_the_quantised_tensors(L):
+    B_, Hq, Hkv, N, D = 4, 32, 8, 16384, 128
+    need = L.sage_attn_fwd_workspace_bytes(B_, Hq, Hkv, N, N, D, None)
+    payload = B_ * Hq * N * D + 2 * B_ * Hkv * N * D + B_ * Hq * N * 4
+    assert payload < need < payload * 1.1
+    assert L.sage_quantize_workspace_bytes(B_, Hkv, N, D) > 0
+    assert L.sage_quantize_workspace_bytes(0, Hkv, N, D) == 0

@@ -1,0 +1,140 @@
+"""Fused INT8-QK / FP8-PV attention on the GPU vs the oracle.
+
+Two entry points: sage_attn_fwd_quantized on the ORACLE's codes (isolates
+the attention kernel) and sage_attn_fwd on bf16/fp16 inputs (the whole
+path).  Bound: max |out - oracle| <= 2e-2 and cosine >= 0.9995, same for the
+LSE; -inf LSE entries (rows with no visible key) must match exactly."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from gpu_util import assert_attention_close, lib, qkv_from_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def S():
+    return lib()
+
+
+CASES = [
+    # (workload, causal, return_lse)
+    (W.TINY, False, True),
+    (W.TINY, True, True),
+    (W.TINY.scaled(B=2, Hq=4, Hkv=2, N=300, D=128, seed=31), False, True),     # ragged, GQA
+    (W.TINY.scaled(B=1, Hq=8, Hkv=2, N=640, D=128, seed=32), True, True),      # odd tile count
+    (W.TINY.scaled(B=1, Hq=2, Hkv=1, N=1000, D=64, seed=33), True, False),
+    (W.VIDEO_DIT.scaled(N=1024, Hq=2, Hkv=2), False, True),                    # V outliers
+]
+
+
+@pytest.mark.parametrize("w,causal,lse", CASES,
+                         ids=lambda c: str(c) if not hasattr(c, "N") else f"{c.B}x{c.Hq}x{c.Hkv}x{c.N}x{c.D}")
+def test_attention_on_oracle_codes(S, w, causal, lse):
+    q, k, v = W.make_qkv(w)
+    oz = O.quantize_qkv_i8f8(q, k, v)
+    ref = O.attention_i8f8(oz, causal=causal, sm_scale=w.sm_scale)
+    z = qkv_from_oracle(S, oz)
+    res = S.sage_attn_fwd_quantized(z, causal=causal, sm_scale=w.sm_scale, return_lse=lse)
+    out, l = res if lse else (res, None)
+    assert_attention_close(out, l, ref, what=w.name)
+
+
+@pytest.mark.parametrize("w,causal,lse", CASES[:4],
+                         ids=lambda c: str(c) if not hasattr(c, "N") else f"{c.B}x{c.Hq}x{c.Hkv}x{c.N}x{c.D}")
+def test_fused_path(S, w, causal, lse):
+    q, k, v = W.make_qkv(w)
+    ref = O.attention_i8f8(O.quantize_qkv_i8f8(q, k, v), causal=causal, sm_scale=w.sm_scale)
+    res = S.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, sm_scale=w.sm_scale,
+                          return_lse=lse)
+    out, l = res if lse else (res, None)
+    assert out.shape == q.shape and out.dtype == q.dtype
+    assert_attention_close(out, l, ref, what=w.name)
+
+
+def test_fused_fp16_nhd(S):
+    w = W.TINY.scaled(B=2, Hq=4, Hkv=2, N=256, D=128, seed=34)
+    q, k, v = W.make_qkv(w, dtype=torch.float16)
+    ref = O.attention_i8f8(O.quantize_qkv_i8f8(q, k, v), causal=True)
+    qn, kn, vn = (t.transpose(1, 2).contiguous().cuda() for t in (q, k, v))
+    out, l = S.sage_attn_fwd(qn, kn, vn, causal=True, return_lse=True, layout="NHD")
+    assert out.shape == qn.shape and out.dtype == torch.float16
+    assert_attention_close(out.transpose(1, 2), l, ref, what="fp16 NHD")
+
+
+def test_mask_second_half_and_random_mask(S):
+    w = W.TINY.scaled(B=2, Hq=4, Hkv=4, N=512, D=128, seed=35, mask="second_half_keys")
+    q, k, v = W.make_qkv(w)
+    oz = O.quantize_qkv_i8f8(q, k, v)
+    z = qkv_from_oracle(S, oz)
+    mask = W.make_mask(w)
+    ref = O.attention_i8f8(oz, mask=mask.numpy())
+    out, l = S.sage_attn_fwd_quantized(z, return_lse=True, mask=mask.cuda())
+    assert_attention_close(out, l, ref, what="second half masked")
+    g = torch.Generator().manual_seed(3)
+    rm = torch.rand(2, 1, 512, 512, generator=g) < 0.5
+    rm[:, :, 7, :] = False                         # a row with no visible key
+    rm[:, :, :, 256:384] = True                    # a fully visible key tile
+    rm[:, :, :, 384:] = False                      # a fully hidden key tile
+    ref = O.attention_i8f8(oz, mask=rm.numpy(), causal=True)
+    out, l = S.sage_attn_fwd_quantized(z, return_lse=True, mask=rm.cuda(), causal=True)
+    assert_attention_close(out, l, ref, what="random mask + causal")
+    assert torch.all(out[:, :, 7] == 0) and torch.all(torch.isneginf(l[:, :, 7]))
+
+
+def test_mask_unaligned_key_length(S):
+    w = W.TINY.scaled(B=1, Hq=2, Hkv=2, N=200, D=64, seed=36)
+    q, k, v = W.make_qkv(w)
+    oz = O.quantize_qkv_i8f8(q, k, v)
+    g = torch.Generator().manual_seed(4)
+    rm = torch.rand(1, 2, 200, 200, generator=g) < 0.6
+    ref = O.attention_i8f8(oz, mask=rm.numpy())
+    out, l = S.sage_attn_fwd_quantized(qkv_from_oracle(S, oz), return_lse=True, mask=rm.cuda())
+    assert_attention_close(out, l, ref, what="per-head mask, Nk=200")
+
+
+def test_causal_bottom_right_when_lengths_differ(S):
+    for Nq, Nk in [(200, 333), (333, 200)]:
+        wq = W.TINY.scaled(B=1, Hq=2, Hkv=1, N=Nq, D=128, seed=37)
+        wk = W.TINY.scaled(B=1, Hq=2, Hkv=1, N=Nk, D=128, seed=38)
+        q = W.make_qkv(wq)[0]
+        _, k, v = W.make_qkv(wk)
+        oz = O.quantize_qkv_i8f8(q, k, v)
+        ref = O.attention_i8f8(oz, causal=True)
+        out, l = S.sage_attn_fwd_quantized(qkv_from_oracle(S, oz), causal=True, return_lse=True)
+        assert_attention_close(out, l, ref, what=f"causal Nq={Nq} Nk={Nk}")
+
+
+def test_lossless_case_matches_exact_attention(S):
+    """On the oracle's lossless inputs the GPU must also land on exact
+    attention (up to its fp32 exp2 and bf16 output rounding)."""
+    from lossless_cases import LN2, i8f8_case
+    q, k, v = i8f8_case(B=1, Hq=2, Hkv=1, N=384, D=64, seed=3)
+    ex, lse = O.exact_attention(q, k, v, causal=True, sm_scale=LN2)
+    out, l = S.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True, sm_scale=LN2, return_lse=True)
+    np.testing.assert_allclose(out.float().cpu().numpy(), ex, atol=2e-2)
+    np.testing.assert_allclose(l.cpu().numpy(), lse, atol=1e-4)
+
+
+@pytest.mark.parametrize("w", [W.LLM_MASK, W.CAUSAL_GQA, W.VIDEO_DIT], ids=lambda w: w.name)
+def test_full_size_sampled(S, w):
+    """The full workload through sage_attn_fwd (the call bench.py times);
+    the oracle checks the sampled rows of the Q heads of two KV heads."""
+    q, k, v = W.make_qkv(w)
+    mask = W.make_mask(w)
+    res = S.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=w.causal, sm_scale=w.sm_scale,
+                          return_lse=True, mask=None if mask is None else mask.cuda())
+    out, l = res
+    torch.cuda.synchronize()
+    rows = W.sample_rows(w)
+    G = w.Hq // w.Hkv
+    b = w.B - 1
+    for g in (0, w.Hkv - 1):
+        hq = list(range(g * G, (g + 1) * G))
+        oz = O.quantize_qkv_i8f8(q[b:b + 1, hq], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1])
+        m = None if mask is None else mask[b:b + 1].numpy()
+        ref = O.attention_i8f8(oz, causal=w.causal, sm_scale=w.sm_scale, mask=m, rows=rows)
+        assert_attention_close(out[b:b + 1, hq], l[b:b + 1, hq], ref, rows=rows, what=w.name)
