@@ -1,0 +1,411 @@
+"""Benchmark of the quantized-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one pass of the whole path over one batch of synthetic input:
+the quantisation stage (sage_quantize_qkv: smooth_k, per-block INT8 Q/K,
+per-channel FP8 V) followed by the fused INT8-QK / FP8-PV attention
+(sage_attn_fwd_quantized), on the causal GQA workload B=4, Hq=32, Hkv=8,
+N=16384, d=128 by default.  The metric is attention TOPS,
+4*B*Hq*N*N*d / step time (halved for causal).
+
+Timing: W warm-up steps, then K steps bracketed by a barrier and
+cuda.synchronize on both sides, CUDA events on the launching stream, max
+over ranks.  Inputs (805 MB of bf16 per step) are larger than L2.  SM clocks
+and throttle reasons are sampled with nvidia-smi during the timed region.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own replica
+of the workload (seeded by rank; the path has no exchange step), so the
+scaling is weak and the value is the ops of all ranks over the max time.
+
+--impl reference times the CPU oracle (the reference arm of this build) on
+rank 0: every step quantises and attends a bounded sample of the workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "attention TOPS at seq 16K hd128 and % of B200 dense INT8/FP8 tensor peak"
+UNIT = "TOPS"
+# dense INT8/FP8 : BF16 tensor throughput on B200 (4.5 vs 2.25 PFLOP/s nominal)
+FP8_PER_BF16 = 2.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ ranks
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(backend):
+    import datetime
+    import torch.distributed as dist
+    ws, rank, _ = dist_env()
+    if ws > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device=None) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def rank_workload(w: W.Workload, rank: int) -> W.Workload:
+    """Replica of the workload for one rank: same shapes, its own seed."""
+    return w.scaled(seed=w.seed + 1000 * rank)
+
+
+# ------------------------------------------------------------------ peaks, clocks
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+CLOCK_FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw",
+                "clocks_event_reasons.sw_power_cap", "clocks_event_reasons.hw_slowdown",
+                "clocks_event_reasons.hw_thermal_slowdown",
+                "clocks_event_reasons.sw_thermal_slowdown",
+                "clocks_event_reasons.hw_power_brake_slowdown"]
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons every 200 ms."""
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = f"/tmp/sage_clocks_{os.getpid()}.csv"
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", "--query-gpu=" + ",".join(CLOCK_FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) == len(CLOCK_FIELDS):
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["sw_power_cap", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "hw_power_brake_slowdown"]
+        reasons = sorted({names[i] for r in rows for i in range(5) if r[3 + i] == "Active"})
+        sm_sorted = sorted(sm)
+        return {"sm_mhz": sm_sorted[len(sm_sorted) // 2] if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_sample(w: W.Workload, tokens: int):
+    """One bounded sample of workload ``w`` for the CPU oracle: the first
+    KV head group (one KV head and its Hq/Hkv Q heads) of batch 0, truncated
+    to the first ``tokens`` tokens; quantised and attended in full.
+    Returns (ops, seconds)."""
+    import oracle as O
+    G = w.Hq // w.Hkv
+    ws = w.scaled(B=1, Hq=G, Hkv=1, N=tokens)
+    q, k, v = W.make_qkv(ws)
+    mask = W.make_mask(ws)
+    t0 = time.perf_counter()
+    oz = O.quantize_qkv_i8f8(q, k, v)
+    O.attention_i8f8(oz, causal=ws.causal, sm_scale=ws.sm_scale,
+                     mask=None if mask is None else mask.numpy())
+    dt = time.perf_counter() - t0
+    return ws.ops, dt
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w: W.Workload, budget_s=15.0):
+    tokens = 2048
+    ops, dt = oracle_sample(w, tokens)
+    reps = max(1, min(8, int(budget_s / max(dt, 1e-3))))
+    tot_ops, tot_t = 0.0, 0.0
+    for _ in range(reps):
+        o, t = oracle_sample(w, tokens)
+        tot_ops += o
+        tot_t += t
+    return {"value": tot_ops / tot_t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{reps} x (first KV-head group of batch 0, {w.Hq // w.Hkv} Q heads, first "
+                      f"{tokens} tokens: oracle quantise + attend in full); {tot_t:.1f} s of CPU work"}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, w):
+    import quantized_attention_05_b200 as S
+    ws_, rank, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if ws_ > 1:
+        init_dist("nccl")
+    S.lib()
+    wr = rank_workload(w, rank)
+    q, k, v = W.make_qkv(wr, device=device)
+    mask = W.make_mask(wr, device=device)
+    z = S.QuantizedQKV.empty(w.B, w.Hq, w.Hkv, w.N, w.N, w.D, device, with_qdk=True)
+    qws = torch.empty(S.lib().sage_quantize_workspace_bytes(w.B, w.Hkv, w.N, w.D),
+                      dtype=torch.uint8, device=device)
+    out = torch.empty_like(q)
+    lse = torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    launches_per_step = 3 + (1 if mask is not None else 0)
+
+    def step(ev_a=None, ev_b=None):
+        S.sage_quantize_qkv(q, k, v, out=z, ws=qws)
+        if ev_a is not None:
+            ev_a.record(stream)
+        S.sage_attn_fwd_quantized(z, causal=w.causal, sm_scale=w.sm_scale, return_lse=True,
+                                  mask=mask, out=out, lse=lse)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    st, site = S.sage_get_device_status()
+    if st != S.SAGE_OK:
+        raise RuntimeError(f"device wait timed out at site {site}")
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local) if rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(*evs[i])
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop() if sampler else None
+    ms_local = e0.elapsed_time(e1)
+    attn_ms_local = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    ms = max_over_ranks(ms_local, device)
+    attn_ms = max_over_ranks(attn_ms_local, device)
+    st, site = S.sage_get_device_status()
+    if st != S.SAGE_OK:
+        raise RuntimeError(f"device wait timed out at site {site}")
+
+    # ---- end to end through the C ABI with host buffers
+    k_e2e = max(1, min(args.steps, 8))
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    outh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    lseh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    maskh = None if mask is None else mask.cpu().pin_memory()
+    nbytes_ws = S.sage_attn_fwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.N, w.D,
+                                               None if mask is None else tuple(mask.shape[:2]))
+    ws_fused = torch.empty(nbytes_ws, dtype=torch.uint8, device=device)
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    md = None if mask is None else torch.empty_like(mask)
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        if md is not None:
+            md.copy_(maskh, non_blocking=True)
+        S.sage_attn_fwd(qd, kd, vd, causal=w.causal, sm_scale=w.sm_scale, return_lse=True,
+                        mask=md, out=out, lse=lse, ws=ws_fused)
+        outh.copy_(out, non_blocking=True)
+        lseh.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(k_e2e):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / k_e2e, device)
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v)) + (0 if mask is None else mask.numel())
+    d2h = out.numel() * out.element_size() + lse.numel() * 4
+
+    ranks = ws_
+    ms_step = ms / args.steps
+    value = ranks * w.ops / (ms_step * 1e-3) / 1e12
+    peaks, src = load_peaks()
+    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP8_PER_BF16
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP8_PER_BF16
+    achieved = w.ops / (attn_ms * 1e-3) / 1e12
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if os.path.exists(tr_path):
+        try:
+            tr = json.load(open(tr_path))
+            if tr.get("workload") == w.name and tr.get("kernel_hash") == kernel_hash():
+                traffic = tr.get("bytes_per_launch")
+        except (OSError, ValueError):
+            traffic = None
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ranks,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "i8xi8->i32 (QK), e4m3xe4m3->f32 (PV)", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "D": w.D,
+                   "causal": w.causal, "return_lse": True, "mask": w.mask, "input_dtype": "bf16",
+                   "l2": "inputs larger than L2 (q/k/v bf16 805 MB per step, not flushed)",
+                   "parallelism": f"replicas x{ranks}"},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_i8f8_kernel<128>",
+                     "achieved": round(achieved, 1), "peak": round(peak_sus, 1), "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_sus, 4), "traffic": traffic,
+                     "peak_source": f"{src} bf16 sustained x{FP8_PER_BF16:g} (dense INT8/FP8:BF16)",
+                     "peak_burst": round(peak_burst, 1), "frac_burst": round(achieved / peak_burst, 4),
+                     "attn_ms": round(attn_ms, 4)},
+        "e2e": {"value": round(ranks * w.ops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 3), "api": "sage_attn_fwd with pinned host buffers"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and ranks == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def kernel_hash():
+    """Hash of the attention kernel source: a recorded DRAM traffic figure is
+    reported only while the kernel it was measured on is unchanged."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("attn_fwd_i8f8.cuh", "sage_ptx.cuh"):
+        with open(os.path.join(ROOT, "quantized_attention_05_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, w):
+    ws_, rank, _ = dist_env()
+    if rank != 0:
+        return
+    tokens = 1024
+    for _ in range(args.warmup):
+        oracle_sample(w, tokens)
+    tot_ops, tot_t = 0.0, 0.0
+    for _ in range(args.steps):
+        o, t = oracle_sample(w, tokens)
+        tot_ops += o
+        tot_t += t
+    value = tot_ops / tot_t / 1e12
+    sample = (f"each step: first KV-head group of batch 0 ({w.Hq // w.Hkv} Q heads), first {tokens} "
+              f"tokens, oracle quantise + attend in full")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * tot_t / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 (oracle)", "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "D": w.D,
+                   "causal": w.causal, "return_lse": True, "mask": w.mask, "input_dtype": "bf16",
+                   "parallelism": "cpu oracle, rank 0"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=W.CAUSAL_GQA.name, choices=sorted(W.BY_NAME))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--B", type=int, default=None,
+                    help="override the batch size (smaller cases for profiling)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = W.BY_NAME[args.workload]
+    if args.B is not None:
+        w = w.scaled(B=args.B, name=w.name.replace(f"_b{w.B}_", f"_b{args.B}_"))
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -115,7 +115,9 @@ def test_lossless_case_matches_exact_attention(S):
     q, k, v = i8f8_case(B=1, Hq=2, Hkv=1, N=384, D=64, seed=3)
     ex, lse = O.exact_attention(q, k, v, causal=True, sm_scale=LN2)
     out, l = S.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True, sm_scale=LN2, return_lse=True)
-    np.testing.assert_allclose(out.float().cpu().numpy(), ex, atol=2e-2)
+    # outputs here reach 448 (V holds +-448), so the bound is bf16-relative:
+    # half a bf16 ulp (2**-8 relative) plus the fp32 exp2 error
+    np.testing.assert_allclose(out.float().cpu().numpy(), ex, rtol=2.0 ** -8 + 1e-4, atol=1e-3)
     np.testing.assert_allclose(l.cpu().numpy(), lse, atol=1e-4)
 
 
