@@ -205,6 +205,37 @@ sage_status sage_debug_pv_fp32(const sage_qkv_i8f8* qkv, const uint8_t* p, int64
  * bounded-wait path without hanging the GPU. */
 sage_status sage_debug_wait_timeout(uint32_t timeout_us, sage_stream_t stream);
 
+/* ------------------------------------------------- allocation-free variant */
+/* No counterpart on the pages: an addition of this library.
+ *
+ * sage_quantize_qkv needs a scratch workspace for its per-split K sums and
+ * V maxima, and the caller has to allocate it.  Some callers cannot: a
+ * plugin inside a host framework that owns every device allocation, or a
+ * latency-critical loop where a cudaMalloc (which may synchronise the
+ * device) is not allowed.  This entry point computes exactly what
+ * sage_quantize_qkv computes, with the same inputs and outputs (still
+ * caller-owned), but keeps its scratch in a fixed array of
+ * SAGE_NOALLOC_SCRATCH_BYTES of device memory that is part of the library
+ * itself: every GPU that loads the library holds that array until the
+ * process exits.  It calls no cudaMalloc, cudaFree or allocating library
+ * routine.
+ *   - Size limit: sage_quantize_workspace_bytes(B, Hkv, Nk, D) must not
+ *     exceed SAGE_NOALLOC_SCRATCH_BYTES; larger problems are rejected with
+ *     SAGE_ERR_WORKSPACE before anything is enqueued (use
+ *     sage_quantize_qkv with a workspace for them).
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress, with that device current) and caches
+ *     it; make that first call before any stream capture.
+ *   - Sharing: every call on a device uses the same array, which keeps the
+ *     contents of the last call.  The kernels overwrite every scratch entry
+ *     they read before reading it, so nothing needs clearing, but calls
+ *     that overlap on the GPU (e.g. on two streams at once) race on the
+ *     array: order them. */
+#define SAGE_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+sage_status sage_quantize_qkv_noalloc(const sage_tensor* q, const sage_tensor* k,
+                                      const sage_tensor* v, int smooth_k,
+                                      const sage_qkv_i8f8* out, sage_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

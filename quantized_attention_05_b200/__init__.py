@@ -86,6 +86,8 @@ def lib():
         "sage_debug_qk_int32": (ctypes.c_int, [P(SageQkvI8F8), _i64, _i64, _i64, _i64, _vp, _vp]),
         "sage_debug_pv_fp32": (ctypes.c_int, [P(SageQkvI8F8), _vp, _i64, _i64, _i64, _vp, _vp]),
         "sage_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, _vp]),
+        "sage_quantize_qkv_noalloc": (ctypes.c_int, [P(SageTensor), P(SageTensor), P(SageTensor),
+                                                     ctypes.c_int, P(SageQkvI8F8), _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -207,6 +209,21 @@ def sage_quantize_qkv(q, k, v, smooth_k=True, layout="HND", with_qdk=True,
     _check(L.sage_quantize_qkv(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
                                int(bool(smooth_k)), ctypes.byref(s), ws.data_ptr(), ws.numel(),
                                _stream(q.device)), "sage_quantize_qkv")
+    return out
+
+
+def sage_quantize_qkv_noalloc(q, k, v, smooth_k=True, layout="HND", with_qdk=True,
+                              out: Optional[QuantizedQKV] = None):
+    """sage_quantize_qkv without a caller workspace: the library's own fixed
+    device scratch is used instead (for callers that cannot allocate)."""
+    L = lib()
+    tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
+    if out is None:
+        out = QuantizedQKV.empty(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D, q.device, with_qdk)
+    s = out.struct()
+    _check(L.sage_quantize_qkv_noalloc(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                                       int(bool(smooth_k)), ctypes.byref(s), _stream(q.device)),
+           "sage_quantize_qkv_noalloc")
     return out
 
 

@@ -476,4 +476,36 @@ sage_status sage_debug_wait_timeout(uint32_t timeout_us, sage_stream_t stream) {
   return launch_status();
 }
 
+// ------------------------------------------------- allocation-free variant
+// The quantiser's scratch (per-split K sums and V maxima) in a fixed array of
+// the library's own device memory, for callers that cannot allocate.  Host
+// code cannot use `g_noalloc_scratch` as a pointer (in host code the name is
+// a host-side stand-in); its device address is looked up once per device
+// with cudaGetSymbolAddress and cached.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SAGE_NOALLOC_SCRATCH_BYTES];
+
+static void* noalloc_scratch_ptr() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<void*> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  void* p = cache[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+  cache[dev].store(p, std::memory_order_release);
+  return p;
+}
+
+sage_status sage_quantize_qkv_noalloc(const sage_tensor* q, const sage_tensor* k,
+                                      const sage_tensor* v, int smooth_k,
+                                      const sage_qkv_i8f8* out, sage_stream_t stream) {
+  sage_status st;
+  if ((st = check_tensor(q)) || (st = check_tensor(k)) || (st = check_tensor(v))) return st;
+  if (quant_plan(k->B, k->H, k->N, k->D).part_bytes > SAGE_NOALLOC_SCRATCH_BYTES)
+    return SAGE_ERR_WORKSPACE;  // the fixed scratch is too small for these sizes
+  void* scratch = noalloc_scratch_ptr();
+  if (!scratch) return SAGE_ERR_CUDA;
+  return run_quantize(q, k, v, smooth_k, out, scratch, SAGE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 }  // extern "C"
