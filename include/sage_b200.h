@@ -136,8 +136,7 @@ sage_status sage_get_device_status(sage_stream_t stream, uint32_t* site);
 size_t sage_quantize_workspace_bytes(int64_t B, int64_t Hkv, int64_t Nk, int64_t D);
 
 /* Quantisation stage: smooth_k + per-block INT8 Q/K, per-channel FP8 V
- * (north-star "sage_quantize_qkv"; pages: "smooth_k", per-block INT8 QK,
- * per-channel FP8 V).  q: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D] (same dtype,
+ * (pages: "smooth_k", per-block INT8 QK, per-channel FP8 V).  q: [B, Hq, Nq, D]; k, v: [B, Hkv, Nk, D] (same dtype,
  * Hq % Hkv == 0, D in {64, 128}).  Writes every array of *out (whose shape
  * fields must match the inputs).  ws: device workspace of at least
  * sage_quantize_workspace_bytes(B, Hkv, Nk, D) bytes, 256-byte aligned. */
@@ -150,8 +149,8 @@ sage_status sage_quantize_qkv(const sage_tensor* q, const sage_tensor* k, const 
  * classification (zero when mask == NULL). */
 size_t sage_attn_quantized_workspace_bytes(const sage_qkv_i8f8* qkv, const sage_mask* mask);
 
-/* Fused attention on quantised inputs (north-star "sage_attn_fwd" second
- * stage: INT8 QK^T, dequantise, online softmax, P -> FP8, FP8 PV with FP32
+/* Fused attention on quantised inputs (the second stage of the path:
+ * INT8 QK^T, dequantise, online softmax, P -> FP8, FP8 PV with FP32
  * accumulation).
  *   causal:   keep key j for query i when j <= i + Nk - Nq.
  *   sm_scale: softmax scale; <= 0 selects 1/sqrt(D).
@@ -173,8 +172,8 @@ sage_status sage_attn_fwd_quantized(const sage_qkv_i8f8* qkv, int causal, float 
 size_t sage_attn_fwd_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
                                      int64_t Nk, int64_t D, const sage_mask* mask);
 
-/* The whole path on FP16/BF16 inputs (north-star "sage_attn_fwd (q, k, v,
- * causal, sm_scale, num_kv_heads, return_lse)"; pages: "sageattn").
+/* The whole path on FP16/BF16 inputs (q, k, v, causal, sm_scale,
+ * num_kv_heads, return_lse; pages: "sageattn").
  * num_kv_heads must equal k->H.  smooth_k as in sage_quantize_qkv (the
  * pages' default is on).  out has q's dtype; the other arguments are those
  * of sage_attn_fwd_quantized.  Quantises into the workspace, then attends. */

@@ -232,8 +232,8 @@ def cosine(a, b):
 
 
 def qk_int32_tile(qz, b, h, qblk, kblk):
-    """Exact integer QK^T of one 128x128 tile of INT8 codes (north-star
-    "int32 QK^T block products"): rows qblk*128.., keys kblk*128.., of the
+    """Exact integer QK^T of one 128x128 tile of INT8 codes (the int32
+    block product the kernel's first MMA chain produces): rows qblk*128.., keys kblk*128.., of the
     Q head h and its KV head h // G.  Returns int64 [128, 128]; the float64
     matmul is exact because |S| < 2**53."""
     G = qz["Hq"] // qz["Hkv"]

@@ -86,7 +86,10 @@ __device__ __forceinline__ void dd_add(DD& acc, const DD& y) {
   dd_add(acc, y.hi);
   acc.lo = __dadd_rn(acc.lo, y.lo);
 }
-// fp32 value of (hi + lo) / n rounded once (see DESIGN notes on exactness).
+// fp32 value of (hi + lo) / n rounded once.  With the remainder of the
+// division carried exactly, this equals the correctly rounded mean unless the
+// exact value lies within ~2^-100 (relative) of an fp32 rounding boundary,
+// which bf16/fp16 sums of fewer than 2^31 terms cannot do.
 __device__ __forceinline__ float dd_mean_f32(const DD& s, double n) {
   const double q1 = __ddiv_rn(s.hi, n);
   const double r = __fma_rn(-q1, n, s.hi);  // exact remainder of the division

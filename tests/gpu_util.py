@@ -1,5 +1,5 @@
 """Helpers shared by the GPU tests: move oracle results onto the device in
-the library's layouts, and the output tolerances of the benchmark spec's bound
+the library's layouts, and the output tolerances of the parity bound
 (max |err| <= 2e-2 and cosine >= 0.9995 against the oracle)."""
 import numpy as np
 import torch
