@@ -33,7 +33,13 @@ namespace sage {
 
 constexpr int ATT_BM = 128, ATT_BN = 128;
 constexpr int ATT_STAGES = 3;
-constexpr int ATT_THREADS = 320;
+constexpr int ATT_THREADS = 384;   // 3 warpgroups: 2 softmax, 1 TMA/MMA (+2 idle warps)
+// Register split between the warpgroups (setmaxnreg): the TMA/MMA warpgroup
+// keeps ATT_REGS_LOW per thread, the softmax warpgroups grow to
+// ATT_REGS_HIGH.  The sum must not exceed what the block is launched with
+// (384 threads x the kernel's compiled register count); the host checks it.
+constexpr int ATT_REGS_LOW = 56;
+constexpr int ATT_REGS_HIGH = 224;
 constexpr int ATT_MAX_NKT = 2048;   // keys <= 262144
 constexpr float LOG2_448 = 8.807354922057604f;
 constexpr float LN2_F = 0.6931471805599453f;
@@ -68,15 +74,26 @@ struct AttnLayout {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + ATT_STAGES * K_BYTES;
-  static constexpr int OFF_P = OFF_V + ATT_STAGES * V_BYTES;
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-  static constexpr int NBAR = 1 + 2 * ATT_STAGES + 8 + 1;
+  static constexpr int OFF_P = OFF_V + ATT_STAGES * V_BYTES;   // [warpgroup][buffer]
+  static constexpr int OFF_BAR = OFF_P + 4 * P_BYTES;
+  // q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2][2],
+  // o_ready[2][2], mma_done
+  static constexpr int NBAR = 1 + 2 * ATT_STAGES + 2 + 2 + 4 + 4 + 1;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_VS = (OFF_TMEM + 16 + 15) / 16 * 16;
   static constexpr int OFF_NLIST = OFF_VS + D * 4;
   static constexpr int OFF_LIST = OFF_NLIST + 16;
   static size_t bytes(int nkt) { return 1024 + OFF_LIST + (size_t)nkt * 4; }
 };
+
+// Exponentials: pairs i of each 32-key chunk with i % POLY_EVERY ==
+// POLY_EVERY - 1 are computed by a polynomial on the FMA pipe, the rest by
+// MUFU ex2, so that neither pipe limits alone.
+constexpr int POLY_EVERY = 4;
+// int32 score S as the float 1.5*2^23 + S (exact for |S| < 2^22): the bit
+// pattern of 1.5*2^23 plus S.
+constexpr uint32_t MAGIC_I = 0x4B400000u;
+constexpr float MAGIC_F = 12582912.0f;
 
 // Write one thread's row of 128 E4M3 probabilities (32 packed words) into a
 // 128x128-byte K-major tile with the 128-byte swizzle: 16-byte chunk c of
@@ -159,6 +176,93 @@ __device__ __forceinline__ void store_out_chunk(const AttnArgs& a, OutT* orow, i
   for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 }
 
+// Visibility of the 128 keys of tile kt for one row (bit j of vis[j / 32]):
+// key length, causal limit and, for mixed mask tiles, the boolean mask.
+__device__ __forceinline__ void tile_visibility(const AttnArgs& a, int kt, int row, bool part,
+                                                const uint8_t* mrow, uint32_t* vis) {
+  const int key0 = kt * ATT_BN;
+  int jmax = min(ATT_BN - 1, a.Nk - 1 - key0);
+  if (a.causal) jmax = min(jmax, row + a.causal_off - key0);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const int hi = jmax - 32 * w;  // keep bits 0..hi
+    vis[w] = hi >= 31 ? ~0u : (hi < 0 ? 0u : ((2u << hi) - 1u));
+  }
+  if (part && mrow) {
+    const uint8_t* mk = mrow + key0;
+    if (a.mask_vec16 && key0 + ATT_BN <= a.Nk) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint4 mv = __ldg(reinterpret_cast<const uint4*>(mk) + q);
+        const uint32_t wds[4] = {mv.x, mv.y, mv.z, mv.w};
+        uint32_t bits = 0;
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          bits |= (((wds[t >> 2] >> (8 * (t & 3))) & 0xFFu) ? 1u : 0u) << t;
+        vis[q >> 1] &= ~(((~bits) & 0xFFFFu) << (16 * (q & 1)));
+      }
+    } else {
+      for (int j = 0; j < ATT_BN; ++j)
+        if (key0 + j < a.Nk && mk[j] == 0) vis[j >> 5] &= ~(1u << (j & 31));
+    }
+  }
+}
+
+// Exponentials, E4M3 P into the swizzled shared-memory tile, and the row sum
+// of one 128-key tile.  sr holds 1.5*2^23 + S as float bits (0 for hidden
+// keys when NEED); p = 2^(S*c + bias) in fp32, P = E4M3(p) (bias includes
+// log2(448) and minus the running max), row sum of the unquantised p.
+template <bool NEED>
+__device__ __forceinline__ float exp_tile(const uint32_t* sr, const uint32_t* vis, float c,
+                                          float bias, uint8_t* ptile, int rt) {
+  const uint64_t c2 = f2_pack(c, c), b2 = f2_pack(bias, bias);
+  const uint64_t nm2 = f2_pack(-MAGIC_F, -MAGIC_F);
+  uint64_t acc = f2_pack(0.f, 0.f);
+  uint8_t* prow = ptile + rt * 128;
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    uint32_t pw[8];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      uint32_t half[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int j = ch * 32 + 2 * (i + u);
+        const uint64_t y = f2_fma(
+            f2_add(f2_pack(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), nm2), c2, b2);
+        float y0, y1;
+        f2_unpack(y, y0, y1);
+        uint64_t p;
+        if ((i + u) % POLY_EVERY == POLY_EVERY - 1) {
+          p = f2_exp2_poly(y0, y1);
+        } else {
+          p = f2_pack(ex2_approx(y0), ex2_approx(y1));
+        }
+        if (NEED) {
+          float p0, p1;
+          f2_unpack(p, p0, p1);
+          if (!((vis[j >> 5] >> (j & 31)) & 1u)) p0 = 0.f;
+          if (!((vis[j >> 5] >> ((j + 1) & 31)) & 1u)) p1 = 0.f;
+          p = f2_pack(p0, p1);
+        }
+        acc = f2_add(acc, p);
+        float p0, p1;
+        f2_unpack(p, p0, p1);
+        half[u] = cvt_e4m3x2(p0, p1);
+      }
+      pw[i >> 1] = half[0] | (half[1] << 16);
+    }
+    // 16-byte chunks 2ch and 2ch+1 of the row, 128-byte swizzle
+    *reinterpret_cast<uint4*>(prow + (((2 * ch) ^ (rt & 7)) << 4)) =
+        make_uint4(pw[0], pw[1], pw[2], pw[3]);
+    *reinterpret_cast<uint4*>(prow + (((2 * ch + 1) ^ (rt & 7)) << 4)) =
+        make_uint4(pw[4], pw[5], pw[6], pw[7]);
+  }
+  float a0, a1;
+  f2_unpack(acc, a0, a1);
+  return a0 + a1;
+}
+
 template <int D>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attn_fwd_i8f8_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -175,11 +279,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + ATT_STAGES;
-  uint64_t* s_full = kv_empty + ATT_STAGES;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* o_ready = p_full + 2;
-  uint64_t* mma_done = o_ready + 2;
+  uint64_t* s_full = kv_empty + ATT_STAGES;   // [wg]
+  uint64_t* s_free = s_full + 2;              // [wg]
+  uint64_t* p_full = s_free + 2;              // [wg * 2 + buffer]
+  uint64_t* o_ready = p_full + 4;             // [wg * 2 + buffer]
+  uint64_t* mma_done = o_ready + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   float* s_vs = reinterpret_cast<float*>(smem + L::OFF_VS);
   int* s_nlist = reinterpret_cast<int*>(smem + L::OFF_NLIST);
@@ -223,6 +327,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
+    }
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&p_full[i], 128);
       mbar_init(&o_ready[i], 1);
     }
@@ -244,114 +350,109 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const int ntile = s_nlist[0];
   const uint32_t orf = (uint32_t)s_nlist[1];
 
-  if (warp == 8) {
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(ATT_REGS_LOW));
+    if (warp == 8) {
     // ---------------------------------------------------------- TMA producer
-    // The whole warp runs the loop and waits; lane 0 issues the copies.
-    const bool act0 = orf & 1u, act1 = (orf >> 1) & 1u;
     if (lane == 0) {
+      const bool act0 = orf & 1u, act1 = (orf >> 1) & 1u;
       mbar_arrive_expect_tx(q_full, (uint32_t)((act0 ? L::Q_BYTES : 0) + (act1 ? L::Q_BYTES : 0)));
       if (act0) tma_load_2d(sQ, &tmQ, q_full, 0, bhq * a.Nqp + qt0 * ATT_BM);
       if (act1) tma_load_2d(sQ + L::Q_BYTES, &tmQ, q_full, 0, bhq * a.Nqp + (qt0 + 1) * ATT_BM);
-    }
-    __syncwarp();
-    for (int idx = 0; idx < ntile; ++idx) {
-      const int st = idx % ATT_STAGES, rd = idx / ATT_STAGES;
-      if (idx >= ATT_STAGES &&
-          !__all_sync(0xffffffffu, mbar_wait(&kv_empty[st], (rd - 1) & 1, SITE_KV_EMPTY)))
-        break;
-      if (lane == 0) {
+      for (int idx = 0; idx < ntile; ++idx) {
+        const int st = idx % ATT_STAGES, rd = idx / ATT_STAGES;
+        if (idx >= ATT_STAGES && !mbar_wait(&kv_empty[st], (rd - 1) & 1, SITE_KV_EMPTY)) break;
         const int kt = (int)(s_list[idx] >> 8);
         mbar_arrive_expect_tx(&kv_full[st], (uint32_t)(L::K_BYTES + L::V_BYTES));
         tma_load_2d(sK + st * L::K_BYTES, &tmK, &kv_full[st], 0, bhk * a.Nkp + kt * ATT_BN);
         tma_load_2d(sV + st * L::V_BYTES, &tmV, &kv_full[st], kt * ATT_BN, bhk * D);
       }
-      __syncwarp();
     }
+    __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
-    // The whole warp runs the schedule and waits; lane 0 issues MMAs/commits.
-    constexpr uint32_t IDESC_QK = instr_desc(kDS32, kS8, kS8, ATT_BM, ATT_BN);
-    constexpr uint32_t IDESC_PV = instr_desc(kDF32, kE4M3, kE4M3, ATT_BM, D);
-    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-    auto issue_qk = [&](int i, int st) {
-      const uint32_t tS = tmem + (uint32_t)(i * 256);
-      const uint32_t qa = aQ + i * L::Q_BYTES, ka = aK + st * L::K_BYTES;
-#pragma unroll
-      for (int k = 0; k < D / 32; ++k)
-        mma_i8(tS, smem_desc(qa + 32 * k, L::QK_SBO, L::QK_SWIZZLE),
-               smem_desc(ka + 32 * k, L::QK_SBO, L::QK_SWIZZLE), IDESC_QK, k > 0 ? 1u : 0u);
-    };
-    auto issue_pv = [&](int i, int st, bool acc) {
-      const uint32_t tO = tmem + (uint32_t)(i * 256 + 128);
-      const uint32_t pa = aP + i * L::P_BYTES, va = aV + st * L::V_BYTES;
-#pragma unroll
-      for (int k = 0; k < ATT_BN / 32; ++k)
-        mma_f8f6f4(tO, smem_desc(pa + 32 * k, 1024, 128), smem_desc(va + 32 * k, 1024, 128),
-                   IDESC_PV, (acc || k > 0) ? 1u : 0u);
-    };
-    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, SITE_Q_FULL));
-    tc_fence_after();
-    uint32_t qk_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
-    if (ok && ntile > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[0], 0, SITE_KV_FULL));
+    // One thread polls the barriers and issues, per Q tile i, the ops
+    // QK(0), QK(1), PV(0), QK(2), PV(1), ... in order, whichever Q tile is
+    // ready first.  A stage of the K/V ring is released once both Q tiles
+    // have issued their PV on it.
+    if (lane == 0) {
+      constexpr uint32_t IDESC_QK = instr_desc(kDS32, kS8, kS8, ATT_BM, ATT_BN);
+      constexpr uint32_t IDESC_PV = instr_desc(kDF32, kE4M3, kE4M3, ATT_BM, D);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      auto next_active = [&](int i, int from) {
+        while (from < ntile && !((s_list[from] >> i) & 1u)) ++from;
+        return from;
+      };
+      bool ok = mbar_wait(q_full, 0, SITE_Q_FULL);
       tc_fence_after();
-      const uint32_t f = s_list[0];
-      for (int i = 0; ok && i < 2; ++i)
-        if ((f >> i) & 1u) {
-          if (lane == 0) {
-            issue_qk(i, 0);
+      int qk_e[2], pv_e[2];
+      uint32_t qk_k[2] = {0, 0}, pv_k[2] = {0, 0};
+      for (int i = 0; i < 2; ++i) qk_e[i] = pv_e[i] = next_active(i, 0);
+      int rel_e = 0;
+      uint32_t idle = 0;
+      uint64_t idle_t0 = 0;
+      while (ok && rel_e < ntile) {
+        bool prog = false;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int e = qk_e[i];
+          if (e < ntile && mbar_test(&kv_full[e % ATT_STAGES], (e / ATT_STAGES) & 1) &&
+              mbar_test(&s_free[i], qk_k[i] & 1)) {
+            tc_fence_after();
+            const uint32_t tS = tmem + (uint32_t)(i * 256);
+            const uint32_t qa = aQ + i * L::Q_BYTES, ka = aK + (e % ATT_STAGES) * L::K_BYTES;
+#pragma unroll
+            for (int k = 0; k < D / 32; ++k)
+              mma_i8(tS, smem_desc(qa + 32 * k, L::QK_SBO, L::QK_SWIZZLE),
+                     smem_desc(ka + 32 * k, L::QK_SBO, L::QK_SWIZZLE), IDESC_QK, 1u);
             tc_commit(&s_full[i]);
+            ++qk_k[i];
+            qk_e[i] = next_active(i, e + 1);
+            prog = true;
           }
-          __syncwarp();
-          ++qk_cnt[i];
+          const uint32_t k = pv_k[i];
+          if (k < qk_k[i] && mbar_test(&p_full[i * 2 + (k & 1)], (k >> 1) & 1)) {
+            tc_fence_after();
+            const int ep = pv_e[i];
+            const uint32_t tO = tmem + (uint32_t)(i * 256 + 128);
+            const uint32_t pa = aP + (i * 2 + (k & 1)) * L::P_BYTES;
+            const uint32_t va = aV + (ep % ATT_STAGES) * L::V_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < ATT_BN / 32; ++kk)
+              mma_f8f6f4(tO, smem_desc(pa + 32 * kk, 1024, 128), smem_desc(va + 32 * kk, 1024, 128),
+                         IDESC_PV, (k > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&o_ready[i * 2 + (k & 1)]);
+            ++pv_k[i];
+            pv_e[i] = next_active(i, ep + 1);
+            prog = true;
+          }
         }
-    }
-    for (int idx = 0; ok && idx < ntile; ++idx) {
-      const int st = idx % ATT_STAGES;
-      const uint32_t f = s_list[idx];
-      const int nx = idx + 1;
-      const uint32_t fn = nx < ntile ? s_list[nx] : 0u;
-      bool next_ready = false;
-      for (int i = 0; ok && i < 2; ++i) {
-        if ((fn >> i) & 1u) {
-          if (!next_ready) {
-            ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[nx % ATT_STAGES],
-                                                   (nx / ATT_STAGES) & 1, SITE_KV_FULL));
-            next_ready = true;
-          }
-          if (ok && qk_cnt[i] > 0)
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(&s_free[i], (qk_cnt[i] - 1) & 1, SITE_S_FREE));
-          if (!ok) break;
-          tc_fence_after();
-          if (lane == 0) {
-            issue_qk(i, nx % ATT_STAGES);
-            tc_commit(&s_full[i]);
-          }
-          __syncwarp();
-          ++qk_cnt[i];
+        while (rel_e < ntile && rel_e < pv_e[0] && rel_e < pv_e[1]) {
+          tc_commit(&kv_empty[rel_e % ATT_STAGES]);
+          ++rel_e;
+          prog = true;
         }
-        if ((f >> i) & 1u) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&p_full[i], pv_cnt[i] & 1, SITE_P_FULL));
-          if (!ok) break;
-          tc_fence_after();
-          if (lane == 0) {
-            issue_pv(i, st, pv_cnt[i] > 0);
-            tc_commit(&o_ready[i]);
+        if (prog) {
+          idle = 0;
+        } else if ((++idle & 255u) == 0) {
+          if (*reinterpret_cast<volatile uint32_t*>(&g_status) != 0u) {
+            ok = false;
+          } else if (idle == 256u) {
+            idle_t0 = globaltimer_ns();
+          } else if (globaltimer_ns() - idle_t0 > 2000000000ull) {
+            report_timeout(SITE_MMA_STALL);
+            ok = false;
           }
-          __syncwarp();
-          ++pv_cnt[i];
         }
       }
-      if (lane == 0) tc_commit(&kv_empty[st]);
-      __syncwarp();
+      // every MMA issued above completes before the CTA tears down TMEM
+      tc_commit(mma_done);
+      mbar_wait(mma_done, 0, SITE_MMA_DONE);
     }
-    // every MMA issued above completes before the CTA tears down TMEM
-    if (lane == 0) tc_commit(mma_done);
     __syncwarp();
-    mbar_wait(mma_done, 0, SITE_MMA_DONE);
-    __syncwarp();
+    }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(ATT_REGS_HIGH));
     // ---------------------------------------------------------- softmax WGs
     const int wg = warp >> 2;
     const int rt = threadIdx.x & 127;
@@ -360,7 +461,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + (uint32_t)(wg * 256);
     const uint32_t tO = tS + 128;
-    uint8_t* sPw = sP + wg * L::P_BYTES;
     const bool tile_exists = qt < a.nqt;
     const float cq = tile_exists ? a.q_scale[(int64_t)bhq * a.nqt + qt] * a.c0 : 0.f;
     const uint8_t* mrow = nullptr;
@@ -368,7 +468,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const int bm = a.m_bcast_b ? 0 : b, hm = a.m_bcast_h ? 0 : h;
       mrow = a.mask + bm * a.m_sb + hm * a.m_sh + (int64_t)row * a.m_sq;
     }
-    float m = -INFINITY, l = 0.f;
+    // S accumulators start at 1.5*2^23 (as int32 bits): the int32 QK^T sum
+    // on top of it is then directly the float 1.5*2^23 + S.  The refill
+    // counts as the first release of S.
+#pragma unroll
+    for (int cb = 0; cb < 128; cb += 32) SAGE_TMEM_ST32_SPLAT(tS + cb, MAGIC_I);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(&s_free[wg]);
+    float m_ref = -INFINITY, l = 0.f;
     uint32_t n = 0;
     bool ok = true;
     for (int idx = 0; idx < ntile; ++idx) {
@@ -378,6 +486,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const bool need = (e >> (2 + wg)) & 1u;
       const bool part = (e >> (4 + wg)) & 1u;
       const float c = cq * a.k_scale[(int64_t)bhk * a.nkt + kt];
+      const uint32_t buf = n & 1u;
+      uint8_t* ptile = sP + (wg * 2 + buf) * L::P_BYTES;
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], n & 1, SITE_S_FULL));
       if (!ok) break;
       tc_fence_after();
@@ -387,91 +497,81 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       SAGE_TMEM_LD32(tS + 64, (sr + 64));
       SAGE_TMEM_LD32(tS + 96, (sr + 96));
       tmem_wait_ld();
+      // refill S with 1.5*2^23 for the next QK^T, which accumulates on top
+#pragma unroll
+      for (int cb = 0; cb < 128; cb += 32) SAGE_TMEM_ST32_SPLAT(tS + cb, MAGIC_I);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&s_free[wg]);
 
-      // visibility of the 128 keys of this tile for this row (bit j of vis[j/32])
+      // sr holds 1.5*2^23 + S as float bits; hidden keys -> 0.0 (below every score)
       uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
       if (need) {
-        const int key0 = kt * ATT_BN;
-        int jmax = min(ATT_BN - 1, a.Nk - 1 - key0);
-        if (a.causal) jmax = min(jmax, row + a.causal_off - key0);
+        tile_visibility(a, kt, row, part, mrow, vis);
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const int hi = jmax - 32 * w;  // keep bits 0..hi
-          vis[w] = hi >= 31 ? ~0u : (hi < 0 ? 0u : ((2u << hi) - 1u));
-        }
-        if (part && mrow) {
-          const uint8_t* mk = mrow + key0;
-          if (a.mask_vec16 && key0 + ATT_BN <= a.Nk) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const uint4 mv = __ldg(reinterpret_cast<const uint4*>(mk) + q);
-              const uint32_t wds[4] = {mv.x, mv.y, mv.z, mv.w};
-              uint32_t bits = 0;
-#pragma unroll
-              for (int t = 0; t < 16; ++t) bits |= (((wds[t >> 2] >> (8 * (t & 3))) & 0xFFu) ? 1u : 0u) << t;
-              vis[q >> 1] &= ~(((~bits) & 0xFFFFu) << (16 * (q & 1)));
-            }
-          } else {
-            for (int j = 0; j < ATT_BN; ++j)
-              if (key0 + j < a.Nk && mk[j] == 0) vis[j >> 5] &= ~(1u << (j & 31));
-          }
-        }
+        for (int j = 0; j < 128; ++j)
+          if (!((vis[j >> 5] >> (j & 31)) & 1u)) sr[j] = 0u;
       }
-      float mx = -INFINITY;
+      float m0 = __uint_as_float(sr[0]), m1 = __uint_as_float(sr[1]);
+      float m2 = __uint_as_float(sr[2]), m3 = __uint_as_float(sr[3]);
 #pragma unroll
-      for (int j = 0; j < 128; ++j) {
-        const float x = (float)(int)sr[j];
-        const bool v = (vis[j >> 5] >> (j & 31)) & 1u;
-        mx = v ? fmaxf(mx, x) : mx;
+      for (int j = 4; j < 128; j += 8) {
+        m0 = max3f(m0, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+        m1 = max3f(m1, __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
+        m2 = max3f(m2, __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
+        m3 = max3f(m3, __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
       }
-      const float mt = mx == -INFINITY ? -INFINITY : mx * c;
-      const float m_new = fmaxf(m, mt);
+      const float mx = max3f(m0, m1, fmaxf(m2, m3));
+      // tile max of the scaled scores (-inf if this row sees no key here)
+      const float mt = mx >= 4194304.f ? (mx - MAGIC_F) * c : -INFINITY;
+      const float m_new = fmaxf(m_ref, mt);
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float alpha = ex2_approx(m - m_use);
+      const float alpha = ex2_approx(m_ref - m_use);
       const float bias = LOG2_448 - m_use;
-      float rs = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int j = 0; j < 128; j += 4) {
-        float p[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const bool v = (vis[(j + t) >> 5] >> ((j + t) & 31)) & 1u;
-          p[t] = v ? ex2_approx(fmaf((float)(int)sr[j + t], c, bias)) : 0.f;
-          rs += p[t];
-        }
-        pk[j >> 2] = (uint32_t)cvt_e4m3x2(p[0], p[1]) | ((uint32_t)cvt_e4m3x2(p[2], p[3]) << 16);
-      }
-      l = l * alpha + rs;
 
-      if (n > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[wg], (n - 1) & 1, SITE_O_READY));
+      // the P buffer being overwritten was read by PV(n-2); O is touched only
+      // once PV(n-1) has completed
+      if (n >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[wg * 2 + buf], ((n - 2) >> 1) & 1,
+                                                SITE_O_READY));
+        if (!ok) break;
+      }
+      const float rs = need ? exp_tile<true>(sr, vis, c, bias, ptile, rt)
+                            : exp_tile<false>(sr, vis, c, bias, ptile, rt);
+      if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        const uint32_t pb = (n - 1) & 1u;
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[wg * 2 + pb], ((n - 1) >> 1) & 1,
+                                                SITE_O_READY));
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-          for (int cb = 0; cb < D; cb += 32) {
-            uint32_t o[32];
-            SAGE_TMEM_LD32(tO + cb, o);
-            tmem_wait_ld();
+        for (int cb = 0; cb < D; cb += 32) {
+          uint32_t o[32];
+          SAGE_TMEM_LD32(tO + cb, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            SAGE_TMEM_ST32(tO + cb, o);
+          for (int i = 0; i < 32; i += 2) {
+            float x0, x1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2), x0, x1);
+            o[i] = __float_as_uint(x0);
+            o[i + 1] = __float_as_uint(x1);
           }
-          tmem_wait_st();
+          SAGE_TMEM_ST32(tO + cb, o);
         }
+        tmem_wait_st();
       }
-      store_p_row(sPw, rt, pk);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[wg]);
-      m = m_new;
+      mbar_arrive(&p_full[wg * 2 + buf]);
+      l = l * alpha + rs;
+      m_ref = m_new;
       ++n;
     }
     if (ok && n > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[wg], (n - 1) & 1, SITE_O_READY));
+      const uint32_t pb = (n - 1) & 1u;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&o_ready[wg * 2 + pb], ((n - 1) >> 1) & 1, SITE_O_READY));
       tc_fence_after();
     }
     if (tile_exists) {
@@ -499,7 +599,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
       if (a.return_lse && row < a.Nq) {
         float v = -INFINITY;
-        if (l > 0.f) v = (m + log2f(l) - LOG2_448) * LN2_F + a.sm_scale * a.qdk[(int64_t)bhq * a.Nq + row];
+        if (l > 0.f)
+          v = (m_ref + log2f(l) - LOG2_448) * LN2_F +
+              a.sm_scale * a.qdk[(int64_t)bhq * a.Nq + row];
         a.lse[(int64_t)bhq * a.Nq + row] = v;
       }
     }

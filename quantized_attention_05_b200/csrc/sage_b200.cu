@@ -297,6 +297,16 @@ sage_status run_attention(const sage_qkv_i8f8* z, int causal, float sm_scale, in
   if (log_enabled())
     std::fprintf(stderr, "[sage] attn B=%d Hq=%d Hkv=%d Nq=%d Nk=%d D=%lld causal=%d grid=%d\n", a.B,
                  a.Hq, a.Hkv, a.Nq, a.Nk, (long long)z->D, a.causal, grid);
+  // the kernel redistributes registers between its warpgroups; that is only
+  // safe if the launch provides at least the sum of their shares
+  {
+    cudaFuncAttributes fa{};
+    const cudaError_t e = z->D == 128 ? cudaFuncGetAttributes(&fa, attn_fwd_i8f8_kernel<128>)
+                                      : cudaFuncGetAttributes(&fa, attn_fwd_i8f8_kernel<64>);
+    if (e != cudaSuccess) return SAGE_ERR_CUDA;
+    if (128 * ATT_REGS_LOW + 256 * ATT_REGS_HIGH > ATT_THREADS * fa.numRegs)
+      return SAGE_ERR_UNSUPPORTED;
+  }
   if (z->D == 128) {
     const size_t smem = AttnLayout<128>::bytes(a.nkt);
     if (!ensure_smem(attn_fwd_i8f8_kernel<128>, AttnLayout<128>::bytes(ATT_MAX_NKT), &g_smem_set_128))

@@ -8,6 +8,7 @@
 
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 namespace sage {
 
@@ -27,6 +28,7 @@ enum WaitSite : uint32_t {
   SITE_O_READY = 7,
   SITE_DEBUG = 8,
   SITE_MMA_DONE = 9,
+  SITE_MMA_STALL = 10,
 };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -71,6 +73,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking check that the phase of `parity` has completed.
+__device__ __forceinline__ bool mbar_test(const uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -223,6 +238,13 @@ constexpr uint32_t kE4M3 = 0;   // kind::f8f6f4 operand
       "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])                               \
       : "memory")
 
+// Store one 32-bit value into 32 consecutive TMEM columns of the warp's lanes.
+#define SAGE_TMEM_ST32_SPLAT(taddr, v)                                                          \
+  asm volatile(                                                                                 \
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"  \
+      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(v)         \
+      : "memory")
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -231,6 +253,93 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 // ---------------------------------------------------------------- math
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): element 0 in the low half.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// Two fp32 values to an f16x2 (round to nearest even); `lo` in the low half.
+__device__ __forceinline__ uint32_t f2_to_h2(uint64_t v) {
+  float lo, hi;
+  f2_unpack(v, lo, hi);
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// 2^x on both halves of an f16x2 (one MUFU instruction for two values).
+__device__ __forceinline__ uint32_t h2_ex2(uint32_t x) {
+  uint32_t r;
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
+__device__ __forceinline__ uint32_t h2_add(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// f16x2 to two E4M3 bytes (round to nearest even, saturating), low half in
+// the low byte.
+__device__ __forceinline__ uint32_t h2_to_e4m3x2(uint32_t x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(x));
+  return r;
+}
+__device__ __forceinline__ float h2_hsum(uint32_t x) {
+  return __half2float(__ushort_as_half((unsigned short)(x & 0xFFFFu))) +
+         __half2float(__ushort_as_half((unsigned short)(x >> 16)));
+}
+
+// 2^y for a pair of fp32 values on the FMA pipe (no MUFU): y is clamped to
+// [-125, ...], split as y = n + f with n = round(y) (via the 1.5*2^23
+// rounding trick) and f in [-0.5, 0.5]; 2^f is a degree-4 polynomial fitted
+// for this library by minimising the maximum relative error on [-0.5, 0.5]
+// (max relative error 2.7e-6 in fp32 Horner form); 2^n is applied by adding
+// n to the exponent field.
+__device__ __forceinline__ uint64_t f2_exp2_poly(float y0, float y1) {
+  y0 = fmaxf(y0, -125.f);
+  y1 = fmaxf(y1, -125.f);
+  const uint64_t y = f2_pack(y0, y1);
+  const uint64_t t = f2_add(y, f2_pack(12582912.f, 12582912.f));       // n in the low mantissa
+  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));     // n as a float
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), y);                // f = y - n
+  uint64_t p = f2_fma(f2_pack(0.009569989517331123f, 0.009569989517331123f), f,
+                      f2_pack(0.05591757968068123f, 0.05591757968068123f));
+  p = f2_fma(p, f, f2_pack(0.240247443318367f, 0.240247443318367f));
+  p = f2_fma(p, f, f2_pack(0.6931218504905701f, 0.6931218504905701f));
+  p = f2_fma(p, f, f2_pack(0.9999992847442627f, 0.9999992847442627f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  // bits(t) = 0x4B400000 + n, and 0x4B400000 << 23 wraps to 0: (bits(t) << 23) = n << 23
+  const uint32_t r0 = __float_as_uint(t0) * (1u << 23) + __float_as_uint(p0);
+  const uint32_t r1 = __float_as_uint(t1) * (1u << 23) + __float_as_uint(p1);
+  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
