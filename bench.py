@@ -44,6 +44,8 @@ METRIC = "attention TOPS at seq 16K hd128 and % of B200 dense INT8/FP8 tensor pe
 UNIT = "TOPS"
 # dense INT8/FP8 : BF16 tensor throughput on B200 (4.5 vs 2.25 PFLOP/s nominal)
 FP8_PER_BF16 = 2.0
+# dense FP4 : BF16 (9 vs 2.25 PFLOP/s nominal)
+FP4_PER_BF16 = 4.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -214,20 +216,35 @@ def run_ours(args, w):
     wr = rank_workload(w, rank)
     q, k, v = W.make_qkv(wr, device=device)
     mask = W.make_mask(wr, device=device)
-    z = S.QuantizedQKV.empty(w.B, w.Hq, w.Hkv, w.N, w.N, w.D, device, with_qdk=True)
-    qws = torch.empty(S.lib().sage_quantize_workspace_bytes(w.B, w.Hkv, w.N, w.D),
-                      dtype=torch.uint8, device=device)
     out = torch.empty_like(q)
     lse = torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
-    launches_per_step = 3 + (1 if mask is not None else 0)
+    if w.nvfp4:
+        ukl = w.unpadded_k_len or w.N
+        z = S.QuantizedNvfp4.empty(w.B, w.Hq, w.Hkv, w.N, w.N, w.D, ukl, w.per_block_mean, device)
+        qws = torch.empty(S.lib().sage_quantize_nvfp4_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.N, w.D),
+                          dtype=torch.uint8, device=device)
+        launches_per_step = 6
+    else:
+        z = S.QuantizedQKV.empty(w.B, w.Hq, w.Hkv, w.N, w.N, w.D, device, with_qdk=True)
+        qws = torch.empty(S.lib().sage_quantize_workspace_bytes(w.B, w.Hkv, w.N, w.D),
+                          dtype=torch.uint8, device=device)
+        launches_per_step = 3 + (1 if mask is not None else 0)
 
     def step(ev_a=None, ev_b=None):
-        S.sage_quantize_qkv(q, k, v, out=z, ws=qws)
+        if w.nvfp4:
+            S.sage_quantize_qkv_nvfp4(q, k, v, per_block_mean=w.per_block_mean,
+                                      unpadded_k_len=w.unpadded_k_len, out=z, ws=qws)
+        else:
+            S.sage_quantize_qkv(q, k, v, out=z, ws=qws)
         if ev_a is not None:
             ev_a.record(stream)
-        S.sage_attn_fwd_quantized(z, causal=w.causal, sm_scale=w.sm_scale, return_lse=True,
-                                  mask=mask, out=out, lse=lse)
+        if w.nvfp4:
+            S.sage_attn_fwd_nvfp4(z, sm_scale=w.sm_scale, causal=w.causal, return_lse=True,
+                                  out=out, lse=lse)
+        else:
+            S.sage_attn_fwd_quantized(z, causal=w.causal, sm_scale=w.sm_scale, return_lse=True,
+                                      mask=mask, out=out, lse=lse)
         if ev_b is not None:
             ev_b.record(stream)
 
@@ -266,8 +283,8 @@ def run_ours(args, w):
     outh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     lseh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     maskh = None if mask is None else mask.cpu().pin_memory()
-    nbytes_ws = S.sage_attn_fwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.N, w.D,
-                                               None if mask is None else tuple(mask.shape[:2]))
+    nbytes_ws = 1 if w.nvfp4 else S.sage_attn_fwd_workspace_bytes(
+        w.B, w.Hq, w.Hkv, w.N, w.N, w.D, None if mask is None else tuple(mask.shape[:2]))
     ws_fused = torch.empty(nbytes_ws, dtype=torch.uint8, device=device)
     qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     md = None if mask is None else torch.empty_like(mask)
@@ -278,8 +295,14 @@ def run_ours(args, w):
         vd.copy_(vh, non_blocking=True)
         if md is not None:
             md.copy_(maskh, non_blocking=True)
-        S.sage_attn_fwd(qd, kd, vd, causal=w.causal, sm_scale=w.sm_scale, return_lse=True,
-                        mask=md, out=out, lse=lse, ws=ws_fused)
+        if w.nvfp4:
+            S.sage_quantize_qkv_nvfp4(qd, kd, vd, per_block_mean=w.per_block_mean,
+                                      unpadded_k_len=w.unpadded_k_len, out=z, ws=qws)
+            S.sage_attn_fwd_nvfp4(z, sm_scale=w.sm_scale, causal=w.causal, return_lse=True,
+                                  out=out, lse=lse)
+        else:
+            S.sage_attn_fwd(qd, kd, vd, causal=w.causal, sm_scale=w.sm_scale, return_lse=True,
+                            mask=md, out=out, lse=lse, ws=ws_fused)
         outh.copy_(out, non_blocking=True)
         lseh.copy_(lse, non_blocking=True)
 
@@ -301,8 +324,9 @@ def run_ours(args, w):
     ms_step = ms / args.steps
     value = ranks * w.ops / (ms_step * 1e-3) / 1e12
     peaks, src = load_peaks()
-    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP8_PER_BF16
-    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP8_PER_BF16
+    ratio = FP4_PER_BF16 if w.nvfp4 else FP8_PER_BF16
+    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * ratio
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * ratio
     achieved = w.ops / (attn_ms * 1e-3) / 1e12
     traffic = None
     tr_path = os.path.join(ROOT, "profiles", "attn_traffic.json")
@@ -317,15 +341,20 @@ def run_ours(args, w):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ranks,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "i8xi8->i32 (QK), e4m3xe4m3->f32 (PV)", "data": "synthetic",
+        "dtype": ("nvfp4 (e2m1 x e2m1, e4m3 block-16 scales) -> f32" if w.nvfp4 else
+                  "i8xi8->i32 (QK), e4m3xe4m3->f32 (PV)"), "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "D": w.D,
                    "causal": w.causal, "return_lse": True, "mask": w.mask, "input_dtype": "bf16",
-                   "l2": "inputs larger than L2 (q/k/v bf16 805 MB per step, not flushed)",
+                   "nvfp4": w.nvfp4, "unpadded_k_len": w.unpadded_k_len,
+                   "l2": f"inputs larger than L2 (q/k/v bf16 "
+                         f"{(w.B * (w.Hq + 2 * w.Hkv) * w.N * w.D * 2) >> 20} MiB per step, not flushed)",
                    "parallelism": f"replicas x{ranks}"},
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_i8f8_kernel<128>",
+        "roofline": {"bound": "tensor",
+                     "kernel": "attn_fwd_nvfp4_kernel<128>" if w.nvfp4 else "attn_fwd_i8f8_kernel<128>",
                      "achieved": round(achieved, 1), "peak": round(peak_sus, 1), "unit": "TFLOP/s",
                      "frac": round(achieved / peak_sus, 4), "traffic": traffic,
-                     "peak_source": f"{src} bf16 sustained x{FP8_PER_BF16:g} (dense INT8/FP8:BF16)",
+                     "peak_source": f"{src} bf16 sustained x{ratio:g} (dense "
+                                    f"{'FP4' if w.nvfp4 else 'INT8/FP8'}:BF16)",
                      "peak_burst": round(peak_burst, 1), "frac_burst": round(achieved / peak_burst, 4),
                      "attn_ms": round(attn_ms, 4)},
         "e2e": {"value": round(ranks * w.ops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,

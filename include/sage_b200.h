@@ -120,6 +120,39 @@ typedef struct {
   int64_t B, Hq, Hkv, Nq, Nk, D;
 } sage_qkv_i8f8;
 
+/* Quantised Q/K/V of the NVFP4 path ("flashinfer.nvfp4_attention_sm120_fwd":
+ * packed FP4 Q/K/V with per-vector FP8 scale factors, V and its scales
+ * stored transposed, a compact FP32 qk_correction with one row per 128-token
+ * Q block, per_block_mean, unpadded_k_len).  Device memory owned by the
+ * caller; Nq_pad / Nk_pad as for sage_qkv_i8f8; every array dense.
+ *   q        u8   [B, Hq,  Nq_pad, D/2]  E2M1 codes, element 2i in the low nibble
+ *   q_sf     u8   [B, Hq,  Nq_pad, D/16] E4M3 scale of each 16-element vector
+ *   k        u8   [B, Hkv, Nk_pad, D/2]  codes of K - kmean (rows >= unpadded_k_len: 0)
+ *   k_sf     u8   [B, Hkv, Nk_pad, D/16]
+ *   v_t      u8   [B, Hkv, D, Nk_pad/2]  V transposed, 16-token vectors
+ *   v_sf_t   u8   [B, Hkv, D, Nk_pad/16]
+ *   qk_correction fp32 [B, Hq, Nq_pad/128, Nk_pad]: qmean(block) . Ks[j]
+ *   q_mean   fp32 [B, Hq, Nq_pad/128, D]: the mean removed from each Q block
+ *                 (the same vector in every block when per_block_mean == 0)
+ *   k_mean   fp32 [B, Hkv, D]
+ *   q_dot_kmean fp32 [B, Hq, Nq] (may be NULL when no LSE is wanted)
+ * The base pointers of q, k, v_t must be 16-byte aligned. */
+typedef struct {
+  uint8_t* q;
+  uint8_t* q_sf;
+  uint8_t* k;
+  uint8_t* k_sf;
+  uint8_t* v_t;
+  uint8_t* v_sf_t;
+  float* qk_correction;
+  float* q_mean;
+  float* k_mean;
+  float* q_dot_kmean;
+  int64_t B, Hq, Hkv, Nq, Nk, D;
+  int64_t unpadded_k_len;
+  int32_t per_block_mean;
+} sage_qkv_nvfp4;
+
 /* ------------------------------------------------------------------ info */
 const char* sage_status_str(sage_status status);
 const char* sage_version(void);
@@ -182,6 +215,37 @@ sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage
                           int smooth_k, const sage_mask* mask, void* out, int64_t out_sb,
                           int64_t out_sh, int64_t out_sn, float* lse, void* ws,
                           size_t ws_bytes, sage_stream_t stream);
+
+/* ------------------------------------------------------------------ NVFP4 */
+/* Workspace bytes of sage_quantize_qkv_nvfp4 (per-split K and Q sums). */
+size_t sage_quantize_nvfp4_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
+                                           int64_t Nk, int64_t D);
+
+/* NVFP4 quantisation ("nvfp4_attention_sm120_quantize_qkv" of the FlashInfer
+ * page, named there): K minus its mean over the first unpadded_k_len tokens
+ * (rows at and beyond it become zero); Q minus its mean over each 128-token
+ * block (per_block_mean != 0) or over all tokens; every 16-element vector
+ * (along D for Q and K, along tokens for the transposed V) gets
+ * sf = e4m3(fp32(amax/6)) and codes e2m1(fp32(x * fp32(1/sf))); then
+ * qk_correction = qmean . Ks^T per Q block.  unpadded_k_len <= 0 means Nk.
+ * out's shape fields, per_block_mean and unpadded_k_len must match the call. */
+sage_status sage_quantize_qkv_nvfp4(const sage_tensor* q, const sage_tensor* k,
+                                    const sage_tensor* v, int per_block_mean,
+                                    int64_t unpadded_k_len, const sage_qkv_nvfp4* out, void* ws,
+                                    size_t ws_bytes, sage_stream_t stream);
+
+/* NVFP4 attention on the output of sage_quantize_qkv_nvfp4
+ * ("nvfp4_attention_sm120_fwd"): scores sm_scale * (deq(Q).deq(K) +
+ * qk_correction[q block, key]), keys at and beyond unpadded_k_len masked,
+ * online softmax over 128-key tiles, P = 2688 * exp(s - running max)
+ * quantised to NVFP4 per 16 keys, block-scaled FP4 PV accumulated in FP32,
+ * out = O / (2688 * l).  per_block_mean must equal the value the quantiser
+ * was called with.  out / lse as in sage_attn_fwd_quantized (lse needs
+ * q_dot_kmean). */
+sage_status sage_attn_fwd_nvfp4(const sage_qkv_nvfp4* qkv, float sm_scale, int causal,
+                                int per_block_mean, int return_lse, void* out, int32_t out_dtype,
+                                int64_t out_sb, int64_t out_sh, int64_t out_sn, float* lse,
+                                sage_stream_t stream);
 
 /* ------------------------------------------------------------ test exports */
 /* Exact int32 QK^T of one 128x128 tile of codes: rows qblk*128.. of Q head

@@ -53,6 +53,13 @@ class SageQkvI8F8(ctypes.Structure):
                 ("B", _i64), ("Hq", _i64), ("Hkv", _i64), ("Nq", _i64), ("Nk", _i64), ("D", _i64)]
 
 
+class SageQkvNvfp4(ctypes.Structure):
+    _fields_ = [("q", _vp), ("q_sf", _vp), ("k", _vp), ("k_sf", _vp), ("v_t", _vp), ("v_sf_t", _vp),
+                ("qk_correction", _vp), ("q_mean", _vp), ("k_mean", _vp), ("q_dot_kmean", _vp),
+                ("B", _i64), ("Hq", _i64), ("Hkv", _i64), ("Nq", _i64), ("Nk", _i64), ("D", _i64),
+                ("unpadded_k_len", _i64), ("per_block_mean", ctypes.c_int32)]
+
+
 _lib = None
 
 
@@ -88,6 +95,13 @@ def lib():
         "sage_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, _vp]),
         "sage_quantize_qkv_noalloc": (ctypes.c_int, [P(SageTensor), P(SageTensor), P(SageTensor),
                                                      ctypes.c_int, P(SageQkvI8F8), _vp]),
+        "sage_quantize_nvfp4_workspace_bytes": (ctypes.c_size_t, [_i64] * 6),
+        "sage_quantize_qkv_nvfp4": (ctypes.c_int, [P(SageTensor), P(SageTensor), P(SageTensor),
+                                                   ctypes.c_int, _i64, P(SageQkvNvfp4), _vp,
+                                                   ctypes.c_size_t, _vp]),
+        "sage_attn_fwd_nvfp4": (ctypes.c_int, [P(SageQkvNvfp4), ctypes.c_float, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int32,
+                                               _i64, _i64, _i64, _vp, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -316,3 +330,84 @@ def sage_get_device_status():
 
 def default_sm_scale(D):
     return 1.0 / math.sqrt(D)
+
+
+@dataclasses.dataclass
+class QuantizedNvfp4:
+    """NVFP4 quantised Q/K/V (device tensors) with the layouts of sage_qkv_nvfp4."""
+    q: torch.Tensor              # u8 [B, Hq, Nq_pad, D/2]   packed E2M1
+    q_sf: torch.Tensor           # u8 [B, Hq, Nq_pad, D/16]  E4M3
+    k: torch.Tensor              # u8 [B, Hkv, Nk_pad, D/2]
+    k_sf: torch.Tensor           # u8 [B, Hkv, Nk_pad, D/16]
+    v_t: torch.Tensor            # u8 [B, Hkv, D, Nk_pad/2]
+    v_sf_t: torch.Tensor         # u8 [B, Hkv, D, Nk_pad/16]
+    qk_correction: torch.Tensor  # fp32 [B, Hq, Nq_pad/128, Nk_pad]
+    q_mean: torch.Tensor         # fp32 [B, Hq, Nq_pad/128, D]
+    k_mean: torch.Tensor         # fp32 [B, Hkv, D]
+    q_dot_kmean: Optional[torch.Tensor]
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    D: int
+    unpadded_k_len: int
+    per_block_mean: bool
+
+    @classmethod
+    def empty(cls, B, Hq, Hkv, Nq, Nk, D, unpadded_k_len, per_block_mean, device, with_qdk=True):
+        Nqp, Nkp = pad128(Nq), pad128(Nk)
+        u8 = dict(dtype=torch.uint8, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
+        return cls(torch.empty(B, Hq, Nqp, D // 2, **u8), torch.empty(B, Hq, Nqp, D // 16, **u8),
+                   torch.empty(B, Hkv, Nkp, D // 2, **u8), torch.empty(B, Hkv, Nkp, D // 16, **u8),
+                   torch.empty(B, Hkv, D, Nkp // 2, **u8), torch.empty(B, Hkv, D, Nkp // 16, **u8),
+                   torch.empty(B, Hq, Nqp // 128, Nkp, **f32), torch.empty(B, Hq, Nqp // 128, D, **f32),
+                   torch.empty(B, Hkv, D, **f32),
+                   torch.empty(B, Hq, Nq, **f32) if with_qdk else None,
+                   B, Hq, Hkv, Nq, Nk, D, unpadded_k_len, bool(per_block_mean))
+
+    def struct(self) -> SageQkvNvfp4:
+        p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        return SageQkvNvfp4(p(self.q), p(self.q_sf), p(self.k), p(self.k_sf), p(self.v_t),
+                            p(self.v_sf_t), p(self.qk_correction), p(self.q_mean), p(self.k_mean),
+                            p(self.q_dot_kmean), self.B, self.Hq, self.Hkv, self.Nq, self.Nk, self.D,
+                            self.unpadded_k_len, int(self.per_block_mean))
+
+
+def sage_quantize_qkv_nvfp4(q, k, v, per_block_mean=True, unpadded_k_len=None, layout="HND",
+                            with_qdk=True, out: Optional[QuantizedNvfp4] = None,
+                            ws: Optional[torch.Tensor] = None):
+    """NVFP4 quantisation (sage_quantize_qkv_nvfp4)."""
+    L = lib()
+    tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
+    ukl = tk.N if unpadded_k_len is None else int(unpadded_k_len)
+    if out is None:
+        out = QuantizedNvfp4.empty(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D, ukl, per_block_mean,
+                                   q.device, with_qdk)
+    if ws is None:
+        ws = _ws(L.sage_quantize_nvfp4_workspace_bytes(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D), q.device)
+    s = out.struct()
+    _check(L.sage_quantize_qkv_nvfp4(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                                     int(bool(per_block_mean)), ukl, ctypes.byref(s), ws.data_ptr(),
+                                     ws.numel(), _stream(q.device)), "sage_quantize_qkv_nvfp4")
+    return out
+
+
+def sage_attn_fwd_nvfp4(qkv: QuantizedNvfp4, sm_scale=None, causal=False, per_block_mean=None,
+                        return_lse=True, out=None, out_dtype=torch.bfloat16, lse=None):
+    """NVFP4 attention on pre-quantised inputs (sage_attn_fwd_nvfp4)."""
+    L = lib()
+    dev = qkv.q.device
+    pbm = qkv.per_block_mean if per_block_mean is None else bool(per_block_mean)
+    if out is None:
+        out = torch.empty(qkv.B, qkv.Hq, qkv.Nq, qkv.D, dtype=out_dtype, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty(qkv.B, qkv.Hq, qkv.Nq, dtype=torch.float32, device=dev)
+    sb, sh, sn, _ = out.stride()
+    s = qkv.struct()
+    _check(L.sage_attn_fwd_nvfp4(ctypes.byref(s), float(sm_scale) if sm_scale else 0.0,
+                                 int(bool(causal)), int(pbm), int(bool(return_lse)), out.data_ptr(),
+                                 _dtype_code(out), sb, sh, sn, lse.data_ptr() if return_lse else None,
+                                 _stream(dev)), "sage_attn_fwd_nvfp4")
+    return (out, lse) if return_lse else out

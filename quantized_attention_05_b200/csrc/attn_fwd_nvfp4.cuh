@@ -1,0 +1,519 @@
+// attn_fwd_nvfp4.cuh -- NVFP4 attention forward for sm_100a
+// ("flashinfer.nvfp4_attention_sm120_fwd": pre-quantised FP4 Q/K/V with
+// per-vector FP8 scale factors, qk_correction with one row per 128-token Q
+// block, unpadded_k_len masking, optional LSE; "sageattn3_blackwell": FP4
+// microscaling for Q/K and V).
+//
+// One CTA owns one 128-row Q tile of one (batch, Q head):
+//   warp 4   producer: TMA for the packed Q, K and V^T tiles, a bulk copy
+//            of the tile's qk_correction row, and the scale factors staged
+//            in shared memory in the layout tcgen05.cp expects (for every
+//            64-element K block a 512-byte block: row r's four scale
+//            factors as one 32-bit word at 16*(r%32) + 4*(r/32));
+//   warp 5   MMA issuer: tcgen05.cp of the scale factors into TMEM and
+//            tcgen05.mma kind::mxf4nvf4 with 16-element E4M3 block scales,
+//            S = Q K^T into a double-buffered TMEM accumulator and
+//            O += P V into TMEM, both fp32;
+//   warps 0-3  softmax, one thread per row: scores S + qk_correction,
+//            masking, exact online softmax with exp2, P' = 2688 * p
+//            quantised per 16 keys to E2M1 with an E4M3 scale (written in the
+//            64-byte-swizzled K-major layout of the MMA), O rescaled in TMEM
+//            when the running max moves, epilogue O / l and LSE.
+// TMEM: S 2 x 128 columns, O D columns, scale factors 32 columns.
+#pragma once
+
+#include "attn_fwd_i8f8.cuh"
+#include "quantize_nvfp4.cuh"
+
+namespace sage {
+
+constexpr int NV_THREADS = 192;
+constexpr int NV_STAGES = 3;
+constexpr float LOG2_2688 = 11.392317422778761f;   // log2(448 * 6)
+
+struct NvAttnArgs {
+  const uint8_t* q_sf;
+  const uint8_t* k_sf;
+  const uint8_t* v_sf_t;
+  const float* corr;
+  const float* qdk;
+  void* out;
+  int64_t out_sb, out_sh, out_sn;
+  int out_fp16;
+  float* lse;
+  int B, Hq, Hkv, G, Nq, Nk, Nqp, Nkp, nqt, nkt, L;
+  int causal, return_lse, causal_off;
+  float c0;       // sm_scale * log2(e)
+  float sm_scale;
+};
+
+template <int D>
+struct NvLayout {
+  static constexpr int ROWB = D / 2;            // bytes per packed Q/K row
+  static constexpr int Q_BYTES = 128 * ROWB;
+  static constexpr int K_BYTES = 128 * ROWB;
+  static constexpr int V_BYTES = D * 64;        // V^T tile: D rows x 128 keys
+  static constexpr int P_BYTES = 128 * 64;      // P tile: 128 rows x 128 keys
+  static constexpr int KB_QK = D / 64;          // 64-element K blocks of QK^T
+  static constexpr int SF_BLK = 512;
+  static constexpr int QK_SWIZZLE = ROWB;       // 64 or 32 bytes
+  static constexpr int QK_SBO = 8 * ROWB;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = (Q_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_V = OFF_K + NV_STAGES * ((K_BYTES + 1023) / 1024 * 1024);
+  static constexpr int OFF_P = OFF_V + NV_STAGES * V_BYTES;
+  static constexpr int OFF_QSF = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_KSF = OFF_QSF + KB_QK * SF_BLK;
+  static constexpr int OFF_VSF = OFF_KSF + NV_STAGES * KB_QK * SF_BLK;
+  static constexpr int OFF_PSF = OFF_VSF + NV_STAGES * 2 * SF_BLK;
+  static constexpr int OFF_CORR = OFF_PSF + 2 * 2 * SF_BLK;
+  static constexpr int OFF_BAR = OFF_CORR + NV_STAGES * 512;
+  // q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2], o_ready[2], mma_done
+  static constexpr int NBAR = 1 + 2 * NV_STAGES + 8 + 1;
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_NLIST = (OFF_TMEM + 16 + 15) / 16 * 16;
+  static constexpr int OFF_LIST = OFF_NLIST + 16;
+  static size_t bytes(int nkt) { return 1024 + OFF_LIST + (size_t)nkt * 4; }
+  // TMEM columns
+  static constexpr uint32_t T_S = 0, T_O = 256, T_SFQ = 384, T_SFK = T_SFQ + 4 * KB_QK,
+                            T_SFV = T_SFK + 4 * KB_QK, T_SFP = T_SFV + 8;
+};
+
+// Block-scaled FP4 MMA: D[tmem] (+)= (A * sfa) (B * sfb)^T, scale factors in TMEM.
+__device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copy one 512-byte scale-factor block (32 rows x 16 bytes in shared memory,
+// no swizzle) into 4 TMEM columns, broadcast to the four lane quarters.
+__device__ __forceinline__ void sf_copy(uint32_t tmem_col, uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128u >> 4) << 32;   // 8-row groups 128 bytes apart
+  d |= (uint64_t)1u << 46;            // descriptor version
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem_col), "l"(d)
+               : "memory");
+}
+
+// Instruction descriptor of the block-scaled MMA: E2M1 A and B (format 1),
+// E4M3 scale factors (bit 23 = 0), K-major, K = 64, N >> 3 at 17, M >> 4 at 24.
+__host__ __device__ constexpr uint32_t nv_idesc(uint32_t M, uint32_t N) {
+  return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Stage the scale factors of 128 rows (row-major, D/16 bytes each, rows from
+// `src` with `row_stride` bytes) into the tcgen05.cp layout at `dst`: the
+// four scale factors of a 64-element block of row r form one word at
+// block*512 + 16*(r % 32) + 4*(r / 32).  Rows >= nrows become 0.
+template <int NSF>
+__device__ __forceinline__ void stage_sf(uint8_t* dst, const uint8_t* src, int64_t row_stride,
+                                         int nrows, int lane) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = lane + 32 * i;
+    uint32_t w[NSF / 4];
+    if (r < nrows) {
+      const uint8_t* p = src + (int64_t)r * row_stride;
+#pragma unroll
+      for (int b = 0; b < NSF / 4; ++b) w[b] = *reinterpret_cast<const uint32_t*>(p + 4 * b);
+    } else {
+#pragma unroll
+      for (int b = 0; b < NSF / 4; ++b) w[b] = 0u;
+    }
+#pragma unroll
+    for (int b = 0; b < NSF / 4; ++b)
+      *reinterpret_cast<uint32_t*>(dst + b * 512 + 16 * (r & 31) + 4 * (r >> 5)) = w[b];
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(NV_THREADS, 1)
+    attn_fwd_nvfp4_kernel(const __grid_constant__ CUtensorMap tmQ,
+                          const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, NvAttnArgs a) {
+  using L = NvLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sQ = smem + L::OFF_Q;
+  uint8_t* sK = smem + L::OFF_K;
+  uint8_t* sV = smem + L::OFF_V;
+  uint8_t* sP = smem + L::OFF_P;
+  uint8_t* sQsf = smem + L::OFF_QSF;
+  uint8_t* sKsf = smem + L::OFF_KSF;
+  uint8_t* sVsf = smem + L::OFF_VSF;
+  uint8_t* sPsf = smem + L::OFF_PSF;
+  float* sCorr = reinterpret_cast<float*>(smem + L::OFF_CORR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + NV_STAGES;
+  uint64_t* s_full = kv_empty + NV_STAGES;   // [S buffer]
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;              // [P buffer]
+  uint64_t* o_ready = p_full + 2;
+  uint64_t* mma_done = o_ready + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
+  int* s_nlist = reinterpret_cast<int*>(smem + L::OFF_NLIST);
+  uint32_t* s_list = reinterpret_cast<uint32_t*>(smem + L::OFF_LIST);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // work: (b, h, qt); causal -> longest rows first
+  int b, h, qt;
+  {
+    const int bid = blockIdx.x, per = a.B * a.Hq;
+    if (a.causal) {
+      qt = a.nqt - 1 - bid / per;
+      b = (bid % per) / a.Hq;
+      h = (bid % per) % a.Hq;
+    } else {
+      const int j = bid % a.G;
+      int t = bid / a.G;
+      qt = t % a.nqt;
+      t /= a.nqt;
+      const int g = t % a.Hkv;
+      b = t / a.Hkv;
+      h = g * a.G + j;
+    }
+  }
+  const int g = h / a.G;
+  const int bhq = b * a.Hq + h, bhk = b * a.Hkv + g;
+  const int row_lo = qt * 128, row_hi = min(row_lo + 127, a.Nq - 1);
+
+  if (warp == 0) {
+    // visible key tiles (bit 2 = needs per-element masking)
+    int count = 0;
+    for (int base = 0; base < a.nkt; base += 32) {
+      const int kt = base + lane;
+      uint32_t f = 0;
+      if (kt < a.nkt) {
+        const int key_lo = kt * 128, key_hi = key_lo + 127;
+        const bool vis = key_lo < a.L && !(a.causal && key_lo > row_hi + a.causal_off);
+        if (vis) {
+          const bool need = key_hi >= a.L || (a.causal && key_hi > row_lo + a.causal_off);
+          f = 1u | (need ? 4u : 0u);
+        }
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, f != 0);
+      if (f) s_list[count + __popc(bal & ((1u << lane) - 1u))] = ((uint32_t)kt << 8) | f;
+      count += __popc(bal);
+    }
+    if (lane == 0) s_nlist[0] = count;
+  } else if (warp == 1 && lane == 0) {
+    mbar_init(q_full, 32);
+    for (int s = 0; s < NV_STAGES; ++s) {
+      mbar_init(&kv_full[s], 32);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_ready[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  } else if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  } else if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int ntile = s_nlist[0];
+
+  if (warp == 4) {
+    // ---------------------------------------------------------- producer
+    stage_sf<D / 16>(sQsf, a.q_sf + ((int64_t)bhq * a.Nqp + qt * 128) * (D / 16), D / 16, 128, lane);
+    fence_proxy_async_smem();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, (uint32_t)L::Q_BYTES);
+      tma_load_2d(sQ, &tmQ, q_full, 0, bhq * a.Nqp + qt * 128);
+    } else {
+      mbar_arrive(q_full);
+    }
+    for (int idx = 0; idx < ntile; ++idx) {
+      const int st = idx % NV_STAGES, rd = idx / NV_STAGES;
+      if (idx >= NV_STAGES &&
+          !__all_sync(0xffffffffu, mbar_wait(&kv_empty[st], (rd - 1) & 1, SITE_KV_EMPTY)))
+        break;
+      const int kt = (int)(s_list[idx] >> 8);
+      stage_sf<D / 16>(sKsf + st * L::KB_QK * L::SF_BLK,
+                       a.k_sf + ((int64_t)bhk * a.Nkp + kt * 128) * (D / 16), D / 16, 128, lane);
+      stage_sf<8>(sVsf + st * 2 * L::SF_BLK, a.v_sf_t + (int64_t)bhk * D * (a.Nkp / 16) + kt * 8,
+                  a.Nkp / 16, D, lane);
+      fence_proxy_async_smem();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&kv_full[st], (uint32_t)(L::K_BYTES + L::V_BYTES + 512));
+        tma_load_2d(sK + st * (L::OFF_V - L::OFF_K) / NV_STAGES, &tmK, &kv_full[st], 0,
+                    bhk * a.Nkp + kt * 128);
+        tma_load_2d(sV + st * L::V_BYTES, &tmV, &kv_full[st], kt * 64, bhk * D);
+        bulk_load(sCorr + st * 128, a.corr + ((int64_t)bhq * a.nqt + qt) * a.Nkp + kt * 128, 512,
+                  &kv_full[st]);
+      } else {
+        mbar_arrive(&kv_full[st]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_QK = nv_idesc(128, 128);
+      constexpr uint32_t ID_PV = nv_idesc(128, D);
+      constexpr int KSTRIDE = (L::OFF_V - L::OFF_K) / NV_STAGES;
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      bool ok = mbar_wait(q_full, 0, SITE_Q_FULL);
+      tc_fence_after();
+#pragma unroll
+      for (int kb = 0; kb < L::KB_QK; ++kb) sf_copy(tmem + L::T_SFQ + 4 * kb, smem_u32(sQsf) + kb * 512);
+      auto do_pv = [&](int j) {
+        ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, SITE_P_FULL);
+        if (!ok) return;
+        tc_fence_after();
+        const int st = j % NV_STAGES;
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+          sf_copy(tmem + L::T_SFV + 4 * kb, smem_u32(sVsf) + (st * 2 + kb) * 512);
+          sf_copy(tmem + L::T_SFP + 4 * kb, smem_u32(sPsf) + ((j & 1) * 2 + kb) * 512);
+        }
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+          mma_nvfp4(tmem + L::T_O, smem_desc(aP + (j & 1) * L::P_BYTES + 32 * kb, 512, 64),
+                    smem_desc(aV + st * L::V_BYTES + 32 * kb, 512, 64), ID_PV,
+                    tmem + L::T_SFP + 4 * kb, tmem + L::T_SFV + 4 * kb, (j > 0 || kb > 0) ? 1u : 0u);
+        tc_commit(&o_ready[j & 1]);
+        tc_commit(&kv_empty[st]);
+      };
+      for (int idx = 0; ok && idx < ntile; ++idx) {
+        const int st = idx % NV_STAGES, buf = idx & 1;
+        ok = mbar_wait(&kv_full[st], (idx / NV_STAGES) & 1, SITE_KV_FULL);
+        if (ok && idx >= 2) ok = mbar_wait(&s_free[buf], ((idx - 2) >> 1) & 1, SITE_S_FREE);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kb = 0; kb < L::KB_QK; ++kb)
+          sf_copy(tmem + L::T_SFK + 4 * kb, smem_u32(sKsf) + (st * L::KB_QK + kb) * 512);
+#pragma unroll
+        for (int kb = 0; kb < L::KB_QK; ++kb)
+          mma_nvfp4(tmem + L::T_S + buf * 128,
+                    smem_desc(aQ + 32 * kb, L::QK_SBO, L::QK_SWIZZLE),
+                    smem_desc(aK + st * KSTRIDE + 32 * kb, L::QK_SBO, L::QK_SWIZZLE), ID_QK,
+                    tmem + L::T_SFQ + 4 * kb, tmem + L::T_SFK + 4 * kb, kb > 0 ? 1u : 0u);
+        tc_commit(&s_full[buf]);
+        if (idx >= 1) do_pv(idx - 1);
+      }
+      if (ok && ntile > 0) do_pv(ntile - 1);
+      tc_commit(mma_done);
+      mbar_wait(mma_done, 0, SITE_MMA_DONE);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- softmax
+    const int rt = threadIdx.x;
+    const int row = row_lo + rt;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tO = tmem + lane_base + L::T_O;
+    const float c = a.c0;
+    const uint64_t c2 = f2_pack(c, c);
+    float m_ref = -INFINITY, l = 0.f;
+    uint32_t n = 0;
+    bool ok = true;
+    for (int idx = 0; idx < ntile; ++idx) {
+      const uint32_t e = s_list[idx];
+      const int kt = (int)(e >> 8);
+      const bool need = (e >> 2) & 1u;
+      const int st = idx % NV_STAGES;
+      const uint32_t buf = n & 1u;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[buf], (n >> 1) & 1, SITE_S_FULL));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[128];
+      const uint32_t tS = tmem + lane_base + L::T_S + buf * 128;
+      SAGE_TMEM_LD32(tS + 0, (sr + 0));
+      SAGE_TMEM_LD32(tS + 32, (sr + 32));
+      SAGE_TMEM_LD32(tS + 64, (sr + 64));
+      SAGE_TMEM_LD32(tS + 96, (sr + 96));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&s_free[buf]);
+      // the tile's correction row arrived with its K/V (bulk copy on kv_full)
+      ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[st], (idx / NV_STAGES) & 1, SITE_KV_FULL));
+      if (!ok) break;
+      const float* corr = sCorr + st * 128;
+#pragma unroll
+      for (int j = 0; j < 128; j += 4) {
+        const float4 cv = *reinterpret_cast<const float4*>(corr + j);
+        sr[j] = __float_as_uint(__uint_as_float(sr[j]) + cv.x);
+        sr[j + 1] = __float_as_uint(__uint_as_float(sr[j + 1]) + cv.y);
+        sr[j + 2] = __float_as_uint(__uint_as_float(sr[j + 2]) + cv.z);
+        sr[j + 3] = __float_as_uint(__uint_as_float(sr[j + 3]) + cv.w);
+      }
+      uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
+      if (need) {
+        const int key0 = kt * 128;
+        int jmax = min(127, a.L - 1 - key0);
+        if (a.causal) jmax = min(jmax, row + a.causal_off - key0);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int hi = jmax - 32 * w;
+          vis[w] = hi >= 31 ? ~0u : (hi < 0 ? 0u : ((2u << hi) - 1u));
+        }
+#pragma unroll
+        for (int j = 0; j < 128; ++j)
+          if (!((vis[j >> 5] >> (j & 31)) & 1u)) sr[j] = __float_as_uint(-INFINITY);
+      }
+      float m0 = __uint_as_float(sr[0]), m1 = __uint_as_float(sr[1]);
+      float m2 = __uint_as_float(sr[2]), m3 = __uint_as_float(sr[3]);
+#pragma unroll
+      for (int j = 4; j < 128; j += 8) {
+        m0 = max3f(m0, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+        m1 = max3f(m1, __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
+        m2 = max3f(m2, __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
+        m3 = max3f(m3, __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
+      }
+      const float mx = max3f(m0, m1, fmaxf(m2, m3));
+      const float mt = mx == -INFINITY ? -INFINITY : mx * c;
+      const float m_new = fmaxf(m_ref, mt);
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = ex2_approx(m_ref - m_use);
+      const float bias = LOG2_2688 - m_use;
+      const uint64_t b2 = f2_pack(bias, bias);
+
+      if (n >= 2) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&o_ready[buf], ((n - 2) >> 1) & 1, SITE_O_READY));
+        if (!ok) break;
+      }
+      // P' = 2688 * p per 16-key vector: E4M3 scale, E2M1 codes
+      uint8_t* prow = sP + buf * L::P_BYTES + rt * 64;
+      uint8_t* psf = sPsf + buf * 2 * L::SF_BLK + 16 * (rt & 31) + 4 * (rt >> 5);
+      uint64_t acc = f2_pack(0.f, 0.f);
+      uint32_t sfw[2] = {0u, 0u};
+#pragma unroll
+      for (int vv = 0; vv < 8; ++vv) {
+        float pv[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int j = vv * 16 + 2 * i;
+          const uint64_t y = f2_fma(f2_pack(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2, b2);
+          float y0, y1;
+          f2_unpack(y, y0, y1);
+          uint64_t p;
+          if (i % POLY_EVERY == POLY_EVERY - 1)
+            p = f2_exp2_poly(y0, y1);
+          else
+            p = f2_pack(ex2_approx(y0), ex2_approx(y1));
+          f2_unpack(p, pv[2 * i], pv[2 * i + 1]);
+          if (need) {
+            if (!((vis[j >> 5] >> (j & 31)) & 1u)) pv[2 * i] = 0.f;
+            if (!((vis[j >> 5] >> ((j + 1) & 31)) & 1u)) pv[2 * i + 1] = 0.f;
+          }
+          acc = f2_add(acc, f2_pack(pv[2 * i], pv[2 * i + 1]));
+        }
+        uint32_t w0, w1;
+        const uint32_t sf = nvfp4_vector(pv, &w0, &w1);
+        sfw[vv >> 2] |= sf << (8 * (vv & 3));
+        // 16-byte chunk vv/2 of the row (64-byte swizzle: chunk ^ ((row >> 1) & 3))
+        uint8_t* dst = prow + ((((vv >> 1) ^ ((rt >> 1) & 3))) << 4) + (vv & 1) * 8;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
+      }
+      *reinterpret_cast<uint32_t*>(psf) = sfw[0];
+      *reinterpret_cast<uint32_t*>(psf + L::SF_BLK) = sfw[1];
+      if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        const uint32_t pb = (n - 1) & 1u;
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[pb], ((n - 1) >> 1) & 1, SITE_O_READY));
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+        for (int cb = 0; cb < D; cb += 32) {
+          uint32_t o[32];
+          SAGE_TMEM_LD32(tO + cb, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float x0, x1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2), x0, x1);
+            o[i] = __float_as_uint(x0);
+            o[i + 1] = __float_as_uint(x1);
+          }
+          SAGE_TMEM_ST32(tO + cb, o);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[buf]);
+      float a0, a1;
+      f2_unpack(acc, a0, a1);
+      l = l * alpha + (a0 + a1);
+      m_ref = m_new;
+      ++n;
+    }
+    if (ok && n > 0) {
+      const uint32_t pb = (n - 1) & 1u;
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[pb], ((n - 1) >> 1) & 1, SITE_O_READY));
+      tc_fence_after();
+    }
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    const bool live = ok && n > 0;
+    char* obase = reinterpret_cast<char*>(a.out) +
+                  ((int64_t)b * a.out_sb + (int64_t)h * a.out_sh + (int64_t)row * a.out_sn) * 2;
+    __shared__ float s_one[D];
+    if (threadIdx.x < D) s_one[threadIdx.x] = 1.f;
+    asm volatile("bar.sync 1, 128;" ::: "memory");   // the softmax warps only
+#pragma unroll
+    for (int cb = 0; cb < D; cb += 32) {
+      uint32_t o[32];
+      if (live) {
+        SAGE_TMEM_LD32(tO + cb, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      if (row < a.Nq) {
+        AttnArgs dummy{};
+        if (a.out_fp16)
+          store_out_chunk<D, __half>(dummy, reinterpret_cast<__half*>(obase), cb, o, s_one, inv_l);
+        else
+          store_out_chunk<D, __nv_bfloat16>(dummy, reinterpret_cast<__nv_bfloat16*>(obase), cb, o,
+                                            s_one, inv_l);
+      }
+    }
+    if (a.return_lse && row < a.Nq) {
+      float v = -INFINITY;
+      if (l > 0.f)
+        v = (m_ref + log2f(l) - LOG2_2688) * LN2_F + a.sm_scale * a.qdk[(int64_t)bhq * a.Nq + row];
+      a.lse[(int64_t)bhq * a.Nq + row] = v;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace sage

@@ -17,6 +17,8 @@
 #include "sage_ptx.cuh"
 #include "quantize_i8f8.cuh"
 #include "attn_fwd_i8f8.cuh"
+#include "quantize_nvfp4.cuh"
+#include "attn_fwd_nvfp4.cuh"
 
 using namespace sage;
 
@@ -321,6 +323,172 @@ sage_status run_attention(const sage_qkv_i8f8* z, int causal, float sm_scale, in
   return launch_status();
 }
 
+// ---------------------------------------------------------------- NVFP4 quantise
+struct NvPlan {
+  QuantPlan k, q;
+  size_t k_bytes, q_bytes, total;
+};
+NvPlan nv_plan(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D) {
+  NvPlan p;
+  p.k = quant_plan(B, Hkv, Nk, D);
+  p.q = quant_plan(B, Hq, Nq, D);
+  const int64_t nqt = pad128(Nq) / 128;
+  // per-block means need one split per 128-token block; the global mean uses
+  // the reduction plan.  Size for the larger of the two.
+  const int64_t qs = std::max<int64_t>(p.q.splits, nqt);
+  p.k_bytes = 2 * align256((size_t)B * Hkv * p.k.splits * D * 8);
+  p.q_bytes = 2 * align256((size_t)B * Hq * qs * D * 8);
+  p.total = p.k_bytes + p.q_bytes;
+  return p;
+}
+
+sage_status check_nvfp4(const sage_qkv_nvfp4* z, bool need_qdk) {
+  if (!z) return SAGE_ERR_INVALID_ARG;
+  sage_status st = check_qkv_shapes(z->B, z->Hq, z->Hkv, z->Nq, z->Nk, z->D);
+  if (st != SAGE_OK) return st;
+  if (!z->q || !z->q_sf || !z->k || !z->k_sf || !z->v_t || !z->v_sf_t || !z->qk_correction ||
+      !z->q_mean || !z->k_mean)
+    return SAGE_ERR_INVALID_ARG;
+  if (need_qdk && !z->q_dot_kmean) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(z->q) || !aligned16(z->k) || !aligned16(z->v_t) || !aligned16(z->qk_correction))
+    return SAGE_ERR_INVALID_ARG;
+  if (z->unpadded_k_len < 1 || z->unpadded_k_len > z->Nk) return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
+}
+
+std::atomic<uint32_t> g_smem_corr{0};
+
+sage_status run_quantize_nvfp4(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                               int per_block_mean, int64_t unpadded_k_len,
+                               const sage_qkv_nvfp4* out, void* ws, size_t ws_bytes,
+                               cudaStream_t stream) {
+  sage_status st;
+  if ((st = check_tensor(q)) || (st = check_tensor(k)) || (st = check_tensor(v))) return st;
+  if (q->dtype != k->dtype || q->dtype != v->dtype) return SAGE_ERR_INVALID_ARG;
+  if (k->B != q->B || v->B != q->B || k->H != v->H || k->N != v->N || k->D != q->D ||
+      v->D != q->D)
+    return SAGE_ERR_INVALID_ARG;
+  const int64_t L = unpadded_k_len <= 0 ? k->N : unpadded_k_len;
+  if (L > k->N) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_nvfp4(out, false))) return st;
+  if (out->B != q->B || out->Hq != q->H || out->Hkv != k->H || out->Nq != q->N ||
+      out->Nk != k->N || out->D != q->D || out->unpadded_k_len != L ||
+      (out->per_block_mean != 0) != (per_block_mean != 0))
+    return SAGE_ERR_INVALID_ARG;
+  const NvPlan plan = nv_plan(q->B, q->H, k->H, q->N, k->N, q->D);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < plan.total) return SAGE_ERR_WORKSPACE;
+
+  NvQuantArgs a{};
+  a.q = q->ptr; a.k = k->ptr; a.v = v->ptr;
+  a.q_sb = q->sb; a.q_sh = q->sh; a.q_sn = q->sn;
+  a.k_sb = k->sb; a.k_sh = k->sh; a.k_sn = k->sn;
+  a.v_sb = v->sb; a.v_sh = v->sh; a.v_sn = v->sn;
+  a.B = (int)q->B; a.Hq = (int)q->H; a.Hkv = (int)k->H; a.G = a.Hq / a.Hkv;
+  a.Nq = (int)q->N; a.Nk = (int)k->N;
+  a.Nqp = (int)pad128(q->N); a.Nkp = (int)pad128(k->N);
+  a.nqt = a.Nqp / 128; a.nkt = a.Nkp / 128;
+  a.L = (int)L;
+  a.per_block_mean = per_block_mean ? 1 : 0;
+  // K sums over the first L tokens
+  const QuantPlan kp = quant_plan(q->B, k->H, L, q->D);
+  a.k_splits = kp.splits; a.k_split_tokens = kp.split_tokens;
+  if (a.per_block_mean) {
+    a.q_splits = a.nqt; a.q_split_tokens = 128;
+  } else {
+    a.q_splits = plan.q.splits; a.q_split_tokens = plan.q.split_tokens;
+  }
+  char* w = static_cast<char*>(ws);
+  const size_t kn = (size_t)a.B * a.Hkv * plan.k.splits * q->D;
+  const size_t qn = (size_t)a.B * a.Hq * std::max(plan.q.splits, a.nqt) * q->D;
+  a.k_hi = reinterpret_cast<double*>(w);
+  a.k_lo = reinterpret_cast<double*>(w + align256(kn * 8));
+  a.q_hi = reinterpret_cast<double*>(w + plan.k_bytes);
+  a.q_lo = reinterpret_cast<double*>(w + plan.k_bytes + align256(qn * 8));
+  a.q4 = out->q; a.q_sf = out->q_sf; a.k4 = out->k; a.k_sf = out->k_sf;
+  a.v4t = out->v_t; a.v_sf_t = out->v_sf_t; a.corr = out->qk_correction;
+  a.q_mean = out->q_mean; a.k_mean = out->k_mean; a.qdk = out->q_dot_kmean;
+
+  const bool fp16 = q->dtype == SAGE_FP16;
+  const int nblocks = a.B * a.Hq * a.nqt + 2 * a.B * a.Hkv * a.nkt;
+  const dim3 gk(a.k_splits, a.B * a.Hkv), gq(a.q_splits, a.B * a.Hq), gc(a.nkt, a.B * a.Hkv);
+  const size_t corr_smem = (size_t)(q->D * 128 + 64 * q->D) * 4;
+#define SAGE_NV_LAUNCH(T, D)                                                                     \
+  do {                                                                                           \
+    nv_colsum_kernel<T, D><<<gk, QUANT_THREADS, 0, stream>>>(a.k, a.k_sb, a.k_sh, a.k_sn, a.Hkv, \
+                                                             a.L, a.k_splits, a.k_split_tokens,  \
+                                                             a.k_hi, a.k_lo);                    \
+    nv_colsum_kernel<T, D><<<gq, QUANT_THREADS, 0, stream>>>(a.q, a.q_sb, a.q_sh, a.q_sn, a.Hq,  \
+                                                             a.Nq, a.q_splits, a.q_split_tokens, \
+                                                             a.q_hi, a.q_lo);                    \
+    nv_means_kernel<D><<<a.B * (a.Hkv + a.Hq), D, 0, stream>>>(a);                               \
+    nv_quant_kernel<T, D><<<nblocks, QUANT_THREADS, 0, stream>>>(a);                             \
+    if (!ensure_smem(nv_corr_kernel<T, D>, corr_smem, &g_smem_corr)) return SAGE_ERR_CUDA;       \
+    nv_corr_kernel<T, D><<<gc, 256, corr_smem, stream>>>(a);                                     \
+  } while (0)
+  if (q->D == 128) {
+    if (fp16) SAGE_NV_LAUNCH(__half, 128); else SAGE_NV_LAUNCH(__nv_bfloat16, 128);
+  } else {
+    if (fp16) SAGE_NV_LAUNCH(__half, 64); else SAGE_NV_LAUNCH(__nv_bfloat16, 64);
+  }
+#undef SAGE_NV_LAUNCH
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- NVFP4 attention
+std::atomic<uint32_t> g_smem_nv64{0}, g_smem_nv128{0};
+
+sage_status run_attention_nvfp4(const sage_qkv_nvfp4* z, float sm_scale, int causal,
+                                int per_block_mean, int return_lse, void* out, int32_t out_dtype,
+                                int64_t out_sb, int64_t out_sh, int64_t out_sn, float* lse,
+                                cudaStream_t stream) {
+  sage_status st;
+  if ((st = check_nvfp4(z, return_lse != 0))) return st;
+  if ((per_block_mean != 0) != (z->per_block_mean != 0)) return SAGE_ERR_INVALID_ARG;
+  if (!out || !aligned16(out)) return SAGE_ERR_INVALID_ARG;
+  if (out_dtype != SAGE_BF16 && out_dtype != SAGE_FP16) return SAGE_ERR_INVALID_ARG;
+  if (out_sn < z->D || out_sn % 8 || out_sh % 8 || out_sb % 8 || out_sh < 0 || out_sb < 0)
+    return SAGE_ERR_INVALID_ARG;
+  if ((return_lse != 0) != (lse != nullptr)) return SAGE_ERR_INVALID_ARG;
+  if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  NvAttnArgs a{};
+  a.q_sf = z->q_sf; a.k_sf = z->k_sf; a.v_sf_t = z->v_sf_t; a.corr = z->qk_correction;
+  a.qdk = z->q_dot_kmean;
+  a.out = out; a.out_sb = out_sb; a.out_sh = out_sh; a.out_sn = out_sn;
+  a.out_fp16 = out_dtype == SAGE_FP16;
+  a.lse = lse;
+  a.B = (int)z->B; a.Hq = (int)z->Hq; a.Hkv = (int)z->Hkv; a.G = a.Hq / a.Hkv;
+  a.Nq = (int)z->Nq; a.Nk = (int)z->Nk;
+  a.Nqp = (int)pad128(z->Nq); a.Nkp = (int)pad128(z->Nk);
+  a.nqt = a.Nqp / 128; a.nkt = a.Nkp / 128;
+  a.L = (int)z->unpadded_k_len;
+  a.causal = causal ? 1 : 0;
+  a.return_lse = return_lse ? 1 : 0;
+  a.causal_off = a.Nk - a.Nq;
+  const float s = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)z->D);
+  a.sm_scale = s;
+  a.c0 = (float)((double)s * 1.4426950408889634);
+  const int64_t D = z->D;
+  const CUtensorMapSwizzle sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_u8(&tq, z->q, D / 2, z->B * z->Hq * a.Nqp, D / 2, (uint32_t)(D / 2), 128, sw) ||
+      !make_tmap_u8(&tk, z->k, D / 2, z->B * z->Hkv * a.Nkp, D / 2, (uint32_t)(D / 2), 128, sw) ||
+      !make_tmap_u8(&tv, z->v_t, a.Nkp / 2, z->B * z->Hkv * D, a.Nkp / 2, 64, (uint32_t)D,
+                    CU_TENSOR_MAP_SWIZZLE_64B))
+    return SAGE_ERR_CUDA;
+  const int grid = a.B * a.Hq * a.nqt;
+  if (D == 128) {
+    if (!ensure_smem(attn_fwd_nvfp4_kernel<128>, NvLayout<128>::bytes(ATT_MAX_NKT), &g_smem_nv128))
+      return SAGE_ERR_CUDA;
+    attn_fwd_nvfp4_kernel<128><<<grid, NV_THREADS, NvLayout<128>::bytes(a.nkt), stream>>>(tq, tk, tv, a);
+  } else {
+    if (!ensure_smem(attn_fwd_nvfp4_kernel<64>, NvLayout<64>::bytes(ATT_MAX_NKT), &g_smem_nv64))
+      return SAGE_ERR_CUDA;
+    attn_fwd_nvfp4_kernel<64><<<grid, NV_THREADS, NvLayout<64>::bytes(a.nkt), stream>>>(tq, tk, tv, a);
+  }
+  return launch_status();
+}
+
 // Carve the fused call's workspace: quantised Q/K/V, then the quantiser's
 // partials, then the mask classes.
 struct FusedLayout {
@@ -433,6 +601,27 @@ sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage
   if ((st = run_quantize(q, k, v, smooth_k, &z, w + f.part, f.cls - f.part, stream))) return st;
   return run_attention(&z, causal, sm_scale, return_lse, mask, out, q->dtype, out_sb, out_sh,
                        out_sn, lse, w + f.cls, f.total - f.cls, stream);
+}
+
+size_t sage_quantize_nvfp4_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
+                                           int64_t Nk, int64_t D) {
+  if (!valid_dims(B, Hq, Nq, D) || !valid_dims(B, Hkv, Nk, D)) return 0;
+  return nv_plan(B, Hq, Hkv, Nq, Nk, D).total;
+}
+
+sage_status sage_quantize_qkv_nvfp4(const sage_tensor* q, const sage_tensor* k,
+                                    const sage_tensor* v, int per_block_mean,
+                                    int64_t unpadded_k_len, const sage_qkv_nvfp4* out, void* ws,
+                                    size_t ws_bytes, sage_stream_t stream) {
+  return run_quantize_nvfp4(q, k, v, per_block_mean, unpadded_k_len, out, ws, ws_bytes, stream);
+}
+
+sage_status sage_attn_fwd_nvfp4(const sage_qkv_nvfp4* qkv, float sm_scale, int causal,
+                                int per_block_mean, int return_lse, void* out, int32_t out_dtype,
+                                int64_t out_sb, int64_t out_sh, int64_t out_sn, float* lse,
+                                sage_stream_t stream) {
+  return run_attention_nvfp4(qkv, sm_scale, causal, per_block_mean, return_lse, out, out_dtype,
+                             out_sb, out_sh, out_sn, lse, stream);
 }
 
 sage_status sage_debug_qk_int32(const sage_qkv_i8f8* z, int64_t b, int64_t h, int64_t qblk,

@@ -47,8 +47,10 @@ def test_ctypes_layout_matches_header(tmp_path):
 #include <stddef.h>
 #include "sage_b200.h"
 int main(void) {
-  printf("%zu %zu %zu\\n", sizeof(sage_tensor), sizeof(sage_mask), sizeof(sage_qkv_i8f8));
-  printf("%zu %zu %zu\\n", offsetof(sage_tensor, B), offsetof(sage_mask, sq), offsetof(sage_qkv_i8f8, D));
+  printf("%zu %zu %zu %zu\\n", sizeof(sage_tensor), sizeof(sage_mask), sizeof(sage_qkv_i8f8),
+         sizeof(sage_qkv_nvfp4));
+  printf("%zu %zu %zu %zu\\n", offsetof(sage_tensor, B), offsetof(sage_mask, sq),
+         offsetof(sage_qkv_i8f8, D), offsetof(sage_qkv_nvfp4, per_block_mean));
   return 0;
 }""")
     exe = tmp_path / "probe"
@@ -57,8 +59,10 @@ int main(void) {
     lines = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
     sizes = list(map(int, lines[0].split()))
     offs = list(map(int, lines[1].split()))
-    assert sizes == [ctypes.sizeof(S.SageTensor), ctypes.sizeof(S.SageMask), ctypes.sizeof(S.SageQkvI8F8)]
-    assert offs == [S.SageTensor.B.offset, S.SageMask.sq.offset, S.SageQkvI8F8.D.offset]
+    assert sizes == [ctypes.sizeof(S.SageTensor), ctypes.sizeof(S.SageMask), ctypes.sizeof(S.SageQkvI8F8),
+                     ctypes.sizeof(S.SageQkvNvfp4)]
+    assert offs == [S.SageTensor.B.offset, S.SageMask.sq.offset, S.SageQkvI8F8.D.offset,
+                    S.SageQkvNvfp4.per_block_mean.offset]
 
 
 def test_status_strings_and_version(L):
@@ -140,3 +144,22 @@ def test_workspace_sizes_cover_the_quantised_tensors(L):
     assert payload < need < payload * 1.1
     assert L.sage_quantize_workspace_bytes(B_, Hkv, N, D) > 0
     assert L.sage_quantize_workspace_bytes(0, Hkv, N, D) == 0
+
+
+def test_nvfp4_rejects_bad_arguments_on_host(L):
+    byref = ctypes.byref
+    q, k, v = _t(H=2), _t(H=2), _t(H=2)
+    z = S.SageQkvNvfp4(256, 256, 256, 256, 256, 256, 256, 256, 256, 256, 1, 2, 2, 256, 256, 64, 256, 1)
+    f = L.sage_quantize_qkv_nvfp4
+    assert f(byref(q), byref(k), byref(v), 1, 300, byref(z), 256, 1 << 30, None) \
+        == S.SAGE_ERR_INVALID_ARG                                   # unpadded length > N
+    assert f(byref(q), byref(k), byref(v), 0, 256, byref(z), 256, 1 << 30, None) \
+        == S.SAGE_ERR_INVALID_ARG                                   # per_block_mean mismatch
+    need = L.sage_quantize_nvfp4_workspace_bytes(1, 2, 2, 256, 256, 64)
+    assert f(byref(q), byref(k), byref(v), 1, 256, byref(z), 256, need - 1, None) == S.SAGE_ERR_WORKSPACE
+    a = L.sage_attn_fwd_nvfp4
+    assert a(byref(z), 0.0, 0, 0, 1, 256, 0, 0, 256 * 64, 64, 512, None) \
+        == S.SAGE_ERR_INVALID_ARG                                   # per_block_mean mismatch
+    zz = S.SageQkvNvfp4(256, 256, 256, 256, 256, 256, 256, 256, 256, None, 1, 2, 2, 256, 256, 64, 256, 1)
+    assert a(byref(zz), 0.0, 0, 1, 1, 256, 0, 0, 256 * 64, 64, 512, None) \
+        == S.SAGE_ERR_INVALID_ARG                                   # LSE without q_dot_kmean
