@@ -98,23 +98,25 @@ typedef struct {
 
 /* Quantised Q/K/V of the INT8/FP8 path, all device memory owned by the
  * caller.  Nq_pad = ceil(Nq/128)*128, Nk_pad = ceil(Nk/128)*128; every
- * array is dense in the order given.
+ * array is dense in the order given.  V keeps its own [token, channel]
+ * order: the PV product reads each 128-token tile as an MN-major operand,
+ * so no transposition is needed.
  *   q        int8  [B, Hq,  Nq_pad, D]   codes; rows >= Nq are 0
  *   q_scale  fp32  [B, Hq,  Nq_pad/128]  one scale per 128-token block
  *   k        int8  [B, Hkv, Nk_pad, D]   codes of K - kmean; rows >= Nk are 0
  *   k_scale  fp32  [B, Hkv, Nk_pad/128]
  *   k_mean   fp32  [B, Hkv, D]
- *   v_t      e4m3  [B, Hkv, D, Nk_pad]   V codes, transposed; tokens >= Nk are 0
+ *   v        e4m3  [B, Hkv, Nk_pad, D]   V codes; rows >= Nk are 0
  *   v_scale  fp32  [B, Hkv, D]
  *   q_dot_kmean fp32 [B, Hq, Nq]  (may be NULL when no LSE is wanted)
- * The base pointers of q, k and v_t must be 16-byte aligned. */
+ * The base pointers of q, k and v must be 16-byte aligned. */
 typedef struct {
   int8_t* q;
   float* q_scale;
   int8_t* k;
   float* k_scale;
   float* k_mean;
-  uint8_t* v_t;
+  uint8_t* v;
   float* v_scale;
   float* q_dot_kmean;
   int64_t B, Hq, Hkv, Nq, Nk, D;

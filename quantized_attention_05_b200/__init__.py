@@ -49,7 +49,7 @@ class SageMask(ctypes.Structure):
 
 class SageQkvI8F8(ctypes.Structure):
     _fields_ = [("q", _vp), ("q_scale", _vp), ("k", _vp), ("k_scale", _vp), ("k_mean", _vp),
-                ("v_t", _vp), ("v_scale", _vp), ("q_dot_kmean", _vp),
+                ("v", _vp), ("v_scale", _vp), ("q_dot_kmean", _vp),
                 ("B", _i64), ("Hq", _i64), ("Hkv", _i64), ("Nq", _i64), ("Nk", _i64), ("D", _i64)]
 
 
@@ -173,7 +173,7 @@ class QuantizedQKV:
     k: torch.Tensor            # int8  [B, Hkv, Nk_pad, D]
     k_scale: torch.Tensor      # fp32  [B, Hkv, Nk_pad/128]
     k_mean: torch.Tensor       # fp32  [B, Hkv, D]
-    v_t: torch.Tensor          # uint8 (E4M3) [B, Hkv, D, Nk_pad]
+    v: torch.Tensor            # uint8 (E4M3) [B, Hkv, Nk_pad, D]
     v_scale: torch.Tensor      # fp32  [B, Hkv, D]
     q_dot_kmean: Optional[torch.Tensor]  # fp32 [B, Hq, Nq]
     B: int
@@ -192,7 +192,7 @@ class QuantizedQKV:
                    torch.empty(B, Hkv, Nkp, D, dtype=torch.int8, **kw),
                    torch.empty(B, Hkv, Nkp // 128, dtype=torch.float32, **kw),
                    torch.empty(B, Hkv, D, dtype=torch.float32, **kw),
-                   torch.empty(B, Hkv, D, Nkp, dtype=torch.uint8, **kw),
+                   torch.empty(B, Hkv, Nkp, D, dtype=torch.uint8, **kw),
                    torch.empty(B, Hkv, D, dtype=torch.float32, **kw),
                    torch.empty(B, Hq, Nq, dtype=torch.float32, **kw) if with_qdk else None,
                    B, Hq, Hkv, Nq, Nk, D)
@@ -200,7 +200,7 @@ class QuantizedQKV:
     def struct(self) -> SageQkvI8F8:
         p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
         return SageQkvI8F8(p(self.q), p(self.q_scale), p(self.k), p(self.k_scale), p(self.k_mean),
-                           p(self.v_t), p(self.v_scale), p(self.q_dot_kmean),
+                           p(self.v), p(self.v_scale), p(self.q_dot_kmean),
                            self.B, self.Hq, self.Hkv, self.Nq, self.Nk, self.D)
 
 

@@ -67,10 +67,14 @@ template <int D>
 struct AttnLayout {
   static constexpr int Q_BYTES = ATT_BM * D;
   static constexpr int K_BYTES = ATT_BN * D;
-  static constexpr int V_BYTES = D * ATT_BN;
+  static constexpr int V_BYTES = ATT_BN * D;
   static constexpr int P_BYTES = ATT_BM * ATT_BN;
   static constexpr int QK_SWIZZLE = D;            // bytes per Q/K row: 128 or 64
   static constexpr int QK_SBO = 8 * D;            // 8-row group stride
+  // V tile: 128 token rows of D bytes, read MN-major by the PV MMA (one
+  // swizzle atom across D, 8-row groups QK_SBO apart); one MMA consumes 32
+  // tokens, i.e. 32 rows.
+  static constexpr int V_KSTEP = 32 * D;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + ATT_STAGES * K_BYTES;
@@ -369,7 +373,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const int kt = (int)(s_list[idx] >> 8);
         mbar_arrive_expect_tx(&kv_full[st], (uint32_t)(L::K_BYTES + L::V_BYTES));
         tma_load_2d(sK + st * L::K_BYTES, &tmK, &kv_full[st], 0, bhk * a.Nkp + kt * ATT_BN);
-        tma_load_2d(sV + st * L::V_BYTES, &tmV, &kv_full[st], kt * ATT_BN, bhk * D);
+        tma_load_2d(sV + st * L::V_BYTES, &tmV, &kv_full[st], 0, bhk * a.Nkp + kt * ATT_BN);
       }
     }
     __syncwarp();
@@ -381,7 +385,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // have issued their PV on it.
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = instr_desc(kDS32, kS8, kS8, ATT_BM, ATT_BN);
-      constexpr uint32_t IDESC_PV = instr_desc(kDF32, kE4M3, kE4M3, ATT_BM, D);
+      constexpr uint32_t IDESC_PV = instr_desc(kDF32, kE4M3, kE4M3, ATT_BM, D) | kBMajorMN;
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
       auto next_active = [&](int i, int from) {
         while (from < ntile && !((s_list[from] >> i) & 1u)) ++from;
@@ -423,8 +427,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const uint32_t va = aV + (ep % ATT_STAGES) * L::V_BYTES;
 #pragma unroll
             for (int kk = 0; kk < ATT_BN / 32; ++kk)
-              mma_f8f6f4(tO, smem_desc(pa + 32 * kk, 1024, 128), smem_desc(va + 32 * kk, 1024, 128),
-                         IDESC_PV, (k > 0 || kk > 0) ? 1u : 0u);
+              mma_f8f6f4(tO, smem_desc(pa + 32 * kk, 1024, 128),
+                         smem_desc(va + L::V_KSTEP * kk, L::QK_SBO, L::QK_SWIZZLE), IDESC_PV,
+                         (k > 0 || kk > 0) ? 1u : 0u);
             tc_commit(&o_ready[i * 2 + (k & 1)]);
             ++pv_k[i];
             pv_e[i] = next_active(i, ep + 1);
@@ -742,11 +747,12 @@ __global__ void __launch_bounds__(128, 1)
     tma_load_2d(sV, &tmV, &bar[0], vcol, vrow);
     if (mbar_wait(&bar[0], 0, SITE_DEBUG)) {
       tc_fence_after();
-      constexpr uint32_t IDESC = instr_desc(kDF32, kE4M3, kE4M3, ATT_BM, D);
+      constexpr uint32_t IDESC = instr_desc(kDF32, kE4M3, kE4M3, ATT_BM, D) | kBMajorMN;
 #pragma unroll
       for (int k = 0; k < ATT_BN / 32; ++k)
         mma_f8f6f4(tmem, smem_desc(smem_u32(sP) + 32 * k, 1024, 128),
-                   smem_desc(smem_u32(sV) + 32 * k, 1024, 128), IDESC, k > 0 ? 1u : 0u);
+                   smem_desc(smem_u32(sV) + L::V_KSTEP * k, L::QK_SBO, L::QK_SWIZZLE), IDESC,
+                   k > 0 ? 1u : 0u);
     }
     tc_commit(&bar[1]);
   }

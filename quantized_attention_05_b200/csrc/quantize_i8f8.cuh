@@ -3,13 +3,15 @@
 // "sageattn_qk_int8_pv_fp16_triton", per-channel FP8 V in
 // "sageattn_qk_int8_pv_fp8_cuda").
 //
-// Two launches, both HBM-bound, 128-bit coalesced loads and stores:
+// Three launches, HBM-bound, 128-bit coalesced loads:
 //   pass A  per (batch, KV head, token split): exact-in-practice K channel
 //           sums (double-double accumulation, fixed reduction order) and V
 //           channel maxima into the workspace;
+//   stats   per (batch, KV head): the splits combined in fixed order into
+//           k_mean, v_scale and the V channel maxima;
 //   pass B  one CTA per 128-token block of Q, K or V: the block's amax,
-//           scale and INT8 codes (Q, K - kmean) or the E4M3 codes of V,
-//           transposed through shared memory.
+//           scale and INT8 codes (Q, K - kmean), or the per-channel E4M3
+//           codes of V, stored in V's own [token, channel] order.
 // Every arithmetic step that decides a code uses an explicitly rounded
 // IEEE operation (__fsub_rn, __fmul_rn, __fdiv_rn, cvt.rn), so the codes and
 // scales are reproducible bit for bit.
@@ -41,8 +43,9 @@ struct QuantArgs {
   int8_t* k8;
   float* k_scale;
   float* k_mean;
-  uint8_t* v8t;
+  uint8_t* v8;
   float* v_scale;
+  float* va;                      // [B*Hkv, D] V channel maxima (workspace)
   float* qdk;                     // may be null
   int kv_limit;                   // tokens of K/V used for the mean / codes (Nk)
 };
@@ -159,21 +162,22 @@ __global__ void __launch_bounds__(QUANT_THREADS) kmean_vamax_partial_kernel(Quan
   }
 }
 
-// Combine the splits of KV head (b, h) in fixed order: kmean and V amax.
+// ------------------------------------------------------------ stats
+// grid B*Hkv, D threads: the splits of KV head bh combined in fixed order
+// into k_mean (0 without smoothing), the V channel maxima and v_scale.
 template <int D>
-__device__ __forceinline__ void combine_splits(const QuantArgs& a, int bh, float* s_km,
-                                               float* s_va) {
-  for (int c = threadIdx.x; c < D; c += blockDim.x) {
-    DD s = {0.0, 0.0};
-    float m = 0.f;
-    for (int sp = 0; sp < a.splits; ++sp) {
-      const int64_t o = ((int64_t)bh * a.splits + sp) * D + c;
-      dd_add(s, DD{a.part_hi[o], a.part_lo[o]});
-      m = fmaxf(m, a.part_amax[o]);
-    }
-    if (s_km) s_km[c] = a.smooth_k ? dd_mean_f32(s, (double)a.kv_limit) : 0.f;
-    if (s_va) s_va[c] = m;
+__global__ void __launch_bounds__(D) kv_stats_kernel(QuantArgs a) {
+  const int bh = blockIdx.x, c = threadIdx.x;
+  DD s = {0.0, 0.0};
+  float m = 0.f;
+  for (int sp = 0; sp < a.splits; ++sp) {
+    const int64_t o = ((int64_t)bh * a.splits + sp) * D + c;
+    dd_add(s, DD{a.part_hi[o], a.part_lo[o]});
+    m = fmaxf(m, a.part_amax[o]);
   }
+  a.k_mean[(int64_t)bh * D + c] = a.smooth_k ? dd_mean_f32(s, (double)a.kv_limit) : 0.f;
+  a.va[(int64_t)bh * D + c] = m;
+  a.v_scale[(int64_t)bh * D + c] = __fdiv_rn(m, 448.f);
 }
 
 __device__ __forceinline__ float block_max(float v, float* s_red) {
@@ -196,16 +200,15 @@ __device__ __forceinline__ int8_t int8_code(float x, float inv) {
 
 // ------------------------------------------------------------ pass B
 // One CTA per 128-token block: [0, nQb) Q blocks, [nQb, nQb+nKb) K blocks,
-// then V blocks.
+// then V blocks.  Each thread keeps its 16-byte loads in registers between
+// the amax and the code pass.
 template <typename T, int D>
-__global__ void __launch_bounds__(QUANT_THREADS) quant_blocks_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArgs a) {
   constexpr int TPR = D / 8;
   constexpr int RPP = QUANT_THREADS / TPR;
   constexpr int ITERS = QB / RPP;
-  __shared__ float s_km[D];
-  __shared__ float s_va[D];
+  __shared__ float s_c[D];      // k_mean (Q with LSE, K) or 448 / V channel max (V)
   __shared__ float s_red[QUANT_THREADS / 32];
-  __shared__ __align__(16) uint8_t s_vt[D][QB + 16];
 
   const int nQb = a.B * a.Hq * a.nqt;
   const int nKb = a.B * a.Hkv * a.nkt;
@@ -217,7 +220,8 @@ __global__ void __launch_bounds__(QUANT_THREADS) quant_blocks_kernel(QuantArgs a
     const int bh = job / a.nqt, qt = job % a.nqt;
     const int b = bh / a.Hq, h = bh % a.Hq;
     const int g = h / a.G;
-    if (a.qdk) combine_splits<D>(a, b * a.Hkv + g, s_km, nullptr);
+    if (a.qdk)
+      for (int c = threadIdx.x; c < D; c += blockDim.x) s_c[c] = a.k_mean[(int64_t)(b * a.Hkv + g) * D + c];
     const char* base = reinterpret_cast<const char*>(a.q) +
                        (b * a.q_sb + h * a.q_sh + cg * 8) * (int64_t)sizeof(T);
     uint4 raw[ITERS];
@@ -226,12 +230,15 @@ __global__ void __launch_bounds__(QUANT_THREADS) quant_blocks_kernel(QuantArgs a
     for (int it = 0; it < ITERS; ++it) {
       const int n = qt * QB + rs + it * RPP;
       raw[it] = n < a.Nq ? ldg16(base + (int64_t)n * a.q_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
       float f[8];
       unpack8<T>(raw[it], f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(f[i]));
     }
-    const float amax = block_max(am, s_red);  // also orders s_km
+    const float amax = block_max(am, s_red);  // also orders s_c
     const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) quant_blocks_kernel(QuantArgs a
       if (a.qdk) {
         float d = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) d = fmaf(f[i], s_km[cg * 8 + i], d);
+        for (int i = 0; i < 8; ++i) d = fmaf(f[i], s_c[cg * 8 + i], d);
 #pragma unroll
         for (int o = TPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
         if (cg == 0 && n < a.Nq) a.qdk[(int64_t)bh * a.Nq + n] = d;
@@ -261,85 +268,86 @@ __global__ void __launch_bounds__(QUANT_THREADS) quant_blocks_kernel(QuantArgs a
     // ---------------- K block: codes of K - kmean
     const int bh = job / a.nkt, kt = job % a.nkt;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
-    combine_splits<D>(a, bh, s_km, nullptr);
-    __syncthreads();
+    for (int c = threadIdx.x; c < D; c += blockDim.x) s_c[c] = a.k_mean[(int64_t)bh * D + c];
     const char* base = reinterpret_cast<const char*>(a.k) +
                        (b * a.k_sb + h * a.k_sh + cg * 8) * (int64_t)sizeof(T);
-    float x[ITERS][8];
+    uint4 raw[ITERS];
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int n = kt * QB + rs + it * RPP;
+      raw[it] = n < a.kv_limit ? ldg16(base + (int64_t)n * a.k_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    float km[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) km[i] = s_c[cg * 8 + i];
     float am = 0.f;
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
       const int n = kt * QB + rs + it * RPP;
+      float f[8];
+      unpack8<T>(raw[it], f);
       if (n < a.kv_limit) {
-        float f[8];
-        unpack8<T>(ldg16(base + (int64_t)n * a.k_sn * sizeof(T)), f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x[it][i] = __fsub_rn(f[i], s_km[cg * 8 + i]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[it][i] = 0.f;
+        for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(__fsub_rn(f[i], km[i])));
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(x[it][i]));
     }
     const float amax = block_max(am, s_red);
     const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
       const int n = kt * QB + rs + it * RPP;
+      float f[8];
+      unpack8<T>(raw[it], f);
       uint32_t w0 = 0, w1 = 0;
+      if (n < a.kv_limit) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) w0 |= (uint32_t)(uint8_t)int8_code(x[it][i], inv) << (8 * i);
+        for (int i = 0; i < 4; ++i)
+          w0 |= (uint32_t)(uint8_t)int8_code(__fsub_rn(f[i], km[i]), inv) << (8 * i);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) w1 |= (uint32_t)(uint8_t)int8_code(x[it][4 + i], inv) << (8 * i);
+        for (int i = 0; i < 4; ++i)
+          w1 |= (uint32_t)(uint8_t)int8_code(__fsub_rn(f[4 + i], km[4 + i]), inv) << (8 * i);
+      }
       *reinterpret_cast<uint2*>(a.k8 + ((int64_t)bh * a.Nkp + n) * D + cg * 8) = make_uint2(w0, w1);
     }
     if (threadIdx.x == 0) a.k_scale[(int64_t)bh * a.nkt + kt] = __fdiv_rn(amax, 127.f);
-    if (kt == 0)
-      for (int c = threadIdx.x; c < D; c += blockDim.x) a.k_mean[(int64_t)bh * D + c] = s_km[c];
     return;
   }
   job -= nKb;
   {
-    // ---------------- V block: E4M3 codes, transposed
+    // ---------------- V block: per-channel E4M3 codes, [token, channel] order
     const int bh = job / a.nkt, vt = job % a.nkt;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
-    combine_splits<D>(a, bh, nullptr, s_va);
-    __syncthreads();
+    for (int c = threadIdx.x; c < D; c += blockDim.x) {
+      const float m = a.va[(int64_t)bh * D + c];
+      s_c[c] = m > 0.f ? __fdiv_rn(448.f, m) : 0.f;
+    }
     const char* base = reinterpret_cast<const char*>(a.v) +
                        (b * a.v_sb + h * a.v_sh + cg * 8) * (int64_t)sizeof(T);
+    uint4 raw[ITERS];
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
-      const int nl = rs + it * RPP;
-      const int n = vt * QB + nl;
-      float f[8];
-      if (n < a.kv_limit) {
-        unpack8<T>(ldg16(base + (int64_t)n * a.v_sn * sizeof(T)), f);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; i += 2) {
-        const float va0 = s_va[cg * 8 + i], va1 = s_va[cg * 8 + i + 1];
-        const float y0 = va0 > 0.f ? __fmul_rn(f[i], __fdiv_rn(448.f, va0)) : 0.f;
-        const float y1 = va1 > 0.f ? __fmul_rn(f[i + 1], __fdiv_rn(448.f, va1)) : 0.f;
-        uint16_t two = cvt_e4m3x2(y0, y1);
-        if (n >= a.kv_limit) two = 0;
-        s_vt[cg * 8 + i][nl] = (uint8_t)(two & 0xFF);
-        s_vt[cg * 8 + i + 1][nl] = (uint8_t)(two >> 8);
-      }
+      const int n = vt * QB + rs + it * RPP;
+      raw[it] = n < a.kv_limit ? ldg16(base + (int64_t)n * a.v_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
-    // write D rows of 128 bytes: 8 threads x 16 bytes per channel row
-    for (int idx = threadIdx.x; idx < D * 8; idx += blockDim.x) {
-      const int c = idx >> 3, ch = idx & 7;
-      const uint4 val = *reinterpret_cast<const uint4*>(&s_vt[c][ch * 16]);
-      *reinterpret_cast<uint4*>(a.v8t + ((int64_t)bh * D + c) * a.Nkp + vt * QB + ch * 16) = val;
+    float inv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) inv[i] = s_c[cg * 8 + i];
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int n = vt * QB + rs + it * RPP;
+      float f[8];
+      unpack8<T>(raw[it], f);
+      uint32_t w[2] = {0u, 0u};
+      if (n < a.kv_limit) {
+#pragma unroll
+        for (int i = 0; i < 8; i += 2)
+          w[i >> 2] |= (uint32_t)cvt_e4m3x2(__fmul_rn(f[i], inv[i]), __fmul_rn(f[i + 1], inv[i + 1]))
+                       << (8 * (i & 3));
+      }
+      *reinterpret_cast<uint2*>(a.v8 + ((int64_t)bh * a.Nkp + n) * D + cg * 8) = make_uint2(w[0], w[1]);
     }
-    if (vt == 0)
-      for (int c = threadIdx.x; c < D; c += blockDim.x)
-        a.v_scale[(int64_t)bh * D + c] = __fdiv_rn(s_va[c], 448.f);
   }
 }
 

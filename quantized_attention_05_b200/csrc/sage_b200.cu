@@ -72,10 +72,10 @@ sage_status check_qkv(const sage_qkv_i8f8* z, bool need_qdk) {
   if (!z) return SAGE_ERR_INVALID_ARG;
   sage_status st = check_qkv_shapes(z->B, z->Hq, z->Hkv, z->Nq, z->Nk, z->D);
   if (st != SAGE_OK) return st;
-  if (!z->q || !z->q_scale || !z->k || !z->k_scale || !z->k_mean || !z->v_t || !z->v_scale)
+  if (!z->q || !z->q_scale || !z->k || !z->k_scale || !z->k_mean || !z->v || !z->v_scale)
     return SAGE_ERR_INVALID_ARG;
   if (need_qdk && !z->q_dot_kmean) return SAGE_ERR_INVALID_ARG;
-  if (!aligned16(z->q) || !aligned16(z->k) || !aligned16(z->v_t)) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(z->q) || !aligned16(z->k) || !aligned16(z->v)) return SAGE_ERR_INVALID_ARG;
   return SAGE_OK;
 }
 
@@ -110,7 +110,7 @@ QuantPlan quant_plan(int64_t B, int64_t Hkv, int64_t Nk, int64_t D) {
   p.splits = (int)s;
   p.split_tokens = (int)t;
   const size_t n = (size_t)bh * s * D;
-  p.part_bytes = align256(n * 8) * 2 + align256(n * 4);
+  p.part_bytes = align256(n * 8) * 2 + align256(n * 4) + align256((size_t)bh * D * 4);
   return p;
 }
 
@@ -154,8 +154,7 @@ bool make_qkv_tmaps(const sage_qkv_i8f8* z, CUtensorMap* tq, CUtensorMap* tk, CU
   const int64_t Nqp = pad128(z->Nq), Nkp = pad128(z->Nk), D = z->D;
   return make_tmap_u8(tq, z->q, D, z->B * z->Hq * Nqp, D, (uint32_t)D, 128, qk_swizzle(D)) &&
          make_tmap_u8(tk, z->k, D, z->B * z->Hkv * Nkp, D, (uint32_t)D, 128, qk_swizzle(D)) &&
-         make_tmap_u8(tv, z->v_t, Nkp, z->B * z->Hkv * D, Nkp, 128, (uint32_t)D,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
+         make_tmap_u8(tv, z->v, D, z->B * z->Hkv * Nkp, D, (uint32_t)D, 128, qk_swizzle(D));
 }
 
 // Dynamic shared memory opt-in, once per device and kernel.
@@ -214,8 +213,9 @@ sage_status run_quantize(const sage_tensor* q, const sage_tensor* k, const sage_
   a.part_hi = reinterpret_cast<double*>(w);
   a.part_lo = reinterpret_cast<double*>(w + align256(n * 8));
   a.part_amax = reinterpret_cast<float*>(w + 2 * align256(n * 8));
+  a.va = reinterpret_cast<float*>(w + 2 * align256(n * 8) + align256(n * 4));
   a.q8 = out->q; a.q_scale = out->q_scale; a.k8 = out->k; a.k_scale = out->k_scale;
-  a.k_mean = out->k_mean; a.v8t = out->v_t; a.v_scale = out->v_scale; a.qdk = out->q_dot_kmean;
+  a.k_mean = out->k_mean; a.v8 = out->v; a.v_scale = out->v_scale; a.qdk = out->q_dot_kmean;
   a.kv_limit = a.Nk;
 
   const dim3 gridA(plan.splits, a.B * a.Hkv);
@@ -227,17 +227,21 @@ sage_status run_quantize(const sage_tensor* q, const sage_tensor* k, const sage_
   if (q->D == 128) {
     if (fp16) {
       kmean_vamax_partial_kernel<__half, 128><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      kv_stats_kernel<128><<<a.B * a.Hkv, 128, 0, stream>>>(a);
       quant_blocks_kernel<__half, 128><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
     } else {
       kmean_vamax_partial_kernel<__nv_bfloat16, 128><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      kv_stats_kernel<128><<<a.B * a.Hkv, 128, 0, stream>>>(a);
       quant_blocks_kernel<__nv_bfloat16, 128><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
     }
   } else {
     if (fp16) {
       kmean_vamax_partial_kernel<__half, 64><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      kv_stats_kernel<64><<<a.B * a.Hkv, 64, 0, stream>>>(a);
       quant_blocks_kernel<__half, 64><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
     } else {
       kmean_vamax_partial_kernel<__nv_bfloat16, 64><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      kv_stats_kernel<64><<<a.B * a.Hkv, 64, 0, stream>>>(a);
       quant_blocks_kernel<__nv_bfloat16, 64><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
     }
   }
@@ -594,7 +598,7 @@ sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage
   z.k = reinterpret_cast<int8_t*>(w + f.k8);
   z.k_scale = reinterpret_cast<float*>(w + f.ks);
   z.k_mean = reinterpret_cast<float*>(w + f.km);
-  z.v_t = reinterpret_cast<uint8_t*>(w + f.v8);
+  z.v = reinterpret_cast<uint8_t*>(w + f.v8);
   z.v_scale = reinterpret_cast<float*>(w + f.vs);
   z.q_dot_kmean = return_lse ? reinterpret_cast<float*>(w + f.qdk) : nullptr;
   z.B = q->B; z.Hq = q->H; z.Hkv = k->H; z.Nq = q->N; z.Nk = k->N; z.D = q->D;
@@ -656,8 +660,8 @@ sage_status sage_debug_pv_fp32(const sage_qkv_i8f8* z, const uint8_t* p, int64_t
     return SAGE_ERR_INVALID_ARG;
   CUtensorMap tq, tk, tv;
   if (!make_qkv_tmaps(z, &tq, &tk, &tv)) return SAGE_ERR_CUDA;
-  const int vrow = (int)((b * z->Hkv + h_kv) * z->D);
-  const int vcol = (int)(kblk * 128);
+  const int vrow = (int)((b * z->Hkv + h_kv) * pad128(z->Nk) + kblk * 128);
+  const int vcol = 0;
   if (z->D == 128) {
     const size_t smem = 1024 + AttnLayout<128>::P_BYTES + AttnLayout<128>::V_BYTES + 64;
     if (!ensure_smem(debug_pv_kernel<128>, smem, &g_smem_dbg_pv)) return SAGE_ERR_CUDA;

@@ -211,6 +211,8 @@ __host__ __device__ constexpr uint32_t instr_desc(uint32_t dfmt, uint32_t afmt, 
   return (dfmt << 4) | (afmt << 7) | (bfmt << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 constexpr uint32_t kDS32 = 2, kDF32 = 1;
+// Bit 16: B operand MN-major (valid for E4M3/E5M2/INT8/F16/BF16/TF32 sources).
+constexpr uint32_t kBMajorMN = 1u << 16;
 constexpr uint32_t kS8 = 1;     // kind::i8 signed operand
 constexpr uint32_t kE4M3 = 0;   // kind::f8f6f4 operand
 

@@ -25,7 +25,7 @@ def qkv_from_oracle(S, oz, device="cuda", with_qdk=True):
     return S.QuantizedQKV(
         q=t(oz["q"], torch.int8), q_scale=t(oz["q_scale"], torch.float32),
         k=t(oz["k"], torch.int8), k_scale=t(oz["k_scale"], torch.float32),
-        k_mean=t(oz["k_mean"], torch.float32), v_t=t(oz["v_t"], torch.uint8),
+        k_mean=t(oz["k_mean"], torch.float32), v=t(np.swapaxes(oz["v_t"], -1, -2), torch.uint8),
         v_scale=t(oz["v_scale"], torch.float32), q_dot_kmean=qdk,
         B=oz["B"], Hq=oz["Hq"], Hkv=oz["Hkv"], Nq=oz["Nq"], Nk=oz["Nk"], D=oz["D"])
 

@@ -25,7 +25,7 @@ def _compare(gz, oz, hq_sel=None, hkv_sel=None):
     np.testing.assert_array_equal(c(gz.k_mean)[:, hkv_sel], oz["k_mean"], err_msg="k mean")
     np.testing.assert_array_equal(c(gz.k)[:, hkv_sel], oz["k"], err_msg="k codes")
     np.testing.assert_array_equal(c(gz.k_scale)[:, hkv_sel], oz["k_scale"], err_msg="k scales")
-    np.testing.assert_array_equal(c(gz.v_t)[:, hkv_sel], oz["v_t"], err_msg="v codes")
+    np.testing.assert_array_equal(c(gz.v)[:, hkv_sel], np.swapaxes(oz["v_t"], -1, -2), err_msg="v codes")
     np.testing.assert_array_equal(c(gz.v_scale)[:, hkv_sel], oz["v_scale"], err_msg="v scales")
     if gz.q_dot_kmean is not None:
         g = c(gz.q_dot_kmean)[:, hq_sel].astype(np.float64)
@@ -79,6 +79,6 @@ def test_quantize_full_size_sampled_heads(S, w):
         oz = O.quantize_qkv_i8f8(q[b:b + 1, hq], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1])
         sub = lambda t: t[b:b + 1]  # noqa: E731
         gsub = S.QuantizedQKV(sub(gz.q), sub(gz.q_scale), sub(gz.k), sub(gz.k_scale),
-                              sub(gz.k_mean), sub(gz.v_t), sub(gz.v_scale), sub(gz.q_dot_kmean),
+                              sub(gz.k_mean), sub(gz.v), sub(gz.v_scale), sub(gz.q_dot_kmean),
                               1, w.Hq, w.Hkv, w.N, w.N, w.D)
         _compare(gsub, oz, hq_sel=hq, hkv_sel=[g])

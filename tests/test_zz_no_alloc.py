@@ -20,7 +20,7 @@ from gpu_util import lib
 
 pytestmark = pytest.mark.gpu
 
-FIELDS = ("q", "q_scale", "k", "k_scale", "k_mean", "v_t", "v_scale", "q_dot_kmean")
+FIELDS = ("q", "q_scale", "k", "k_scale", "k_mean", "v", "v_scale", "q_dot_kmean")
 
 
 def _call_noalloc(S, q, k, v, out):
