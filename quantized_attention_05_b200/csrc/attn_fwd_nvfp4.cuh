@@ -5,20 +5,26 @@
 // microscaling for Q/K and V).
 //
 // One CTA owns one 128-row Q tile of one (batch, Q head):
-//   warp 4   producer: TMA for the packed Q, K and V^T tiles, a bulk copy
+//   warp 8   producer: TMA for the packed Q, K and V^T tiles, a bulk copy
 //            of the tile's qk_correction row, and the scale factors staged
 //            in shared memory in the layout tcgen05.cp expects (for every
 //            64-element K block a 512-byte block: row r's four scale
 //            factors as one 32-bit word at 16*(r%32) + 4*(r/32));
-//   warp 5   MMA issuer: tcgen05.cp of the scale factors into TMEM and
+//   warp 9   MMA issuer: tcgen05.cp of the scale factors into TMEM and
 //            tcgen05.mma kind::mxf4nvf4 with 16-element E4M3 block scales,
 //            S = Q K^T into a double-buffered TMEM accumulator and
 //            O += P V into TMEM, both fp32;
-//   warps 0-3  softmax, one thread per row: scores S + qk_correction,
-//            masking, exact online softmax with exp2, P' = 2688 * p
+//   warps 0-7  softmax, two threads per row: warps q and q+4 share the
+//            TMEM lane quarter q and take keys 0-63 and 64-127 of each
+//            tile (four 16-key vectors each).  Per tile: scores S +
+//            qk_correction, masking, the row max from the two partial maxima
+//            (exchanged through shared memory on an mbarrier per warp pair
+//            and tile parity, so the wait is bounded like every other),
+//            exact online softmax with exp2, P' = 2688 * p
 //            quantised per 16 keys to E2M1 with an E4M3 scale (written in the
-//            64-byte-swizzled K-major layout of the MMA), O rescaled in TMEM
-//            when the running max moves, epilogue O / l and LSE.
+//            64-byte-swizzled K-major layout of the MMA), each half of O's
+//            columns rescaled by its own thread when the running max moves;
+//            epilogue O / l (the two partial sums added once) and LSE.
 // TMEM: S 2 x 128 columns, O D columns, scale factors 32 columns.
 #pragma once
 
@@ -27,7 +33,8 @@
 
 namespace sage {
 
-constexpr int NV_THREADS = 192;
+constexpr int NV_THREADS = 320;
+constexpr int NV_PRODUCER_WARP = 8, NV_MMA_WARP = 9;
 constexpr int NV_STAGES = 3;
 constexpr float LOG2_2688 = 11.392317422778761f;   // log2(448 * 6)
 
@@ -68,10 +75,14 @@ struct NvLayout {
   static constexpr int OFF_PSF = OFF_VSF + NV_STAGES * 2 * SF_BLK;
   static constexpr int OFF_CORR = OFF_PSF + 2 * 2 * SF_BLK;
   static constexpr int OFF_BAR = OFF_CORR + NV_STAGES * 512;
-  // q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2], o_ready[2], mma_done
-  static constexpr int NBAR = 1 + 2 * NV_STAGES + 8 + 1;
+  // q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2], o_ready[2], mma_done,
+  // pmax_full[quarter][tile parity]
+  static constexpr int NBAR = 1 + 2 * NV_STAGES + 8 + 1 + 8;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
-  static constexpr int OFF_NLIST = (OFF_TMEM + 16 + 15) / 16 * 16;
+  // partial row maxima [tile parity][half][row], partial row sums [half][row]
+  static constexpr int OFF_PMAX = (OFF_TMEM + 16 + 15) / 16 * 16;
+  static constexpr int OFF_PSUM = OFF_PMAX + 2 * 2 * 128 * 4;
+  static constexpr int OFF_NLIST = OFF_PSUM + 2 * 128 * 4;
   static constexpr int OFF_LIST = OFF_NLIST + 16;
   static size_t bytes(int nkt) { return 1024 + OFF_LIST + (size_t)nkt * 4; }
   // TMEM columns
@@ -167,7 +178,10 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
   uint64_t* p_full = s_free + 2;              // [P buffer]
   uint64_t* o_ready = p_full + 2;
   uint64_t* mma_done = o_ready + 2;
+  uint64_t* pmax_full = mma_done + 1;         // [quarter * 2 + tile parity]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
+  float* s_pmax = reinterpret_cast<float*>(smem + L::OFF_PMAX);
+  float* s_psum = reinterpret_cast<float*>(smem + L::OFF_PSUM);
   int* s_nlist = reinterpret_cast<int*>(smem + L::OFF_NLIST);
   uint32_t* s_list = reinterpret_cast<uint32_t*>(smem + L::OFF_LIST);
 
@@ -221,16 +235,17 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&s_free[i], 256);
+      mbar_init(&p_full[i], 256);
       mbar_init(&o_ready[i], 1);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&pmax_full[i], 64);
     fence_mbar_init();
-  } else if (warp == 5) {
+  } else if (warp == NV_MMA_WARP) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
-  } else if (warp == 4 && lane == 0) {
+  } else if (warp == NV_PRODUCER_WARP && lane == 0) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
@@ -241,7 +256,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const int ntile = s_nlist[0];
 
-  if (warp == 4) {
+  if (warp == NV_PRODUCER_WARP) {
     // ---------------------------------------------------------- producer
     stage_sf<D / 16>(sQsf, a.q_sf + ((int64_t)bhq * a.Nqp + qt * 128) * (D / 16), D / 16, 128, lane);
     fence_proxy_async_smem();
@@ -274,7 +289,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == NV_MMA_WARP) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t ID_QK = nv_idesc(128, 128);
@@ -328,9 +343,11 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- softmax
-    const int rt = threadIdx.x;
+    const int half = warp >> 2;               // keys [64*half, 64*half + 64) of a tile
+    const int quarter = warp & 3;
+    const int rt = quarter * 32 + lane;
     const int row = row_lo + rt;
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t tO = tmem + lane_base + L::T_O;
     const float c = a.c0;
     const uint64_t c2 = f2_pack(c, c);
@@ -346,51 +363,58 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[buf], (n >> 1) & 1, SITE_S_FULL));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[128];
-      const uint32_t tS = tmem + lane_base + L::T_S + buf * 128;
+      uint32_t sr[64];
+      const uint32_t tS = tmem + lane_base + L::T_S + buf * 128 + half * 64;
       SAGE_TMEM_LD32(tS + 0, (sr + 0));
       SAGE_TMEM_LD32(tS + 32, (sr + 32));
-      SAGE_TMEM_LD32(tS + 64, (sr + 64));
-      SAGE_TMEM_LD32(tS + 96, (sr + 96));
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&s_free[buf]);
       // the tile's correction row arrived with its K/V (bulk copy on kv_full)
       ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[st], (idx / NV_STAGES) & 1, SITE_KV_FULL));
       if (!ok) break;
-      const float* corr = sCorr + st * 128;
+      const float* corr = sCorr + st * 128 + half * 64;
 #pragma unroll
-      for (int j = 0; j < 128; j += 4) {
+      for (int j = 0; j < 64; j += 4) {
         const float4 cv = *reinterpret_cast<const float4*>(corr + j);
         sr[j] = __float_as_uint(__uint_as_float(sr[j]) + cv.x);
         sr[j + 1] = __float_as_uint(__uint_as_float(sr[j + 1]) + cv.y);
         sr[j + 2] = __float_as_uint(__uint_as_float(sr[j + 2]) + cv.z);
         sr[j + 3] = __float_as_uint(__uint_as_float(sr[j + 3]) + cv.w);
       }
-      uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
+      uint32_t vis[2] = {~0u, ~0u};
       if (need) {
-        const int key0 = kt * 128;
-        int jmax = min(127, a.L - 1 - key0);
+        const int key0 = kt * 128 + half * 64;
+        int jmax = min(63, a.L - 1 - key0);
         if (a.causal) jmax = min(jmax, row + a.causal_off - key0);
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < 2; ++w) {
           const int hi = jmax - 32 * w;
           vis[w] = hi >= 31 ? ~0u : (hi < 0 ? 0u : ((2u << hi) - 1u));
         }
 #pragma unroll
-        for (int j = 0; j < 128; ++j)
+        for (int j = 0; j < 64; ++j)
           if (!((vis[j >> 5] >> (j & 31)) & 1u)) sr[j] = __float_as_uint(-INFINITY);
       }
       float m0 = __uint_as_float(sr[0]), m1 = __uint_as_float(sr[1]);
       float m2 = __uint_as_float(sr[2]), m3 = __uint_as_float(sr[3]);
 #pragma unroll
-      for (int j = 4; j < 128; j += 8) {
+      for (int j = 4; j < 64; j += 8) {
         m0 = max3f(m0, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
         m1 = max3f(m1, __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
         m2 = max3f(m2, __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
         m3 = max3f(m3, __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
       }
-      const float mx = max3f(m0, m1, fmaxf(m2, m3));
+      // row max of the tile: this thread's 64 keys and its partner's (the
+      // slot of tile n is rewritten at tile n+2, after the partner has
+      // passed tile n+1's exchange, hence after it read this one)
+      float* pm = s_pmax + (buf * 2) * 128;
+      pm[half * 128 + rt] = max3f(m0, m1, fmaxf(m2, m3));
+      mbar_arrive(&pmax_full[quarter * 2 + buf]);
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&pmax_full[quarter * 2 + buf], (n >> 1) & 1, SITE_ROW_MAX));
+      if (!ok) break;
+      const float mx = fmaxf(pm[rt], pm[128 + rt]);
       const float mt = mx == -INFINITY ? -INFINITY : mx * c;
       const float m_new = fmaxf(m_ref, mt);
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
@@ -405,11 +429,11 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       }
       // P' = 2688 * p per 16-key vector: E4M3 scale, E2M1 codes
       uint8_t* prow = sP + buf * L::P_BYTES + rt * 64;
-      uint8_t* psf = sPsf + buf * 2 * L::SF_BLK + 16 * (rt & 31) + 4 * (rt >> 5);
+      uint8_t* psf = sPsf + buf * 2 * L::SF_BLK + half * L::SF_BLK + 16 * (rt & 31) + 4 * (rt >> 5);
       uint64_t acc = f2_pack(0.f, 0.f);
-      uint32_t sfw[2] = {0u, 0u};
+      uint32_t sfw = 0u;
 #pragma unroll
-      for (int vv = 0; vv < 8; ++vv) {
+      for (int vv = 0; vv < 4; ++vv) {
         float pv[16];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -431,13 +455,13 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
         }
         uint32_t w0, w1;
         const uint32_t sf = nvfp4_vector(pv, &w0, &w1);
-        sfw[vv >> 2] |= sf << (8 * (vv & 3));
-        // 16-byte chunk vv/2 of the row (64-byte swizzle: chunk ^ ((row >> 1) & 3))
-        uint8_t* dst = prow + ((((vv >> 1) ^ ((rt >> 1) & 3))) << 4) + (vv & 1) * 8;
+        sfw |= sf << (8 * vv);
+        // 16-byte chunk (4*half + vv)/2 of the row (64-byte swizzle: chunk ^ ((row >> 1) & 3))
+        const int v16 = 4 * half + vv;
+        uint8_t* dst = prow + ((((v16 >> 1) ^ ((rt >> 1) & 3))) << 4) + (v16 & 1) * 8;
         *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
       }
-      *reinterpret_cast<uint32_t*>(psf) = sfw[0];
-      *reinterpret_cast<uint32_t*>(psf + L::SF_BLK) = sfw[1];
+      *reinterpret_cast<uint32_t*>(psf) = sfw;
       if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         const uint32_t pb = (n - 1) & 1u;
         ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[pb], ((n - 1) >> 1) & 1, SITE_O_READY));
@@ -445,7 +469,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
         tc_fence_after();
         const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-        for (int cb = 0; cb < D; cb += 32) {
+        for (int cb = half * (D / 2); cb < (half + 1) * (D / 2); cb += 32) {
           uint32_t o[32];
           SAGE_TMEM_LD32(tO + cb, o);
           tmem_wait_ld();
@@ -474,15 +498,18 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[pb], ((n - 1) >> 1) & 1, SITE_O_READY));
       tc_fence_after();
     }
+    // the row sum is the two halves' partial sums, added in one order
+    s_psum[half * 128 + rt] = l;
+    __shared__ float s_one[D];
+    if (threadIdx.x < D) s_one[threadIdx.x] = 1.f;
+    asm volatile("bar.sync 1, 256;" ::: "memory");   // the softmax warps only
+    l = s_psum[rt] + s_psum[128 + rt];
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     const bool live = ok && n > 0;
     char* obase = reinterpret_cast<char*>(a.out) +
                   ((int64_t)b * a.out_sb + (int64_t)h * a.out_sh + (int64_t)row * a.out_sn) * 2;
-    __shared__ float s_one[D];
-    if (threadIdx.x < D) s_one[threadIdx.x] = 1.f;
-    asm volatile("bar.sync 1, 128;" ::: "memory");   // the softmax warps only
 #pragma unroll
-    for (int cb = 0; cb < D; cb += 32) {
+    for (int cb = half * (D / 2); cb < (half + 1) * (D / 2); cb += 32) {
       uint32_t o[32];
       if (live) {
         SAGE_TMEM_LD32(tO + cb, o);
@@ -500,7 +527,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
                                             s_one, inv_l);
       }
     }
-    if (a.return_lse && row < a.Nq) {
+    if (half == 0 && a.return_lse && row < a.Nq) {
       float v = -INFINITY;
       if (l > 0.f)
         v = (m_ref + log2f(l) - LOG2_2688) * LN2_F + a.sm_scale * a.qdk[(int64_t)bhq * a.Nq + row];
@@ -510,7 +537,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == NV_MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -29,6 +29,7 @@ enum WaitSite : uint32_t {
   SITE_DEBUG = 8,
   SITE_MMA_DONE = 9,
   SITE_MMA_STALL = 10,
+  SITE_ROW_MAX = 11,
 };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
