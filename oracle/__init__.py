@@ -14,6 +14,8 @@ quantize   the quantisation stage (smooth_k, per-block INT8 Q/K, per-channel
            FP8 V; NVFP4 with per-block Q mean and qk_correction).
 attention  exact fp64 attention and the tile-ordered online-softmax
            attention over the quantised codes (INT8-QK/FP8-PV and NVFP4).
+varlen     packed variable-length batches (cu_seqlens): every sequence its
+           own dense problem.
 
 Every function states the passage of the SageAttention / FlashInfer pages it
 follows.  Where the pages are silent the plainest reading is taken; those
@@ -31,3 +33,4 @@ from .quantize import (BLOCK, fp4_vector_quant, fp8_channel_quant, int8_block_qu
                        quantize_qkv_i8f8, quantize_qkv_nvfp4)
 from .attention import (attention_i8f8, attention_nvfp4, cosine, default_sm_scale,  # noqa: F401
                         exact_attention, qk_int32_tile)
+from .varlen import attention_varlen_i8f8, block_diagonal_mask, check_cu_seqlens  # noqa: F401

@@ -138,3 +138,24 @@ def test_nvfp4_full_size_sampled(S):
         _compare_quant(gsub, oz)
         ref = O.attention_nvfp4(oz, rows=rows)
         assert_attention_close(out[:, h:h + 1], lse[:, h:h + 1], ref, rows=rows, what=f"nvfp4 h{h}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_nvfp4_without_lse_matches_with_lse(S, causal):
+    """return_lse=False (no LSE, no q.kmean needed) gives the same output as
+    the LSE run, bit for bit, and needs no q_dot_kmean array."""
+    w = W.NVFP4.scaled(B=1, Hq=2, Hkv=2, N=384, D=128, unpadded_k_len=350, seed=13)
+    q, k, v = W.make_qkv(w)
+    z = S.sage_quantize_qkv_nvfp4(q.cuda(), k.cuda(), v.cuda(), per_block_mean=True,
+                                  unpadded_k_len=w.unpadded_k_len)
+    out_lse, _ = S.sage_attn_fwd_nvfp4(z, causal=causal, return_lse=True)
+    z.q_dot_kmean = None
+    out = S.sage_attn_fwd_nvfp4(z, causal=causal, return_lse=False)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out_lse)
+    oz = O.quantize_qkv_nvfp4(q, k, v, per_block_mean=True, unpadded_k_len=w.unpadded_k_len)
+    ref = O.attention_nvfp4(oz, causal=causal)
+    o = out.float().cpu().numpy()
+    assert O.cosine(o, ref["out"]) >= 0.9995
+    if not causal:
+        assert np.abs(o - ref["out"]).max() <= 2e-2
