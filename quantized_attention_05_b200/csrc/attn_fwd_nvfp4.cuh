@@ -152,6 +152,23 @@ __device__ __forceinline__ void stage_sf(uint8_t* dst, const uint8_t* src, int64
   }
 }
 
+// P' vector quantisation when the vector's amax is already known: scale
+// factor sf = E4M3(amax / 6), codes E2M1(x * (1 / value(sf))) with the
+// correctly rounded reciprocal taken from `inv_tab` (0 for a zero scale, so
+// the codes of an all-zero vector are 0).
+__device__ __forceinline__ uint32_t nvfp4_vector_amax(const float* x, float amax,
+                                                      const float* inv_tab, uint32_t* w0,
+                                                      uint32_t* w1) {
+  const uint32_t sf = e4m3_code(__fdiv_rn(amax, 6.f));
+  const float inv = inv_tab[sf];
+  float y[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(x[i], inv);
+  *w0 = e2m1x8(y);
+  *w1 = e2m1x8(y + 8);
+  return sf;
+}
+
 template <int D>
 __global__ void __launch_bounds__(NV_THREADS, 1)
     attn_fwd_nvfp4_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -186,6 +203,11 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
   uint32_t* s_list = reinterpret_cast<uint32_t*>(smem + L::OFF_LIST);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float s_inv[256];   // 1 / value(E4M3 code), 0 for code 0
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+    const float v = i < 128 ? e4m3_value((uint32_t)i) : 0.f;
+    s_inv[i] = v > 0.f ? __frcp_rn(v) : 0.f;
+  }
   // work: (b, h, qt); causal -> longest rows first
   int b, h, qt;
   {
@@ -396,15 +418,18 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
         for (int j = 0; j < 64; ++j)
           if (!((vis[j >> 5] >> (j & 31)) & 1u)) sr[j] = __float_as_uint(-INFINITY);
       }
-      float m0 = __uint_as_float(sr[0]), m1 = __uint_as_float(sr[1]);
-      float m2 = __uint_as_float(sr[2]), m3 = __uint_as_float(sr[3]);
+      // maxima of the four 16-key vectors (they also give each vector's
+      // P' amax: p is increasing in the score), then of the thread's 64 keys
+      float vmax[4];
 #pragma unroll
-      for (int j = 4; j < 64; j += 8) {
-        m0 = max3f(m0, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
-        m1 = max3f(m1, __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
-        m2 = max3f(m2, __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
-        m3 = max3f(m3, __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
+      for (int vv = 0; vv < 4; ++vv) {
+        const float* x = reinterpret_cast<const float*>(sr) + 16 * vv;
+        const float t0 = max3f(x[0], x[1], x[2]), t1 = max3f(x[3], x[4], x[5]);
+        const float t2 = max3f(x[6], x[7], x[8]), t3 = max3f(x[9], x[10], x[11]);
+        const float t4 = max3f(x[12], x[13], x[14]);
+        vmax[vv] = max3f(max3f(t0, t1, t2), max3f(t3, t4, x[15]), -INFINITY);
       }
+      const float m0 = vmax[0], m1 = vmax[1], m2 = vmax[2], m3 = vmax[3];
       // row max of the tile: this thread's 64 keys and its partner's (the
       // slot of tile n is rewritten at tile n+2, after the partner has
       // passed tile n+1's exchange, hence after it read this one)
@@ -453,8 +478,11 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
           }
           acc = f2_add(acc, f2_pack(pv[2 * i], pv[2 * i + 1]));
         }
+        // amax of the vector: the p of its largest score (same fma and ex2
+        // as the element itself; 0 when every key of the vector is hidden)
+        const float pmax = ex2_approx(fmaf(vmax[vv], c, bias));
         uint32_t w0, w1;
-        const uint32_t sf = nvfp4_vector(pv, &w0, &w1);
+        const uint32_t sf = nvfp4_vector_amax(pv, pmax, s_inv, &w0, &w1);
         sfw |= sf << (8 * vv);
         // 16-byte chunk (4*half + vv)/2 of the row (64-byte swizzle: chunk ^ ((row >> 1) & 3))
         const int v16 = 4 * half + vv;

@@ -300,17 +300,20 @@ __global__ void __launch_bounds__(256) nv_corr_kernel(NvQuantArgs a) {
   float* s_qm = s_kt + D * 128;                        // [64][D]
   const int kt = blockIdx.x, bg = blockIdx.y;
   const int b = bg / a.Hkv, g = bg % a.Hkv;
-  // Ks = fp32(K - kmean) for keys < L, 0 beyond
+  // Ks = fp32(K - kmean) for keys < L, 0 beyond; consecutive threads take
+  // consecutive keys, so the transposed shared-memory stores are
+  // conflict-free
   for (int idx = threadIdx.x; idx < 128 * (D / 8); idx += blockDim.x) {
-    const int key = idx / (D / 8), cg = idx % (D / 8);
+    const int key = idx % 128, cg = idx / 128;
     const int n = kt * 128 + key;
     float f[8];
     if (n < a.L) {
       unpack8<T>(ldg16(reinterpret_cast<const char*>(a.k) +
                        (b * a.k_sb + g * a.k_sh + (int64_t)n * a.k_sn + cg * 8) * (int64_t)sizeof(T)),
                  f);
+      const float* km = a.k_mean + (int64_t)bg * D + cg * 8;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) f[i] = __fsub_rn(f[i], a.k_mean[(int64_t)bg * D + cg * 8 + i]);
+      for (int i = 0; i < 8; ++i) f[i] = __fsub_rn(f[i], __ldg(km + i));
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) f[i] = 0.f;
