@@ -28,6 +28,7 @@
 #include <cuda_fp16.h>
 
 #include "sage_ptx.cuh"
+#include "seqs.cuh"
 
 namespace sage {
 
@@ -61,7 +62,41 @@ struct AttnArgs {
   int causal, return_lse, causal_off;
   float c0;                        // sm_scale * log2(e)
   float sm_scale;
+  // B sequences; `seqs` (device table, see seqs.cuh) for a packed
+  // variable-length call, null for a dense one; max_nqp bounds the Q-tile
+  // pairs of any sequence (the grid is sized by it).
+  const int* seqs;
+  int max_nqp;
 };
+
+// The sequence a CTA works on: its sizes and where its head's rows start in
+// the quantised arrays, the scales, q.kmean / LSE and the output.
+struct CtaSeq {
+  int Nq, Nk, nqt, nkt, Nqp, Nkp, causal_off;
+  int64_t qrow0, krow0;   // q8 row, k8/v8 row of token 0
+  int64_t qs0, ks0;       // q_scale, k_scale index of block 0
+  int64_t tok0;           // q_dot_kmean / lse index of token 0
+  int64_t out0;           // out element offset of token 0
+};
+
+__device__ __forceinline__ CtaSeq cta_seq(const AttnArgs& a, int s, int h, int g) {
+  const SeqView v = seq_view(a.seqs, s, a.Nq, a.Nk);
+  CtaSeq c;
+  c.Nq = v.nq;
+  c.Nk = v.nk;
+  c.nqt = (v.nq + ATT_BM - 1) / ATT_BM;
+  c.nkt = (v.nk + ATT_BN - 1) / ATT_BN;
+  c.Nqp = c.nqt * ATT_BM;
+  c.Nkp = c.nkt * ATT_BN;
+  c.causal_off = v.nk - v.nq;
+  c.qrow0 = (int64_t)a.Hq * v.cqp + (int64_t)h * c.Nqp;
+  c.krow0 = (int64_t)a.Hkv * v.ckp + (int64_t)g * c.Nkp;
+  c.qs0 = (int64_t)a.Hq * (v.cqp / ATT_BM) + (int64_t)h * c.nqt;
+  c.ks0 = (int64_t)a.Hkv * (v.ckp / ATT_BN) + (int64_t)g * c.nkt;
+  c.tok0 = (int64_t)a.Hq * v.cq + (int64_t)h * v.nq;
+  c.out0 = (a.seqs ? v.cq * a.out_sn : (int64_t)s * a.out_sb) + (int64_t)h * a.out_sh;
+  return c;
+}
 
 template <int D>
 struct AttnLayout {
@@ -117,15 +152,15 @@ __device__ __forceinline__ void store_p_row(uint8_t* tile, int r, const uint32_t
 // Flags of key tile kt for Q tile qt (0 if nothing in it is visible):
 // bit 0 visible, bit 2 needs per-element masking, bit 4 reads the boolean
 // mask; shifted left by `wg` (0 or 1).
-__device__ __forceinline__ uint32_t tile_flags(const AttnArgs& a, int b, int h, int qt, int wg,
-                                               int kt) {
+__device__ __forceinline__ uint32_t tile_flags(const AttnArgs& a, const CtaSeq& cs, int b, int h,
+                                               int qt, int wg, int kt) {
   const int row_lo = qt * ATT_BM;
-  if (row_lo >= a.Nq) return 0;
-  const int row_hi = min(row_lo + ATT_BM - 1, a.Nq - 1);
+  if (row_lo >= cs.Nq) return 0;
+  const int row_hi = min(row_lo + ATT_BM - 1, cs.Nq - 1);
   const int key_lo = kt * ATT_BN, key_hi = key_lo + ATT_BN - 1;
-  if (key_lo >= a.Nk) return 0;
-  if (a.causal && key_lo > row_hi + a.causal_off) return 0;
-  bool need = key_hi >= a.Nk || (a.causal && key_hi > row_lo + a.causal_off);
+  if (key_lo >= cs.Nk) return 0;
+  if (a.causal && key_lo > row_hi + cs.causal_off) return 0;
+  bool need = key_hi >= cs.Nk || (a.causal && key_hi > row_lo + cs.causal_off);
   bool part = false;
   if (a.tile_class) {
     const int bm = a.m_bcast_b ? 0 : b, hm = a.m_bcast_h ? 0 : h;
@@ -139,9 +174,9 @@ __device__ __forceinline__ uint32_t tile_flags(const AttnArgs& a, int b, int h, 
 }
 
 __device__ __forceinline__ void decode_work(const AttnArgs& a, int bid, int& qp, int& b, int& h) {
-  if (a.causal) {  // longest rows first
+  if (a.causal || a.seqs) {  // longest rows first
     const int per = a.B * a.Hq;
-    qp = a.nqp - 1 - bid / per;
+    qp = a.max_nqp - 1 - bid / per;
     const int r = bid % per;
     b = r / a.Hq;
     h = r % a.Hq;
@@ -186,11 +221,12 @@ __device__ __forceinline__ void store_out_chunk(const AttnArgs& a, OutT* orow, i
 
 // Visibility of the 128 keys of tile kt for one row (bit j of vis[j / 32]):
 // key length, causal limit and, for mixed mask tiles, the boolean mask.
-__device__ __forceinline__ void tile_visibility(const AttnArgs& a, int kt, int row, bool part,
-                                                const uint8_t* mrow, uint32_t* vis) {
+__device__ __forceinline__ void tile_visibility(const AttnArgs& a, const CtaSeq& cs, int kt,
+                                                int row, bool part, const uint8_t* mrow,
+                                                uint32_t* vis) {
   const int key0 = kt * ATT_BN;
-  int jmax = min(ATT_BN - 1, a.Nk - 1 - key0);
-  if (a.causal) jmax = min(jmax, row + a.causal_off - key0);
+  int jmax = min(ATT_BN - 1, cs.Nk - 1 - key0);
+  if (a.causal) jmax = min(jmax, row + cs.causal_off - key0);
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     const int hi = jmax - 32 * w;  // keep bits 0..hi
@@ -198,7 +234,7 @@ __device__ __forceinline__ void tile_visibility(const AttnArgs& a, int kt, int r
   }
   if (part && mrow) {
     const uint8_t* mk = mrow + key0;
-    if (a.mask_vec16 && key0 + ATT_BN <= a.Nk) {
+    if (a.mask_vec16 && key0 + ATT_BN <= cs.Nk) {
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const uint4 mv = __ldg(reinterpret_cast<const uint4*>(mk) + q);
@@ -211,7 +247,7 @@ __device__ __forceinline__ void tile_visibility(const AttnArgs& a, int kt, int r
       }
     } else {
       for (int j = 0; j < ATT_BN; ++j)
-        if (key0 + j < a.Nk && mk[j] == 0) vis[j >> 5] &= ~(1u << (j & 31));
+        if (key0 + j < cs.Nk && mk[j] == 0) vis[j >> 5] &= ~(1u << (j & 31));
     }
   }
 }
@@ -301,20 +337,24 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   int qp, b, h;
   decode_work(a, blockIdx.x, qp, b, h);
   const int g = h / a.G;
-  const int bhq = b * a.Hq + h, bhk = b * a.Hkv + g;
+  const int bhk = b * a.Hkv + g;
+  const CtaSeq cs = cta_seq(a, b, h, g);
   const int qt0 = 2 * qp;
-  const bool has1 = qt0 + 1 < a.nqt;
+  // a variable-length call sizes the grid by its longest sequence: CTAs
+  // beyond this sequence's tiles leave before any setup
+  if (qt0 >= cs.nqt) return;
+  const bool has1 = qt0 + 1 < cs.nqt;
 
   // ------------------------------------------------------------ setup
   if (warp == 0) {
     int count = 0;
     uint32_t orf = 0;
-    for (int base = 0; base < a.nkt; base += 32) {
+    for (int base = 0; base < cs.nkt; base += 32) {
       const int kt = base + lane;
       uint32_t f = 0;
-      if (kt < a.nkt) {
-        f = tile_flags(a, b, h, qt0, 0, kt);
-        if (has1) f |= tile_flags(a, b, h, qt0 + 1, 1, kt);
+      if (kt < cs.nkt) {
+        f = tile_flags(a, cs, b, h, qt0, 0, kt);
+        if (has1) f |= tile_flags(a, cs, b, h, qt0 + 1, 1, kt);
       }
       const unsigned bal = __ballot_sync(0xffffffffu, (f & 3u) != 0);
       if (f & 3u) s_list[count + __popc(bal & ((1u << lane) - 1u))] = ((uint32_t)kt << 8) | f;
@@ -365,15 +405,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (lane == 0) {
       const bool act0 = orf & 1u, act1 = (orf >> 1) & 1u;
       mbar_arrive_expect_tx(q_full, (uint32_t)((act0 ? L::Q_BYTES : 0) + (act1 ? L::Q_BYTES : 0)));
-      if (act0) tma_load_2d(sQ, &tmQ, q_full, 0, bhq * a.Nqp + qt0 * ATT_BM);
-      if (act1) tma_load_2d(sQ + L::Q_BYTES, &tmQ, q_full, 0, bhq * a.Nqp + (qt0 + 1) * ATT_BM);
+      if (act0) tma_load_2d(sQ, &tmQ, q_full, 0, (int)(cs.qrow0 + qt0 * ATT_BM));
+      if (act1) tma_load_2d(sQ + L::Q_BYTES, &tmQ, q_full, 0, (int)(cs.qrow0 + (qt0 + 1) * ATT_BM));
       for (int idx = 0; idx < ntile; ++idx) {
         const int st = idx % ATT_STAGES, rd = idx / ATT_STAGES;
         if (idx >= ATT_STAGES && !mbar_wait(&kv_empty[st], (rd - 1) & 1, SITE_KV_EMPTY)) break;
         const int kt = (int)(s_list[idx] >> 8);
         mbar_arrive_expect_tx(&kv_full[st], (uint32_t)(L::K_BYTES + L::V_BYTES));
-        tma_load_2d(sK + st * L::K_BYTES, &tmK, &kv_full[st], 0, bhk * a.Nkp + kt * ATT_BN);
-        tma_load_2d(sV + st * L::V_BYTES, &tmV, &kv_full[st], 0, bhk * a.Nkp + kt * ATT_BN);
+        tma_load_2d(sK + st * L::K_BYTES, &tmK, &kv_full[st], 0, (int)(cs.krow0 + kt * ATT_BN));
+        tma_load_2d(sV + st * L::V_BYTES, &tmV, &kv_full[st], 0, (int)(cs.krow0 + kt * ATT_BN));
       }
     }
     __syncwarp();
@@ -470,10 +510,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + (uint32_t)(wg * 256);
     const uint32_t tO = tS + 128;
-    const bool tile_exists = qt < a.nqt;
-    const float cq = tile_exists ? a.q_scale[(int64_t)bhq * a.nqt + qt] * a.c0 : 0.f;
+    const bool tile_exists = qt < cs.nqt;
+    const float cq = tile_exists ? a.q_scale[cs.qs0 + qt] * a.c0 : 0.f;
     const uint8_t* mrow = nullptr;
-    if (a.mask && row < a.Nq) {
+    if (a.mask && row < cs.Nq) {
       const int bm = a.m_bcast_b ? 0 : b, hm = a.m_bcast_h ? 0 : h;
       mrow = a.mask + bm * a.m_sb + hm * a.m_sh + (int64_t)row * a.m_sq;
     }
@@ -494,7 +534,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const int kt = (int)(e >> 8);
       const bool need = (e >> (2 + wg)) & 1u;
       const bool part = (e >> (4 + wg)) & 1u;
-      const float c = cq * a.k_scale[(int64_t)bhk * a.nkt + kt];
+      const float c = cq * a.k_scale[cs.ks0 + kt];
       const uint32_t buf = n & 1u;
       uint8_t* ptile = sP + (wg * 2 + buf) * L::P_BYTES;
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], n & 1, SITE_S_FULL));
@@ -516,7 +556,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       // sr holds 1.5*2^23 + S as float bits; hidden keys -> 0.0 (below every score)
       uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
       if (need) {
-        tile_visibility(a, kt, row, part, mrow, vis);
+        tile_visibility(a, cs, kt, row, part, mrow, vis);
 #pragma unroll
         for (int j = 0; j < 128; ++j)
           if (!((vis[j >> 5] >> (j & 31)) & 1u)) sr[j] = 0u;
@@ -586,8 +626,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (tile_exists) {
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const bool live = ok && n > 0;
-      char* obase = reinterpret_cast<char*>(a.out) +
-                    ((int64_t)b * a.out_sb + (int64_t)h * a.out_sh + (int64_t)row * a.out_sn) * 2;
+      char* obase = reinterpret_cast<char*>(a.out) + (cs.out0 + (int64_t)row * a.out_sn) * 2;
 #pragma unroll
       for (int cb = 0; cb < D; cb += 32) {
         uint32_t o[32];
@@ -598,7 +637,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0u;
         }
-        if (row < a.Nq) {
+        if (row < cs.Nq) {
           if (a.out_fp16)
             store_out_chunk<D, __half>(a, reinterpret_cast<__half*>(obase), cb, o, s_vs, inv_l);
           else
@@ -606,12 +645,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                               s_vs, inv_l);
         }
       }
-      if (a.return_lse && row < a.Nq) {
+      if (a.return_lse && row < cs.Nq) {
         float v = -INFINITY;
         if (l > 0.f)
-          v = (m_ref + log2f(l) - LOG2_448) * LN2_F +
-              a.sm_scale * a.qdk[(int64_t)bhq * a.Nq + row];
-        a.lse[(int64_t)bhq * a.Nq + row] = v;
+          v = (m_ref + log2f(l) - LOG2_448) * LN2_F + a.sm_scale * a.qdk[cs.tok0 + row];
+        a.lse[cs.tok0 + row] = v;
       }
     }
   }

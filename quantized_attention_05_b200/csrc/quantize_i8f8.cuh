@@ -21,6 +21,7 @@
 #include <cuda_fp16.h>
 
 #include "sage_ptx.cuh"
+#include "seqs.cuh"
 
 namespace sage {
 
@@ -48,7 +49,19 @@ struct QuantArgs {
   float* va;                      // [B*Hkv, D] V channel maxima (workspace)
   float* qdk;                     // may be null
   int kv_limit;                   // tokens of K/V used for the mean / codes (Nk)
+  // sequences: B of them; `seqs` (device table, see seqs.cuh) for a packed
+  // variable-length call, null for a dense one.  max_nqt / max_nkt bound
+  // the 128-token blocks of any sequence (the block grid is sized by them).
+  const int* seqs;
+  int max_nqt, max_nkt;
 };
+
+// Element offset of sequence s in an input tensor: packed tokens for a
+// variable-length call, the batch stride for a dense one.
+__device__ __forceinline__ int64_t seq_in_offset(const QuantArgs& a, int64_t tok0, int s,
+                                                 int64_t sn, int64_t sb) {
+  return a.seqs ? tok0 * sn : (int64_t)s * sb;
+}
 
 template <typename T>
 __device__ __forceinline__ float to_f32(T x);
@@ -114,9 +127,10 @@ __global__ void __launch_bounds__(QUANT_THREADS) kmean_vamax_partial_kernel(Quan
   const int split = blockIdx.x;
   const int bh = blockIdx.y;
   const int b = bh / a.Hkv, h = bh % a.Hkv;
+  const SeqView sq = seq_view(a.seqs, b, a.Nq, a.kv_limit);
   const int cg = threadIdx.x % TPR, rs = threadIdx.x / TPR;
   const int n0 = split * a.split_tokens;
-  const int n1 = min(a.kv_limit, n0 + a.split_tokens);
+  const int n1 = min(sq.nk, n0 + a.split_tokens);
 
   DD acc[8];
   float am[8];
@@ -126,9 +140,11 @@ __global__ void __launch_bounds__(QUANT_THREADS) kmean_vamax_partial_kernel(Quan
     am[i] = 0.f;
   }
   const char* kb = reinterpret_cast<const char*>(a.k) +
-                   (b * a.k_sb + h * a.k_sh + cg * 8) * (int64_t)sizeof(T);
+                   (seq_in_offset(a, sq.ck, b, a.k_sn, a.k_sb) + h * a.k_sh + cg * 8) *
+                       (int64_t)sizeof(T);
   const char* vb = reinterpret_cast<const char*>(a.v) +
-                   (b * a.v_sb + h * a.v_sh + cg * 8) * (int64_t)sizeof(T);
+                   (seq_in_offset(a, sq.ck, b, a.v_sn, a.v_sb) + h * a.v_sh + cg * 8) *
+                       (int64_t)sizeof(T);
   for (int n = n0 + rs; n < n1; n += RPP) {
     float f[8];
     if (a.smooth_k) {
@@ -168,6 +184,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) kmean_vamax_partial_kernel(Quan
 template <int D>
 __global__ void __launch_bounds__(D) kv_stats_kernel(QuantArgs a) {
   const int bh = blockIdx.x, c = threadIdx.x;
+  const int nk = seq_view(a.seqs, bh / a.Hkv, a.Nq, a.kv_limit).nk;
   DD s = {0.0, 0.0};
   float m = 0.f;
   for (int sp = 0; sp < a.splits; ++sp) {
@@ -175,7 +192,7 @@ __global__ void __launch_bounds__(D) kv_stats_kernel(QuantArgs a) {
     dd_add(s, DD{a.part_hi[o], a.part_lo[o]});
     m = fmaxf(m, a.part_amax[o]);
   }
-  a.k_mean[(int64_t)bh * D + c] = a.smooth_k ? dd_mean_f32(s, (double)a.kv_limit) : 0.f;
+  a.k_mean[(int64_t)bh * D + c] = a.smooth_k && nk > 0 ? dd_mean_f32(s, (double)nk) : 0.f;
   a.va[(int64_t)bh * D + c] = m;
   a.v_scale[(int64_t)bh * D + c] = __fdiv_rn(m, 448.f);
 }
@@ -210,26 +227,31 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
   __shared__ float s_c[D];      // k_mean (Q with LSE, K) or 448 / V channel max (V)
   __shared__ float s_red[QUANT_THREADS / 32];
 
-  const int nQb = a.B * a.Hq * a.nqt;
-  const int nKb = a.B * a.Hkv * a.nkt;
+  const int nQb = a.B * a.Hq * a.max_nqt;
+  const int nKb = a.B * a.Hkv * a.max_nkt;
   int job = blockIdx.x;
   const int cg = threadIdx.x % TPR, rs = threadIdx.x / TPR;
 
   if (job < nQb) {
     // ---------------- Q block
-    const int bh = job / a.nqt, qt = job % a.nqt;
+    const int bh = job / a.max_nqt, qt = job % a.max_nqt;
     const int b = bh / a.Hq, h = bh % a.Hq;
     const int g = h / a.G;
+    const SeqView sq = seq_view(a.seqs, b, a.Nq, a.kv_limit);
+    const int nqt = (sq.nq + 127) / 128, Nqp = nqt * 128;
+    if (qt >= nqt) return;                  // beyond this sequence (whole CTA)
+    const int64_t row0 = (int64_t)a.Hq * sq.cqp + (int64_t)h * Nqp;   // q8 row of token 0
     if (a.qdk)
       for (int c = threadIdx.x; c < D; c += blockDim.x) s_c[c] = a.k_mean[(int64_t)(b * a.Hkv + g) * D + c];
     const char* base = reinterpret_cast<const char*>(a.q) +
-                       (b * a.q_sb + h * a.q_sh + cg * 8) * (int64_t)sizeof(T);
+                       (seq_in_offset(a, sq.cq, b, a.q_sn, a.q_sb) + h * a.q_sh + cg * 8) *
+                           (int64_t)sizeof(T);
     uint4 raw[ITERS];
     float am = 0.f;
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
       const int n = qt * QB + rs + it * RPP;
-      raw[it] = n < a.Nq ? ldg16(base + (int64_t)n * a.q_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
+      raw[it] = n < sq.nq ? ldg16(base + (int64_t)n * a.q_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
@@ -250,32 +272,38 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
       for (int i = 0; i < 4; ++i) w0 |= (uint32_t)(uint8_t)int8_code(f[i], inv) << (8 * i);
 #pragma unroll
       for (int i = 0; i < 4; ++i) w1 |= (uint32_t)(uint8_t)int8_code(f[4 + i], inv) << (8 * i);
-      *reinterpret_cast<uint2*>(a.q8 + ((int64_t)bh * a.Nqp + n) * D + cg * 8) = make_uint2(w0, w1);
+      *reinterpret_cast<uint2*>(a.q8 + (row0 + n) * D + cg * 8) = make_uint2(w0, w1);
       if (a.qdk) {
         float d = 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) d = fmaf(f[i], s_c[cg * 8 + i], d);
 #pragma unroll
         for (int o = TPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-        if (cg == 0 && n < a.Nq) a.qdk[(int64_t)bh * a.Nq + n] = d;
+        if (cg == 0 && n < sq.nq) a.qdk[(int64_t)a.Hq * sq.cq + (int64_t)h * sq.nq + n] = d;
       }
     }
-    if (threadIdx.x == 0) a.q_scale[(int64_t)bh * a.nqt + qt] = __fdiv_rn(amax, 127.f);
+    if (threadIdx.x == 0)
+      a.q_scale[(int64_t)a.Hq * (sq.cqp / 128) + (int64_t)h * nqt + qt] = __fdiv_rn(amax, 127.f);
     return;
   }
   job -= nQb;
   if (job < nKb) {
     // ---------------- K block: codes of K - kmean
-    const int bh = job / a.nkt, kt = job % a.nkt;
+    const int bh = job / a.max_nkt, kt = job % a.max_nkt;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const SeqView sq = seq_view(a.seqs, b, a.Nq, a.kv_limit);
+    const int nkt = (sq.nk + 127) / 128, Nkp = nkt * 128;
+    if (kt >= nkt) return;                  // beyond this sequence (whole CTA)
+    const int64_t row0 = (int64_t)a.Hkv * sq.ckp + (int64_t)h * Nkp;
     for (int c = threadIdx.x; c < D; c += blockDim.x) s_c[c] = a.k_mean[(int64_t)bh * D + c];
     const char* base = reinterpret_cast<const char*>(a.k) +
-                       (b * a.k_sb + h * a.k_sh + cg * 8) * (int64_t)sizeof(T);
+                       (seq_in_offset(a, sq.ck, b, a.k_sn, a.k_sb) + h * a.k_sh + cg * 8) *
+                           (int64_t)sizeof(T);
     uint4 raw[ITERS];
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
       const int n = kt * QB + rs + it * RPP;
-      raw[it] = n < a.kv_limit ? ldg16(base + (int64_t)n * a.k_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
+      raw[it] = n < sq.nk ? ldg16(base + (int64_t)n * a.k_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
     float km[8];
@@ -287,7 +315,7 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
       const int n = kt * QB + rs + it * RPP;
       float f[8];
       unpack8<T>(raw[it], f);
-      if (n < a.kv_limit) {
+      if (n < sq.nk) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(__fsub_rn(f[i], km[i])));
       }
@@ -300,7 +328,7 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
       float f[8];
       unpack8<T>(raw[it], f);
       uint32_t w0 = 0, w1 = 0;
-      if (n < a.kv_limit) {
+      if (n < sq.nk) {
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           w0 |= (uint32_t)(uint8_t)int8_code(__fsub_rn(f[i], km[i]), inv) << (8 * i);
@@ -308,27 +336,33 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
         for (int i = 0; i < 4; ++i)
           w1 |= (uint32_t)(uint8_t)int8_code(__fsub_rn(f[4 + i], km[4 + i]), inv) << (8 * i);
       }
-      *reinterpret_cast<uint2*>(a.k8 + ((int64_t)bh * a.Nkp + n) * D + cg * 8) = make_uint2(w0, w1);
+      *reinterpret_cast<uint2*>(a.k8 + (row0 + n) * D + cg * 8) = make_uint2(w0, w1);
     }
-    if (threadIdx.x == 0) a.k_scale[(int64_t)bh * a.nkt + kt] = __fdiv_rn(amax, 127.f);
+    if (threadIdx.x == 0)
+      a.k_scale[(int64_t)a.Hkv * (sq.ckp / 128) + (int64_t)h * nkt + kt] = __fdiv_rn(amax, 127.f);
     return;
   }
   job -= nKb;
   {
     // ---------------- V block: per-channel E4M3 codes, [token, channel] order
-    const int bh = job / a.nkt, vt = job % a.nkt;
+    const int bh = job / a.max_nkt, vt = job % a.max_nkt;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const SeqView sq = seq_view(a.seqs, b, a.Nq, a.kv_limit);
+    const int nkt = (sq.nk + 127) / 128, Nkp = nkt * 128;
+    if (vt >= nkt) return;                  // beyond this sequence (whole CTA)
+    const int64_t row0 = (int64_t)a.Hkv * sq.ckp + (int64_t)h * Nkp;
     for (int c = threadIdx.x; c < D; c += blockDim.x) {
       const float m = a.va[(int64_t)bh * D + c];
       s_c[c] = m > 0.f ? __fdiv_rn(448.f, m) : 0.f;
     }
     const char* base = reinterpret_cast<const char*>(a.v) +
-                       (b * a.v_sb + h * a.v_sh + cg * 8) * (int64_t)sizeof(T);
+                       (seq_in_offset(a, sq.ck, b, a.v_sn, a.v_sb) + h * a.v_sh + cg * 8) *
+                           (int64_t)sizeof(T);
     uint4 raw[ITERS];
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
       const int n = vt * QB + rs + it * RPP;
-      raw[it] = n < a.kv_limit ? ldg16(base + (int64_t)n * a.v_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
+      raw[it] = n < sq.nk ? ldg16(base + (int64_t)n * a.v_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
     float inv[8];
@@ -340,13 +374,13 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
       float f[8];
       unpack8<T>(raw[it], f);
       uint32_t w[2] = {0u, 0u};
-      if (n < a.kv_limit) {
+      if (n < sq.nk) {
 #pragma unroll
         for (int i = 0; i < 8; i += 2)
           w[i >> 2] |= (uint32_t)cvt_e4m3x2(__fmul_rn(f[i], inv[i]), __fmul_rn(f[i + 1], inv[i + 1]))
                        << (8 * (i & 3));
       }
-      *reinterpret_cast<uint2*>(a.v8 + ((int64_t)bh * a.Nkp + n) * D + cg * 8) = make_uint2(w[0], w[1]);
+      *reinterpret_cast<uint2*>(a.v8 + (row0 + n) * D + cg * 8) = make_uint2(w[0], w[1]);
     }
   }
 }

@@ -217,6 +217,9 @@ sage_status run_quantize(const sage_tensor* q, const sage_tensor* k, const sage_
   a.q8 = out->q; a.q_scale = out->q_scale; a.k8 = out->k; a.k_scale = out->k_scale;
   a.k_mean = out->k_mean; a.v8 = out->v; a.v_scale = out->v_scale; a.qdk = out->q_dot_kmean;
   a.kv_limit = a.Nk;
+  a.seqs = nullptr;
+  a.max_nqt = a.nqt;
+  a.max_nkt = a.nkt;
 
   const dim3 gridA(plan.splits, a.B * a.Hkv);
   const int nblocks = a.B * a.Hq * a.nqt + 2 * a.B * a.Hkv * a.nkt;
@@ -280,6 +283,8 @@ sage_status run_attention(const sage_qkv_i8f8* z, int causal, float sm_scale, in
   a.causal = causal ? 1 : 0;
   a.return_lse = return_lse ? 1 : 0;
   a.causal_off = a.Nk - a.Nq;
+  a.seqs = nullptr;
+  a.max_nqp = a.nqp;
   const float s = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)z->D);
   a.sm_scale = s;
   a.c0 = (float)((double)s * 1.4426950408889634);
@@ -360,7 +365,12 @@ sage_status check_nvfp4(const sage_qkv_nvfp4* z, bool need_qdk) {
   return SAGE_OK;
 }
 
-std::atomic<uint32_t> g_smem_corr{0};
+// one opt-in flag per instantiation of the correction kernel
+template <typename T, int D>
+std::atomic<uint32_t>& corr_smem_flag() {
+  static std::atomic<uint32_t> flag{0};
+  return flag;
+}
 
 sage_status run_quantize_nvfp4(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
                                int per_block_mean, int64_t unpadded_k_len,
@@ -427,7 +437,8 @@ sage_status run_quantize_nvfp4(const sage_tensor* q, const sage_tensor* k, const
                                                              a.q_hi, a.q_lo);                    \
     nv_means_kernel<D><<<a.B * (a.Hkv + a.Hq), D, 0, stream>>>(a);                               \
     nv_quant_kernel<T, D><<<nblocks, QUANT_THREADS, 0, stream>>>(a);                             \
-    if (!ensure_smem(nv_corr_kernel<T, D>, corr_smem, &g_smem_corr)) return SAGE_ERR_CUDA;       \
+    if (!ensure_smem(nv_corr_kernel<T, D>, corr_smem, &corr_smem_flag<T, D>()))                  \
+      return SAGE_ERR_CUDA;                                                                      \
     nv_corr_kernel<T, D><<<gc, 256, corr_smem, stream>>>(a);                                     \
   } while (0)
   if (q->D == 128) {

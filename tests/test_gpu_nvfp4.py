@@ -159,3 +159,16 @@ def test_nvfp4_without_lse_matches_with_lse(S, causal):
     assert O.cosine(o, ref["out"]) >= 0.9995
     if not causal:
         assert np.abs(o - ref["out"]).max() <= 2e-2
+
+
+def test_nvfp4_quantize_fp16_and_both_head_dims(S):
+    """Every (dtype, head_dim) instantiation of the quantiser launches (each
+    sets its own shared-memory size), in an order that starts with d=64."""
+    for D, dt in [(64, torch.float16), (128, torch.float16), (64, torch.bfloat16), (128, torch.bfloat16)]:
+        w = W.NVFP4.scaled(B=1, Hq=2, Hkv=1, N=256, D=D, unpadded_k_len=256, seed=17)
+        q, k, v = W.make_qkv(w, dtype=dt)
+        oz = O.quantize_qkv_nvfp4(q, k, v, per_block_mean=True, unpadded_k_len=256)
+        gz = S.sage_quantize_qkv_nvfp4(q.cuda(), k.cuda(), v.cuda(), per_block_mean=True,
+                                       unpadded_k_len=256)
+        torch.cuda.synchronize()
+        _compare_quant(gz, oz)
