@@ -218,6 +218,49 @@ sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage
                           int64_t out_sh, int64_t out_sn, float* lse, void* ws,
                           size_t ws_bytes, sage_stream_t stream);
 
+/* --------------------------------------------------------- variable length */
+/* Workspace bytes of sage_attn_fwd_varlen: the sequence table, quantised
+ * Q/K/V of the packed sequences (each padded to 128 tokens per head), the
+ * quantiser's reductions and, with return_lse, q.kmean.  0 for invalid
+ * sizes. */
+size_t sage_attn_fwd_varlen_workspace_bytes(int64_t nseq, int64_t Hq, int64_t Hkv,
+                                            int64_t total_q, int64_t total_k,
+                                            int64_t max_seqlen_q, int64_t max_seqlen_k,
+                                            int64_t D, int return_lse);
+
+/* Attention over a batch of variable-length sequences packed into flat
+ * tensors (pages: "sageattn_varlen": packed q/k/v, cumulative length
+ * arrays cu_seqlens_q/k starting at 0, max_seqlen_q/k, is_causal,
+ * smooth_k; INT8 QK with per-block scales).  Every sequence is its own
+ * problem: its own K mean, 128-token quantisation blocks from its first
+ * token, per-channel V scales, and bottom-right causal alignment.
+ *   q:        [total_q, Hq, D] as a sage_tensor with B = 1, N = total_q (any
+ *             token / head strides, channel stride 1, 16-byte aligned);
+ *   k, v:     [total_k, Hkv, D] likewise, q's dtype, Hq % Hkv == 0;
+ *   cu_seqlens_q/k: DEVICE int32 [nseq + 1]; sequence s holds tokens
+ *             [cu[s], cu[s+1]).  They are read on the device: offsets are
+ *             clamped to [0, total] and lengths to [0, max_seqlen] and to
+ *             the tokens left, so out-of-range values cannot make the
+ *             kernels leave the buffers, but only the rows of valid
+ *             sequences are defined;
+ *   max_seqlen_q/k: bounds of the sequence lengths (they size the grids);
+ *   out:      device [total_q, Hq, D] in q's dtype, token stride out_sn and
+ *             head stride out_sh (elements, multiples of 8), 16-byte aligned;
+ *             rows of empty-key sequences are 0;
+ *   lse:      device fp32, written iff return_lse: one [Hq, len_s] block per
+ *             sequence in sequence order (Hq * total_q values), natural-log
+ *             LSE of the unsmoothed scores, -inf for rows that see no key;
+ *   ws:       device workspace (256-byte aligned) of
+ *             sage_attn_fwd_varlen_workspace_bytes bytes.
+ * sm_scale <= 0 selects 1/sqrt(D).  Returns SAGE_ERR_INVALID_ARG /
+ * _UNSUPPORTED / _WORKSPACE on the host before any launch. */
+sage_status sage_attn_fwd_varlen(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                 int64_t nseq, int64_t max_seqlen_q, int64_t max_seqlen_k,
+                                 int causal, float sm_scale, int smooth_k, int return_lse,
+                                 void* out, int64_t out_sn, int64_t out_sh, float* lse, void* ws,
+                                 size_t ws_bytes, sage_stream_t stream);
+
 /* ------------------------------------------------------------------ NVFP4 */
 /* Workspace bytes of sage_quantize_qkv_nvfp4 (per-split K and Q sums). */
 size_t sage_quantize_nvfp4_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,

@@ -90,6 +90,11 @@ def lib():
                                          ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          P(SageMask), _vp, _i64, _i64, _i64, _vp, _vp,
                                          ctypes.c_size_t, _vp]),
+        "sage_attn_fwd_varlen_workspace_bytes": (ctypes.c_size_t, [_i64] * 8 + [ctypes.c_int]),
+        "sage_attn_fwd_varlen": (ctypes.c_int, [P(SageTensor), P(SageTensor), P(SageTensor), _vp, _vp,
+                                                _i64, _i64, _i64, ctypes.c_int, ctypes.c_float,
+                                                ctypes.c_int, ctypes.c_int, _vp, _i64, _i64, _vp,
+                                                _vp, ctypes.c_size_t, _vp]),
         "sage_debug_qk_int32": (ctypes.c_int, [P(SageQkvI8F8), _i64, _i64, _i64, _i64, _vp, _vp]),
         "sage_debug_pv_fp32": (ctypes.c_int, [P(SageQkvI8F8), _vp, _i64, _i64, _i64, _vp, _vp]),
         "sage_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, _vp]),
@@ -297,6 +302,55 @@ def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, num_kv_heads=None, retur
                            int(bool(return_lse)), int(bool(smooth_k)), mstruct, to.ptr, to.sb,
                            to.sh, to.sn, lse.data_ptr() if return_lse else None, ws.data_ptr(),
                            ws.numel(), _stream(q.device)), "sage_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def _packed(t: torch.Tensor) -> SageTensor:
+    """Describe a packed [total, H, D] tensor (B = 1)."""
+    if t.dim() != 3:
+        raise ValueError("expected a packed [total, H, D] tensor")
+    sn, sh, sd = t.stride()
+    if sd != 1:
+        raise ValueError("the channel stride must be 1")
+    return SageTensor(t.data_ptr(), _dtype_code(t), 1, t.shape[1], t.shape[0], t.shape[2],
+                      0, sh, sn)
+
+
+def sage_attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                         causal=False, sm_scale=None, smooth_k=True, return_lse=False,
+                         out=None, lse=None, ws=None):
+    """Variable-length attention on packed sequences (sage_attn_fwd_varlen).
+
+    q: [total_q, Hq, D], k/v: [total_k, Hkv, D] (bf16/fp16, CUDA);
+    cu_seqlens_q/k: int32 CUDA tensors [nseq + 1].  Returns out
+    [total_q, Hq, D] and, with return_lse, lse (fp32, one [Hq, len_s] block
+    per sequence, flat)."""
+    L = lib()
+    tq, tk, tv = _packed(q), _packed(k), _packed(v)
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    nseq = cu_seqlens_q.numel() - 1
+    if cu_seqlens_k.numel() != nseq + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k describe different numbers of sequences")
+    cq, ck = cu_seqlens_q.contiguous(), cu_seqlens_k.contiguous()
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    sn, sh, sd = out.stride()
+    if sd != 1:
+        raise ValueError("out: the channel stride must be 1")
+    if return_lse and lse is None:
+        lse = torch.empty(q.shape[0] * q.shape[1], dtype=torch.float32, device=q.device)
+    nbytes = L.sage_attn_fwd_varlen_workspace_bytes(nseq, tq.H, tk.H, tq.N, tk.N, int(max_seqlen_q),
+                                                    int(max_seqlen_k), tq.D, int(bool(return_lse)))
+    if ws is None or ws.numel() < nbytes:
+        ws = _ws(nbytes, q.device)
+    _check(L.sage_attn_fwd_varlen(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                                  cq.data_ptr(), ck.data_ptr(), nseq, int(max_seqlen_q),
+                                  int(max_seqlen_k), int(bool(causal)),
+                                  float(sm_scale) if sm_scale else 0.0, int(bool(smooth_k)),
+                                  int(bool(return_lse)), out.data_ptr(), sn, sh,
+                                  lse.data_ptr() if return_lse else None, ws.data_ptr(),
+                                  ws.numel(), _stream(q.device)), "sage_attn_fwd_varlen")
     return (out, lse) if return_lse else out
 
 

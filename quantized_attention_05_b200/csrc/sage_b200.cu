@@ -15,6 +15,7 @@
 
 #include "sage_b200.h"
 #include "sage_ptx.cuh"
+#include "seqs.cuh"
 #include "quantize_i8f8.cuh"
 #include "attn_fwd_i8f8.cuh"
 #include "quantize_nvfp4.cuh"
@@ -176,6 +177,42 @@ sage_status launch_status() {
 }
 
 // ---------------------------------------------------------------- quantise
+// Pass A, stats and pass B for B sequences (dense batch entries or the rows
+// of a sequence table); the grids are sized by the longest sequence.
+sage_status launch_quantize(const QuantArgs& a, const QuantPlan& plan, int64_t D, bool fp16,
+                            cudaStream_t stream) {
+  const dim3 gridA(plan.splits, a.B * a.Hkv);
+  const int64_t nblocks = (int64_t)a.B * a.Hq * a.max_nqt + 2 * (int64_t)a.B * a.Hkv * a.max_nkt;
+  if (nblocks >= (int64_t(1) << 31)) return SAGE_ERR_UNSUPPORTED;
+  if (log_enabled())
+    std::fprintf(stderr, "[sage] quantize B=%d Hq=%d Hkv=%d Nq=%d Nk=%d D=%lld splits=%d x %d, blocks=%lld\n",
+                 a.B, a.Hq, a.Hkv, a.Nq, a.Nk, (long long)D, plan.splits, plan.split_tokens,
+                 (long long)nblocks);
+  const int nb = (int)nblocks;
+  if (D == 128) {
+    if (fp16) {
+      kmean_vamax_partial_kernel<__half, 128><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      kv_stats_kernel<128><<<a.B * a.Hkv, 128, 0, stream>>>(a);
+      quant_blocks_kernel<__half, 128><<<nb, QUANT_THREADS, 0, stream>>>(a);
+    } else {
+      kmean_vamax_partial_kernel<__nv_bfloat16, 128><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      kv_stats_kernel<128><<<a.B * a.Hkv, 128, 0, stream>>>(a);
+      quant_blocks_kernel<__nv_bfloat16, 128><<<nb, QUANT_THREADS, 0, stream>>>(a);
+    }
+  } else {
+    if (fp16) {
+      kmean_vamax_partial_kernel<__half, 64><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      kv_stats_kernel<64><<<a.B * a.Hkv, 64, 0, stream>>>(a);
+      quant_blocks_kernel<__half, 64><<<nb, QUANT_THREADS, 0, stream>>>(a);
+    } else {
+      kmean_vamax_partial_kernel<__nv_bfloat16, 64><<<gridA, QUANT_THREADS, 0, stream>>>(a);
+      kv_stats_kernel<64><<<a.B * a.Hkv, 64, 0, stream>>>(a);
+      quant_blocks_kernel<__nv_bfloat16, 64><<<nb, QUANT_THREADS, 0, stream>>>(a);
+    }
+  }
+  return launch_status();
+}
+
 sage_status run_quantize(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
                          int smooth_k, const sage_qkv_i8f8* out, void* ws, size_t ws_bytes,
                          cudaStream_t stream) {
@@ -221,38 +258,39 @@ sage_status run_quantize(const sage_tensor* q, const sage_tensor* k, const sage_
   a.max_nqt = a.nqt;
   a.max_nkt = a.nkt;
 
-  const dim3 gridA(plan.splits, a.B * a.Hkv);
-  const int nblocks = a.B * a.Hq * a.nqt + 2 * a.B * a.Hkv * a.nkt;
-  if (log_enabled())
-    std::fprintf(stderr, "[sage] quantize B=%d Hq=%d Hkv=%d Nq=%d Nk=%d D=%lld splits=%d x %d, blocks=%d\n",
-                 a.B, a.Hq, a.Hkv, a.Nq, a.Nk, (long long)q->D, plan.splits, plan.split_tokens, nblocks);
-  const bool fp16 = q->dtype == SAGE_FP16;
-  if (q->D == 128) {
-    if (fp16) {
-      kmean_vamax_partial_kernel<__half, 128><<<gridA, QUANT_THREADS, 0, stream>>>(a);
-      kv_stats_kernel<128><<<a.B * a.Hkv, 128, 0, stream>>>(a);
-      quant_blocks_kernel<__half, 128><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
-    } else {
-      kmean_vamax_partial_kernel<__nv_bfloat16, 128><<<gridA, QUANT_THREADS, 0, stream>>>(a);
-      kv_stats_kernel<128><<<a.B * a.Hkv, 128, 0, stream>>>(a);
-      quant_blocks_kernel<__nv_bfloat16, 128><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
-    }
-  } else {
-    if (fp16) {
-      kmean_vamax_partial_kernel<__half, 64><<<gridA, QUANT_THREADS, 0, stream>>>(a);
-      kv_stats_kernel<64><<<a.B * a.Hkv, 64, 0, stream>>>(a);
-      quant_blocks_kernel<__half, 64><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
-    } else {
-      kmean_vamax_partial_kernel<__nv_bfloat16, 64><<<gridA, QUANT_THREADS, 0, stream>>>(a);
-      kv_stats_kernel<64><<<a.B * a.Hkv, 64, 0, stream>>>(a);
-      quant_blocks_kernel<__nv_bfloat16, 64><<<nblocks, QUANT_THREADS, 0, stream>>>(a);
-    }
-  }
-  return launch_status();
+  return launch_quantize(a, plan, q->D, q->dtype == SAGE_FP16, stream);
 }
 
 // ---------------------------------------------------------------- attention
 std::atomic<uint32_t> g_smem_set_64{0}, g_smem_set_128{0};
+
+sage_status launch_attention(const AttnArgs& a, int64_t D, const CUtensorMap& tq,
+                             const CUtensorMap& tk, const CUtensorMap& tv, int64_t grid,
+                             cudaStream_t stream) {
+  if (grid >= (int64_t(1) << 31)) return SAGE_ERR_UNSUPPORTED;
+  // the kernel redistributes registers between its warpgroups; that is only
+  // safe if the launch provides at least the sum of their shares
+  {
+    cudaFuncAttributes fa{};
+    const cudaError_t e = D == 128 ? cudaFuncGetAttributes(&fa, attn_fwd_i8f8_kernel<128>)
+                                   : cudaFuncGetAttributes(&fa, attn_fwd_i8f8_kernel<64>);
+    if (e != cudaSuccess) return SAGE_ERR_CUDA;
+    if (128 * ATT_REGS_LOW + 256 * ATT_REGS_HIGH > ATT_THREADS * fa.numRegs)
+      return SAGE_ERR_UNSUPPORTED;
+  }
+  if (D == 128) {
+    const size_t smem = AttnLayout<128>::bytes(a.nkt);
+    if (!ensure_smem(attn_fwd_i8f8_kernel<128>, AttnLayout<128>::bytes(ATT_MAX_NKT), &g_smem_set_128))
+      return SAGE_ERR_CUDA;
+    attn_fwd_i8f8_kernel<128><<<(unsigned)grid, ATT_THREADS, smem, stream>>>(tq, tk, tv, a);
+  } else {
+    const size_t smem = AttnLayout<64>::bytes(a.nkt);
+    if (!ensure_smem(attn_fwd_i8f8_kernel<64>, AttnLayout<64>::bytes(ATT_MAX_NKT), &g_smem_set_64))
+      return SAGE_ERR_CUDA;
+    attn_fwd_i8f8_kernel<64><<<(unsigned)grid, ATT_THREADS, smem, stream>>>(tq, tk, tv, a);
+  }
+  return launch_status();
+}
 
 sage_status run_attention(const sage_qkv_i8f8* z, int causal, float sm_scale, int return_lse,
                           const sage_mask* mask, void* out, int32_t out_dtype, int64_t out_sb,
@@ -308,28 +346,7 @@ sage_status run_attention(const sage_qkv_i8f8* z, int causal, float sm_scale, in
   if (log_enabled())
     std::fprintf(stderr, "[sage] attn B=%d Hq=%d Hkv=%d Nq=%d Nk=%d D=%lld causal=%d grid=%d\n", a.B,
                  a.Hq, a.Hkv, a.Nq, a.Nk, (long long)z->D, a.causal, grid);
-  // the kernel redistributes registers between its warpgroups; that is only
-  // safe if the launch provides at least the sum of their shares
-  {
-    cudaFuncAttributes fa{};
-    const cudaError_t e = z->D == 128 ? cudaFuncGetAttributes(&fa, attn_fwd_i8f8_kernel<128>)
-                                      : cudaFuncGetAttributes(&fa, attn_fwd_i8f8_kernel<64>);
-    if (e != cudaSuccess) return SAGE_ERR_CUDA;
-    if (128 * ATT_REGS_LOW + 256 * ATT_REGS_HIGH > ATT_THREADS * fa.numRegs)
-      return SAGE_ERR_UNSUPPORTED;
-  }
-  if (z->D == 128) {
-    const size_t smem = AttnLayout<128>::bytes(a.nkt);
-    if (!ensure_smem(attn_fwd_i8f8_kernel<128>, AttnLayout<128>::bytes(ATT_MAX_NKT), &g_smem_set_128))
-      return SAGE_ERR_CUDA;
-    attn_fwd_i8f8_kernel<128><<<grid, ATT_THREADS, smem, stream>>>(tq, tk, tv, a);
-  } else {
-    const size_t smem = AttnLayout<64>::bytes(a.nkt);
-    if (!ensure_smem(attn_fwd_i8f8_kernel<64>, AttnLayout<64>::bytes(ATT_MAX_NKT), &g_smem_set_64))
-      return SAGE_ERR_CUDA;
-    attn_fwd_i8f8_kernel<64><<<grid, ATT_THREADS, smem, stream>>>(tq, tk, tv, a);
-  }
-  return launch_status();
+  return launch_attention(a, z->D, tq, tk, tv, grid, stream);
 }
 
 // ---------------------------------------------------------------- NVFP4 quantise
@@ -530,6 +547,47 @@ FusedLayout fused_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t
 
 std::atomic<uint32_t> g_smem_dbg_qk{0}, g_smem_dbg_pv{0};
 
+// ---------------------------------------------------------------- varlen
+// Workspace of a variable-length call: the sequence table, then the
+// quantised arrays sized for the worst padding (every sequence wastes up to
+// 127 rows per head), the quantiser's reductions and q.kmean.
+struct VarlenLayout {
+  size_t table, q8, qs, k8, ks, km, v8, vs, qdk, part, total;
+  int64_t rows_q, rows_k;   // row capacity of q8 and of k8 / v8
+};
+
+VarlenLayout varlen_layout(int64_t nseq, int64_t Hq, int64_t Hkv, int64_t total_q,
+                           int64_t total_k, int64_t max_k, int64_t D, bool with_qdk) {
+  VarlenLayout f{};
+  f.rows_q = Hq * (total_q + 128 * nseq);
+  f.rows_k = Hkv * (total_k + 128 * nseq);
+  size_t o = 0;
+  f.table = o; o += align256((size_t)nseq * SEQ_STRIDE * 4);
+  f.q8 = o; o += align256((size_t)f.rows_q * D);
+  f.qs = o; o += align256((size_t)(f.rows_q / 128) * 4);
+  f.k8 = o; o += align256((size_t)f.rows_k * D);
+  f.ks = o; o += align256((size_t)(f.rows_k / 128) * 4);
+  f.km = o; o += align256((size_t)nseq * Hkv * D * 4);
+  f.v8 = o; o += align256((size_t)f.rows_k * D);
+  f.vs = o; o += align256((size_t)nseq * Hkv * D * 4);
+  f.qdk = o; o += with_qdk ? align256((size_t)Hq * total_q * 4) : 0;
+  f.part = o; o += quant_plan(nseq, Hkv, max_k, D).part_bytes;
+  f.total = o;
+  return f;
+}
+
+// A packed [total, H, D] tensor of a variable-length call (B = 1).
+sage_status check_packed(const sage_tensor* t) {
+  if (!t || !t->ptr) return SAGE_ERR_INVALID_ARG;
+  if (t->dtype != SAGE_BF16 && t->dtype != SAGE_FP16) return SAGE_ERR_INVALID_ARG;
+  if (t->B != 1 || t->H < 1 || t->H > (1 << 12) || t->N < 1 || t->N >= (int64_t(1) << 30))
+    return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(t->ptr)) return SAGE_ERR_INVALID_ARG;
+  if (t->sn < t->D || t->sn % 8 || t->sh % 8 || t->sh < 0) return SAGE_ERR_INVALID_ARG;
+  if (t->D != 64 && t->D != 128) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -688,6 +746,118 @@ sage_status sage_debug_wait_timeout(uint32_t timeout_us, sage_stream_t stream) {
   if (timeout_us == 0 || timeout_us > 10000000u) return SAGE_ERR_INVALID_ARG;
   debug_wait_kernel<<<1, 32, 0, stream>>>((uint64_t)timeout_us * 1000ull);
   return launch_status();
+}
+
+// ------------------------------------------------- variable length
+size_t sage_attn_fwd_varlen_workspace_bytes(int64_t nseq, int64_t Hq, int64_t Hkv,
+                                            int64_t total_q, int64_t total_k,
+                                            int64_t max_seqlen_q, int64_t max_seqlen_k,
+                                            int64_t D, int return_lse) {
+  (void)max_seqlen_q;
+  if (nseq < 1 || Hq < 1 || Hkv < 1 || total_q < 1 || total_k < 1 || max_seqlen_k < 1 ||
+      (D != 64 && D != 128))
+    return 0;
+  return varlen_layout(nseq, Hq, Hkv, total_q, total_k, max_seqlen_k, D, return_lse != 0).total;
+}
+
+sage_status sage_attn_fwd_varlen(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                 int64_t nseq, int64_t max_seqlen_q, int64_t max_seqlen_k,
+                                 int causal, float sm_scale, int smooth_k, int return_lse,
+                                 void* out, int64_t out_sn, int64_t out_sh, float* lse, void* ws,
+                                 size_t ws_bytes, sage_stream_t stream) {
+  sage_status st;
+  if ((st = check_packed(q)) || (st = check_packed(k)) || (st = check_packed(v))) return st;
+  if (q->dtype != k->dtype || q->dtype != v->dtype) return SAGE_ERR_INVALID_ARG;
+  if (k->H != v->H || k->N != v->N || k->D != q->D || v->D != q->D || q->H % k->H)
+    return SAGE_ERR_INVALID_ARG;
+  if (nseq < 1 || nseq > (1 << 20) || !cu_seqlens_q || !cu_seqlens_k ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return SAGE_ERR_INVALID_ARG;
+  if (max_seqlen_q < 1 || max_seqlen_k < 1) return SAGE_ERR_INVALID_ARG;
+  if (max_seqlen_q > 128 * ATT_MAX_NKT || max_seqlen_k > 128 * ATT_MAX_NKT)
+    return SAGE_ERR_UNSUPPORTED;
+  if (!out || !aligned16(out) || out_sn < q->D || out_sn % 8 || out_sh % 8 || out_sh < 0)
+    return SAGE_ERR_INVALID_ARG;
+  if ((return_lse != 0) != (lse != nullptr)) return SAGE_ERR_INVALID_ARG;
+  if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  const int64_t D = q->D, Hq = q->H, Hkv = k->H, total_q = q->N, total_k = k->N;
+  const VarlenLayout f = varlen_layout(nseq, Hq, Hkv, total_q, total_k, max_seqlen_k, D,
+                                       return_lse != 0);
+  // TMA row coordinates and the LSE index are int32
+  if (f.rows_q >= (int64_t(1) << 31) || f.rows_k >= (int64_t(1) << 31) ||
+      Hq * total_q >= (int64_t(1) << 31))
+    return SAGE_ERR_UNSUPPORTED;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < f.total) return SAGE_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  int* table = reinterpret_cast<int*>(w + f.table);
+  seq_table_kernel<<<1, 32, 0, stream>>>(cu_seqlens_q, cu_seqlens_k, (int)nseq, (int)total_q,
+                                         (int)total_k, (int)max_seqlen_q, (int)max_seqlen_k,
+                                         table);
+  if ((st = launch_status())) return st;
+
+  // quantise: every sequence its own K mean, blocks and V scales
+  const QuantPlan plan = quant_plan(nseq, Hkv, max_seqlen_k, D);
+  QuantArgs a{};
+  a.q = q->ptr; a.k = k->ptr; a.v = v->ptr;
+  a.q_sh = q->sh; a.q_sn = q->sn;
+  a.k_sh = k->sh; a.k_sn = k->sn;
+  a.v_sh = v->sh; a.v_sn = v->sn;
+  a.B = (int)nseq; a.Hq = (int)Hq; a.Hkv = (int)Hkv; a.G = a.Hq / a.Hkv;
+  a.Nq = (int)max_seqlen_q; a.Nk = (int)max_seqlen_k;
+  a.Nqp = (int)pad128(max_seqlen_q); a.Nkp = (int)pad128(max_seqlen_k);
+  a.nqt = a.Nqp / 128; a.nkt = a.Nkp / 128;
+  a.smooth_k = smooth_k ? 1 : 0;
+  a.splits = plan.splits;
+  a.split_tokens = plan.split_tokens;
+  const size_t n = (size_t)nseq * Hkv * plan.splits * D;
+  char* wp = w + f.part;
+  a.part_hi = reinterpret_cast<double*>(wp);
+  a.part_lo = reinterpret_cast<double*>(wp + align256(n * 8));
+  a.part_amax = reinterpret_cast<float*>(wp + 2 * align256(n * 8));
+  a.va = reinterpret_cast<float*>(wp + 2 * align256(n * 8) + align256(n * 4));
+  a.q8 = reinterpret_cast<int8_t*>(w + f.q8);
+  a.q_scale = reinterpret_cast<float*>(w + f.qs);
+  a.k8 = reinterpret_cast<int8_t*>(w + f.k8);
+  a.k_scale = reinterpret_cast<float*>(w + f.ks);
+  a.k_mean = reinterpret_cast<float*>(w + f.km);
+  a.v8 = reinterpret_cast<uint8_t*>(w + f.v8);
+  a.v_scale = reinterpret_cast<float*>(w + f.vs);
+  a.qdk = return_lse ? reinterpret_cast<float*>(w + f.qdk) : nullptr;
+  a.kv_limit = a.Nk;
+  a.seqs = table;
+  a.max_nqt = a.nqt;
+  a.max_nkt = a.nkt;
+  if ((st = launch_quantize(a, plan, D, q->dtype == SAGE_FP16, stream))) return st;
+
+  // attention over the quantised sequences
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_u8(&tq, a.q8, D, f.rows_q, D, (uint32_t)D, 128, qk_swizzle(D)) ||
+      !make_tmap_u8(&tk, a.k8, D, f.rows_k, D, (uint32_t)D, 128, qk_swizzle(D)) ||
+      !make_tmap_u8(&tv, a.v8, D, f.rows_k, D, (uint32_t)D, 128, qk_swizzle(D)))
+    return SAGE_ERR_CUDA;
+  AttnArgs b{};
+  b.q_scale = a.q_scale; b.k_scale = a.k_scale; b.v_scale = a.v_scale; b.qdk = a.qdk;
+  b.out = out; b.out_sh = out_sh; b.out_sn = out_sn;
+  b.out_fp16 = q->dtype == SAGE_FP16;
+  b.lse = lse;
+  b.B = (int)nseq; b.Hq = (int)Hq; b.Hkv = (int)Hkv; b.G = b.Hq / b.Hkv;
+  b.Nq = a.Nq; b.Nk = a.Nk; b.Nqp = a.Nqp; b.Nkp = a.Nkp;
+  b.nqt = a.nqt; b.nkt = a.nkt; b.nqp = (b.nqt + 1) / 2;
+  b.causal = causal ? 1 : 0;
+  b.return_lse = return_lse ? 1 : 0;
+  const float s = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)D);
+  b.sm_scale = s;
+  b.c0 = (float)((double)s * 1.4426950408889634);
+  b.seqs = table;
+  b.max_nqp = b.nqp;
+  const int64_t grid = (int64_t)b.max_nqp * nseq * Hq;
+  if (log_enabled())
+    std::fprintf(stderr, "[sage] attn varlen nseq=%lld Hq=%d Hkv=%d max_q=%d max_k=%d causal=%d grid=%lld\n",
+                 (long long)nseq, b.Hq, b.Hkv, b.Nq, b.Nk, b.causal, (long long)grid);
+  return launch_attention(b, D, tq, tk, tv, grid, stream);
 }
 
 // ------------------------------------------------- allocation-free variant

@@ -163,3 +163,32 @@ def test_nvfp4_rejects_bad_arguments_on_host(L):
     zz = S.SageQkvNvfp4(256, 256, 256, 256, 256, 256, 256, 256, 256, None, 1, 2, 2, 256, 256, 64, 256, 1)
     assert a(byref(zz), 0.0, 0, 1, 1, 256, 0, 0, 256 * 64, 64, 512, None) \
         == S.SAGE_ERR_INVALID_ARG                                   # LSE without q_dot_kmean
+
+
+def test_varlen_rejects_bad_arguments_on_host(L):
+    byref = ctypes.byref
+    pq = _t(B=1, H=4, N=1000, D=64, sn=4 * 64, sh=64)
+    pk = _t(B=1, H=2, N=900, D=64, sn=2 * 64, sh=64)
+    f = L.sage_attn_fwd_varlen
+    need = L.sage_attn_fwd_varlen_workspace_bytes(3, 4, 2, 1000, 900, 512, 512, 64, 1)
+    assert need > 0
+    ok = dict(cu_q=256, cu_k=256, nseq=3, mq=512, mk=512, out=256, sn=4 * 64, sh=64, lse=512,
+              ws=256, nb=need)
+
+    def call(q=pq, k=pk, v=pk, **kw):
+        a = dict(ok, **kw)
+        return f(byref(q), byref(k), byref(v), a["cu_q"], a["cu_k"], a["nseq"], a["mq"], a["mk"], 0,
+                 0.0, 1, 1, a["out"], a["sn"], a["sh"], a["lse"], a["ws"], a["nb"], None)
+    assert call(q=_t(B=2, H=4, N=1000, D=64)) == S.SAGE_ERR_INVALID_ARG      # not packed (B=2)
+    assert call(cu_q=0) == S.SAGE_ERR_INVALID_ARG                            # no cu_seqlens_q
+    assert call(cu_k=258) == S.SAGE_ERR_INVALID_ARG                          # misaligned cu_seqlens_k
+    assert call(nseq=0) == S.SAGE_ERR_INVALID_ARG
+    assert call(mq=0) == S.SAGE_ERR_INVALID_ARG
+    assert call(mk=128 * 4096) == S.SAGE_ERR_UNSUPPORTED                     # longer than supported
+    assert call(lse=0) == S.SAGE_ERR_INVALID_ARG                             # return_lse without lse
+    assert call(sn=60) == S.SAGE_ERR_INVALID_ARG                             # out stride
+    assert call(nb=need - 1) == S.SAGE_ERR_WORKSPACE
+    assert call(q=_t(B=1, H=3, N=1000, D=64)) == S.SAGE_ERR_INVALID_ARG      # Hq % Hkv
+    assert call(q=_t(B=1, H=4, N=1000, D=96), k=_t(B=1, H=2, N=900, D=96),
+                v=_t(B=1, H=2, N=900, D=96)) == S.SAGE_ERR_UNSUPPORTED      # head_dim 96
+    assert L.sage_attn_fwd_varlen_workspace_bytes(0, 4, 2, 1000, 900, 512, 512, 64, 1) == 0
