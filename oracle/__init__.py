@@ -16,6 +16,7 @@ attention  exact fp64 attention and the tile-ordered online-softmax
            attention over the quantised codes (INT8-QK/FP8-PV and NVFP4).
 varlen     packed variable-length batches (cu_seqlens): every sequence its
            own dense problem.
+merge      the LSE merge of partial results over key shards.
 
 Every function states the passage of the SageAttention / FlashInfer pages it
 follows.  Where the pages are silent the plainest reading is taken; those
@@ -34,3 +35,4 @@ from .quantize import (BLOCK, fp4_vector_quant, fp8_channel_quant, int8_block_qu
 from .attention import (attention_i8f8, attention_nvfp4, cosine, default_sm_scale,  # noqa: F401
                         exact_attention, qk_int32_tile)
 from .varlen import attention_varlen_i8f8, block_diagonal_mask, check_cu_seqlens  # noqa: F401
+from .merge import merge_partials, merge_step  # noqa: F401
