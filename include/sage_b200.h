@@ -261,6 +261,32 @@ sage_status sage_attn_fwd_varlen(const sage_tensor* q, const sage_tensor* k, con
                                  void* out, int64_t out_sn, int64_t out_sh, float* lse, void* ws,
                                  size_t ws_bytes, sage_stream_t stream);
 
+/* ------------------------------------------------- merge over key shards */
+/* Running merge of attention results computed over disjoint parts of the
+ * keys (pages: "Utilize SageAttention for Distributed Inference", the
+ * return_lse of "sageattn_qk_int8_pv_fp8_cuda"): per row
+ *   lse' = log(exp(lse) + exp(lse_part)),
+ *   acc' = exp(lse - lse') * acc + exp(lse_part - lse') * part,
+ * -inf meaning "no key seen" (weight 0; a row with no key anywhere stays
+ * 0 / -inf).
+ *   acc:      device fp32 [B, H, N, D] dense, 16-byte aligned, updated in place;
+ *   acc_lse:  device fp32 [B, H, N], updated in place;
+ *   part:     device bf16/fp16 [B, H, N, D], element strides (sb, sh, sn),
+ *             multiples of 8, channel stride 1, 16-byte aligned (the output
+ *             of the attention calls);
+ *   part_lse: device fp32 [B, H, N] (their LSE);
+ *   init:     non-zero for the first part (acc, acc_lse take its values).
+ * D in {64, 128}. */
+sage_status sage_lse_merge(float* acc, float* acc_lse, const void* part, int32_t part_dtype,
+                           int64_t sb, int64_t sh, int64_t sn, const float* part_lse, int64_t B,
+                           int64_t H, int64_t N, int64_t D, int init, sage_stream_t stream);
+
+/* The merged result converted to bf16/fp16 (round to nearest even) with
+ * element strides (sb, sh, sn). */
+sage_status sage_lse_merge_finalize(const float* acc, void* out, int32_t out_dtype, int64_t sb,
+                                    int64_t sh, int64_t sn, int64_t B, int64_t H, int64_t N,
+                                    int64_t D, sage_stream_t stream);
+
 /* ------------------------------------------------------------------ NVFP4 */
 /* Workspace bytes of sage_quantize_qkv_nvfp4 (per-split K and Q sums). */
 size_t sage_quantize_nvfp4_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,

@@ -95,6 +95,10 @@ def lib():
                                                 _i64, _i64, _i64, ctypes.c_int, ctypes.c_float,
                                                 ctypes.c_int, ctypes.c_int, _vp, _i64, _i64, _vp,
                                                 _vp, ctypes.c_size_t, _vp]),
+        "sage_lse_merge": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int32, _i64, _i64, _i64, _vp,
+                                          _i64, _i64, _i64, _i64, ctypes.c_int, _vp]),
+        "sage_lse_merge_finalize": (ctypes.c_int, [_vp, _vp, ctypes.c_int32, _i64, _i64, _i64,
+                                                   _i64, _i64, _i64, _i64, _vp]),
         "sage_debug_qk_int32": (ctypes.c_int, [P(SageQkvI8F8), _i64, _i64, _i64, _i64, _vp, _vp]),
         "sage_debug_pv_fp32": (ctypes.c_int, [P(SageQkvI8F8), _vp, _i64, _i64, _i64, _vp, _vp]),
         "sage_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, _vp]),
@@ -352,6 +356,32 @@ def sage_attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_
                                   lse.data_ptr() if return_lse else None, ws.data_ptr(),
                                   ws.numel(), _stream(q.device)), "sage_attn_fwd_varlen")
     return (out, lse) if return_lse else out
+
+
+def sage_lse_merge(acc, acc_lse, part, part_lse, init=False):
+    """Merge a partial attention result (part [B, H, N, D] bf16/fp16 in any
+    layout with channel stride 1, part_lse [B, H, N]) into the running fp32
+    (acc [B, H, N, D] contiguous, acc_lse [B, H, N]) in place."""
+    B, H, N, D = part.shape
+    sb, sh, sn, sd = part.stride()
+    if sd != 1 or not acc.is_contiguous() or acc.dtype != torch.float32 or acc_lse.dtype != torch.float32:
+        raise ValueError("acc must be contiguous fp32 and part must have channel stride 1")
+    if part_lse.dtype != torch.float32 or not part_lse.is_contiguous() or not acc_lse.is_contiguous():
+        raise ValueError("the LSE tensors must be contiguous fp32")
+    _check(lib().sage_lse_merge(acc.data_ptr(), acc_lse.data_ptr(), part.data_ptr(), _dtype_code(part),
+                                sb, sh, sn, part_lse.data_ptr(), B, H, N, D, int(bool(init)),
+                                _stream(part.device)), "sage_lse_merge")
+
+
+def sage_lse_merge_finalize(acc, out):
+    """Write the merged fp32 result into ``out`` (bf16/fp16 [B, H, N, D])."""
+    B, H, N, D = out.shape
+    sb, sh, sn, sd = out.stride()
+    if sd != 1 or not acc.is_contiguous():
+        raise ValueError("out must have channel stride 1 and acc be contiguous")
+    _check(lib().sage_lse_merge_finalize(acc.data_ptr(), out.data_ptr(), _dtype_code(out), sb, sh, sn,
+                                         B, H, N, D, _stream(out.device)), "sage_lse_merge_finalize")
+    return out
 
 
 def sage_debug_qk_int32(qkv: QuantizedQKV, b, h, qblk, kblk):

@@ -20,6 +20,7 @@
 #include "attn_fwd_i8f8.cuh"
 #include "quantize_nvfp4.cuh"
 #include "attn_fwd_nvfp4.cuh"
+#include "merge.cuh"
 
 using namespace sage;
 
@@ -858,6 +859,56 @@ sage_status sage_attn_fwd_varlen(const sage_tensor* q, const sage_tensor* k, con
     std::fprintf(stderr, "[sage] attn varlen nseq=%lld Hq=%d Hkv=%d max_q=%d max_k=%d causal=%d grid=%lld\n",
                  (long long)nseq, b.Hq, b.Hkv, b.Nq, b.Nk, b.causal, (long long)grid);
   return launch_attention(b, D, tq, tk, tv, grid, stream);
+}
+
+// ------------------------------------------------- merge over key shards
+sage_status sage_lse_merge(float* acc, float* acc_lse, const void* part, int32_t part_dtype,
+                           int64_t sb, int64_t sh, int64_t sn, const float* part_lse, int64_t B,
+                           int64_t H, int64_t N, int64_t D, int init, sage_stream_t stream) {
+  if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+  if (!valid_dims(B, H, N, D)) return SAGE_ERR_INVALID_ARG;
+  if (!acc || !acc_lse || !part || !part_lse || !aligned16(acc) || !aligned16(part))
+    return SAGE_ERR_INVALID_ARG;
+  if (part_dtype != SAGE_BF16 && part_dtype != SAGE_FP16) return SAGE_ERR_INVALID_ARG;
+  if (sn < D || sn % 8 || sh % 8 || sb % 8 || sh < 0 || sb < 0) return SAGE_ERR_INVALID_ARG;
+  MergeArgs a{};
+  a.acc = acc; a.acc_lse = acc_lse; a.part = part; a.sb = sb; a.sh = sh; a.sn = sn;
+  a.part_lse = part_lse; a.B = (int)B; a.H = (int)H; a.N = (int)N; a.init = init ? 1 : 0;
+  const int64_t rows = B * H * N;
+  const int64_t blocks = (rows + (256 / (D / 8)) - 1) / (256 / (D / 8));
+  if (blocks >= (int64_t(1) << 31)) return SAGE_ERR_UNSUPPORTED;
+  const bool fp16 = part_dtype == SAGE_FP16;
+  if (D == 128) {
+    if (fp16) lse_merge_kernel<__half, 128><<<(unsigned)blocks, 256, 0, stream>>>(a);
+    else lse_merge_kernel<__nv_bfloat16, 128><<<(unsigned)blocks, 256, 0, stream>>>(a);
+  } else {
+    if (fp16) lse_merge_kernel<__half, 64><<<(unsigned)blocks, 256, 0, stream>>>(a);
+    else lse_merge_kernel<__nv_bfloat16, 64><<<(unsigned)blocks, 256, 0, stream>>>(a);
+  }
+  return launch_status();
+}
+
+sage_status sage_lse_merge_finalize(const float* acc, void* out, int32_t out_dtype, int64_t sb,
+                                    int64_t sh, int64_t sn, int64_t B, int64_t H, int64_t N,
+                                    int64_t D, sage_stream_t stream) {
+  if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+  if (!valid_dims(B, H, N, D) || !acc || !out || !aligned16(acc) || !aligned16(out))
+    return SAGE_ERR_INVALID_ARG;
+  if (out_dtype != SAGE_BF16 && out_dtype != SAGE_FP16) return SAGE_ERR_INVALID_ARG;
+  if (sn < D || sn % 8 || sh % 8 || sb % 8 || sh < 0 || sb < 0) return SAGE_ERR_INVALID_ARG;
+  const int64_t rows = B * H * N;
+  const int64_t blocks = (rows + (256 / (D / 8)) - 1) / (256 / (D / 8));
+  if (blocks >= (int64_t(1) << 31)) return SAGE_ERR_UNSUPPORTED;
+  const bool fp16 = out_dtype == SAGE_FP16;
+  const int b = (int)B, h = (int)H, n = (int)N;
+  if (D == 128) {
+    if (fp16) lse_merge_finalize_kernel<__half, 128><<<(unsigned)blocks, 256, 0, stream>>>(acc, out, sb, sh, sn, b, h, n);
+    else lse_merge_finalize_kernel<__nv_bfloat16, 128><<<(unsigned)blocks, 256, 0, stream>>>(acc, out, sb, sh, sn, b, h, n);
+  } else {
+    if (fp16) lse_merge_finalize_kernel<__half, 64><<<(unsigned)blocks, 256, 0, stream>>>(acc, out, sb, sh, sn, b, h, n);
+    else lse_merge_finalize_kernel<__nv_bfloat16, 64><<<(unsigned)blocks, 256, 0, stream>>>(acc, out, sb, sh, sn, b, h, n);
+  }
+  return launch_status();
 }
 
 // ------------------------------------------------- allocation-free variant
