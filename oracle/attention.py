@@ -65,12 +65,14 @@ def _visible(rows, keys, Nq, Nk, causal, mask_rows, kv_limit=None):
 
 
 def exact_attention(q, k, v, causal=False, sm_scale=None, mask=None, rows=None,
-                    kv_len=None):
+                    kv_len=None, bias=None):
     """Unquantised attention in float64.
 
     q [B,Hq,Nq,D], k/v [B,Hkv,Nk,D]; mask broadcastable to [B,Hq,Nq,Nk]
-    (True = attend); ``kv_len`` masks keys >= kv_len.  Returns (out
-    [B,Hq,R,D], lse [B,Hq,R]) for the query rows ``rows`` (default all).
+    (True = attend); ``bias`` a float mask broadcastable to [B,Hq,Nq,Nk]
+    added to the scaled scores (-inf hides a key); ``kv_len`` masks keys
+    >= kv_len.  Returns (out [B,Hq,R,D], lse [B,Hq,R]) for the query rows
+    ``rows`` (default all).
     """
     q, k, v = _np64(q), _np64(k), _np64(v)
     B, Hq, Nq, D = q.shape
@@ -81,14 +83,18 @@ def exact_attention(q, k, v, causal=False, sm_scale=None, mask=None, rows=None,
     keys = np.arange(Nk)
     L = Nk if kv_len is None else kv_len
     m4 = None if mask is None else np.broadcast_to(np.asarray(mask, bool), (B, Hq, Nq, Nk))
+    b4 = None if bias is None else np.broadcast_to(_np64(bias), (B, Hq, Nq, Nk))
     out = np.zeros((B, Hq, len(rows), D))
     lse = np.full((B, Hq, len(rows)), -np.inf)
     for b in range(B):
         for h in range(Hq):
             g = h // G
             s = sm_scale * (q[b, h, rows] @ k[b, g].T)
+            if b4 is not None:
+                s = s + b4[b, h][rows]
             vis = _visible(rows, keys, Nq, Nk, causal,
                            None if m4 is None else m4[b, h][rows], kv_limit=L)
+            vis = vis & (s > -np.inf)
             s = np.where(vis, s, -np.inf)
             mx = s.max(axis=1)
             ok = np.isfinite(mx)
@@ -155,11 +161,14 @@ def _p_nvfp4(pp):
 
 
 def attention_i8f8(qz, causal=False, sm_scale=None, mask=None, rows=None, heads=None,
-                   return_internal=False):
+                   return_internal=False, bias=None):
     """Oracle of the fused INT8-QK / FP8-PV attention on quantised inputs.
 
     qz: dict from ``quantize_qkv_i8f8``.  mask: boolean broadcastable to
-    [B, Hq, Nq, Nk] or None.  rows: query rows to compute (default all).
+    [B, Hq, Nq, Nk] or None.  bias: float mask broadcastable to
+    [B, Hq, Nq, Nk] added to the scaled scores ("sageattn_qk_int8_pv_fp16_triton":
+    an optional boolean or float32 attention mask; -inf hides a key), or
+    None.  rows: query rows to compute (default all).
     heads: iterable of (b, h) pairs (default all).  Returns dict with
     ``out`` (bf16-rounded, float64 array [B, Hq, R, D]), ``out_f64`` (before
     rounding), ``lse`` [B, Hq, R]; entries for heads not computed are NaN.
@@ -171,6 +180,7 @@ def attention_i8f8(qz, causal=False, sm_scale=None, mask=None, rows=None, heads=
     keys = np.arange(Nk)
     heads = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else list(heads)
     m4 = None if mask is None else np.broadcast_to(np.asarray(mask, bool), (B, Hq, Nq, Nk))
+    b4 = None if bias is None else np.broadcast_to(np.asarray(bias, np.float64), (B, Hq, Nq, Nk))
     out = np.full((B, Hq, len(rows), D), np.nan)
     lse = np.full((B, Hq, len(rows)), np.nan)
     for b, h in heads:
@@ -181,7 +191,10 @@ def attention_i8f8(qz, causal=False, sm_scale=None, mask=None, rows=None, heads=
         qs = qz["q_scale"][b, h, rows // BLOCK].astype(np.float64)
         ks = qz["k_scale"][b, g, keys // BLOCK].astype(np.float64)
         s = S * qs[:, None] * ks[None, :] * sm_scale
+        if b4 is not None:
+            s = s + b4[b, h][rows]
         vis = _visible(rows, keys, Nq, Nk, causal, None if m4 is None else m4[b, h][rows])
+        vis &= s > -np.inf
         vdec = F.e4m3_decode(qz["v_t"][b, g, :, :Nk]).T          # [Nk, D]
         acc, l, m = _online_softmax_rows(s, vis, vdec, _p_e4m3, 448.0)
         vs = qz["v_scale"][b, g].astype(np.float64)

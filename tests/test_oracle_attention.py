@@ -220,3 +220,70 @@ def test_nvfp4_short_causal_rows_are_tie_sensitive():
     d = np.abs(alt["out"] - ref["out"])
     assert d.max() > 2e-2 and O.cosine(alt["out"], ref["out"]) > 0.9999
     assert np.all(np.argwhere(d > 2e-2)[:, 2] < 127)     # only rows that see < 128 keys
+
+
+# ------------------------------------------------------------ float additive mask
+# ("sageattn_qk_int8_pv_fp16_triton": an optional boolean or float32 attention
+# mask; the float mask is added to the scaled scores, -inf hides a key)
+def _bias_case(seed=71):
+    w = W.TINY.scaled(B=1, Hq=2, Hkv=1, N=256, D=64, seed=seed)
+    q, k, v = W.make_qkv(w)
+    g = torch.Generator().manual_seed(seed)
+    bias = torch.randn(1, 2, 256, 256, generator=g).double()
+    bias[..., 200:] = float("-inf")
+    bias[0, 1, 7, :] = float("-inf")                     # a row that sees nothing
+    return q, k, v, bias
+
+
+def test_exact_attention_float_mask_matches_torch_sdpa():
+    q, k, v, bias = _bias_case()
+    out, lse = O.exact_attention(q, k, v, bias=bias.numpy())
+    qq, kk, vv = (t.double() for t in (q, k, v))
+    kk = kk.repeat_interleave(2, dim=1)
+    vv = vv.repeat_interleave(2, dim=1)
+    ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=bias)
+    ok = np.isfinite(lse)
+    np.testing.assert_allclose(out[ok], ref.numpy()[ok], rtol=0, atol=1e-12)
+    assert np.all(out[~ok] == 0) and not ok[0, 1, 7]
+
+
+def test_float_mask_zero_and_minus_inf_reduce_to_no_mask_and_bool_mask():
+    q, k, v, _ = _bias_case(72)
+    z = O.quantize_qkv_i8f8(q, k, v)
+    plain = O.attention_i8f8(z)
+    zero = O.attention_i8f8(z, bias=np.zeros((1, 1, 256, 256)))
+    np.testing.assert_array_equal(zero["out"], plain["out"])
+    np.testing.assert_array_equal(zero["lse"], plain["lse"])
+    keep = np.ones((1, 1, 256, 256), bool)
+    keep[..., 100:180] = False
+    bias = np.where(keep, 0.0, -np.inf)
+    a = O.attention_i8f8(z, mask=keep)
+    b = O.attention_i8f8(z, bias=bias)
+    np.testing.assert_array_equal(a["out"], b["out"])
+    np.testing.assert_array_equal(a["lse"], b["lse"])
+
+
+def test_float_mask_lossless_equals_exact():
+    """Lossless codes and a bias of 0 or -ln 2: the quantised oracle must
+    equal exact attention with the same bias.  (Integer scores in [-7, 7]
+    plus the bias keep every exponent gap within 15, and 448 * 2**-k is an
+    exact E4M3 value for k <= 15.)"""
+    q, k, v = i8f8_case(B=1, Hq=2, Hkv=2, N=256, D=64, seed=73)
+    g = torch.Generator().manual_seed(73)
+    bias = -LN2 * torch.randint(0, 2, (1, 2, 256, 256), generator=g).double().numpy()
+    bias[..., 240:] = -np.inf
+    r = O.attention_i8f8(O.quantize_qkv_i8f8(q, k, v), sm_scale=LN2, bias=bias)
+    ex, ex_lse = O.exact_attention(q, k, v, sm_scale=LN2, bias=bias)
+    np.testing.assert_allclose(r["out_f64"], ex, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["lse"], ex_lse, rtol=0, atol=1e-12)
+
+
+def test_float_mask_row_constant_shifts_only_the_lse():
+    q, k, v, _ = _bias_case(74)
+    z = O.quantize_qkv_i8f8(q, k, v)
+    shift = np.linspace(-3, 5, 256)[None, None, :, None]
+    a = O.attention_i8f8(z)
+    b = O.attention_i8f8(z, bias=np.broadcast_to(shift, (1, 1, 256, 256)))
+    np.testing.assert_allclose(b["out_f64"], a["out_f64"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(b["lse"] - a["lse"], np.broadcast_to(shift[..., 0], a["lse"].shape),
+                               rtol=0, atol=1e-12)
