@@ -84,16 +84,23 @@ typedef struct {
   int64_t sb, sh, sn;
 } sage_tensor;
 
-/* Boolean attention mask, one byte per element, nonzero = attend
- * ("mask[..., seq_len // 2:] = False  # mask out second half of keys").
+/* Attention mask ("sageattn_qk_int8_pv_fp16_triton": an optional boolean or
+ * float32 attention mask broadcastable to [batch, heads, q_len, k_len]).
+ *   kind SAGE_MASK_BOOL: one byte per element, nonzero = attend
+ *     ("mask[..., seq_len // 2:] = False  # mask out second half of keys");
+ *   kind SAGE_MASK_FLOAT: fp32 added to the scaled scores (natural-log
+ *     units, as a float attention mask adds to q.k^T * sm_scale); -inf hides
+ *     a key; +inf and NaN are not allowed.  4-byte aligned.
  * Logical shape [B, H, Nq, Nk] broadcast over batch and heads: B is 1 or the
- * attention's batch, H is 1 or the number of Q heads.  sb, sh, sq: byte
- * strides (ignored for a broadcast dimension of size 1); the key stride is 1.
- * Device memory, owned by the caller, read-only. */
+ * attention's batch, H is 1 or the number of Q heads.  sb, sh, sq: strides
+ * in elements (ignored for a broadcast dimension of size 1); the key stride
+ * is 1.  Device memory, owned by the caller, read-only. */
+typedef enum { SAGE_MASK_BOOL = 0, SAGE_MASK_FLOAT = 1 } sage_mask_kind;
 typedef struct {
-  const uint8_t* ptr;
+  const void* ptr;
   int64_t B, H, Nq, Nk;
   int64_t sb, sh, sq;
+  int32_t kind; /* sage_mask_kind */
 } sage_mask;
 
 /* Quantised Q/K/V of the INT8/FP8 path, all device memory owned by the

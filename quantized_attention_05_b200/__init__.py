@@ -44,7 +44,10 @@ class SageTensor(ctypes.Structure):
 
 class SageMask(ctypes.Structure):
     _fields_ = [("ptr", _vp), ("B", _i64), ("H", _i64), ("Nq", _i64), ("Nk", _i64),
-                ("sb", _i64), ("sh", _i64), ("sq", _i64)]
+                ("sb", _i64), ("sh", _i64), ("sq", _i64), ("kind", ctypes.c_int32)]
+
+
+SAGE_MASK_BOOL, SAGE_MASK_FLOAT = 0, 1
 
 
 class SageQkvI8F8(ctypes.Structure):
@@ -157,8 +160,9 @@ def _as_tensor(t: torch.Tensor, layout: str = "HND") -> SageTensor:
 def _as_mask(mask: Optional[torch.Tensor], B, Hq, Nq, Nk):
     if mask is None:
         return None
-    if mask.dtype != torch.bool and mask.dtype != torch.uint8:
-        raise TypeError("mask must be bool or uint8 (nonzero = attend)")
+    if mask.dtype not in (torch.bool, torch.uint8, torch.float32):
+        raise TypeError("mask must be bool/uint8 (nonzero = attend) or float32 (added to the scores)")
+    kind = SAGE_MASK_FLOAT if mask.dtype == torch.float32 else SAGE_MASK_BOOL
     m = mask
     while m.dim() < 4:
         m = m.unsqueeze(0)
@@ -167,7 +171,7 @@ def _as_mask(mask: Optional[torch.Tensor], B, Hq, Nq, Nk):
         m = m.contiguous()
     mb, mh = m.shape[0], m.shape[1]
     return SageMask(m.data_ptr(), mb, mh, Nq, Nk, m.stride(0) if mb > 1 else 0,
-                    m.stride(1) if mh > 1 else 0, m.stride(2)), m
+                    m.stride(1) if mh > 1 else 0, m.stride(2), kind), m
 
 
 def pad128(n):

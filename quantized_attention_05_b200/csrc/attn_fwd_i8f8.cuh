@@ -44,6 +44,7 @@ constexpr int ATT_REGS_HIGH = 224;
 constexpr int ATT_MAX_NKT = 2048;   // keys <= 262144
 constexpr float LOG2_448 = 8.807354922057604f;
 constexpr float LN2_F = 0.6931471805599453f;
+constexpr float LOG2E_F = 1.4426950408889634f;
 
 struct AttnArgs {
   const float* q_scale;
@@ -55,9 +56,10 @@ struct AttnArgs {
   int out_fp16;
   float* lse;
   const uint8_t* tile_class;       // [Bm, Hm, nqt, nkt] or null
-  const uint8_t* mask;
+  const void* mask;                // bool bytes or fp32 (mask_kind), element strides
   int64_t m_sb, m_sh, m_sq;
   int m_bcast_b, m_bcast_h, mask_vec16;
+  int mask_kind;                   // 0: boolean, 1: fp32 added to the scaled scores
   int B, Hq, Hkv, G, Nq, Nk, Nqp, Nkp, nqt, nkt, nqp;
   int causal, return_lse, causal_off;
   float c0;                        // sm_scale * log2(e)
@@ -256,7 +258,9 @@ __device__ __forceinline__ void tile_visibility(const AttnArgs& a, const CtaSeq&
 // of one 128-key tile.  sr holds 1.5*2^23 + S as float bits (0 for hidden
 // keys when NEED); p = 2^(S*c + bias) in fp32, P = E4M3(p) (bias includes
 // log2(448) and minus the running max), row sum of the unquantised p.
-template <bool NEED>
+// BIASED: sr already holds the scaled score plus the mask's bias (log2
+// units, -inf for hidden keys) as float bits; p = 2^(sr + bias).
+template <bool NEED, bool BIASED = false>
 __device__ __forceinline__ float exp_tile(const uint32_t* sr, const uint32_t* vis, float c,
                                           float bias, uint8_t* ptile, int rt) {
   const uint64_t c2 = f2_pack(c, c), b2 = f2_pack(bias, bias);
@@ -272,8 +276,10 @@ __device__ __forceinline__ float exp_tile(const uint32_t* sr, const uint32_t* vi
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int j = ch * 32 + 2 * (i + u);
-        const uint64_t y = f2_fma(
-            f2_add(f2_pack(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), nm2), c2, b2);
+        const uint64_t y =
+            BIASED ? f2_add(f2_pack(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), b2)
+                   : f2_fma(f2_add(f2_pack(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), nm2),
+                            c2, b2);
         float y0, y1;
         f2_unpack(y, y0, y1);
         uint64_t p;
@@ -512,10 +518,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t tO = tS + 128;
     const bool tile_exists = qt < cs.nqt;
     const float cq = tile_exists ? a.q_scale[cs.qs0 + qt] * a.c0 : 0.f;
-    const uint8_t* mrow = nullptr;
+    const uint8_t* mrow = nullptr;           // this row of the mask (bytes or floats)
     if (a.mask && row < cs.Nq) {
       const int bm = a.m_bcast_b ? 0 : b, hm = a.m_bcast_h ? 0 : h;
-      mrow = a.mask + bm * a.m_sb + hm * a.m_sh + (int64_t)row * a.m_sq;
+      const int64_t el = (int64_t)bm * a.m_sb + (int64_t)hm * a.m_sh + (int64_t)row * a.m_sq;
+      mrow = reinterpret_cast<const uint8_t*>(a.mask) + el * (a.mask_kind ? 4 : 1);
     }
     // S accumulators start at 1.5*2^23 (as int32 bits): the int32 QK^T sum
     // on top of it is then directly the float 1.5*2^23 + S.  The refill
@@ -555,24 +562,60 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
       // sr holds 1.5*2^23 + S as float bits; hidden keys -> 0.0 (below every score)
       uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
+      const bool biased = part && a.mask_kind == 1;
       if (need) {
-        tile_visibility(a, cs, kt, row, part, mrow, vis);
+        tile_visibility(a, cs, kt, row, part && a.mask_kind == 0, mrow, vis);
+        if (!biased) {
 #pragma unroll
-        for (int j = 0; j < 128; ++j)
-          if (!((vis[j >> 5] >> (j & 31)) & 1u)) sr[j] = 0u;
+          for (int j = 0; j < 128; ++j)
+            if (!((vis[j >> 5] >> (j & 31)) & 1u)) sr[j] = 0u;
+        }
       }
-      float m0 = __uint_as_float(sr[0]), m1 = __uint_as_float(sr[1]);
-      float m2 = __uint_as_float(sr[2]), m3 = __uint_as_float(sr[3]);
+      float mt;   // tile max of the scaled scores (-inf if this row sees no key here)
+      if (biased) {
+        // float mask: sr <- S * c + bias * log2(e) (-inf for hidden keys),
+        // in 32-key chunks of 16-byte bias loads
+        const float* brow = mrow ? reinterpret_cast<const float*>(mrow) + kt * ATT_BN : nullptr;
+        float bm0 = -INFINITY, bm1 = -INFINITY;
 #pragma unroll
-      for (int j = 4; j < 128; j += 8) {
-        m0 = max3f(m0, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
-        m1 = max3f(m1, __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
-        m2 = max3f(m2, __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
-        m3 = max3f(m3, __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
+        for (int ch = 0; ch < 4; ++ch) {
+          float bb[32];
+          const int key0 = kt * ATT_BN + ch * 32;
+          if (brow && key0 + 32 <= cs.Nk && (reinterpret_cast<uintptr_t>(brow) & 15u) == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 f = __ldg(reinterpret_cast<const float4*>(brow + ch * 32) + i);
+              bb[4 * i] = f.x; bb[4 * i + 1] = f.y; bb[4 * i + 2] = f.z; bb[4 * i + 3] = f.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              bb[i] = (brow && key0 + i < cs.Nk) ? __ldg(brow + ch * 32 + i) : -INFINITY;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int j = ch * 32 + i;
+            const float t = ((vis[j >> 5] >> (j & 31)) & 1u)
+                                ? fmaf(__uint_as_float(sr[j]) - MAGIC_F, c, bb[i] * LOG2E_F)
+                                : -INFINITY;
+            sr[j] = __float_as_uint(t);
+            if (i & 1) bm1 = fmaxf(bm1, t); else bm0 = fmaxf(bm0, t);
+          }
+        }
+        mt = fmaxf(bm0, bm1);
+      } else {
+        float m0 = __uint_as_float(sr[0]), m1 = __uint_as_float(sr[1]);
+        float m2 = __uint_as_float(sr[2]), m3 = __uint_as_float(sr[3]);
+#pragma unroll
+        for (int j = 4; j < 128; j += 8) {
+          m0 = max3f(m0, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+          m1 = max3f(m1, __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
+          m2 = max3f(m2, __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
+          m3 = max3f(m3, __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
+        }
+        const float mx = max3f(m0, m1, fmaxf(m2, m3));
+        mt = mx >= 4194304.f ? (mx - MAGIC_F) * c : -INFINITY;
       }
-      const float mx = max3f(m0, m1, fmaxf(m2, m3));
-      // tile max of the scaled scores (-inf if this row sees no key here)
-      const float mt = mx >= 4194304.f ? (mx - MAGIC_F) * c : -INFINITY;
       const float m_new = fmaxf(m_ref, mt);
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
       const float alpha = ex2_approx(m_ref - m_use);
@@ -585,8 +628,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                                 SITE_O_READY));
         if (!ok) break;
       }
-      const float rs = need ? exp_tile<true>(sr, vis, c, bias, ptile, rt)
-                            : exp_tile<false>(sr, vis, c, bias, ptile, rt);
+      const float rs = biased ? exp_tile<true, true>(sr, vis, c, bias, ptile, rt)
+                       : need ? exp_tile<true>(sr, vis, c, bias, ptile, rt)
+                              : exp_tile<false>(sr, vis, c, bias, ptile, rt);
       if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         const uint32_t pb = (n - 1) & 1u;
         ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[wg * 2 + pb], ((n - 1) >> 1) & 1,
@@ -665,20 +709,30 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 // ------------------------------------------------------------ mask classes
 // One CTA per (mask batch/head, q tile, k tile): 0 = nothing visible,
 // 1 = everything visible, 2 = mixed.  Only rows < Nq and keys < Nk count.
-__global__ void __launch_bounds__(256) mask_classify_kernel(const uint8_t* __restrict__ mask,
-                                                            int64_t sb, int64_t sh, int64_t sq,
-                                                            int Hm, int Nq, int Nk, int nqt,
-                                                            int nkt, uint8_t* __restrict__ cls) {
+// For a float mask: 0 = every entry -inf, 1 = every entry 0 (no bias),
+// 2 = otherwise.  Strides in elements.
+__global__ void __launch_bounds__(256) mask_classify_kernel(const void* __restrict__ mask,
+                                                            int kind, int64_t sb, int64_t sh,
+                                                            int64_t sq, int Hm, int Nq, int Nk,
+                                                            int nqt, int nkt,
+                                                            uint8_t* __restrict__ cls) {
   const int kt = blockIdx.x, qt = blockIdx.y, bhm = blockIdx.z;
   const int bm = bhm / Hm, hm = bhm % Hm;
-  const uint8_t* base = mask + bm * sb + hm * sh;
+  const int64_t base = (int64_t)bm * sb + (int64_t)hm * sh;
   int any = 0, all = 1;
   for (int idx = threadIdx.x; idx < ATT_BM * ATT_BN; idx += blockDim.x) {
     const int r = qt * ATT_BM + idx / ATT_BN, c = kt * ATT_BN + idx % ATT_BN;
     if (r < Nq && c < Nk) {
-      const int v = base[(int64_t)r * sq + c] != 0;
-      any |= v;
-      all &= v;
+      const int64_t e = base + (int64_t)r * sq + c;
+      if (kind == 0) {
+        const int v = static_cast<const uint8_t*>(mask)[e] != 0;
+        any |= v;
+        all &= v;
+      } else {
+        const float x = static_cast<const float*>(mask)[e];
+        any |= x != -INFINITY;
+        all &= x == 0.f;
+      }
     }
   }
   any = __syncthreads_or(any);

@@ -84,6 +84,9 @@ sage_status check_qkv(const sage_qkv_i8f8* z, bool need_qdk) {
 sage_status check_mask(const sage_mask* m, int64_t B, int64_t Hq, int64_t Nq, int64_t Nk) {
   if (!m) return SAGE_OK;
   if (!m->ptr) return SAGE_ERR_INVALID_ARG;
+  if (m->kind != SAGE_MASK_BOOL && m->kind != SAGE_MASK_FLOAT) return SAGE_ERR_INVALID_ARG;
+  if (m->kind == SAGE_MASK_FLOAT && (reinterpret_cast<uintptr_t>(m->ptr) & 3u))
+    return SAGE_ERR_INVALID_ARG;
   if (!(m->B == 1 || m->B == B) || !(m->H == 1 || m->H == Hq)) return SAGE_ERR_INVALID_ARG;
   if (m->Nq != Nq || m->Nk != Nk) return SAGE_ERR_INVALID_ARG;
   if (m->sq < Nk || (m->B > 1 && m->sb < 0) || (m->H > 1 && m->sh < 0)) return SAGE_ERR_INVALID_ARG;
@@ -329,16 +332,17 @@ sage_status run_attention(const sage_qkv_i8f8* z, int causal, float sm_scale, in
   a.c0 = (float)((double)s * 1.4426950408889634);
   if (mask) {
     a.mask = mask->ptr;
+    a.mask_kind = mask->kind;
     a.m_sb = mask->sb; a.m_sh = mask->sh; a.m_sq = mask->sq;
     a.m_bcast_b = mask->B == 1; a.m_bcast_h = mask->H == 1;
-    a.mask_vec16 = aligned16(mask->ptr) && mask->sq % 16 == 0 &&
+    a.mask_vec16 = mask->kind == SAGE_MASK_BOOL && aligned16(mask->ptr) && mask->sq % 16 == 0 &&
                    (mask->B == 1 || mask->sb % 16 == 0) && (mask->H == 1 || mask->sh % 16 == 0);
     uint8_t* cls = static_cast<uint8_t*>(ws);
     a.tile_class = cls;
     const int Hm = (int)mask->H;
     mask_classify_kernel<<<dim3(a.nkt, a.nqt, (unsigned)(mask->B * mask->H)), 256, 0, stream>>>(
-        mask->ptr, mask->B == 1 ? 0 : mask->sb, mask->H == 1 ? 0 : mask->sh, mask->sq, Hm, a.Nq,
-        a.Nk, a.nqt, a.nkt, cls);
+        mask->ptr, mask->kind, mask->B == 1 ? 0 : mask->sb, mask->H == 1 ? 0 : mask->sh, mask->sq,
+        Hm, a.Nq, a.Nk, a.nqt, a.nkt, cls);
     if ((st = launch_status())) return st;
   }
   CUtensorMap tq, tk, tv;

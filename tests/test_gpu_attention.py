@@ -96,6 +96,45 @@ def test_mask_unaligned_key_length(S):
     assert_attention_close(out, l, ref, what="per-head mask, Nk=200")
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_float_mask(S, causal):
+    """Float additive mask ("sageattn_qk_int8_pv_fp16_triton": boolean or
+    float32 attention mask): random biases, -inf regions (a hidden key
+    tile, a row that sees nothing), an all-zero tile, broadcast over heads."""
+    w = W.TINY.scaled(B=2, Hq=4, Hkv=2, N=512, D=128, seed=37)
+    q, k, v = W.make_qkv(w)
+    oz = O.quantize_qkv_i8f8(q, k, v)
+    g = torch.Generator().manual_seed(5)
+    bias = 2.0 * torch.randn(2, 1, 512, 512, generator=g)
+    bias[:, :, :, 384:] = float("-inf")           # a fully hidden key tile
+    bias[:, :, :, 128:256] = 0.0                   # a tile without bias
+    bias[:, :, 9, :] = float("-inf")               # a row with no visible key
+    bias[:, :, :, 40:60] = float("-inf")
+    ref = O.attention_i8f8(oz, bias=bias.double().numpy(), causal=causal)
+    out, l = S.sage_attn_fwd_quantized(qkv_from_oracle(S, oz), return_lse=True, mask=bias.cuda(),
+                                       causal=causal)
+    assert_attention_close(out, l, ref, what=f"float mask causal={causal}")
+    assert torch.all(out[:, :, 9] == 0) and torch.all(torch.isneginf(l[:, :, 9]))
+
+
+def test_float_mask_unaligned_rows_and_zero_bias(S):
+    """A per-head bias whose rows are not 16-byte aligned (scalar loads) on
+    a ragged key length; and an all-zero bias equals no mask bit for bit."""
+    w = W.TINY.scaled(B=1, Hq=2, Hkv=2, N=203, D=64, seed=38)
+    q, k, v = W.make_qkv(w)
+    oz = O.quantize_qkv_i8f8(q, k, v)
+    z = qkv_from_oracle(S, oz)
+    g = torch.Generator().manual_seed(6)
+    bias = torch.randn(1, 2, 203, 203, generator=g)
+    ref = O.attention_i8f8(oz, bias=bias.double().numpy())
+    out, l = S.sage_attn_fwd_quantized(z, return_lse=True, mask=bias.cuda())
+    assert_attention_close(out, l, ref, what="float mask, unaligned rows")
+    plain, pl = S.sage_attn_fwd_quantized(z, return_lse=True)
+    zero, zl = S.sage_attn_fwd_quantized(z, return_lse=True, mask=torch.zeros(1, 1, 203, 203).cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(plain, zero) and torch.equal(pl, zl)
+
+
 def test_causal_bottom_right_when_lengths_differ(S):
     for Nq, Nk in [(200, 333), (333, 200)]:
         wq = W.TINY.scaled(B=1, Hq=2, Hkv=1, N=Nq, D=128, seed=37)
