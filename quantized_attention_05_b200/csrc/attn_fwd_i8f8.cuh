@@ -313,7 +313,9 @@ __device__ __forceinline__ float exp_tile(const uint32_t* sr, const uint32_t* vi
   return a0 + a1;
 }
 
-template <int D>
+// FMASK: the instantiation for a float mask (its biased softmax path is
+// compiled only there, so the kernel without it keeps its code size).
+template <int D, bool FMASK>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attn_fwd_i8f8_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
@@ -345,6 +347,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const int g = h / a.G;
   const int bhk = b * a.Hkv + g;
   const CtaSeq cs = cta_seq(a, b, h, g);
+  // the softmax warps read the sequence view from shared memory when they
+  // need it (fewer registers held through their loop)
+  __shared__ CtaSeq s_cs;
   const int qt0 = 2 * qp;
   // a variable-length call sizes the grid by its longest sequence: CTAs
   // beyond this sequence's tiles leave before any setup
@@ -373,6 +378,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       s_nlist[1] = (int)orf;
     }
   } else if (warp == 1 && lane == 0) {
+    s_cs = cs;
     mbar_init(q_full, 1);
     for (int s = 0; s < ATT_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -509,6 +515,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(ATT_REGS_HIGH));
     // ---------------------------------------------------------- softmax WGs
+    const CtaSeq& cs = s_cs;
     const int wg = warp >> 2;
     const int rt = threadIdx.x & 127;
     const int qt = qt0 + wg;
@@ -562,9 +569,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
       // sr holds 1.5*2^23 + S as float bits; hidden keys -> 0.0 (below every score)
       uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
-      const bool biased = part && a.mask_kind == 1;
+      const bool biased = FMASK && part;
       if (need) {
-        tile_visibility(a, cs, kt, row, part && a.mask_kind == 0, mrow, vis);
+        tile_visibility(a, cs, kt, row, part && !FMASK, mrow, vis);
         if (!biased) {
 #pragma unroll
           for (int j = 0; j < 128; ++j)
@@ -572,7 +579,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
       }
       float mt;   // tile max of the scaled scores (-inf if this row sees no key here)
-      if (biased) {
+      if (FMASK && biased) {
         // float mask: sr <- S * c + bias * log2(e) (-inf for hidden keys),
         // in 32-key chunks of 16-byte bias loads
         const float* brow = mrow ? reinterpret_cast<const float*>(mrow) + kt * ATT_BN : nullptr;
@@ -628,9 +635,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                                 SITE_O_READY));
         if (!ok) break;
       }
-      const float rs = biased ? exp_tile<true, true>(sr, vis, c, bias, ptile, rt)
-                       : need ? exp_tile<true>(sr, vis, c, bias, ptile, rt)
-                              : exp_tile<false>(sr, vis, c, bias, ptile, rt);
+      float rs;
+      if constexpr (FMASK) {
+        rs = biased ? exp_tile<true, true>(sr, vis, c, bias, ptile, rt)
+                    : need ? exp_tile<true>(sr, vis, c, bias, ptile, rt)
+                           : exp_tile<false>(sr, vis, c, bias, ptile, rt);
+      } else {
+        rs = need ? exp_tile<true>(sr, vis, c, bias, ptile, rt)
+                  : exp_tile<false>(sr, vis, c, bias, ptile, rt);
+      }
       if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         const uint32_t pb = (n - 1) & 1u;
         ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[wg * 2 + pb], ((n - 1) >> 1) & 1,

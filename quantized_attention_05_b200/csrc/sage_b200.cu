@@ -266,33 +266,29 @@ sage_status run_quantize(const sage_tensor* q, const sage_tensor* k, const sage_
 }
 
 // ---------------------------------------------------------------- attention
-std::atomic<uint32_t> g_smem_set_64{0}, g_smem_set_128{0};
+std::atomic<uint32_t> g_smem_set_64{0}, g_smem_set_128{0}, g_smem_set_64f{0}, g_smem_set_128f{0};
 
 sage_status launch_attention(const AttnArgs& a, int64_t D, const CUtensorMap& tq,
                              const CUtensorMap& tk, const CUtensorMap& tv, int64_t grid,
                              cudaStream_t stream) {
   if (grid >= (int64_t(1) << 31)) return SAGE_ERR_UNSUPPORTED;
+  const bool fmask = a.mask && a.mask_kind == SAGE_MASK_FLOAT;
+  auto kernel = D == 128 ? (fmask ? attn_fwd_i8f8_kernel<128, true> : attn_fwd_i8f8_kernel<128, false>)
+                         : (fmask ? attn_fwd_i8f8_kernel<64, true> : attn_fwd_i8f8_kernel<64, false>);
+  std::atomic<uint32_t>* flag = D == 128 ? (fmask ? &g_smem_set_128f : &g_smem_set_128)
+                                         : (fmask ? &g_smem_set_64f : &g_smem_set_64);
   // the kernel redistributes registers between its warpgroups; that is only
   // safe if the launch provides at least the sum of their shares
   {
     cudaFuncAttributes fa{};
-    const cudaError_t e = D == 128 ? cudaFuncGetAttributes(&fa, attn_fwd_i8f8_kernel<128>)
-                                   : cudaFuncGetAttributes(&fa, attn_fwd_i8f8_kernel<64>);
-    if (e != cudaSuccess) return SAGE_ERR_CUDA;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return SAGE_ERR_CUDA;
     if (128 * ATT_REGS_LOW + 256 * ATT_REGS_HIGH > ATT_THREADS * fa.numRegs)
       return SAGE_ERR_UNSUPPORTED;
   }
-  if (D == 128) {
-    const size_t smem = AttnLayout<128>::bytes(a.nkt);
-    if (!ensure_smem(attn_fwd_i8f8_kernel<128>, AttnLayout<128>::bytes(ATT_MAX_NKT), &g_smem_set_128))
-      return SAGE_ERR_CUDA;
-    attn_fwd_i8f8_kernel<128><<<(unsigned)grid, ATT_THREADS, smem, stream>>>(tq, tk, tv, a);
-  } else {
-    const size_t smem = AttnLayout<64>::bytes(a.nkt);
-    if (!ensure_smem(attn_fwd_i8f8_kernel<64>, AttnLayout<64>::bytes(ATT_MAX_NKT), &g_smem_set_64))
-      return SAGE_ERR_CUDA;
-    attn_fwd_i8f8_kernel<64><<<(unsigned)grid, ATT_THREADS, smem, stream>>>(tq, tk, tv, a);
-  }
+  const size_t smem = D == 128 ? AttnLayout<128>::bytes(a.nkt) : AttnLayout<64>::bytes(a.nkt);
+  const size_t smem_max = D == 128 ? AttnLayout<128>::bytes(ATT_MAX_NKT) : AttnLayout<64>::bytes(ATT_MAX_NKT);
+  if (!ensure_smem(kernel, smem_max, flag)) return SAGE_ERR_CUDA;
+  kernel<<<(unsigned)grid, ATT_THREADS, smem, stream>>>(tq, tk, tv, a);
   return launch_status();
 }
 
