@@ -145,16 +145,30 @@ __global__ void __launch_bounds__(QUANT_THREADS) kmean_vamax_partial_kernel(Quan
   const char* vb = reinterpret_cast<const char*>(a.v) +
                    (seq_in_offset(a, sq.ck, b, a.v_sn, a.v_sb) + h * a.v_sh + cg * 8) *
                        (int64_t)sizeof(T);
-  for (int n = n0 + rs; n < n1; n += RPP) {
-    float f[8];
-    if (a.smooth_k) {
-      unpack8<T>(ldg16(kb + (int64_t)n * a.k_sn * sizeof(T)), f);
+  // four rows per iteration, their loads issued before any arithmetic (the
+  // accumulation order per channel is the same fixed row order as one by one)
+  constexpr int UNR = 4;
+  for (int nb = n0 + rs; nb < n1; nb += UNR * RPP) {
+    uint4 kr[UNR], vr[UNR];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dd_add(acc[i], (double)f[i]);
+    for (int u = 0; u < UNR; ++u) {
+      const int n = nb + u * RPP;
+      kr[u] = (a.smooth_k && n < n1) ? ldg16(kb + (int64_t)n * a.k_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
+      vr[u] = n < n1 ? ldg16(vb + (int64_t)n * a.v_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
     }
-    unpack8<T>(ldg16(vb + (int64_t)n * a.v_sn * sizeof(T)), f);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) am[i] = fmaxf(am[i], fabsf(f[i]));
+    for (int u = 0; u < UNR; ++u) {
+      if (nb + u * RPP >= n1) break;
+      float f[8];
+      if (a.smooth_k) {
+        unpack8<T>(kr[u], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dd_add(acc[i], (double)f[i]);
+      }
+      unpack8<T>(vr[u], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) am[i] = fmaxf(am[i], fabsf(f[i]));
+    }
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -209,10 +223,19 @@ __device__ __forceinline__ float block_max(float v, float* s_red) {
   return r;
 }
 
-__device__ __forceinline__ int8_t int8_code(float x, float inv) {
-  int c = __float2int_rn(__fmul_rn(x, inv));
-  c = max(-127, min(127, c));
-  return (int8_t)c;
+// Four INT8 codes rint(fp32(x[i] * inv)) (round half to even) packed into a
+// word, x[0] in the low byte.  |x * inv| <= 127 by construction (inv =
+// 127/amax of the block), so adding 1.5*2^23 to the fp32 product leaves the
+// integer in the low mantissa bits and their low byte is the two's-complement
+// code: FMA-pipe arithmetic and byte permutes instead of float-to-int
+// conversions.
+__device__ __forceinline__ uint32_t int8x4_codes(float x0, float x1, float x2, float x3,
+                                                 float inv) {
+  const uint32_t t0 = __float_as_uint(__fadd_rn(__fmul_rn(x0, inv), 12582912.f));
+  const uint32_t t1 = __float_as_uint(__fadd_rn(__fmul_rn(x1, inv), 12582912.f));
+  const uint32_t t2 = __float_as_uint(__fadd_rn(__fmul_rn(x2, inv), 12582912.f));
+  const uint32_t t3 = __float_as_uint(__fadd_rn(__fmul_rn(x3, inv), 12582912.f));
+  return __byte_perm(__byte_perm(t0, t1, 0x0040), __byte_perm(t2, t3, 0x0040), 0x5410);
 }
 
 // ------------------------------------------------------------ pass B
@@ -267,11 +290,8 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
       const int n = qt * QB + rs + it * RPP;
       float f[8];
       unpack8<T>(raw[it], f);
-      uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) w0 |= (uint32_t)(uint8_t)int8_code(f[i], inv) << (8 * i);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) w1 |= (uint32_t)(uint8_t)int8_code(f[4 + i], inv) << (8 * i);
+      const uint32_t w0 = int8x4_codes(f[0], f[1], f[2], f[3], inv);
+      const uint32_t w1 = int8x4_codes(f[4], f[5], f[6], f[7], inv);
       *reinterpret_cast<uint2*>(a.q8 + (row0 + n) * D + cg * 8) = make_uint2(w0, w1);
       if (a.qdk) {
         float d = 0.f;
@@ -329,12 +349,10 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
       unpack8<T>(raw[it], f);
       uint32_t w0 = 0, w1 = 0;
       if (n < sq.nk) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          w0 |= (uint32_t)(uint8_t)int8_code(__fsub_rn(f[i], km[i]), inv) << (8 * i);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          w1 |= (uint32_t)(uint8_t)int8_code(__fsub_rn(f[4 + i], km[4 + i]), inv) << (8 * i);
+        w0 = int8x4_codes(__fsub_rn(f[0], km[0]), __fsub_rn(f[1], km[1]), __fsub_rn(f[2], km[2]),
+                          __fsub_rn(f[3], km[3]), inv);
+        w1 = int8x4_codes(__fsub_rn(f[4], km[4]), __fsub_rn(f[5], km[5]), __fsub_rn(f[6], km[6]),
+                          __fsub_rn(f[7], km[7]), inv);
       }
       *reinterpret_cast<uint2*>(a.k8 + (row0 + n) * D + cg * 8) = make_uint2(w0, w1);
     }

@@ -107,7 +107,7 @@ struct QuantPlan {
 QuantPlan quant_plan(int64_t B, int64_t Hkv, int64_t Nk, int64_t D) {
   const int64_t bh = B * Hkv;
   const int64_t max_split = std::max<int64_t>(1, (Nk + 255) / 256);
-  const int64_t want = std::max<int64_t>(1, (2 * kSMs + bh - 1) / bh);
+  const int64_t want = std::max<int64_t>(1, (8 * kSMs + bh - 1) / bh);
   int64_t s = std::min(want, max_split);
   int64_t t = ((Nk + s - 1) / s + 31) / 32 * 32;
   s = (Nk + t - 1) / t;
