@@ -32,7 +32,8 @@
  * Conventions (all entry points):
  *   - Every pointer argument named as device memory must point to memory
  *     of the device that is current on the calling thread; host pointers
- *     are only the descriptor structs themselves.  The library never
+ *     are the descriptor structs themselves and the tensors of
+ *     sage_attn_fwd_host, whose arguments say which side each is on.  The library never
  *     allocates device memory: the caller owns every buffer, including the
  *     workspace, whose size the matching *_workspace_bytes query returns.
  *   - Work is enqueued asynchronously on `stream` (NULL = legacy default
@@ -44,7 +45,10 @@
  *     CUDA call failed at launch).  Device-side failures (a bounded wait that
  *     ran out) set a device status word read by sage_get_device_status.
  *   - The calls are thread-safe.  Calls that share a workspace or outputs
- *     must be ordered by the caller (same stream or events).
+ *     must be ordered by the caller (same stream or events).  Library state:
+ *     the kernels' shared-memory opt-ins (set once) and, for
+ *     sage_attn_fwd_host, two copy streams and a few events per device,
+ *     created on first use and kept for the life of the process.
  */
 #ifndef SAGE_B200_H
 #define SAGE_B200_H
@@ -224,6 +228,47 @@ sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage
                           int smooth_k, const sage_mask* mask, void* out, int64_t out_sb,
                           int64_t out_sh, int64_t out_sn, float* lse, void* ws,
                           size_t ws_bytes, sage_stream_t stream);
+
+/* ------------------------------------------------------- host-resident inputs */
+/* Workspace bytes of sage_attn_fwd_host for chunks of `chunk_groups` (batch
+ * entry, KV head) groups (0 = automatic, about 64 MB of inputs per chunk):
+ * three staging slots, each holding one chunk's Q/K/V, output and LSE, plus
+ * the quantise + attend workspace of one chunk.  mask as for the call (only
+ * its B and H matter).  0 for invalid sizes. */
+size_t sage_attn_fwd_host_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
+                                          int64_t Nk, int64_t D, const sage_mask* mask,
+                                          int64_t chunk_groups);
+
+/* sage_attn_fwd for Q/K/V and outputs held in HOST memory ("sageattn" with
+ * tensors that live on the host): the same arguments and results as
+ * sage_attn_fwd, with these differences.
+ *   q, k, v:  HOST tensors (sage_tensor ptr is a host address; same shapes,
+ *             strides and alignment rules as sage_attn_fwd; q, k and v share
+ *             the dtype);
+ *   out, lse: HOST buffers, out with element strides (out_sb, out_sh, out_sn),
+ *             lse [B, Hq, Nq] contiguous fp32 (written iff return_lse);
+ *   mask:     DEVICE memory, as in sage_attn_fwd (or NULL);
+ *   chunk_groups: (batch entry, KV head) groups per chunk, 0 = automatic;
+ *   ws:       DEVICE workspace (256-byte aligned) of
+ *             sage_attn_fwd_host_workspace_bytes(..., chunk_groups) bytes.
+ * The problem is streamed through the GPU a chunk at a time.  Each group is a
+ * problem of its own (its K mean, V channel scales and Q blocks), so the
+ * result equals sage_attn_fwd's bit for bit.  The copies of later and
+ * earlier chunks run on two library-owned streams, overlapped with the
+ * kernels of the current chunk, which run on `stream`; `stream` waits for
+ * every copy before it proceeds, so an event recorded on `stream` after the
+ * call completes after the last byte has reached `out` and `lse`.
+ * The host buffers must stay valid and unmodified until then.  Page-locked
+ * host memory is needed for the copies to overlap; pageable memory gives the
+ * same result with the copies serialised by the driver.  Concurrent calls are
+ * serialised while they enqueue (the copy streams are shared per device).
+ * On SAGE_ERR_CUDA, work already enqueued still runs and `stream` still waits
+ * for it; out and lse are then undefined. */
+sage_status sage_attn_fwd_host(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                               int causal, float sm_scale, int num_kv_heads, int return_lse,
+                               int smooth_k, const sage_mask* mask, void* out, int64_t out_sb,
+                               int64_t out_sh, int64_t out_sn, float* lse, int64_t chunk_groups,
+                               void* ws, size_t ws_bytes, sage_stream_t stream);
 
 /* --------------------------------------------------------- variable length */
 /* Workspace bytes of sage_attn_fwd_varlen: the sequence table, quantised

@@ -93,6 +93,12 @@ def lib():
                                          ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          P(SageMask), _vp, _i64, _i64, _i64, _vp, _vp,
                                          ctypes.c_size_t, _vp]),
+        "sage_attn_fwd_host_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, _i64, _i64, _i64,
+                                                                 P(SageMask), _i64]),
+        "sage_attn_fwd_host": (ctypes.c_int, [P(SageTensor), P(SageTensor), P(SageTensor), ctypes.c_int,
+                                              ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              P(SageMask), _vp, _i64, _i64, _i64, _vp, _i64, _vp,
+                                              ctypes.c_size_t, _vp]),
         "sage_attn_fwd_varlen_workspace_bytes": (ctypes.c_size_t, [_i64] * 8 + [ctypes.c_int]),
         "sage_attn_fwd_varlen": (ctypes.c_int, [P(SageTensor), P(SageTensor), P(SageTensor), _vp, _vp,
                                                 _i64, _i64, _i64, ctypes.c_int, ctypes.c_float,
@@ -310,6 +316,68 @@ def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, num_kv_heads=None, retur
                            int(bool(return_lse)), int(bool(smooth_k)), mstruct, to.ptr, to.sb,
                            to.sh, to.sn, lse.data_ptr() if return_lse else None, ws.data_ptr(),
                            ws.numel(), _stream(q.device)), "sage_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def sage_attn_fwd_host_workspace_bytes(B, Hq, Hkv, Nq, Nk, D, mask_shape=None, chunk_groups=0):
+    """Device workspace bytes of sage_attn_fwd_host (mask_shape: the mask's
+    leading (B, H) or None)."""
+    m = None
+    if mask_shape is not None:
+        m = ctypes.byref(SageMask(None, mask_shape[0], mask_shape[1], Nq, Nk, 0, 0, Nk,
+                                  SAGE_MASK_BOOL))
+    return lib().sage_attn_fwd_host_workspace_bytes(B, Hq, Hkv, Nq, Nk, D, m, chunk_groups)
+
+
+def sage_attn_fwd_host(q, k, v, causal=False, sm_scale=None, num_kv_heads=None, return_lse=False,
+                       smooth_k=True, mask=None, layout="HND", out=None, lse=None, ws=None,
+                       chunk_groups=0, device=None):
+    """The whole path on bf16/fp16 Q/K/V held in host memory
+    (sage_attn_fwd_host): the problem is streamed through the GPU in chunks of
+    (batch entry, KV head) groups with the copies overlapped with the
+    kernels.  q/k/v and out/lse are CPU tensors (page-locked for the
+    overlap; out and lse are allocated page-locked when not given); mask, if
+    any, is a CUDA tensor.  Work is enqueued on the current stream of
+    `device` (default: the current device); synchronise it before reading
+    out.  Returns out (q's shape, layout and dtype) and, with return_lse,
+    lse [B, Hq, Nq] fp32."""
+    L = lib()
+    for t in (q, k, v):
+        if t.is_cuda:
+            raise ValueError("sage_attn_fwd_host takes host tensors (use sage_attn_fwd for CUDA tensors)")
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
+    if num_kv_heads is None:
+        num_kv_heads = tk.H
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if out.is_cuda:
+        raise ValueError("out must be a host tensor")
+    to = _as_tensor(out, layout)
+    if return_lse:
+        if lse is None:
+            lse = torch.empty(tq.B, tq.H, tq.N, dtype=torch.float32, pin_memory=True)
+        if lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous() or \
+                lse.numel() != tq.B * tq.H * tq.N:
+            raise ValueError("lse must be a contiguous fp32 host tensor [B, Hq, Nq]")
+    mk = _as_mask(mask, tq.B, tq.H, tq.N, tk.N)
+    if mk is not None and not mask.is_cuda:
+        raise ValueError("mask must be a CUDA tensor")
+    mstruct = ctypes.byref(mk[0]) if mk else None
+    nbytes = L.sage_attn_fwd_host_workspace_bytes(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D, mstruct,
+                                                  int(chunk_groups))
+    if nbytes == 0:
+        raise SageError(SAGE_ERR_INVALID_ARG, "sage_attn_fwd_host: invalid sizes")
+    if ws is None or ws.numel() < nbytes:
+        ws = _ws(nbytes, device)
+    with torch.cuda.device(device):
+        _check(L.sage_attn_fwd_host(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                                    int(bool(causal)), float(sm_scale) if sm_scale else 0.0,
+                                    int(num_kv_heads), int(bool(return_lse)), int(bool(smooth_k)),
+                                    mstruct, to.ptr, to.sb, to.sh, to.sn,
+                                    lse.data_ptr() if return_lse else None, int(chunk_groups),
+                                    ws.data_ptr(), ws.numel(), _stream(device)),
+               "sage_attn_fwd_host")
     return (out, lse) if return_lse else out
 
 

@@ -589,6 +589,234 @@ sage_status check_packed(const sage_tensor* t) {
   return SAGE_OK;
 }
 
+// ---------------------------------------------------------------- fused path
+// Quantise into the workspace laid out by `f` (at `w`), then attend.
+sage_status run_fused(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v, int causal,
+                      float sm_scale, int return_lse, int smooth_k, const sage_mask* mask,
+                      void* out, int64_t out_sb, int64_t out_sh, int64_t out_sn, float* lse,
+                      const FusedLayout& f, char* w, cudaStream_t stream) {
+  sage_status st;
+  sage_qkv_i8f8 z{};
+  z.q = reinterpret_cast<int8_t*>(w + f.q8);
+  z.q_scale = reinterpret_cast<float*>(w + f.qs);
+  z.k = reinterpret_cast<int8_t*>(w + f.k8);
+  z.k_scale = reinterpret_cast<float*>(w + f.ks);
+  z.k_mean = reinterpret_cast<float*>(w + f.km);
+  z.v = reinterpret_cast<uint8_t*>(w + f.v8);
+  z.v_scale = reinterpret_cast<float*>(w + f.vs);
+  z.q_dot_kmean = return_lse ? reinterpret_cast<float*>(w + f.qdk) : nullptr;
+  z.B = q->B; z.Hq = q->H; z.Hkv = k->H; z.Nq = q->N; z.Nk = k->N; z.D = q->D;
+  if ((st = run_quantize(q, k, v, smooth_k, &z, w + f.part, f.cls - f.part, stream))) return st;
+  return run_attention(&z, causal, sm_scale, return_lse, mask, out, q->dtype, out_sb, out_sh,
+                       out_sn, lse, w + f.cls, f.total - f.cls, stream);
+}
+
+// ---------------------------------------------------------------- host pipeline
+// sage_attn_fwd_host streams a problem held in host memory through the GPU in
+// chunks of (batch entry, KV head) groups.  Every group is a problem of its
+// own (its K mean, its V channel scales, the 128-token blocks of its Q heads),
+// so a chunk computed alone gives the bits the whole call gives.  Chunk c
+// passes through three streams:
+//   copy-in stream:  Q/K/V of chunk c into input slot c % kPipeSlots;
+//   caller's stream: quantise + attend chunk c into output slot c % kPipeSlots;
+//   copy-out stream: output slot to the host out / lse;
+// so the copy in of a later chunk, the kernels of chunk c and the copy out of
+// an earlier chunk overlap (the host link carries both directions at once).
+constexpr int kPipeSlots = 3;
+constexpr int kPipeRing = kPipeSlots + 1;            // events of one kind in flight
+constexpr size_t kPipeChunkInBytes = size_t(64) << 20;  // automatic chunk: input bytes
+constexpr int kPipeMaxDevices = 64;
+
+// Staging order of heads [h0, h0 + nh) of one batch entry: token-major
+// ([N, nh, D]) when the caller's tensor keeps all heads of a token together
+// in one row (head stride D, token stride at least H * D: the NHD layout),
+// else head-major ([nh, N, D]).
+bool token_major(int64_t H, int64_t D, int64_t sh, int64_t sn) {
+  return H > 1 && sh == D && sn >= H * D;
+}
+struct Stage {
+  int64_t sh, sn;
+};
+Stage stage_of(bool tm, int64_t N, int64_t nh, int64_t D) {
+  return tm ? Stage{D, nh * D} : Stage{N * D, D};
+}
+
+// Heads [h0, h0 + nh) of batch entry b between the caller's strided tensor
+// (host side) and its contiguous staging copy (device side).
+cudaError_t copy_heads(char* dev, char* host, bool tm, int64_t sb, int64_t sh, int64_t sn,
+                       int64_t b, int64_t h0, int64_t nh, int64_t N, int64_t D, size_t es,
+                       bool to_dev, cudaStream_t s) {
+  char* hb = host + (b * sb + h0 * sh) * (int64_t)es;
+  auto copy2d = [&](char* d, char* h, size_t width, size_t dpitch, size_t hpitch, size_t rows) {
+    return to_dev ? cudaMemcpy2DAsync(d, dpitch, h, hpitch, width, rows, cudaMemcpyDefault, s)
+                  : cudaMemcpy2DAsync(h, hpitch, d, dpitch, width, rows, cudaMemcpyDefault, s);
+  };
+  if (tm)  // token-major: one 2-D copy, a row per token
+    return copy2d(dev, hb, nh * D * es, nh * D * es, sn * es, N);
+  if (sn == D && sh == N * D)  // the chunk's heads are one contiguous range
+    return copy2d(dev, hb, nh * N * D * es, nh * N * D * es, nh * N * D * es, 1);
+  for (int64_t i = 0; i < nh; ++i) {
+    const cudaError_t e =
+        copy2d(dev + i * N * D * (int64_t)es, hb + i * sh * (int64_t)es, D * es, D * es, sn * es, N);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// The caller's mask restricted to heads [h0, h0 + nh) of batch entry b.
+sage_mask chunk_mask(const sage_mask& m, int64_t b, int64_t h0, int64_t nh) {
+  sage_mask c = m;
+  const int64_t el = (m.B > 1 ? b * m.sb : 0) + (m.H > 1 ? h0 * m.sh : 0);
+  c.ptr = static_cast<const char*>(m.ptr) + el * (m.kind == SAGE_MASK_FLOAT ? 4 : 1);
+  c.B = 1;
+  c.H = m.H > 1 ? nh : 1;
+  return c;
+}
+
+struct PipeLayout {
+  int64_t gpc;                 // KV-head groups per chunk
+  size_t q, k, v, o, l, slot;  // offsets in a slot, slot bytes
+  size_t fused, total;         // one chunk's quantise + attend workspace
+};
+
+PipeLayout pipe_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
+                       const sage_mask* mask, int64_t chunk_groups) {
+  const int64_t G = Hq / Hkv;
+  const size_t per_group = (size_t)(G * Nq + 2 * Nk) * D * 2;
+  int64_t gpc = chunk_groups > 0 ? chunk_groups
+                                  : std::max<int64_t>(1, (int64_t)(kPipeChunkInBytes / per_group));
+  gpc = std::min(gpc, Hkv);
+  PipeLayout p{};
+  p.gpc = gpc;
+  size_t o = 0;
+  p.q = o; o += align256((size_t)gpc * G * Nq * D * 2);
+  p.k = o; o += align256((size_t)gpc * Nk * D * 2);
+  p.v = o; o += align256((size_t)gpc * Nk * D * 2);
+  p.o = o; o += align256((size_t)gpc * G * Nq * D * 2);
+  p.l = o; o += align256((size_t)gpc * G * Nq * 4);
+  p.slot = o;
+  p.fused = kPipeSlots * p.slot;
+  size_t fw = 0;
+  for (const int64_t ng : {gpc, Hkv % gpc}) {  // full chunks and the last of a batch entry
+    if (ng == 0) continue;
+    sage_mask cm{};
+    if (mask) cm = chunk_mask(*mask, 0, 0, ng * G);
+    fw = std::max(fw, fused_layout(1, ng * G, ng, Nq, Nk, D, mask ? &cm : nullptr).total);
+  }
+  p.total = p.fused + fw;
+  return p;
+}
+
+// Copy streams and events, created once per device on first use.
+struct PipeStreams {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, join_in = nullptr, join_out = nullptr;
+  cudaEvent_t copied[kPipeRing], computed[kPipeRing], drained[kPipeRing];
+};
+std::mutex g_pipe_mu;  // held while a call enqueues (the events are shared)
+PipeStreams g_pipe[kPipeMaxDevices];
+
+sage_status pipe_streams(PipeStreams** res) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kPipeMaxDevices)
+    return SAGE_ERR_CUDA;
+  PipeStreams& p = g_pipe[dev];
+  if (!p.in) {
+    PipeStreams n;
+    bool ok = cudaStreamCreateWithFlags(&n.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&n.out, cudaStreamNonBlocking) == cudaSuccess;
+    cudaEvent_t* evs[] = {&n.start, &n.join_in, &n.join_out};
+    for (cudaEvent_t* e : evs)
+      ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < kPipeRing; ++i)
+      ok = ok && cudaEventCreateWithFlags(&n.copied[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&n.computed[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&n.drained[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) return SAGE_ERR_CUDA;  // a failed creation leaks what it made; it does not recur
+    p = n;
+  }
+  *res = &p;
+  return SAGE_OK;
+}
+
+sage_status run_host_pipeline(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                              int causal, float sm_scale, int return_lse, int smooth_k,
+                              const sage_mask* mask, void* out, int64_t out_sb, int64_t out_sh,
+                              int64_t out_sn, float* lse, const PipeLayout& p, char* w,
+                              cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  PipeStreams* ps = nullptr;
+  sage_status st = pipe_streams(&ps);
+  if (st) return st;
+  const int64_t B = q->B, Hq = q->H, Hkv = k->H, Nq = q->N, Nk = k->N, D = q->D;
+  const int64_t G = Hq / Hkv;
+  const size_t es = 2;
+  char* hq = static_cast<char*>(const_cast<void*>(q->ptr));
+  char* hk = static_cast<char*>(const_cast<void*>(k->ptr));
+  char* hv = static_cast<char*>(const_cast<void*>(v->ptr));
+  char* ho = static_cast<char*>(out);
+  const bool tq = token_major(Hq, D, q->sh, q->sn), tk = token_major(Hkv, D, k->sh, k->sn),
+             tv = token_major(Hkv, D, v->sh, v->sn), to = token_major(Hq, D, out_sh, out_sn);
+  bool ok = cudaEventRecord(ps->start, stream) == cudaSuccess &&
+            cudaStreamWaitEvent(ps->in, ps->start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(ps->out, ps->start, 0) == cudaSuccess;
+  int64_t c = 0;
+  for (int64_t b = 0; ok && b < B; ++b) {
+    for (int64_t g0 = 0; ok && g0 < Hkv; g0 += p.gpc, ++c) {
+      const int64_t ng = std::min(p.gpc, Hkv - g0), nh = ng * G, h0 = g0 * G;
+      const int r = (int)(c % kPipeRing);
+      char* sl = w + (c % kPipeSlots) * p.slot;
+      // copy in, once the chunk that last used this slot has been computed
+      if (c >= kPipeSlots)
+        ok = cudaStreamWaitEvent(ps->in, ps->computed[(c - kPipeSlots) % kPipeRing], 0) ==
+             cudaSuccess;
+      ok = ok && copy_heads(sl + p.q, hq, tq, q->sb, q->sh, q->sn, b, h0, nh, Nq, D, es, true,
+                            ps->in) == cudaSuccess;
+      ok = ok && copy_heads(sl + p.k, hk, tk, k->sb, k->sh, k->sn, b, g0, ng, Nk, D, es, true,
+                            ps->in) == cudaSuccess;
+      ok = ok && copy_heads(sl + p.v, hv, tv, v->sb, v->sh, v->sn, b, g0, ng, Nk, D, es, true,
+                            ps->in) == cudaSuccess;
+      ok = ok && cudaEventRecord(ps->copied[r], ps->in) == cudaSuccess;
+      // quantise + attend, once the output slot has been drained
+      ok = ok && cudaStreamWaitEvent(stream, ps->copied[r], 0) == cudaSuccess;
+      if (ok && c >= kPipeSlots)
+        ok = cudaStreamWaitEvent(stream, ps->drained[(c - kPipeSlots) % kPipeRing], 0) ==
+             cudaSuccess;
+      if (!ok) break;
+      const Stage sq = stage_of(tq, Nq, nh, D), sk = stage_of(tk, Nk, ng, D),
+                  sv = stage_of(tv, Nk, ng, D), so = stage_of(to, Nq, nh, D);
+      const sage_tensor cq{sl + p.q, q->dtype, 1, nh, Nq, D, nh * Nq * D, sq.sh, sq.sn};
+      const sage_tensor ck{sl + p.k, k->dtype, 1, ng, Nk, D, ng * Nk * D, sk.sh, sk.sn};
+      const sage_tensor cv{sl + p.v, v->dtype, 1, ng, Nk, D, ng * Nk * D, sv.sh, sv.sn};
+      sage_mask cm{};
+      if (mask) cm = chunk_mask(*mask, b, h0, nh);
+      const FusedLayout f = fused_layout(1, nh, ng, Nq, Nk, D, mask ? &cm : nullptr);
+      st = run_fused(&cq, &ck, &cv, causal, sm_scale, return_lse, smooth_k, mask ? &cm : nullptr,
+                     sl + p.o, nh * Nq * D, so.sh, so.sn,
+                     return_lse ? reinterpret_cast<float*>(sl + p.l) : nullptr, f, w + p.fused,
+                     stream);
+      if (st) break;
+      ok = cudaEventRecord(ps->computed[r], stream) == cudaSuccess;
+      // copy out
+      ok = ok && cudaStreamWaitEvent(ps->out, ps->computed[r], 0) == cudaSuccess;
+      ok = ok && copy_heads(sl + p.o, ho, to, out_sb, out_sh, out_sn, b, h0, nh, Nq, D, es, false,
+                            ps->out) == cudaSuccess;
+      if (ok && return_lse)
+        ok = cudaMemcpyAsync(lse + (b * Hq + h0) * Nq, sl + p.l, (size_t)nh * Nq * 4,
+                             cudaMemcpyDefault, ps->out) == cudaSuccess;
+      ok = ok && cudaEventRecord(ps->drained[r], ps->out) == cudaSuccess;
+    }
+  }
+  // the caller's stream continues only after everything enqueued on the copy
+  // streams, whatever happened above
+  const bool joined = cudaEventRecord(ps->join_in, ps->in) == cudaSuccess &&
+                      cudaEventRecord(ps->join_out, ps->out) == cudaSuccess &&
+                      cudaStreamWaitEvent(stream, ps->join_in, 0) == cudaSuccess &&
+                      cudaStreamWaitEvent(stream, ps->join_out, 0) == cudaSuccess;
+  if (st) return st;
+  return ok && joined ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -661,20 +889,41 @@ sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage
   const FusedLayout f = fused_layout(q->B, q->H, k->H, q->N, k->N, q->D, mask);
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SAGE_ERR_INVALID_ARG;
   if (ws_bytes < f.total) return SAGE_ERR_WORKSPACE;
-  char* w = static_cast<char*>(ws);
-  sage_qkv_i8f8 z{};
-  z.q = reinterpret_cast<int8_t*>(w + f.q8);
-  z.q_scale = reinterpret_cast<float*>(w + f.qs);
-  z.k = reinterpret_cast<int8_t*>(w + f.k8);
-  z.k_scale = reinterpret_cast<float*>(w + f.ks);
-  z.k_mean = reinterpret_cast<float*>(w + f.km);
-  z.v = reinterpret_cast<uint8_t*>(w + f.v8);
-  z.v_scale = reinterpret_cast<float*>(w + f.vs);
-  z.q_dot_kmean = return_lse ? reinterpret_cast<float*>(w + f.qdk) : nullptr;
-  z.B = q->B; z.Hq = q->H; z.Hkv = k->H; z.Nq = q->N; z.Nk = k->N; z.D = q->D;
-  if ((st = run_quantize(q, k, v, smooth_k, &z, w + f.part, f.cls - f.part, stream))) return st;
-  return run_attention(&z, causal, sm_scale, return_lse, mask, out, q->dtype, out_sb, out_sh,
-                       out_sn, lse, w + f.cls, f.total - f.cls, stream);
+  return run_fused(q, k, v, causal, sm_scale, return_lse, smooth_k, mask, out, out_sb, out_sh,
+                   out_sn, lse, f, static_cast<char*>(ws), stream);
+}
+
+size_t sage_attn_fwd_host_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
+                                          int64_t Nk, int64_t D, const sage_mask* mask,
+                                          int64_t chunk_groups) {
+  if (!valid_dims(B, Hq, Nq, D) || !valid_dims(B, Hkv, Nk, D) || Hq % Hkv || chunk_groups < 0)
+    return 0;
+  return pipe_layout(B, Hq, Hkv, Nq, Nk, D, mask, chunk_groups).total;
+}
+
+sage_status sage_attn_fwd_host(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                               int causal, float sm_scale, int num_kv_heads, int return_lse,
+                               int smooth_k, const sage_mask* mask, void* out, int64_t out_sb,
+                               int64_t out_sh, int64_t out_sn, float* lse, int64_t chunk_groups,
+                               void* ws, size_t ws_bytes, sage_stream_t stream) {
+  sage_status st;
+  if ((st = check_tensor(q)) || (st = check_tensor(k)) || (st = check_tensor(v))) return st;
+  if (num_kv_heads != k->H || k->dtype != q->dtype || v->dtype != q->dtype)
+    return SAGE_ERR_INVALID_ARG;
+  if (k->B != q->B || v->B != q->B || v->H != k->H || v->N != k->N || k->D != q->D ||
+      v->D != q->D)
+    return SAGE_ERR_INVALID_ARG;
+  if ((st = check_qkv_shapes(q->B, q->H, k->H, q->N, k->N, q->D))) return st;
+  if ((st = check_mask(mask, q->B, q->H, q->N, k->N))) return st;
+  if (!out || chunk_groups < 0 || (return_lse && !lse)) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(out) || out_sn < q->D || out_sn % 8 || out_sh % 8 || out_sb % 8 || out_sh < 0 ||
+      out_sb < 0)
+    return SAGE_ERR_INVALID_ARG;
+  const PipeLayout p = pipe_layout(q->B, q->H, k->H, q->N, k->N, q->D, mask, chunk_groups);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < p.total) return SAGE_ERR_WORKSPACE;
+  return run_host_pipeline(q, k, v, causal, sm_scale, return_lse, smooth_k, mask, out, out_sb,
+                           out_sh, out_sn, lse, p, static_cast<char*>(ws), stream);
 }
 
 size_t sage_quantize_nvfp4_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,

@@ -192,3 +192,51 @@ def test_varlen_rejects_bad_arguments_on_host(L):
     assert call(q=_t(B=1, H=4, N=1000, D=96), k=_t(B=1, H=2, N=900, D=96),
                 v=_t(B=1, H=2, N=900, D=96)) == S.SAGE_ERR_UNSUPPORTED      # head_dim 96
     assert L.sage_attn_fwd_varlen_workspace_bytes(0, 4, 2, 1000, 900, 512, 512, 64, 1) == 0
+
+
+def test_host_call_rejects_bad_arguments_on_host(L):
+    byref = ctypes.byref
+    q, k, v = _t(H=4), _t(H=2), _t(H=2)
+    f = L.sage_attn_fwd_host
+    need = L.sage_attn_fwd_host_workspace_bytes(1, 4, 2, 256, 256, 64, None, 0)
+    assert need > 0
+    ok = dict(q=q, k=k, v=v, nkv=2, lse_flag=1, out=256, sn=64, sh=256 * 64, lse=512, chunk=0,
+              ws=256, nb=need)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(byref(a["q"]), byref(a["k"]), byref(a["v"]), 1, 0.0, a["nkv"], a["lse_flag"], 1, None,
+                 a["out"], 4 * 256 * 64, a["sh"], a["sn"], a["lse"], a["chunk"], a["ws"], a["nb"], None)
+    assert call(nkv=3) == S.SAGE_ERR_INVALID_ARG                     # num_kv_heads != k.H
+    assert call(k=_t(H=2, dtype=1)) == S.SAGE_ERR_INVALID_ARG        # k dtype differs from q
+    assert call(v=_t(H=2, N=128)) == S.SAGE_ERR_INVALID_ARG          # v length differs from k
+    assert call(lse=0) == S.SAGE_ERR_INVALID_ARG                     # return_lse without lse
+    assert call(out=0) == S.SAGE_ERR_INVALID_ARG
+    assert call(sn=60) == S.SAGE_ERR_INVALID_ARG                     # out token stride
+    assert call(chunk=-1) == S.SAGE_ERR_INVALID_ARG
+    assert call(ws=0) == S.SAGE_ERR_INVALID_ARG
+    assert call(ws=384) == S.SAGE_ERR_INVALID_ARG                    # workspace not 256-aligned
+    assert call(nb=need - 1) == S.SAGE_ERR_WORKSPACE
+    assert call(q=_t(H=4, D=96), k=_t(H=2, D=96), v=_t(H=2, D=96)) == S.SAGE_ERR_UNSUPPORTED
+    assert L.sage_attn_fwd_host_workspace_bytes(1, 4, 2, 256, 256, 64, None, -1) == 0
+    assert L.sage_attn_fwd_host_workspace_bytes(1, 3, 2, 256, 256, 64, None, 0) == 0
+
+
+def test_host_call_workspace_is_three_chunk_slots_plus_one_chunk_workspace(L):
+    B_, Hq, Hkv, N, D = 4, 32, 8, 16384, 128
+    G = Hq // Hkv
+    # automatic chunk: as many KV-head groups as fit 64 MB of bf16 inputs (2 here)
+    per_group_in = (G * N + 2 * N) * D * 2
+    gpc = max(1, (64 << 20) // per_group_in)
+    assert gpc == 2
+    slot = gpc * (G * N * D * 2 + 2 * N * D * 2 + G * N * D * 2 + G * N * 4)
+    one_chunk = L.sage_attn_fwd_workspace_bytes(1, gpc * G, gpc, N, N, D, None)
+    need = L.sage_attn_fwd_host_workspace_bytes(B_, Hq, Hkv, N, N, D, None, 0)
+    assert need == pytest.approx(3 * slot + one_chunk, abs=3 * 5 * 256)
+    # explicit chunking, with a smaller last chunk per batch entry (8 = 3 + 3 + 2)
+    need3 = L.sage_attn_fwd_host_workspace_bytes(B_, Hq, Hkv, N, N, D, None, 3)
+    assert need3 == pytest.approx(3 * slot * 3 // 2 + L.sage_attn_fwd_workspace_bytes(
+        1, 3 * G, 3, N, N, D, None), abs=3 * 5 * 256 + 4096)
+    # one chunk of everything when the chunk size exceeds the heads
+    assert L.sage_attn_fwd_host_workspace_bytes(1, 4, 2, 256, 256, 64, None, 99) == \
+        L.sage_attn_fwd_host_workspace_bytes(1, 4, 2, 256, 256, 64, None, 2)
