@@ -116,7 +116,8 @@ struct AttnLayout {
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + ATT_STAGES * K_BYTES;
   static constexpr int OFF_P = OFF_V + ATT_STAGES * V_BYTES;   // [warpgroup][buffer]
-  static constexpr int OFF_BAR = OFF_P + 4 * P_BYTES;
+  static constexpr int OFF_INIT = OFF_P + 4 * P_BYTES;   // f16 A (4 KB) and B (4 KB) of the S init
+  static constexpr int OFF_BAR = OFF_INIT + 8192;
   // q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2][2],
   // o_ready[2][2], mma_done
   static constexpr int NBAR = 1 + 2 * ATT_STAGES + 2 + 2 + 4 + 4 + 1;
@@ -135,9 +136,9 @@ struct AttnLayout {
 // 16K workload without it), so the period is set beyond the 16 pairs of a
 // chunk: every exponential is MUFU.
 constexpr int POLY_EVERY = 1000;
-// int32 score S as the float 1.5*2^23 + S (exact for |S| < 2^22): the bit
-// pattern of 1.5*2^23 plus S.
-constexpr uint32_t MAGIC_I = 0x4B400000u;
+// int32 score S as the float 1.5*2^23 + S (exact for |S| < 2^22): the QK^T
+// MMA accumulates the int32 S onto the bit pattern of 1.5*2^23 (0x4B400000),
+// which an f16 MMA (512 x 1536 summed over K = 16) writes into S first.
 constexpr float MAGIC_F = 12582912.0f;
 
 // Write one thread's row of 128 E4M3 probabilities (32 packed words) into a
@@ -328,6 +329,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint8_t* sV = smem + L::OFF_V;
   uint8_t* sP = smem + L::OFF_P;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint8_t* sInit = smem + L::OFF_INIT;
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + ATT_STAGES;
@@ -403,6 +405,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     prefetch_tmap(&tmV);
   }
   for (int c = threadIdx.x; c < D; c += blockDim.x) s_vs[c] = a.v_scale[(int64_t)bhk * D + c];
+  // operands of the S init: f16 512.0 (0x6000) everywhere in A, 1536.0
+  // (0x6600) in B; K = 16 products of 786432 sum exactly to 1.5*2^23
+  for (int i = threadIdx.x; i < 2048; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(sInit)[i] = i < 1024 ? 0x60006000u : 0x66006600u;
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -434,9 +441,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // One thread polls the barriers and issues, per Q tile i, the ops
     // QK(0), QK(1), PV(0), QK(2), PV(1), ... in order, whichever Q tile is
     // ready first.  A stage of the K/V ring is released once both Q tiles
-    // have issued their PV on it.
+    // have issued their PV on it.  Each QK(n) starts with an f16 MMA that
+    // overwrites S with 1.5*2^23 (every operand element equal, so the
+    // operand layout does not matter); the int8 MMAs accumulate onto it.
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = instr_desc(kDS32, kS8, kS8, ATT_BM, ATT_BN);
+      constexpr uint32_t IDESC_INIT = instr_desc(kDF32, 0u, 0u, ATT_BM, ATT_BN);
+      const uint64_t dInitA = smem_desc(smem_u32(sInit), 256, 32);
+      const uint64_t dInitB = smem_desc(smem_u32(sInit) + 4096, 256, 32);
       constexpr uint32_t IDESC_PV = instr_desc(kDF32, kE4M3, kE4M3, ATT_BM, D) | kBMajorMN;
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
       auto next_active = [&](int i, int from) {
@@ -461,6 +473,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             tc_fence_after();
             const uint32_t tS = tmem + (uint32_t)(i * 256);
             const uint32_t qa = aQ + i * L::Q_BYTES, ka = aK + (e % ATT_STAGES) * L::K_BYTES;
+            mma_f16(tS, dInitA, dInitB, IDESC_INIT, 0u);
 #pragma unroll
             for (int k = 0; k < D / 32; ++k)
               mma_i8(tS, smem_desc(qa + 32 * k, L::QK_SBO, L::QK_SWIZZLE),
@@ -531,13 +544,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const int64_t el = (int64_t)bm * a.m_sb + (int64_t)hm * a.m_sh + (int64_t)row * a.m_sq;
       mrow = reinterpret_cast<const uint8_t*>(a.mask) + el * (a.mask_kind ? 4 : 1);
     }
-    // S accumulators start at 1.5*2^23 (as int32 bits): the int32 QK^T sum
-    // on top of it is then directly the float 1.5*2^23 + S.  The refill
-    // counts as the first release of S.
-#pragma unroll
-    for (int cb = 0; cb < 128; cb += 32) SAGE_TMEM_ST32_SPLAT(tS + cb, MAGIC_I);
-    tmem_wait_st();
-    tc_fence_before();
+    // S starts free; each QK^T is preceded by an f16 MMA that sets S to
+    // 1.5*2^23, so the int32 sum on top reads as the float 1.5*2^23 + S.
     mbar_arrive(&s_free[wg]);
     float m_ref = -INFINITY, l = 0.f;
     uint32_t n = 0;
@@ -560,10 +568,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       SAGE_TMEM_LD32(tS + 64, (sr + 64));
       SAGE_TMEM_LD32(tS + 96, (sr + 96));
       tmem_wait_ld();
-      // refill S with 1.5*2^23 for the next QK^T, which accumulates on top
-#pragma unroll
-      for (int cb = 0; cb < 128; cb += 32) SAGE_TMEM_ST32_SPLAT(tS + cb, MAGIC_I);
-      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&s_free[wg]);
 
