@@ -125,15 +125,22 @@ struct AttnLayout {
   static constexpr int OFF_VS = (OFF_TMEM + 16 + 15) / 16 * 16;
   static constexpr int OFF_NLIST = OFF_VS + D * 4;
   static constexpr int OFF_LIST = OFF_NLIST + 16;
-  static size_t bytes(int nkt) { return 1024 + OFF_LIST + (size_t)nkt * 4; }
+  // the list of visible key tiles, then their K scales
+  static constexpr size_t bytes(int nkt) { return 1024 + OFF_LIST + (size_t)nkt * 8; }
 };
+// the longest key list must fit the 227 KB of shared memory a CTA can have
+static_assert(AttnLayout<128>::bytes(ATT_MAX_NKT) <= 232448, "attention smem");
+static_assert(AttnLayout<64>::bytes(ATT_MAX_NKT) <= 232448, "attention smem");
 
 // Exponentials: pairs i of each 32-key chunk with i % POLY_EVERY ==
 // POLY_EVERY - 1 would be computed by the FMA-pipe polynomial instead of MUFU
 // ex2.  Measured on B200 this kernel is not MUFU-throughput bound (MUFU about
 // half busy), and the polynomial's extra instructions, its clamp among them,
 // cost more than the MUFU time they save (8.43 -> 7.81 ms on the causal GQA
-// 16K workload without it), so the period is set beyond the 16 pairs of a
+// 16K workload without it).  A clamp-free degree-3 polynomial (sat-FMA
+// clamp, relative error 8e-5) on one pair in 8 gained under 1 % and moved
+// enough E4M3 roundings of P to break the parity bound on a small case; on
+// one pair in 4 it was slower.  The period is set beyond the 16 pairs of a
 // chunk: every exponential is MUFU.
 constexpr int POLY_EVERY = 1000;
 // int32 score S as the float 1.5*2^23 + S (exact for |S| < 2^22): the QK^T
@@ -342,6 +349,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   float* s_vs = reinterpret_cast<float*>(smem + L::OFF_VS);
   int* s_nlist = reinterpret_cast<int*>(smem + L::OFF_NLIST);
   uint32_t* s_list = reinterpret_cast<uint32_t*>(smem + L::OFF_LIST);
+  float* s_ks = reinterpret_cast<float*>(s_list + a.nkt);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int qp, b, h;
@@ -370,7 +378,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (has1) f |= tile_flags(a, cs, b, h, qt0 + 1, 1, kt);
       }
       const unsigned bal = __ballot_sync(0xffffffffu, (f & 3u) != 0);
-      if (f & 3u) s_list[count + __popc(bal & ((1u << lane) - 1u))] = ((uint32_t)kt << 8) | f;
+      if (f & 3u) {
+        const int pos = count + __popc(bal & ((1u << lane) - 1u));
+        s_list[pos] = ((uint32_t)kt << 8) | f;
+        s_ks[pos] = a.k_scale[cs.ks0 + kt];
+      }
       count += __popc(bal);
       orf |= f;
     }
@@ -556,7 +568,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const int kt = (int)(e >> 8);
       const bool need = (e >> (2 + wg)) & 1u;
       const bool part = (e >> (4 + wg)) & 1u;
-      const float c = cq * a.k_scale[cs.ks0 + kt];
+      const float c = cq * s_ks[idx];
       const uint32_t buf = n & 1u;
       uint8_t* ptile = sP + (wg * 2 + buf) * L::P_BYTES;
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], n & 1, SITE_S_FULL));
