@@ -256,8 +256,14 @@ __device__ __forceinline__ void tile_visibility(const AttnArgs& a, const CtaSeq&
         vis[q >> 1] &= ~(((~bits) & 0xFFFFu) << (16 * (q & 1)));
       }
     } else {
-      for (int j = 0; j < ATT_BN; ++j)
-        if (key0 + j < cs.Nk && mk[j] == 0) vis[j >> 5] &= ~(1u << (j & 31));
+      // word index unrolled, so vis stays in registers
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t bits = vis[w];
+        for (int t = 0; t < 32; ++t)
+          if (key0 + 32 * w + t < cs.Nk && mk[32 * w + t] == 0) bits &= ~(1u << t);
+        vis[w] = bits;
+      }
     }
   }
 }
