@@ -231,7 +231,9 @@ def run_ours(args, w):
                           dtype=torch.uint8, device=device)
         launches_per_step = 3 + (1 if mask is not None else 0)
 
-    def step(ev_a=None, ev_b=None):
+    def step(ev_q=None, ev_a=None, ev_b=None):
+        if ev_q is not None:
+            ev_q.record(stream)
         if w.nvfp4:
             S.sage_quantize_qkv_nvfp4(q, k, v, per_block_mean=w.per_block_mean,
                                       unpadded_k_len=w.unpadded_k_len, out=z, ws=qws)
@@ -255,8 +257,7 @@ def run_ours(args, w):
     if st != S.SAGE_OK:
         raise RuntimeError(f"device wait timed out at site {site}")
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local) if rank == 0 else None
     time.sleep(0.3 if sampler else 0)
@@ -270,9 +271,11 @@ def run_ours(args, w):
     barrier(device)
     clocks = sampler.stop() if sampler else None
     ms_local = e0.elapsed_time(e1)
-    attn_ms_local = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    attn_ms_local = sum(a.elapsed_time(b) for _, a, b in evs) / args.steps
+    quant_ms_local = sum(q.elapsed_time(a) for q, a, _ in evs) / args.steps
     ms = max_over_ranks(ms_local, device)
     attn_ms = max_over_ranks(attn_ms_local, device)
+    quant_ms = max_over_ranks(quant_ms_local, device)
     st, site = S.sage_get_device_status()
     if st != S.SAGE_OK:
         raise RuntimeError(f"device wait timed out at site {site}")
@@ -342,6 +345,18 @@ def run_ours(args, w):
                 traffic = tr.get("bytes_per_launch")
         except (OSError, ValueError):
             traffic = None
+    # the quantiser's algorithmic bytes: bf16 Q/K/V read once, codes, scales,
+    # means, q.kmean and (NVFP4) qk_correction written once
+    eq, ekv = w.B * w.Hq * w.N * w.D, w.B * w.Hkv * w.N * w.D
+    nqb = (w.N + 127) // 128
+    if w.nvfp4:
+        qbytes = (2 * (eq + 2 * ekv) + (eq + 2 * ekv) // 2 + (eq + 2 * ekv) // 16
+                  + w.B * w.Hq * nqb * (nqb * 128) * 4 + w.B * w.Hq * nqb * w.D * 4
+                  + w.B * w.Hkv * w.D * 4 + w.B * w.Hq * w.N * 4)
+    else:
+        qbytes = (3 * (eq + 2 * ekv) + (w.B * w.Hq + w.B * w.Hkv) * nqb * 4
+                  + 2 * w.B * w.Hkv * w.D * 4 + w.B * w.Hq * w.N * 4)
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ranks,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -365,6 +380,11 @@ def run_ours(args, w):
         "e2e": {"value": round(ranks * w.ops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 3), "api": e2e_api},
+        "quantize": {"kernels": "all quantiser kernels of the step", "ms": round(quant_ms, 4),
+                     "algorithmic_bytes": qbytes, "achieved": round(qbytes / (quant_ms * 1e-3) / 1e9, 1),
+                     "peak": hbm, "unit": "GB/s",
+                     "frac": round(qbytes / (quant_ms * 1e-3) / 1e9 / hbm, 4),
+                     "peak_source": f"{src} HBM copy bandwidth"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }

@@ -149,7 +149,8 @@ typedef struct {
  *                 (the same vector in every block when per_block_mean == 0)
  *   k_mean   fp32 [B, Hkv, D]
  *   q_dot_kmean fp32 [B, Hq, Nq] (may be NULL when no LSE is wanted)
- * The base pointers of q, k, v_t must be 16-byte aligned. */
+ * The base pointers of q, k, v_t, qk_correction and q_mean must be 16-byte
+ * aligned. */
 typedef struct {
   uint8_t* q;
   uint8_t* q_sf;

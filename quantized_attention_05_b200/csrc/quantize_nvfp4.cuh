@@ -13,7 +13,8 @@
 //                        codes e2m1(fp32(x * fp32(1/sf))), packed two per byte
 //                        (element 2i in the low nibble); V is transposed so
 //                        its vectors run along tokens;
-//   nv_corr_kernel       qk_correction = qmean . Ks^T in fp32, register-blocked.
+//   nv_corr_kernel       qk_correction = qmean . Ks^T on the tensor pipe (tcgen05
+//                        bf16 MMAs of hi/lo splits, fp32 accumulation in TMEM).
 // Every step that decides a code or a scale uses an explicitly rounded IEEE
 // operation, so codes and scale factors are reproducible bit for bit.
 #pragma once
@@ -137,7 +138,10 @@ __global__ void __launch_bounds__(QUANT_THREADS)
   }
 }
 
-// grid (B*Hkv + B*Hq): the K mean of each KV head, the Q mean(s) of each Q head.
+// grid (B*Hkv + B*Hq*ceil(nqt/NVM_QBLOCKS)): the K mean of each KV head, then
+// the Q means of NVM_QBLOCKS consecutive 128-token blocks of one Q head per
+// CTA (the global mean, when asked for, is formed by each of the head's CTAs).
+constexpr int NVM_QBLOCKS = 8;
 template <int D>
 __global__ void __launch_bounds__(D) nv_means_kernel(NvQuantArgs a) {
   const int c = threadIdx.x;
@@ -152,9 +156,13 @@ __global__ void __launch_bounds__(D) nv_means_kernel(NvQuantArgs a) {
     return;
   }
   id -= a.B * a.Hkv;
+  const int ngrp = (a.nqt + NVM_QBLOCKS - 1) / NVM_QBLOCKS;
+  const int grp = id % ngrp;
+  id /= ngrp;
+  const int qb0 = grp * NVM_QBLOCKS, qb1 = min(a.nqt, qb0 + NVM_QBLOCKS);
   float* qm = a.q_mean + (int64_t)id * a.nqt * D;
   if (a.per_block_mean) {  // q splits are exactly the 128-token blocks
-    for (int qb = 0; qb < a.nqt; ++qb) {
+    for (int qb = qb0; qb < qb1; ++qb) {
       const int64_t o = ((int64_t)id * a.q_splits + qb) * D + c;
       const int cnt = min(a.Nq, (qb + 1) * QB) - qb * QB;
       qm[qb * D + c] = dd_mean_f32(DD{a.q_hi[o], a.q_lo[o]}, (double)cnt);
@@ -166,7 +174,7 @@ __global__ void __launch_bounds__(D) nv_means_kernel(NvQuantArgs a) {
       dd_add(s, DD{a.q_hi[o], a.q_lo[o]});
     }
     const float m = dd_mean_f32(s, (double)a.Nq);
-    for (int qb = 0; qb < a.nqt; ++qb) qm[qb * D + c] = m;
+    for (int qb = qb0; qb < qb1; ++qb) qm[qb * D + c] = m;
   }
 }
 
@@ -290,84 +298,192 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
 }
 
 // ------------------------------------------------------------ qk_correction
-// grid (nkt, B*Hkv), 256 threads, dynamic smem: Ks^T tile [D][128] fp32 and
-// 64 Q-mean vectors [64][D].  Thread: 4 consecutive keys x 8 Q-mean vectors.
-// Rows are (Q head of the group, Q block) pairs, G * nqt of them.
+// qk_correction[b,h,qb,j] = qmean[b,h,qb] . Ks[b,g,j] on the tensor pipe.
+// Both operands are split into bf16 parts, x = hi + lo with
+// |x - hi - lo| <= 2^-18 |x|, and the MMAs hi.hi + hi.lo + lo.hi accumulate
+// in fp32 in TMEM; the omitted lo.lo and the split leave a relative error of
+// about 2^-16 per product (the fp32 reference sum rounds at 2^-24).
+// grid (nkt, B*Hkv), 256 threads: all threads stage the operands with
+// coalesced 16/32-byte loads; thread 0 issues the MMAs; warps w and w + 4
+// read TMEM lane quarter w%4 back, 64 of the 128 key columns each.
+// Shared memory: B_hi, B_lo (128 keys x D), A_hi, A_lo (128 vectors x D),
+// bf16, K-major with the 128-byte swizzle in 64-channel atoms of 16 KB: row r
+// at r * 128, 16-byte chunk c at (c ^ (r % 8)) * 16; then the fp32 output
+// tile, staged so that the correction rows are written coalesced.
+constexpr int NVC_THREADS = 256;
+template <int D>
+struct NvCorrLayout {
+  static constexpr int TILE = 128 * D * 2;   // one operand: 128 rows x D bf16
+  static constexpr int OFF_BHI = 0, OFF_BLO = TILE, OFF_AHI = 2 * TILE, OFF_ALO = 3 * TILE;
+  static constexpr int OFF_OUT = 4 * TILE;        // 128 rows x 132 fp32 (output staging)
+  static constexpr int BYTES = OFF_OUT + 128 * 132 * 4 + 1024;   // + alignment slack
+};
+
+// Channels 8*cg .. 8*cg+7 of row r into a swizzled operand tile.
+__device__ __forceinline__ void nvc_put(uint8_t* tile, int r, int cg, const uint4& v) {
+  const int atom = cg >> 3, c = cg & 7;
+  *reinterpret_cast<uint4*>(tile + atom * 16384 + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+}
+
+// bf16 hi / lo parts of 8 floats, two per word (lower channel in the low half).
+// x - hi is exact in fp32, so lo = bf16(x - hi) is x's next 8 bits.
+__device__ __forceinline__ void nvc_split8(const float* x, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * i]), h1 = __float2bfloat16_rn(x[2 * i + 1]);
+    const __nv_bfloat16 l0 = __float2bfloat16_rn(__fsub_rn(x[2 * i], __bfloat162float(h0)));
+    const __nv_bfloat16 l1 = __float2bfloat16_rn(__fsub_rn(x[2 * i + 1], __bfloat162float(h1)));
+    h[i] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+    l[i] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
 template <typename T, int D>
-__global__ void __launch_bounds__(256) nv_corr_kernel(NvQuantArgs a) {
-  extern __shared__ float4 corr_smem[];
-  float* s_kt = reinterpret_cast<float*>(corr_smem);  // [D][128]
-  float* s_qm = s_kt + D * 128;                        // [64][D]
+__global__ void __launch_bounds__(NVC_THREADS, 1) nv_corr_kernel(NvQuantArgs a) {
+  using L = NvCorrLayout<D>;
+  extern __shared__ uint8_t nvc_raw[];
+  uint8_t* sm = nvc_raw + ((1024u - (smem_u32(nvc_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ float s_km[D];
   const int kt = blockIdx.x, bg = blockIdx.y;
   const int b = bg / a.Hkv, g = bg % a.Hkv;
-  // Ks = fp32(K - kmean) for keys < L, 0 beyond; consecutive threads take
-  // consecutive keys, so the transposed shared-memory stores are
-  // conflict-free
-  for (int idx = threadIdx.x; idx < 128 * (D / 8); idx += blockDim.x) {
-    const int key = idx % 128, cg = idx / 128;
-    const int n = kt * 128 + key;
-    float f[8];
-    if (n < a.L) {
-      unpack8<T>(ldg16(reinterpret_cast<const char*>(a.k) +
-                       (b * a.k_sb + g * a.k_sh + (int64_t)n * a.k_sn + cg * 8) * (int64_t)sizeof(T)),
-                 f);
-      const float* km = a.k_mean + (int64_t)bg * D + cg * 8;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) f[i] = __fsub_rn(f[i], __ldg(km + i));
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) f[i] = 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) s_kt[(cg * 8 + i) * 128 + key] = f[i];
+  const int t = threadIdx.x, warp = t >> 5;
+  constexpr int CG = D / 8;                          // 16-byte bf16 chunks per row
+  constexpr int PER = 128 * CG / NVC_THREADS;        // chunks per thread per operand
+  for (int c = t; c < D; c += NVC_THREADS) s_km[c] = a.k_mean[(int64_t)bg * D + c];
+  if (t == 0) {
+    mbar_init(&mma_bar, 1);
+    fence_mbar_init();
   }
-  const int kq = threadIdx.x % 32;   // keys 4*kq .. 4*kq+3
-  const int vq = threadIdx.x / 32;   // vectors 8*vq .. 8*vq+7 of the chunk
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, 128);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  // B: Ks = fp32(K - kmean) for keys < L, 0 beyond.  Chunk q = t + 256 i is
+  // channels 8*(q % CG).. of key q / CG: consecutive threads read consecutive
+  // 16 bytes of a key row, and every load is in flight before the first use.
+  {
+    uint4 raw[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int q = t + NVC_THREADS * i, key = q / CG, cg = q % CG;
+      const int n = kt * 128 + key;
+      raw[i] = n < a.L ? ldg16(reinterpret_cast<const char*>(a.k) +
+                               (b * a.k_sb + g * a.k_sh + (int64_t)n * a.k_sn + cg * 8) *
+                                   (int64_t)sizeof(T))
+                       : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int q = t + NVC_THREADS * i, key = q / CG, cg = q % CG;
+      const bool live = kt * 128 + key < a.L;
+      float f[8];
+      unpack8<T>(raw[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = live ? __fsub_rn(f[e], s_km[cg * 8 + e]) : 0.f;
+      uint4 hi, lo;
+      nvc_split8(f, hi, lo);
+      nvc_put(sm + L::OFF_BHI, key, cg, hi);
+      nvc_put(sm + L::OFF_BLO, key, cg, lo);
+    }
+  }
+  // the Q means of a chunk are 128 consecutive rows of q_mean: vector v of
+  // KV head g is row (b*Hq + g*G)*nqt + v
   const int nvec = a.G * a.nqt;
-  for (int v0 = 0; v0 < nvec; v0 += 64) {
+  const float* qm_base = a.q_mean + ((int64_t)b * a.Hq + (int64_t)g * a.G) * a.nqt * D;
+  float* corr_base = a.corr + ((int64_t)b * a.Hq + (int64_t)g * a.G) * a.nqt * a.Nkp + kt * 128;
+  // output staging: 128 rows of 128 fp32, rows 132 floats apart (conflict-free
+  // 16-byte stores)
+  float* s_out = reinterpret_cast<float*>(sm + L::OFF_OUT);
+  uint32_t phase = 0;
+  bool ok = true;
+  for (int v0 = 0; ok && v0 < nvec; v0 += 128) {
+    {
+      float4 raw[2 * PER];
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int q = t + NVC_THREADS * i, row = q / CG, cg = q % CG;
+        const bool live = v0 + row < nvec;
+        const float4* src = reinterpret_cast<const float4*>(qm_base + (int64_t)(v0 + row) * D + cg * 8);
+        raw[2 * i] = live ? __ldg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+        raw[2 * i + 1] = live ? __ldg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int q = t + NVC_THREADS * i, row = q / CG, cg = q % CG;
+        const float f[8] = {raw[2 * i].x, raw[2 * i].y, raw[2 * i].z, raw[2 * i].w,
+                            raw[2 * i + 1].x, raw[2 * i + 1].y, raw[2 * i + 1].z, raw[2 * i + 1].w};
+        uint4 hi, lo;
+        nvc_split8(f, hi, lo);
+        nvc_put(sm + L::OFF_AHI, row, cg, hi);
+        nvc_put(sm + L::OFF_ALO, row, cg, lo);
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
-    for (int idx = threadIdx.x; idx < 64 * D; idx += blockDim.x) {
-      const int vv = idx / D, c = idx % D;
-      const int v = v0 + vv;
-      float val = 0.f;
-      if (v < nvec) {
-        const int h = g * a.G + v / a.nqt, qb = v % a.nqt;
-        val = a.q_mean[(((int64_t)b * a.Hq + h) * a.nqt + qb) * D + c];
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    if (t == 0) {
+      constexpr uint32_t ID = instr_desc(kDF32, 1u, 1u, 128, 128);   // bf16 x bf16 -> fp32
+      const uint32_t ah = smem_u32(sm + L::OFF_AHI), al = smem_u32(sm + L::OFF_ALO);
+      const uint32_t bh = smem_u32(sm + L::OFF_BHI), bl = smem_u32(sm + L::OFF_BLO);
+      const uint32_t pa[3] = {ah, ah, al}, pb[3] = {bh, bl, bh};
+#pragma unroll
+      for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+        for (int atom = 0; atom < D / 64; ++atom)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_f16(tmem, smem_desc(pa[pass] + atom * 16384 + 32 * k, 1024, 128),
+                    smem_desc(pb[pass] + atom * 16384 + 32 * k, 1024, 128), ID,
+                    (pass | atom | k) ? 1u : 0u);
+      tc_commit(&mma_bar);
+    }
+    __syncwarp();
+    ok = __all_sync(0xffffffffu, mbar_wait(&mma_bar, phase & 1, SITE_MMA_DONE));
+    ++phase;
+    tc_fence_after();
+    // the MMAs are done with the operand tiles: TMEM rows -> s_out
+    // (warps w and w + 4 share lane quarter w % 4, 64 key columns each)
+    if (ok) {
+      const int rr = (warp & 3) * 32 + (t & 31);
+      const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+#pragma unroll
+      for (int cb = (warp >> 2) * 64; cb < (warp >> 2) * 64 + 64; cb += 32) {
+        uint32_t o[32];
+        SAGE_TMEM_LD32(tl + cb, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          *reinterpret_cast<float4*>(s_out + rr * 132 + cb + 4 * e) =
+              make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                          __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
       }
-      s_qm[vv * D + c] = val;
     }
     __syncthreads();
-    float acc[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-    for (int c = 0; c < D; c += 4) {
-      float4 kv[4];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) kv[cc] = *reinterpret_cast<const float4*>(&s_kt[(c + cc) * 128 + 4 * kq]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 qv = *reinterpret_cast<const float4*>(&s_qm[(vq * 8 + i) * D + c]);
-        const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          acc[i][0] = fmaf(qa[cc], kv[cc].x, acc[i][0]);
-          acc[i][1] = fmaf(qa[cc], kv[cc].y, acc[i][1]);
-          acc[i][2] = fmaf(qa[cc], kv[cc].z, acc[i][2]);
-          acc[i][3] = fmaf(qa[cc], kv[cc].w, acc[i][3]);
-        }
+    // coalesced rows of the correction: 32 threads write one 512-byte row
+    if (ok) {
+      for (int q = t; q < 128 * 32; q += NVC_THREADS) {
+        const int row = q >> 5, c4 = q & 31;
+        if (v0 + row < nvec)
+          *reinterpret_cast<float4*>(corr_base + (int64_t)(v0 + row) * a.Nkp + 4 * c4) =
+              *reinterpret_cast<const float4*>(s_out + row * 132 + 4 * c4);
       }
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int v = v0 + vq * 8 + i;
-      if (v < nvec) {
-        const int h = g * a.G + v / a.nqt, qb = v % a.nqt;
-        float* dst = a.corr + (((int64_t)b * a.Hq + h) * a.nqt + qb) * a.Nkp + kt * 128 + 4 * kq;
-        *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-      }
-    }
+    // TMEM, s_out and the A tiles are rewritten by the next chunk
+    tc_fence_before();
+    __syncthreads();
+  }
+  // every MMA issued above has completed (each chunk waited for its commit)
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_slot, 128);
   }
 }
 

@@ -377,7 +377,8 @@ sage_status check_nvfp4(const sage_qkv_nvfp4* z, bool need_qdk) {
       !z->q_mean || !z->k_mean)
     return SAGE_ERR_INVALID_ARG;
   if (need_qdk && !z->q_dot_kmean) return SAGE_ERR_INVALID_ARG;
-  if (!aligned16(z->q) || !aligned16(z->k) || !aligned16(z->v_t) || !aligned16(z->qk_correction))
+  if (!aligned16(z->q) || !aligned16(z->k) || !aligned16(z->v_t) || !aligned16(z->qk_correction) ||
+      !aligned16(z->q_mean))
     return SAGE_ERR_INVALID_ARG;
   if (z->unpadded_k_len < 1 || z->unpadded_k_len > z->Nk) return SAGE_ERR_INVALID_ARG;
   return SAGE_OK;
@@ -444,7 +445,7 @@ sage_status run_quantize_nvfp4(const sage_tensor* q, const sage_tensor* k, const
   const bool fp16 = q->dtype == SAGE_FP16;
   const int nblocks = a.B * a.Hq * a.nqt + 2 * a.B * a.Hkv * a.nkt;
   const dim3 gk(a.k_splits, a.B * a.Hkv), gq(a.q_splits, a.B * a.Hq), gc(a.nkt, a.B * a.Hkv);
-  const size_t corr_smem = (size_t)(q->D * 128 + 64 * q->D) * 4;
+  const size_t corr_smem = q->D == 128 ? NvCorrLayout<128>::BYTES : NvCorrLayout<64>::BYTES;
 #define SAGE_NV_LAUNCH(T, D)                                                                     \
   do {                                                                                           \
     nv_colsum_kernel<T, D><<<gk, QUANT_THREADS, 0, stream>>>(a.k, a.k_sb, a.k_sh, a.k_sn, a.Hkv, \
@@ -453,11 +454,12 @@ sage_status run_quantize_nvfp4(const sage_tensor* q, const sage_tensor* k, const
     nv_colsum_kernel<T, D><<<gq, QUANT_THREADS, 0, stream>>>(a.q, a.q_sb, a.q_sh, a.q_sn, a.Hq,  \
                                                              a.Nq, a.q_splits, a.q_split_tokens, \
                                                              a.q_hi, a.q_lo);                    \
-    nv_means_kernel<D><<<a.B * (a.Hkv + a.Hq), D, 0, stream>>>(a);                               \
+    nv_means_kernel<D><<<a.B * a.Hkv + a.B * a.Hq * ((a.nqt + NVM_QBLOCKS - 1) / NVM_QBLOCKS), D, \
+                         0, stream>>>(a);                                                        \
     nv_quant_kernel<T, D><<<nblocks, QUANT_THREADS, 0, stream>>>(a);                             \
     if (!ensure_smem(nv_corr_kernel<T, D>, corr_smem, &corr_smem_flag<T, D>()))                  \
       return SAGE_ERR_CUDA;                                                                      \
-    nv_corr_kernel<T, D><<<gc, 256, corr_smem, stream>>>(a);                                     \
+    nv_corr_kernel<T, D><<<gc, NVC_THREADS, corr_smem, stream>>>(a);                             \
   } while (0)
   if (q->D == 128) {
     if (fp16) SAGE_NV_LAUNCH(__half, 128); else SAGE_NV_LAUNCH(__nv_bfloat16, 128);
