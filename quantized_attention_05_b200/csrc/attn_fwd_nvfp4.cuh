@@ -152,23 +152,6 @@ __device__ __forceinline__ void stage_sf(uint8_t* dst, const uint8_t* src, int64
   }
 }
 
-// P' vector quantisation when the vector's amax is already known: scale
-// factor sf = E4M3(amax / 6), codes E2M1(x * (1 / value(sf))) with the
-// correctly rounded reciprocal taken from `inv_tab` (0 for a zero scale, so
-// the codes of an all-zero vector are 0).
-__device__ __forceinline__ uint32_t nvfp4_vector_amax(const float* x, float amax,
-                                                      const float* inv_tab, uint32_t* w0,
-                                                      uint32_t* w1) {
-  const uint32_t sf = e4m3_code(__fdiv_rn(amax, 6.f));
-  const float inv = inv_tab[sf];
-  float y[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(x[i], inv);
-  *w0 = e2m1x8(y);
-  *w1 = e2m1x8(y + 8);
-  return sf;
-}
-
 template <int D>
 __global__ void __launch_bounds__(NV_THREADS, 1)
     attn_fwd_nvfp4_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -399,10 +382,16 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
 #pragma unroll
       for (int j = 0; j < 64; j += 4) {
         const float4 cv = *reinterpret_cast<const float4*>(corr + j);
-        sr[j] = __float_as_uint(__uint_as_float(sr[j]) + cv.x);
-        sr[j + 1] = __float_as_uint(__uint_as_float(sr[j + 1]) + cv.y);
-        sr[j + 2] = __float_as_uint(__uint_as_float(sr[j + 2]) + cv.z);
-        sr[j + 3] = __float_as_uint(__uint_as_float(sr[j + 3]) + cv.w);
+        float x0, x1, x2, x3;
+        f2_unpack(f2_add(f2_pack(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), f2_pack(cv.x, cv.y)),
+                  x0, x1);
+        f2_unpack(f2_add(f2_pack(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])),
+                         f2_pack(cv.z, cv.w)),
+                  x2, x3);
+        sr[j] = __float_as_uint(x0);
+        sr[j + 1] = __float_as_uint(x1);
+        sr[j + 2] = __float_as_uint(x2);
+        sr[j + 3] = __float_as_uint(x3);
       }
       uint32_t vis[2] = {~0u, ~0u};
       if (need) {
@@ -456,10 +445,23 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       uint8_t* prow = sP + buf * L::P_BYTES + rt * 64;
       uint8_t* psf = sPsf + buf * 2 * L::SF_BLK + half * L::SF_BLK + 16 * (rt & 31) + 4 * (rt >> 5);
       uint64_t acc = f2_pack(0.f, 0.f);
+      // the scale of each 16-key vector depends only on its largest score:
+      // amax = the p of that score (same fma and ex2 as the element itself;
+      // 0 when every key of the vector is hidden), sf = e4m3(amax / 6).  The
+      // four scales come first, so the codes below wait on no long chain.
       uint32_t sfw = 0u;
+      float inv[4];
 #pragma unroll
       for (int vv = 0; vv < 4; ++vv) {
-        float pv[16];
+        const float pmax = ex2_approx(fmaf(vmax[vv], c, bias));
+        const uint32_t sf = e4m3_code(__fdiv_rn(pmax, 6.f));
+        inv[vv] = s_inv[sf];
+        sfw |= sf << (8 * vv);
+      }
+#pragma unroll
+      for (int vv = 0; vv < 4; ++vv) {
+        const uint64_t inv2 = f2_pack(inv[vv], inv[vv]);
+        float yq[16];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int j = vv * 16 + 2 * i;
@@ -471,19 +473,18 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
             p = f2_exp2_poly(y0, y1);
           else
             p = f2_pack(ex2_approx(y0), ex2_approx(y1));
-          f2_unpack(p, pv[2 * i], pv[2 * i + 1]);
           if (need) {
-            if (!((vis[j >> 5] >> (j & 31)) & 1u)) pv[2 * i] = 0.f;
-            if (!((vis[j >> 5] >> ((j + 1) & 31)) & 1u)) pv[2 * i + 1] = 0.f;
+            float p0, p1;
+            f2_unpack(p, p0, p1);
+            if (!((vis[j >> 5] >> (j & 31)) & 1u)) p0 = 0.f;
+            if (!((vis[j >> 5] >> ((j + 1) & 31)) & 1u)) p1 = 0.f;
+            p = f2_pack(p0, p1);
           }
-          acc = f2_add(acc, f2_pack(pv[2 * i], pv[2 * i + 1]));
+          acc = f2_add(acc, p);
+          // P' / scale, rounded to E2M1 below
+          f2_unpack(f2_mul(p, inv2), yq[2 * i], yq[2 * i + 1]);
         }
-        // amax of the vector: the p of its largest score (same fma and ex2
-        // as the element itself; 0 when every key of the vector is hidden)
-        const float pmax = ex2_approx(fmaf(vmax[vv], c, bias));
-        uint32_t w0, w1;
-        const uint32_t sf = nvfp4_vector_amax(pv, pmax, s_inv, &w0, &w1);
-        sfw |= sf << (8 * vv);
+        const uint32_t w0 = e2m1x8(yq), w1 = e2m1x8(yq + 8);
         // 16-byte chunk (4*half + vv)/2 of the row (64-byte swizzle: chunk ^ ((row >> 1) & 3))
         const int v16 = 4 * half + vv;
         uint8_t* dst = prow + ((((v16 >> 1) ^ ((rt >> 1) & 3))) << 4) + (v16 & 1) * 8;
