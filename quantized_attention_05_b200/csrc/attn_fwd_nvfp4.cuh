@@ -5,19 +5,21 @@
 // microscaling for Q/K and V).
 //
 // One CTA owns one 128-row Q tile of one (batch, Q head):
-//   warp 8   producer: TMA for the packed Q, K and V^T tiles, a bulk copy
-//            of the tile's qk_correction row, and the scale factors staged
-//            in shared memory in the layout tcgen05.cp expects (for every
-//            64-element K block a 512-byte block: row r's four scale
-//            factors as one 32-bit word at 16*(r%32) + 4*(r/32));
+//   warp 8   producer: TMA for the packed Q, K and V^T tiles, the tile's
+//            qk_correction row as bf16 hi + lo (the B operand of one bf16
+//            MMA that adds it to S), and the scale factors staged in shared
+//            memory in the layout tcgen05.cp expects (for every 64-element K
+//            block a 512-byte block: row r's four scale factors as one
+//            32-bit word at 16*(r%32) + 4*(r/32));
 //   warp 9   MMA issuer: tcgen05.cp of the scale factors into TMEM and
 //            tcgen05.mma kind::mxf4nvf4 with 16-element E4M3 block scales,
-//            S = Q K^T into a double-buffered TMEM accumulator and
-//            O += P V into TMEM, both fp32;
+//            S = Q K^T into a double-buffered TMEM accumulator, then
+//            S += qk_correction (kind::f16 bf16 MMA onto the same fp32
+//            accumulator), and O += P V into TMEM, both fp32;
 //   warps 0-7  softmax, two threads per row: warps q and q+4 share the
 //            TMEM lane quarter q and take keys 0-63 and 64-127 of each
-//            tile (four 16-key vectors each).  Per tile: scores S +
-//            qk_correction, masking, the row max from the two partial maxima
+//            tile (four 16-key vectors each).  Per tile: the scores (the
+//            correction already in S), masking, the row max from the two partial maxima
 //            (exchanged through shared memory on an mbarrier per warp pair
 //            and tile parity, so the wait is bounded like every other),
 //            exact online softmax with exp2, P' = 2688 * p
@@ -73,8 +75,13 @@ struct NvLayout {
   static constexpr int OFF_KSF = OFF_QSF + KB_QK * SF_BLK;
   static constexpr int OFF_VSF = OFF_KSF + NV_STAGES * KB_QK * SF_BLK;
   static constexpr int OFF_PSF = OFF_VSF + NV_STAGES * 2 * SF_BLK;
+  // qk_correction row of each stage as the B operand of one bf16 MMA
+  // (128 keys x K = 16, 32-byte rows: (hi, lo, 0, ...) in one 16-byte chunk,
+  // zeros in the other), and the A operand (1, 1, 0, ...) in both chunks of
+  // every row: the MMA adds hi + lo of key j's correction to every S row.
   static constexpr int OFF_CORR = OFF_PSF + 2 * 2 * SF_BLK;
-  static constexpr int OFF_BAR = OFF_CORR + NV_STAGES * 512;
+  static constexpr int OFF_ONES = OFF_CORR + NV_STAGES * 4096;
+  static constexpr int OFF_BAR = OFF_ONES + 4096;
   // q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2], o_ready[2], mma_done,
   // pmax_full[quarter][tile parity]
   static constexpr int NBAR = 1 + 2 * NV_STAGES + 8 + 1 + 8;
@@ -119,14 +126,6 @@ __host__ __device__ constexpr uint32_t nv_idesc(uint32_t M, uint32_t N) {
   return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // Stage the scale factors of 128 rows (row-major, D/16 bytes each, rows from
 // `src` with `row_stride` bytes) into the tcgen05.cp layout at `dst`: the
 // four scale factors of a 64-element block of row r form one word at
@@ -168,7 +167,8 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
   uint8_t* sKsf = smem + L::OFF_KSF;
   uint8_t* sVsf = smem + L::OFF_VSF;
   uint8_t* sPsf = smem + L::OFF_PSF;
-  float* sCorr = reinterpret_cast<float*>(smem + L::OFF_CORR);
+  uint8_t* sCorrB = smem + L::OFF_CORR;
+  uint8_t* sOnes = smem + L::OFF_ONES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
@@ -255,6 +255,11 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
   }
+  // A operand of the correction MMA: bf16 1.0 (0x3F80) at k = 0 and 1 of
+  // both 16-byte chunks of every row
+  for (int u = threadIdx.x; u < 256; u += blockDim.x)
+    *reinterpret_cast<uint4*>(sOnes + 16 * u) = make_uint4(0x3F803F80u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -281,14 +286,32 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
                        a.k_sf + ((int64_t)bhk * a.Nkp + kt * 128) * (D / 16), D / 16, 128, lane);
       stage_sf<8>(sVsf + st * 2 * L::SF_BLK, a.v_sf_t + (int64_t)bhk * D * (a.Nkp / 16) + kt * 8,
                   a.Nkp / 16, D, lane);
+      {
+        // the correction of keys 4*lane .. 4*lane+3 as bf16 hi + lo
+        // (|x - hi - lo| <= 2^-18 |x|), row j of the B tile
+        const float4 cv = __ldg(reinterpret_cast<const float4*>(
+                                    a.corr + ((int64_t)bhq * a.nqt + qt) * a.Nkp + kt * 128) +
+                                lane);
+        const float x[4] = {cv.x, cv.y, cv.z, cv.w};
+        uint8_t* tile = sCorrB + st * 4096;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = 4 * lane + i;
+          const __nv_bfloat16 hi = __float2bfloat16_rn(x[i]);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(x[i], __bfloat162float(hi)));
+          const uint32_t w =
+              (uint32_t)__bfloat16_as_ushort(hi) | ((uint32_t)__bfloat16_as_ushort(lo) << 16);
+          const int sw = (j >> 2) & 1;   // 32-byte swizzle: chunk c of row j at (c ^ sw) * 16
+          *reinterpret_cast<uint4*>(tile + j * 32 + (sw << 4)) = make_uint4(w, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(tile + j * 32 + ((1 ^ sw) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       fence_proxy_async_smem();
       if (lane == 0) {
-        mbar_arrive_expect_tx(&kv_full[st], (uint32_t)(L::K_BYTES + L::V_BYTES + 512));
+        mbar_arrive_expect_tx(&kv_full[st], (uint32_t)(L::K_BYTES + L::V_BYTES));
         tma_load_2d(sK + st * (L::OFF_V - L::OFF_K) / NV_STAGES, &tmK, &kv_full[st], 0,
                     bhk * a.Nkp + kt * 128);
         tma_load_2d(sV + st * L::V_BYTES, &tmV, &kv_full[st], kt * 64, bhk * D);
-        bulk_load(sCorr + st * 128, a.corr + ((int64_t)bhq * a.nqt + qt) * a.Nkp + kt * 128, 512,
-                  &kv_full[st]);
       } else {
         mbar_arrive(&kv_full[st]);
       }
@@ -338,6 +361,10 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
                     smem_desc(aQ + 32 * kb, L::QK_SBO, L::QK_SWIZZLE),
                     smem_desc(aK + st * KSTRIDE + 32 * kb, L::QK_SBO, L::QK_SWIZZLE), ID_QK,
                     tmem + L::T_SFQ + 4 * kb, tmem + L::T_SFK + 4 * kb, kb > 0 ? 1u : 0u);
+        // S += qk_correction of each key (one bf16 MMA onto the fp32 scores)
+        mma_f16(tmem + L::T_S + buf * 128, smem_desc(smem_u32(sOnes), 256, 32),
+                smem_desc(smem_u32(sCorrB) + st * 4096, 256, 32), instr_desc(kDF32, 1u, 1u, 128, 128),
+                1u);
         tc_commit(&s_full[buf]);
         if (idx >= 1) do_pv(idx - 1);
       }
@@ -375,24 +402,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&s_free[buf]);
-      // the tile's correction row arrived with its K/V (bulk copy on kv_full)
-      ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[st], (idx / NV_STAGES) & 1, SITE_KV_FULL));
-      if (!ok) break;
-      const float* corr = sCorr + st * 128 + half * 64;
-#pragma unroll
-      for (int j = 0; j < 64; j += 4) {
-        const float4 cv = *reinterpret_cast<const float4*>(corr + j);
-        float x0, x1, x2, x3;
-        f2_unpack(f2_add(f2_pack(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), f2_pack(cv.x, cv.y)),
-                  x0, x1);
-        f2_unpack(f2_add(f2_pack(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])),
-                         f2_pack(cv.z, cv.w)),
-                  x2, x3);
-        sr[j] = __float_as_uint(x0);
-        sr[j + 1] = __float_as_uint(x1);
-        sr[j + 2] = __float_as_uint(x2);
-        sr[j + 3] = __float_as_uint(x3);
-      }
+      // S already holds the scores plus qk_correction (added by the MMA)
       uint32_t vis[2] = {~0u, ~0u};
       if (need) {
         const int key0 = kt * 128 + half * 64;
