@@ -56,6 +56,18 @@ struct NvAttnArgs {
   float sm_scale;
 };
 
+// x / 6 rounded to nearest even, for every fp32 x whose quotient is normal
+// (checked exhaustively against the IEEE division by tests/test_div6.py):
+// the product with RN(1/6), then one correction with the exact residual
+// fma(-q0, 6, x).  Smaller quotients can be one unit off, which no E4M3 code
+// sees (they are below half its smallest subnormal, 2^-10).
+__device__ __forceinline__ float div6_rn(float x) {
+  const float c = 0.16666667f;   // RN(1/6) = 0x1.555556p-3
+  const float q0 = __fmul_rn(x, c);
+  const float r = __fmaf_rn(-q0, 6.f, x);
+  return __fmaf_rn(r, c, q0);
+}
+
 template <int D>
 struct NvLayout {
   static constexpr int ROWB = D / 2;            // bytes per packed Q/K row
@@ -464,7 +476,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
 #pragma unroll
       for (int vv = 0; vv < 4; ++vv) {
         const float pmax = ex2_approx(fmaf(vmax[vv], c, bias));
-        const uint32_t sf = e4m3_code(__fdiv_rn(pmax, 6.f));
+        const uint32_t sf = e4m3_code(div6_rn(pmax));
         inv[vv] = s_inv[sf];
         sfw |= sf << (8 * vv);
       }
