@@ -288,8 +288,9 @@ def run_ours(args, w):
     maskh = None if mask is None else mask.cpu().pin_memory()
     md = None if mask is None else torch.empty_like(mask)
     if w.nvfp4:
-        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        e2e_api = "device copies + sage_quantize_qkv_nvfp4 + sage_attn_fwd_nvfp4, pinned host buffers"
+        ws_host = torch.empty(S.sage_attn_fwd_nvfp4_host_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.N, w.D),
+                              dtype=torch.uint8, device=device)
+        e2e_api = "sage_attn_fwd_nvfp4_host on pinned host buffers (chunked, copies overlapped)"
     else:
         # the host-resident entry point: chunked, copies overlapped with the kernels
         ws_host = torch.empty(S.sage_attn_fwd_host_workspace_bytes(
@@ -301,15 +302,10 @@ def run_ours(args, w):
         if md is not None:
             md.copy_(maskh, non_blocking=True)
         if w.nvfp4:
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            S.sage_quantize_qkv_nvfp4(qd, kd, vd, per_block_mean=w.per_block_mean,
-                                      unpadded_k_len=w.unpadded_k_len, out=z, ws=qws)
-            S.sage_attn_fwd_nvfp4(z, sm_scale=w.sm_scale, causal=w.causal, return_lse=True,
-                                  out=out, lse=lse)
-            outh.copy_(out, non_blocking=True)
-            lseh.copy_(lse, non_blocking=True)
+            S.sage_attn_fwd_nvfp4_host(qh, kh, vh, sm_scale=w.sm_scale, causal=w.causal,
+                                       per_block_mean=w.per_block_mean,
+                                       unpadded_k_len=w.unpadded_k_len, return_lse=True, out=outh,
+                                       lse=lseh, ws=ws_host, device=device)
         else:
             S.sage_attn_fwd_host(qh, kh, vh, causal=w.causal, sm_scale=w.sm_scale, return_lse=True,
                                  mask=md, out=outh, lse=lseh, ws=ws_host, device=device)

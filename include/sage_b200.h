@@ -271,6 +271,31 @@ sage_status sage_attn_fwd_host(const sage_tensor* q, const sage_tensor* k, const
                                int64_t out_sh, int64_t out_sn, float* lse, int64_t chunk_groups,
                                void* ws, size_t ws_bytes, sage_stream_t stream);
 
+/* Workspace bytes of sage_attn_fwd_nvfp4_host for chunks of `chunk_groups`
+ * (batch entry, KV head) groups (0 = automatic): three staging slots plus
+ * one chunk's quantised NVFP4 arrays and quantiser sums.  0 for invalid
+ * sizes. */
+size_t sage_attn_fwd_nvfp4_host_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
+                                                int64_t Nk, int64_t D, int64_t chunk_groups);
+
+/* The NVFP4 path (sage_quantize_qkv_nvfp4 then sage_attn_fwd_nvfp4) on Q/K/V
+ * and outputs held in HOST memory, streamed through the GPU a chunk of (batch
+ * entry, KV head) groups at a time exactly as sage_attn_fwd_host does; every
+ * group is a problem of its own (its K mean over the first unpadded_k_len
+ * keys, its Q means, its V vectors), so the result equals the two device calls
+ * bit for bit.  q, k, v: HOST tensors of one dtype; out, lse: HOST buffers (out
+ * with element strides out_sb/out_sh/out_sn, lse [B, Hq, Nq] contiguous fp32,
+ * written iff return_lse); unpadded_k_len <= 0 means Nk; sm_scale <= 0
+ * selects 1/sqrt(D); ws: DEVICE workspace (256-byte aligned) of
+ * sage_attn_fwd_nvfp4_host_workspace_bytes(..., chunk_groups) bytes.  Streams,
+ * ordering, host-memory kinds and errors as for sage_attn_fwd_host. */
+sage_status sage_attn_fwd_nvfp4_host(const sage_tensor* q, const sage_tensor* k,
+                                     const sage_tensor* v, float sm_scale, int causal,
+                                     int per_block_mean, int64_t unpadded_k_len, int return_lse,
+                                     void* out, int64_t out_sb, int64_t out_sh, int64_t out_sn,
+                                     float* lse, int64_t chunk_groups, void* ws, size_t ws_bytes,
+                                     sage_stream_t stream);
+
 /* --------------------------------------------------------- variable length */
 /* Workspace bytes of sage_attn_fwd_varlen: the sequence table, quantised
  * Q/K/V of the packed sequences (each padded to 128 tokens per head), the

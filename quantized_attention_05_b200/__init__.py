@@ -99,6 +99,11 @@ def lib():
                                               ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                               P(SageMask), _vp, _i64, _i64, _i64, _vp, _i64, _vp,
                                               ctypes.c_size_t, _vp]),
+        "sage_attn_fwd_nvfp4_host_workspace_bytes": (ctypes.c_size_t, [_i64] * 7),
+        "sage_attn_fwd_nvfp4_host": (ctypes.c_int, [P(SageTensor), P(SageTensor), P(SageTensor),
+                                                    ctypes.c_float, ctypes.c_int, ctypes.c_int, _i64,
+                                                    ctypes.c_int, _vp, _i64, _i64, _i64, _vp, _i64, _vp,
+                                                    ctypes.c_size_t, _vp]),
         "sage_attn_fwd_varlen_workspace_bytes": (ctypes.c_size_t, [_i64] * 8 + [ctypes.c_int]),
         "sage_attn_fwd_varlen": (ctypes.c_int, [P(SageTensor), P(SageTensor), P(SageTensor), _vp, _vp,
                                                 _i64, _i64, _i64, ctypes.c_int, ctypes.c_float,
@@ -349,17 +354,7 @@ def sage_attn_fwd_host(q, k, v, causal=False, sm_scale=None, num_kv_heads=None, 
     tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
     if num_kv_heads is None:
         num_kv_heads = tk.H
-    if out is None:
-        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-    if out.is_cuda:
-        raise ValueError("out must be a host tensor")
-    to = _as_tensor(out, layout)
-    if return_lse:
-        if lse is None:
-            lse = torch.empty(tq.B, tq.H, tq.N, dtype=torch.float32, pin_memory=True)
-        if lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous() or \
-                lse.numel() != tq.B * tq.H * tq.N:
-            raise ValueError("lse must be a contiguous fp32 host tensor [B, Hq, Nq]")
+    out, to, lse = _host_outputs(q, tq, layout, out, lse, return_lse)
     mk = _as_mask(mask, tq.B, tq.H, tq.N, tk.N)
     if mk is not None and not mask.is_cuda:
         raise ValueError("mask must be a CUDA tensor")
@@ -378,6 +373,59 @@ def sage_attn_fwd_host(q, k, v, causal=False, sm_scale=None, num_kv_heads=None, 
                                     lse.data_ptr() if return_lse else None, int(chunk_groups),
                                     ws.data_ptr(), ws.numel(), _stream(device)),
                "sage_attn_fwd_host")
+    return (out, lse) if return_lse else out
+
+
+def _host_outputs(q, tq, layout, out, lse, return_lse):
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if out.is_cuda:
+        raise ValueError("out must be a host tensor")
+    to = _as_tensor(out, layout)
+    if return_lse:
+        if lse is None:
+            lse = torch.empty(tq.B, tq.H, tq.N, dtype=torch.float32, pin_memory=True)
+        if lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous() or \
+                lse.numel() != tq.B * tq.H * tq.N:
+            raise ValueError("lse must be a contiguous fp32 host tensor [B, Hq, Nq]")
+    return out, to, lse
+
+
+def sage_attn_fwd_nvfp4_host_workspace_bytes(B, Hq, Hkv, Nq, Nk, D, chunk_groups=0):
+    """Device workspace bytes of sage_attn_fwd_nvfp4_host."""
+    return lib().sage_attn_fwd_nvfp4_host_workspace_bytes(B, Hq, Hkv, Nq, Nk, D, chunk_groups)
+
+
+def sage_attn_fwd_nvfp4_host(q, k, v, sm_scale=None, causal=False, per_block_mean=True,
+                             unpadded_k_len=None, return_lse=False, layout="HND", out=None, lse=None,
+                             ws=None, chunk_groups=0, device=None):
+    """The NVFP4 path (quantise, then attend) on bf16/fp16 Q/K/V held in host
+    memory (sage_attn_fwd_nvfp4_host), streamed through the GPU in chunks of
+    (batch entry, KV head) groups with the copies overlapped with the kernels.
+    Host tensors as for sage_attn_fwd_host; out has q's dtype.  Returns out
+    and, with return_lse, lse [B, Hq, Nq] fp32."""
+    L = lib()
+    for t in (q, k, v):
+        if t.is_cuda:
+            raise ValueError("sage_attn_fwd_nvfp4_host takes host tensors")
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
+    out, to, lse = _host_outputs(q, tq, layout, out, lse, return_lse)
+    nbytes = L.sage_attn_fwd_nvfp4_host_workspace_bytes(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D,
+                                                        int(chunk_groups))
+    if nbytes == 0:
+        raise SageError(SAGE_ERR_INVALID_ARG, "sage_attn_fwd_nvfp4_host: invalid sizes")
+    if ws is None or ws.numel() < nbytes:
+        ws = _ws(nbytes, device)
+    with torch.cuda.device(device):
+        _check(L.sage_attn_fwd_nvfp4_host(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                                          float(sm_scale) if sm_scale else 0.0, int(bool(causal)),
+                                          int(bool(per_block_mean)),
+                                          int(unpadded_k_len) if unpadded_k_len else 0,
+                                          int(bool(return_lse)), to.ptr, to.sb, to.sh, to.sn,
+                                          lse.data_ptr() if return_lse else None, int(chunk_groups),
+                                          ws.data_ptr(), ws.numel(), _stream(device)),
+               "sage_attn_fwd_nvfp4_host")
     return (out, lse) if return_lse else out
 
 

@@ -681,8 +681,13 @@ struct PipeLayout {
   size_t fused, total;         // one chunk's quantise + attend workspace
 };
 
-PipeLayout pipe_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
-                       const sage_mask* mask, int64_t chunk_groups) {
+// Staging slots for chunks of `chunk_groups` KV-head groups (0: automatic)
+// and, after them, the largest per-chunk quantise + attend workspace that
+// `chunk_ws(ng)` reports for ng groups (full chunks and the last, smaller
+// chunk of a batch entry).
+template <typename ChunkWs>
+PipeLayout pipe_layout(int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
+                       int64_t chunk_groups, ChunkWs chunk_ws) {
   const int64_t G = Hq / Hkv;
   const size_t per_group = (size_t)(G * Nq + 2 * Nk) * D * 2;
   int64_t gpc = chunk_groups > 0 ? chunk_groups
@@ -699,14 +704,42 @@ PipeLayout pipe_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t N
   p.slot = o;
   p.fused = kPipeSlots * p.slot;
   size_t fw = 0;
-  for (const int64_t ng : {gpc, Hkv % gpc}) {  // full chunks and the last of a batch entry
-    if (ng == 0) continue;
-    sage_mask cm{};
-    if (mask) cm = chunk_mask(*mask, 0, 0, ng * G);
-    fw = std::max(fw, fused_layout(1, ng * G, ng, Nq, Nk, D, mask ? &cm : nullptr).total);
-  }
+  for (const int64_t ng : {gpc, Hkv % gpc})
+    if (ng > 0) fw = std::max(fw, chunk_ws(ng));
   p.total = p.fused + fw;
   return p;
+}
+
+// The INT8/FP8 path's per-chunk workspace (sage_attn_fwd's layout for one chunk).
+size_t i8_chunk_ws(int64_t G, int64_t Nq, int64_t Nk, int64_t D, const sage_mask* mask,
+                   int64_t ng) {
+  sage_mask cm{};
+  if (mask) cm = chunk_mask(*mask, 0, 0, ng * G);
+  return fused_layout(1, ng * G, ng, Nq, Nk, D, mask ? &cm : nullptr).total;
+}
+
+// The NVFP4 path's per-chunk workspace: the quantised arrays of one chunk
+// (sage_qkv_nvfp4 of B = 1, nh Q heads, ng KV heads) and the quantiser's sums.
+struct NvChunkLayout {
+  size_t q4, qsf, k4, ksf, vt, vsft, corr, qm, km, qdk, part, total;
+};
+NvChunkLayout nv_chunk_layout(int64_t nh, int64_t ng, int64_t Nq, int64_t Nk, int64_t D) {
+  const int64_t Nqp = pad128(Nq), Nkp = pad128(Nk), nqt = Nqp / 128;
+  NvChunkLayout f{};
+  size_t o = 0;
+  f.q4 = o; o += align256((size_t)nh * Nqp * D / 2);
+  f.qsf = o; o += align256((size_t)nh * Nqp * D / 16);
+  f.k4 = o; o += align256((size_t)ng * Nkp * D / 2);
+  f.ksf = o; o += align256((size_t)ng * Nkp * D / 16);
+  f.vt = o; o += align256((size_t)ng * D * Nkp / 2);
+  f.vsft = o; o += align256((size_t)ng * D * Nkp / 16);
+  f.corr = o; o += align256((size_t)nh * nqt * Nkp * 4);
+  f.qm = o; o += align256((size_t)nh * nqt * D * 4);
+  f.km = o; o += align256((size_t)ng * D * 4);
+  f.qdk = o; o += align256((size_t)nh * Nq * 4);
+  f.part = o; o += nv_plan(1, nh, ng, Nq, Nk, D).total;
+  f.total = o;
+  return f;
 }
 
 // Copy streams and events, created once per device on first use.
@@ -741,11 +774,16 @@ sage_status pipe_streams(PipeStreams** res) {
   return SAGE_OK;
 }
 
+// `compute(b, h0, g0, cq, ck, cv, out_slot, out_sh, out_sn, lse_slot)`
+// enqueues the quantise + attend of one chunk (heads h0.. of batch entry b,
+// KV heads g0..) on `stream`, reading the staged cq/ck/cv and writing the
+// staged output (strides in elements) and LSE, with its workspace at
+// w + p.fused.
+template <typename Compute>
 sage_status run_host_pipeline(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
-                              int causal, float sm_scale, int return_lse, int smooth_k,
-                              const sage_mask* mask, void* out, int64_t out_sb, int64_t out_sh,
+                              int return_lse, void* out, int64_t out_sb, int64_t out_sh,
                               int64_t out_sn, float* lse, const PipeLayout& p, char* w,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, Compute compute) {
   std::lock_guard<std::mutex> lock(g_pipe_mu);
   PipeStreams* ps = nullptr;
   sage_status st = pipe_streams(&ps);
@@ -790,13 +828,8 @@ sage_status run_host_pipeline(const sage_tensor* q, const sage_tensor* k, const 
       const sage_tensor cq{sl + p.q, q->dtype, 1, nh, Nq, D, nh * Nq * D, sq.sh, sq.sn};
       const sage_tensor ck{sl + p.k, k->dtype, 1, ng, Nk, D, ng * Nk * D, sk.sh, sk.sn};
       const sage_tensor cv{sl + p.v, v->dtype, 1, ng, Nk, D, ng * Nk * D, sv.sh, sv.sn};
-      sage_mask cm{};
-      if (mask) cm = chunk_mask(*mask, b, h0, nh);
-      const FusedLayout f = fused_layout(1, nh, ng, Nq, Nk, D, mask ? &cm : nullptr);
-      st = run_fused(&cq, &ck, &cv, causal, sm_scale, return_lse, smooth_k, mask ? &cm : nullptr,
-                     sl + p.o, nh * Nq * D, so.sh, so.sn,
-                     return_lse ? reinterpret_cast<float*>(sl + p.l) : nullptr, f, w + p.fused,
-                     stream);
+      st = compute(b, h0, g0, cq, ck, cv, sl + p.o, so.sh, so.sn,
+                   return_lse ? reinterpret_cast<float*>(sl + p.l) : nullptr);
       if (st) break;
       ok = cudaEventRecord(ps->computed[r], stream) == cudaSuccess;
       // copy out
@@ -817,6 +850,18 @@ sage_status run_host_pipeline(const sage_tensor* q, const sage_tensor* k, const 
                       cudaStreamWaitEvent(stream, ps->join_out, 0) == cudaSuccess;
   if (st) return st;
   return ok && joined ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+// Arguments of the host-resident calls' outputs: out (host, q's logical
+// shape, element strides, 16-byte aligned rows), lse (host, when asked for),
+// a non-negative chunk size.
+sage_status check_host_out(const sage_tensor* q, const void* out, int64_t out_sb, int64_t out_sh,
+                           int64_t out_sn, int return_lse, const float* lse, int64_t chunk_groups) {
+  if (!out || chunk_groups < 0 || (return_lse && !lse)) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(out) || out_sn < q->D || out_sn % 8 || out_sh % 8 || out_sb % 8 || out_sh < 0 ||
+      out_sb < 0)
+    return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
 }
 
 }  // namespace
@@ -900,7 +945,10 @@ size_t sage_attn_fwd_host_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, in
                                           int64_t chunk_groups) {
   if (!valid_dims(B, Hq, Nq, D) || !valid_dims(B, Hkv, Nk, D) || Hq % Hkv || chunk_groups < 0)
     return 0;
-  return pipe_layout(B, Hq, Hkv, Nq, Nk, D, mask, chunk_groups).total;
+  const int64_t G = Hq / Hkv;
+  return pipe_layout(Hq, Hkv, Nq, Nk, D, chunk_groups,
+                     [&](int64_t ng) { return i8_chunk_ws(G, Nq, Nk, D, mask, ng); })
+      .total;
 }
 
 sage_status sage_attn_fwd_host(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
@@ -917,15 +965,84 @@ sage_status sage_attn_fwd_host(const sage_tensor* q, const sage_tensor* k, const
     return SAGE_ERR_INVALID_ARG;
   if ((st = check_qkv_shapes(q->B, q->H, k->H, q->N, k->N, q->D))) return st;
   if ((st = check_mask(mask, q->B, q->H, q->N, k->N))) return st;
-  if (!out || chunk_groups < 0 || (return_lse && !lse)) return SAGE_ERR_INVALID_ARG;
-  if (!aligned16(out) || out_sn < q->D || out_sn % 8 || out_sh % 8 || out_sb % 8 || out_sh < 0 ||
-      out_sb < 0)
-    return SAGE_ERR_INVALID_ARG;
-  const PipeLayout p = pipe_layout(q->B, q->H, k->H, q->N, k->N, q->D, mask, chunk_groups);
+  if ((st = check_host_out(q, out, out_sb, out_sh, out_sn, return_lse, lse, chunk_groups))) return st;
+  const int64_t Nq = q->N, Nk = k->N, D = q->D, G = q->H / k->H;
+  const PipeLayout p = pipe_layout(q->H, k->H, Nq, Nk, D, chunk_groups, [&](int64_t ng) {
+    return i8_chunk_ws(G, Nq, Nk, D, mask, ng);
+  });
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SAGE_ERR_INVALID_ARG;
   if (ws_bytes < p.total) return SAGE_ERR_WORKSPACE;
-  return run_host_pipeline(q, k, v, causal, sm_scale, return_lse, smooth_k, mask, out, out_sb,
-                           out_sh, out_sn, lse, p, static_cast<char*>(ws), stream);
+  char* fw = static_cast<char*>(ws) + p.fused;
+  return run_host_pipeline(
+      q, k, v, return_lse, out, out_sb, out_sh, out_sn, lse, p, static_cast<char*>(ws), stream,
+      [&](int64_t b, int64_t h0, int64_t, const sage_tensor& cq, const sage_tensor& ck,
+          const sage_tensor& cv, char* o, int64_t o_sh, int64_t o_sn, float* l) {
+        sage_mask cm{};
+        if (mask) cm = chunk_mask(*mask, b, h0, cq.H);
+        const FusedLayout f = fused_layout(1, cq.H, ck.H, Nq, Nk, D, mask ? &cm : nullptr);
+        return run_fused(&cq, &ck, &cv, causal, sm_scale, return_lse, smooth_k,
+                         mask ? &cm : nullptr, o, cq.H * Nq * D, o_sh, o_sn, l, f, fw, stream);
+      });
+}
+
+size_t sage_attn_fwd_nvfp4_host_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
+                                                int64_t Nk, int64_t D, int64_t chunk_groups) {
+  if (!valid_dims(B, Hq, Nq, D) || !valid_dims(B, Hkv, Nk, D) || Hq % Hkv || chunk_groups < 0)
+    return 0;
+  const int64_t G = Hq / Hkv;
+  return pipe_layout(Hq, Hkv, Nq, Nk, D, chunk_groups,
+                     [&](int64_t ng) { return nv_chunk_layout(ng * G, ng, Nq, Nk, D).total; })
+      .total;
+}
+
+sage_status sage_attn_fwd_nvfp4_host(const sage_tensor* q, const sage_tensor* k,
+                                     const sage_tensor* v, float sm_scale, int causal,
+                                     int per_block_mean, int64_t unpadded_k_len, int return_lse,
+                                     void* out, int64_t out_sb, int64_t out_sh, int64_t out_sn,
+                                     float* lse, int64_t chunk_groups, void* ws, size_t ws_bytes,
+                                     sage_stream_t stream) {
+  sage_status st;
+  if ((st = check_tensor(q)) || (st = check_tensor(k)) || (st = check_tensor(v))) return st;
+  if (k->dtype != q->dtype || v->dtype != q->dtype) return SAGE_ERR_INVALID_ARG;
+  if (k->B != q->B || v->B != q->B || v->H != k->H || v->N != k->N || k->D != q->D ||
+      v->D != q->D)
+    return SAGE_ERR_INVALID_ARG;
+  if ((st = check_qkv_shapes(q->B, q->H, k->H, q->N, k->N, q->D))) return st;
+  const int64_t L = unpadded_k_len <= 0 ? k->N : unpadded_k_len;
+  if (L > k->N) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_host_out(q, out, out_sb, out_sh, out_sn, return_lse, lse, chunk_groups))) return st;
+  const int64_t Nq = q->N, Nk = k->N, D = q->D, G = q->H / k->H;
+  const PipeLayout p = pipe_layout(q->H, k->H, Nq, Nk, D, chunk_groups, [&](int64_t ng) {
+    return nv_chunk_layout(ng * G, ng, Nq, Nk, D).total;
+  });
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < p.total) return SAGE_ERR_WORKSPACE;
+  char* fw = static_cast<char*>(ws) + p.fused;
+  return run_host_pipeline(
+      q, k, v, return_lse, out, out_sb, out_sh, out_sn, lse, p, static_cast<char*>(ws), stream,
+      [&](int64_t, int64_t, int64_t, const sage_tensor& cq, const sage_tensor& ck,
+          const sage_tensor& cv, char* o, int64_t o_sh, int64_t o_sn, float* l) {
+        const NvChunkLayout f = nv_chunk_layout(cq.H, ck.H, Nq, Nk, D);
+        sage_qkv_nvfp4 z{};
+        z.q = reinterpret_cast<uint8_t*>(fw + f.q4);
+        z.q_sf = reinterpret_cast<uint8_t*>(fw + f.qsf);
+        z.k = reinterpret_cast<uint8_t*>(fw + f.k4);
+        z.k_sf = reinterpret_cast<uint8_t*>(fw + f.ksf);
+        z.v_t = reinterpret_cast<uint8_t*>(fw + f.vt);
+        z.v_sf_t = reinterpret_cast<uint8_t*>(fw + f.vsft);
+        z.qk_correction = reinterpret_cast<float*>(fw + f.corr);
+        z.q_mean = reinterpret_cast<float*>(fw + f.qm);
+        z.k_mean = reinterpret_cast<float*>(fw + f.km);
+        z.q_dot_kmean = return_lse ? reinterpret_cast<float*>(fw + f.qdk) : nullptr;
+        z.B = 1; z.Hq = cq.H; z.Hkv = ck.H; z.Nq = Nq; z.Nk = Nk; z.D = D;
+        z.unpadded_k_len = L;
+        z.per_block_mean = per_block_mean ? 1 : 0;
+        sage_status s2 = run_quantize_nvfp4(&cq, &ck, &cv, per_block_mean, L, &z, fw + f.part,
+                                            f.total - f.part, stream);
+        if (s2) return s2;
+        return run_attention_nvfp4(&z, sm_scale, causal, per_block_mean, return_lse, o, q->dtype,
+                                   cq.H * Nq * D, o_sh, o_sn, l, stream);
+      });
 }
 
 size_t sage_quantize_nvfp4_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,

@@ -240,3 +240,26 @@ def test_host_call_workspace_is_three_chunk_slots_plus_one_chunk_workspace(L):
     # one chunk of everything when the chunk size exceeds the heads
     assert L.sage_attn_fwd_host_workspace_bytes(1, 4, 2, 256, 256, 64, None, 99) == \
         L.sage_attn_fwd_host_workspace_bytes(1, 4, 2, 256, 256, 64, None, 2)
+
+
+def test_nvfp4_host_call_rejects_bad_arguments_on_host(L):
+    byref = ctypes.byref
+    q, k, v = _t(H=4), _t(H=2), _t(H=2)
+    f = L.sage_attn_fwd_nvfp4_host
+    need = L.sage_attn_fwd_nvfp4_host_workspace_bytes(1, 4, 2, 256, 256, 64, 0)
+    assert need > L.sage_attn_fwd_host_workspace_bytes(1, 4, 2, 256, 256, 64, None, 0) // 4
+    ok = dict(q=q, k=k, v=v, ukl=0, lse_flag=1, out=256, sn=64, lse=512, chunk=0, ws=256, nb=need)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(byref(a["q"]), byref(a["k"]), byref(a["v"]), 0.0, 0, 1, a["ukl"], a["lse_flag"],
+                 a["out"], 4 * 256 * 64, 256 * 64, a["sn"], a["lse"], a["chunk"], a["ws"], a["nb"], None)
+    assert call(ukl=257) == S.SAGE_ERR_INVALID_ARG                   # unpadded length > Nk
+    assert call(k=_t(H=2, dtype=1)) == S.SAGE_ERR_INVALID_ARG        # dtype differs from q
+    assert call(q=_t(H=3)) == S.SAGE_ERR_INVALID_ARG                 # Hq % Hkv
+    assert call(lse=0) == S.SAGE_ERR_INVALID_ARG
+    assert call(sn=60) == S.SAGE_ERR_INVALID_ARG
+    assert call(chunk=-2) == S.SAGE_ERR_INVALID_ARG
+    assert call(ws=384) == S.SAGE_ERR_INVALID_ARG
+    assert call(nb=need - 1) == S.SAGE_ERR_WORKSPACE
+    assert L.sage_attn_fwd_nvfp4_host_workspace_bytes(1, 4, 2, 256, 256, 64, -1) == 0

@@ -118,3 +118,37 @@ def test_host_path_back_to_back_calls_share_streams(S):
     assert torch.equal(o1, d1.cpu()) and torch.equal(o2, d2.cpu())
     st, site = S.sage_get_device_status()
     assert st == S.SAGE_OK, site
+
+
+NV_CASES = [
+    # (workload, per_block_mean, causal, chunk_groups, layout)
+    (W.NVFP4.scaled(B=2, Hq=4, Hkv=2, N=300, D=128, unpadded_k_len=260, seed=81), True, False, 1, "HND"),
+    (W.NVFP4.scaled(B=1, Hq=6, Hkv=3, N=384, D=64, unpadded_k_len=384, seed=82), False, True, 2, "NHD"),
+    (W.NVFP4.scaled(B=1, Hq=2, Hkv=2, N=256, D=128, unpadded_k_len=200, seed=83), True, True, 0, "HND"),
+]
+
+
+@pytest.mark.parametrize("w,pbm,causal,chunk,layout", NV_CASES,
+                         ids=lambda c: str(c) if not hasattr(c, "N") else f"{c.B}x{c.Hq}x{c.Hkv}x{c.N}x{c.D}")
+def test_nvfp4_host_path_equals_device_calls(S, w, pbm, causal, chunk, layout):
+    """sage_attn_fwd_nvfp4_host gives the bits of sage_quantize_qkv_nvfp4 +
+    sage_attn_fwd_nvfp4 on the device, for every chunking and layout."""
+    q, k, v = W.make_qkv(w)
+    if layout == "NHD":
+        q, k, v = (t.transpose(1, 2).contiguous() for t in (q, k, v))
+    z = S.sage_quantize_qkv_nvfp4(q.cuda(), k.cuda(), v.cuda(), per_block_mean=pbm,
+                                  unpadded_k_len=w.unpadded_k_len, layout=layout)
+    d_out, d_lse = S.sage_attn_fwd_nvfp4(z, sm_scale=w.sm_scale, causal=causal, return_lse=True,
+                                         out_dtype=q.dtype)
+    torch.cuda.synchronize()
+    out, lse = S.sage_attn_fwd_nvfp4_host(_host(q), _host(k), _host(v), sm_scale=w.sm_scale,
+                                          causal=causal, per_block_mean=pbm,
+                                          unpadded_k_len=w.unpadded_k_len, return_lse=True,
+                                          layout=layout, chunk_groups=chunk)
+    torch.cuda.synchronize()
+    d_out = d_out.cpu() if layout == "HND" else d_out.transpose(1, 2).cpu()
+    assert out.shape == q.shape and out.dtype == q.dtype
+    assert torch.equal(out, d_out)
+    assert torch.equal(lse, d_lse.cpu())
+    st, site = S.sage_get_device_status()
+    assert st == S.SAGE_OK, site
