@@ -225,17 +225,17 @@ def test_host_call_rejects_bad_arguments_on_host(L):
 def test_host_call_workspace_is_three_chunk_slots_plus_one_chunk_workspace(L):
     B_, Hq, Hkv, N, D = 4, 32, 8, 16384, 128
     G = Hq // Hkv
-    # automatic chunk: as many KV-head groups as fit 64 MB of bf16 inputs (2 here)
+    # automatic chunk: the number of KV-head groups nearest to 100 MB of bf16 inputs (4 here)
     per_group_in = (G * N + 2 * N) * D * 2
-    gpc = max(1, (64 << 20) // per_group_in)
-    assert gpc == 2
+    gpc = max(1, ((100 << 20) + per_group_in // 2) // per_group_in)
+    assert gpc == 4
     slot = gpc * (G * N * D * 2 + 2 * N * D * 2 + G * N * D * 2 + G * N * 4)
     one_chunk = L.sage_attn_fwd_workspace_bytes(1, gpc * G, gpc, N, N, D, None)
     need = L.sage_attn_fwd_host_workspace_bytes(B_, Hq, Hkv, N, N, D, None, 0)
     assert need == pytest.approx(3 * slot + one_chunk, abs=3 * 5 * 256)
     # explicit chunking, with a smaller last chunk per batch entry (8 = 3 + 3 + 2)
     need3 = L.sage_attn_fwd_host_workspace_bytes(B_, Hq, Hkv, N, N, D, None, 3)
-    assert need3 == pytest.approx(3 * slot * 3 // 2 + L.sage_attn_fwd_workspace_bytes(
+    assert need3 == pytest.approx(3 * slot * 3 // 4 + L.sage_attn_fwd_workspace_bytes(
         1, 3 * G, 3, N, N, D, None), abs=3 * 5 * 256 + 4096)
     # one chunk of everything when the chunk size exceeds the heads
     assert L.sage_attn_fwd_host_workspace_bytes(1, 4, 2, 256, 256, 64, None, 99) == \
