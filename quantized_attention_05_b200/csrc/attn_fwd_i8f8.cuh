@@ -588,6 +588,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&s_free[wg]);
+      // the P buffer this tile writes was read by PV(n-2): test it now (its
+      // latency overlaps the row max), wait below only if it was not done
+      const bool pbuf_free =
+          n < 2 || mbar_test(&o_ready[wg * 2 + buf], ((n - 2) >> 1) & 1);
 
       // sr holds 1.5*2^23 + S as float bits; hidden keys -> 0.0 (below every score)
       uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
@@ -652,7 +656,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
       // the P buffer being overwritten was read by PV(n-2); O is touched only
       // once PV(n-1) has completed
-      if (n >= 2) {
+      if (!__all_sync(0xffffffffu, pbuf_free)) {
         ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[wg * 2 + buf], ((n - 2) >> 1) & 1,
                                                 SITE_O_READY));
         if (!ok) break;

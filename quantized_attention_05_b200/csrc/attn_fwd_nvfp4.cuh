@@ -414,6 +414,9 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&s_free[buf]);
+      // the P buffer this tile writes was read by PV(n-2): test it now (its
+      // latency overlaps the row max), wait below only if it was not done
+      const bool pbuf_free = n < 2 || mbar_test(&o_ready[buf], ((n - 2) >> 1) & 1);
       // S already holds the scores plus qk_correction (added by the MMA)
       uint32_t vis[2] = {~0u, ~0u};
       if (need) {
@@ -458,7 +461,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       const float bias = LOG2_2688 - m_use;
       const uint64_t b2 = f2_pack(bias, bias);
 
-      if (n >= 2) {
+      if (!__all_sync(0xffffffffu, pbuf_free)) {
         ok = __all_sync(0xffffffffu,
                         mbar_wait(&o_ready[buf], ((n - 2) >> 1) & 1, SITE_O_READY));
         if (!ok) break;
