@@ -1,5 +1,6 @@
 // sage_b200.cu -- the C ABI of include/sage_b200.h: argument validation,
-// workspace layout, TMA descriptors and kernel launches.  Built as one
+// workspace layout, TMA descriptors, kernel launches, and the chunked
+// copy/compute pipeline of the host-buffer calls.  Built as one
 // translation unit with the kernel headers (device state such as the status
 // word lives here once).
 #include <cuda.h>
