@@ -6,13 +6,15 @@
 //
 // One CTA owns two 128-row Q tiles of one (batch, Q head) and streams the
 // 128-key K/V tiles of its KV head:
-//   warp 8      TMA producer: Q tiles once, then K and V^T tiles into a
+//   warp 8      TMA producer: Q tiles once, then K and V tiles (V in
+//               [token, channel] order, read MN-major by the PV MMA) into a
 //               3-stage ring;
-//   warp 9      MMA issuer (one thread): S_i = Q_i K^T with tcgen05
-//               kind::i8 into TMEM (int32, exact), O_i += P_i V with
-//               kind::f8f6f4 (E4M3 x E4M3 -> FP32 in TMEM); it issues the
-//               next tile's QK^T of a Q tile as soon as that tile's S has
-//               been read, so the tensor pipe runs while softmax works;
+//   warp 9      MMA issuer (one thread): S_i = 1.5*2^23 (one f16 MMA) +
+//               Q_i K^T with tcgen05 kind::i8 into TMEM (int32, exact, read
+//               back as a float), O_i += P_i V with kind::f8f6f4 (E4M3 x
+//               E4M3 -> FP32 in TMEM); it issues the next tile's QK^T of a
+//               Q tile as soon as that tile's S has been read, so the tensor
+//               pipe runs while softmax works;
 //   warps 0..7  two softmax warpgroups, one per Q tile, one thread per row:
 //               tcgen05.ld of the int32 scores, dequantisation by
 //               q_scale*k_scale*sm_scale*log2(e), masking, online softmax
@@ -132,17 +134,10 @@ struct AttnLayout {
 static_assert(AttnLayout<128>::bytes(ATT_MAX_NKT) <= 232448, "attention smem");
 static_assert(AttnLayout<64>::bytes(ATT_MAX_NKT) <= 232448, "attention smem");
 
-// Exponentials: pairs i of each 32-key chunk with i % POLY_EVERY ==
-// POLY_EVERY - 1 would be computed by the FMA-pipe polynomial instead of MUFU
-// ex2.  Measured on B200 this kernel is not MUFU-throughput bound (MUFU about
-// half busy), and the polynomial's extra instructions, its clamp among them,
-// cost more than the MUFU time they save (8.43 -> 7.81 ms on the causal GQA
-// 16K workload without it).  A clamp-free degree-3 polynomial (sat-FMA
-// clamp, relative error 8e-5) on one pair in 8 gained under 1 % and moved
-// enough E4M3 roundings of P to break the parity bound on a small case; on
-// one pair in 4 it was slower.  The period is set beyond the 16 pairs of a
-// chunk: every exponential is MUFU.
-constexpr int POLY_EVERY = 1000;
+// Exponentials: every one on MUFU ex2.  Measured on B200 this kernel is
+// not MUFU-throughput bound (MUFU about half busy); FMA-pipe polynomials for
+// a share of them cost more than the MUFU time they saved, and their error
+// moved enough E4M3 roundings of P to break the parity bound on small cases.
 // int32 score S as the float 1.5*2^23 + S (exact for |S| < 2^22): the QK^T
 // MMA accumulates the int32 S onto the bit pattern of 1.5*2^23 (0x4B400000),
 // which an f16 MMA (512 x 1536 summed over K = 16) writes into S first.
@@ -296,12 +291,7 @@ __device__ __forceinline__ float exp_tile(const uint32_t* sr, const uint32_t* vi
                             c2, b2);
         float y0, y1;
         f2_unpack(y, y0, y1);
-        uint64_t p;
-        if ((i + u) % POLY_EVERY == POLY_EVERY - 1) {
-          p = f2_exp2_poly(y0, y1);
-        } else {
-          p = f2_pack(ex2_approx(y0), ex2_approx(y1));
-        }
+        uint64_t p = f2_pack(ex2_approx(y0), ex2_approx(y1));
         if (NEED) {
           float p0, p1;
           f2_unpack(p, p0, p1);

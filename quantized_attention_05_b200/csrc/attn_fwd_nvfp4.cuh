@@ -493,11 +493,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
           const uint64_t y = f2_fma(f2_pack(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2, b2);
           float y0, y1;
           f2_unpack(y, y0, y1);
-          uint64_t p;
-          if (i % POLY_EVERY == POLY_EVERY - 1)
-            p = f2_exp2_poly(y0, y1);
-          else
-            p = f2_pack(ex2_approx(y0), ex2_approx(y1));
+          uint64_t p = f2_pack(ex2_approx(y0), ex2_approx(y1));
           if (need) {
             float p0, p1;
             f2_unpack(p, p0, p1);

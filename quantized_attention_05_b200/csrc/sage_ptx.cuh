@@ -320,33 +320,6 @@ __device__ __forceinline__ float h2_hsum(uint32_t x) {
          __half2float(__ushort_as_half((unsigned short)(x >> 16)));
 }
 
-// 2^y for a pair of fp32 values on the FMA pipe (no MUFU): y is clamped to
-// [-125, ...], split as y = n + f with n = round(y) (via the 1.5*2^23
-// rounding trick) and f in [-0.5, 0.5]; 2^f is a degree-4 polynomial fitted
-// for this library by minimising the maximum relative error on [-0.5, 0.5]
-// (max relative error 2.7e-6 in fp32 Horner form); 2^n is applied by adding
-// n to the exponent field.
-__device__ __forceinline__ uint64_t f2_exp2_poly(float y0, float y1) {
-  y0 = fmaxf(y0, -125.f);
-  y1 = fmaxf(y1, -125.f);
-  const uint64_t y = f2_pack(y0, y1);
-  const uint64_t t = f2_add(y, f2_pack(12582912.f, 12582912.f));       // n in the low mantissa
-  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));     // n as a float
-  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), y);                // f = y - n
-  uint64_t p = f2_fma(f2_pack(0.009569989517331123f, 0.009569989517331123f), f,
-                      f2_pack(0.05591757968068123f, 0.05591757968068123f));
-  p = f2_fma(p, f, f2_pack(0.240247443318367f, 0.240247443318367f));
-  p = f2_fma(p, f, f2_pack(0.6931218504905701f, 0.6931218504905701f));
-  p = f2_fma(p, f, f2_pack(0.9999992847442627f, 0.9999992847442627f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  // bits(t) = 0x4B400000 + n, and 0x4B400000 << 23 wraps to 0: (bits(t) << 23) = n << 23
-  const uint32_t r0 = __float_as_uint(t0) * (1u << 23) + __float_as_uint(p0);
-  const uint32_t r1 = __float_as_uint(t1) * (1u << 23) + __float_as_uint(p1);
-  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
-}
-
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
