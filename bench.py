@@ -331,7 +331,7 @@ def run_ours(args, w):
     ratio = FP4_PER_BF16 if w.nvfp4 else FP8_PER_BF16
     peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * ratio
     peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * ratio
-    achieved = w.ops / (attn_ms * 1e-3) / 1e12
+    achieved = w.visible_ops / (attn_ms * 1e-3) / 1e12
     traffic = None
     tr_path = os.path.join(ROOT, "profiles", "attn_traffic.json")
     if os.path.exists(tr_path):

@@ -55,6 +55,13 @@ class Workload:
         o = 4.0 * self.B * self.Hq * self.N * self.N * self.D
         return o / 2 if self.causal else o
 
+    @property
+    def visible_ops(self) -> float:
+        """Operations on the (query, key) pairs the attention can see: ops,
+        halved again when the mask hides the second half of the keys (the
+        kernels skip key tiles a mask hides entirely)."""
+        return self.ops / 2 if self.mask == "second_half_keys" else self.ops
+
     def scaled(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
 
