@@ -193,7 +193,7 @@ def blas_threads():
 def cpu_baseline(w: W.Workload, budget_s=15.0):
     tokens = 2048
     ops, dt = oracle_sample(w, tokens)
-    reps = max(1, min(8, int(budget_s / max(dt, 1e-3))))
+    reps = max(1, min(64, int(budget_s / max(dt, 1e-3))))   # ~budget_s of CPU work
     tot_ops, tot_t = 0.0, 0.0
     for _ in range(reps):
         o, t = oracle_sample(w, tokens)
