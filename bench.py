@@ -224,12 +224,14 @@ def run_ours(args, w):
         z = S.QuantizedNvfp4.empty(w.B, w.Hq, w.Hkv, w.N, w.N, w.D, ukl, w.per_block_mean, device)
         qws = torch.empty(S.lib().sage_quantize_nvfp4_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.N, w.D),
                           dtype=torch.uint8, device=device)
-        launches_per_step = 6
+        launches_per_step = 6       # column sums x2, means, codes, correction; attention
     else:
         z = S.QuantizedQKV.empty(w.B, w.Hq, w.Hkv, w.N, w.N, w.D, device, with_qdk=True)
         qws = torch.empty(S.lib().sage_quantize_workspace_bytes(w.B, w.Hkv, w.N, w.D),
                           dtype=torch.uint8, device=device)
-        launches_per_step = 3 + (1 if mask is not None else 0)
+        # K-mean/V-amax partials, their combination, block codes; attention
+        # (+ the mask's tile classification)
+        launches_per_step = 4 + (1 if mask is not None else 0)
 
     def step(ev_q=None, ev_a=None, ev_b=None):
         if ev_q is not None:
