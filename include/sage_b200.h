@@ -223,7 +223,12 @@ size_t sage_attn_fwd_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t
  * num_kv_heads, return_lse; pages: "sageattn").
  * num_kv_heads must equal k->H.  smooth_k as in sage_quantize_qkv (the
  * pages' default is on).  out has q's dtype; the other arguments are those
- * of sage_attn_fwd_quantized.  Quantises into the workspace, then attends. */
+ * of sage_attn_fwd_quantized.  Quantises into the workspace, then attends.
+ * A call without queries (q->B == 0 or q->N == 0) has nothing to compute: its
+ * sizes are checked (one dtype, matching batch, Hq % Hkv == 0, k and v of one
+ * length, D 64 or 128, num_kv_heads == k->H), no pointer is looked at, and it
+ * returns SAGE_OK without enqueuing anything.  Keys are required otherwise:
+ * k->N == 0 with queries present is SAGE_ERR_INVALID_ARG. */
 sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
                           int causal, float sm_scale, int num_kv_heads, int return_lse,
                           int smooth_k, const sage_mask* mask, void* out, int64_t out_sb,
@@ -264,7 +269,8 @@ size_t sage_attn_fwd_host_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, in
  * same result with the copies serialised by the driver.  Concurrent calls are
  * serialised while they enqueue (the copy streams are shared per device).
  * On SAGE_ERR_CUDA, work already enqueued still runs and `stream` still waits
- * for it; out and lse are then undefined. */
+ * for it; out and lse are then undefined.  A call without queries returns as
+ * sage_attn_fwd's does. */
 sage_status sage_attn_fwd_host(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
                                int causal, float sm_scale, int num_kv_heads, int return_lse,
                                int smooth_k, const sage_mask* mask, void* out, int64_t out_sb,
@@ -289,7 +295,8 @@ size_t sage_attn_fwd_nvfp4_host_workspace_bytes(int64_t B, int64_t Hq, int64_t H
  * written iff return_lse); unpadded_k_len <= 0 means Nk; sm_scale <= 0
  * selects 1/sqrt(D); ws: DEVICE workspace (256-byte aligned) of
  * sage_attn_fwd_nvfp4_host_workspace_bytes(..., chunk_groups) bytes.  Streams,
- * ordering, host-memory kinds and errors as for sage_attn_fwd_host. */
+ * ordering, host-memory kinds, errors and calls without queries as for
+ * sage_attn_fwd_host (unpadded_k_len must still not exceed k->N). */
 sage_status sage_attn_fwd_nvfp4_host(const sage_tensor* q, const sage_tensor* k,
                                      const sage_tensor* v, float sm_scale, int causal,
                                      int per_block_mean, int64_t unpadded_k_len, int return_lse,

@@ -361,7 +361,7 @@ def sage_attn_fwd_host(q, k, v, causal=False, sm_scale=None, num_kv_heads=None, 
     mstruct = ctypes.byref(mk[0]) if mk else None
     nbytes = L.sage_attn_fwd_host_workspace_bytes(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D, mstruct,
                                                   int(chunk_groups))
-    if nbytes == 0:
+    if nbytes == 0 and tq.B * tq.N:                       # (no queries: nothing to size)
         raise SageError(SAGE_ERR_INVALID_ARG, "sage_attn_fwd_host: invalid sizes")
     if ws is None or ws.numel() < nbytes:
         ws = _ws(nbytes, device)
@@ -413,7 +413,7 @@ def sage_attn_fwd_nvfp4_host(q, k, v, sm_scale=None, causal=False, per_block_mea
     out, to, lse = _host_outputs(q, tq, layout, out, lse, return_lse)
     nbytes = L.sage_attn_fwd_nvfp4_host_workspace_bytes(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D,
                                                         int(chunk_groups))
-    if nbytes == 0:
+    if nbytes == 0 and tq.B * tq.N:
         raise SageError(SAGE_ERR_INVALID_ARG, "sage_attn_fwd_nvfp4_host: invalid sizes")
     if ws is None or ws.numel() < nbytes:
         ws = _ws(nbytes, device)

@@ -858,6 +858,28 @@ sage_status run_host_pipeline(const sage_tensor* q, const sage_tensor* k, const 
   return ok && joined ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
+// A whole-path call without queries (q->B == 0 or q->N == 0) has no output to
+// compute.  Returns true for such a call, with *st set to SAGE_OK when its
+// sizes are consistent (q, k, v of one dtype, matching batch, head counts
+// with Hq % Hkv == 0, k and v of one length, D 64 or 128) and to the error
+// otherwise.  Pointers are not looked at: an empty tensor has no storage.
+// Nothing is launched or enqueued for it.
+bool empty_call(const sage_tensor* q, const sage_tensor* k, const sage_tensor* v,
+                sage_status* st) {
+  if (!q || !k || !v || (q->B != 0 && q->N != 0)) return false;
+  *st = SAGE_ERR_INVALID_ARG;
+  for (const sage_tensor* t : {q, k, v}) {
+    if (t->dtype != SAGE_BF16 && t->dtype != SAGE_FP16) return true;
+    if (t->B < 0 || t->B > (1 << 16) || t->H < 1 || t->H > (1 << 12) || t->N < 0 || t->D < 1)
+      return true;
+  }
+  if (k->dtype != q->dtype || v->dtype != q->dtype || k->B != q->B || v->B != q->B ||
+      v->H != k->H || v->N != k->N || k->D != q->D || v->D != q->D || q->H % k->H)
+    return true;
+  *st = q->D == 64 || q->D == 128 ? SAGE_OK : SAGE_ERR_UNSUPPORTED;
+  return true;
+}
+
 // Arguments of the host-resident calls' outputs: out (host, q's logical
 // shape, element strides, 16-byte aligned rows), lse (host, when asked for),
 // a non-negative chunk size.
@@ -935,6 +957,7 @@ sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage
                           int64_t out_sh, int64_t out_sn, float* lse, void* ws, size_t ws_bytes,
                           sage_stream_t stream) {
   sage_status st;
+  if (empty_call(q, k, v, &st)) return st ? st : num_kv_heads == k->H ? SAGE_OK : SAGE_ERR_INVALID_ARG;
   if ((st = check_tensor(q)) || (st = check_tensor(k)) || (st = check_tensor(v))) return st;
   if (num_kv_heads != k->H) return SAGE_ERR_INVALID_ARG;
   if ((st = check_qkv_shapes(q->B, q->H, k->H, q->N, k->N, q->D))) return st;
@@ -963,6 +986,7 @@ sage_status sage_attn_fwd_host(const sage_tensor* q, const sage_tensor* k, const
                                int64_t out_sh, int64_t out_sn, float* lse, int64_t chunk_groups,
                                void* ws, size_t ws_bytes, sage_stream_t stream) {
   sage_status st;
+  if (empty_call(q, k, v, &st)) return st ? st : num_kv_heads == k->H ? SAGE_OK : SAGE_ERR_INVALID_ARG;
   if ((st = check_tensor(q)) || (st = check_tensor(k)) || (st = check_tensor(v))) return st;
   if (num_kv_heads != k->H || k->dtype != q->dtype || v->dtype != q->dtype)
     return SAGE_ERR_INVALID_ARG;
@@ -1007,6 +1031,7 @@ sage_status sage_attn_fwd_nvfp4_host(const sage_tensor* q, const sage_tensor* k,
                                      float* lse, int64_t chunk_groups, void* ws, size_t ws_bytes,
                                      sage_stream_t stream) {
   sage_status st;
+  if (empty_call(q, k, v, &st)) return st ? st : unpadded_k_len <= k->N ? SAGE_OK : SAGE_ERR_INVALID_ARG;
   if ((st = check_tensor(q)) || (st = check_tensor(k)) || (st = check_tensor(v))) return st;
   if (k->dtype != q->dtype || v->dtype != q->dtype) return SAGE_ERR_INVALID_ARG;
   if (k->B != q->B || v->B != q->B || v->H != k->H || v->N != k->N || k->D != q->D ||

@@ -263,3 +263,37 @@ def test_nvfp4_host_call_rejects_bad_arguments_on_host(L):
     assert call(ws=384) == S.SAGE_ERR_INVALID_ARG
     assert call(nb=need - 1) == S.SAGE_ERR_WORKSPACE
     assert L.sage_attn_fwd_nvfp4_host_workspace_bytes(1, 4, 2, 256, 256, 64, -1) == 0
+
+
+def test_calls_without_queries_return_ok_without_touching_the_device(L):
+    """B == 0 or Nq == 0: the whole-path calls check the sizes, look at no
+    pointer (null here, as for empty tensors) and return SAGE_OK; no CUDA
+    call is made, which is what lets this run on a machine without a GPU."""
+    byref = ctypes.byref
+
+    def fused(q, k, v, nkv=2):
+        return L.sage_attn_fwd(byref(q), byref(k), byref(v), 1, 0.0, nkv, 1, 1, None,
+                               None, 0, 0, 64, None, None, 0, None)
+
+    def host(q, k, v, nkv=2):
+        return L.sage_attn_fwd_host(byref(q), byref(k), byref(v), 1, 0.0, nkv, 1, 1, None,
+                                    None, 0, 0, 64, None, 0, None, 0, None)
+
+    def nvfp4(q, k, v, ukl=0):
+        return L.sage_attn_fwd_nvfp4_host(byref(q), byref(k), byref(v), 0.0, 1, 1, ukl, 1,
+                                          None, 0, 0, 64, None, 0, None, 0, None)
+
+    for f in (fused, host, nvfp4):
+        assert f(_t(ptr=0, H=4, N=0), _t(ptr=0), _t(ptr=0)) == S.SAGE_OK              # no queries
+        assert f(_t(ptr=0, B=0, H=4), _t(ptr=0, B=0), _t(ptr=0, B=0)) == S.SAGE_OK     # no batch
+        assert f(_t(ptr=0, H=4, N=0), _t(ptr=0, N=0), _t(ptr=0, N=0)) == S.SAGE_OK     # no keys either
+        assert f(_t(ptr=0, H=3, N=0), _t(ptr=0), _t(ptr=0)) == S.SAGE_ERR_INVALID_ARG  # Hq % Hkv
+        assert f(_t(ptr=0, H=4, N=0), _t(ptr=0, dtype=1), _t(ptr=0)) == S.SAGE_ERR_INVALID_ARG
+        assert f(_t(ptr=0, H=4, N=0), _t(ptr=0), _t(ptr=0, N=128)) == S.SAGE_ERR_INVALID_ARG
+        assert f(_t(ptr=0, B=0, H=4), _t(ptr=0), _t(ptr=0)) == S.SAGE_ERR_INVALID_ARG  # batch mismatch
+        assert f(_t(ptr=0, H=4, N=0, D=96), _t(ptr=0, D=96), _t(ptr=0, D=96)) == S.SAGE_ERR_UNSUPPORTED
+        # keys are required when there are queries
+        assert f(_t(H=4), _t(N=0), _t(N=0)) == S.SAGE_ERR_INVALID_ARG
+    assert fused(_t(ptr=0, H=4, N=0), _t(ptr=0), _t(ptr=0), nkv=1) == S.SAGE_ERR_INVALID_ARG
+    assert host(_t(ptr=0, H=4, N=0), _t(ptr=0), _t(ptr=0), nkv=1) == S.SAGE_ERR_INVALID_ARG
+    assert nvfp4(_t(ptr=0, H=4, N=0), _t(ptr=0), _t(ptr=0), ukl=257) == S.SAGE_ERR_INVALID_ARG

@@ -147,6 +147,27 @@ def test_causal_bottom_right_when_lengths_differ(S):
         assert_attention_close(out, l, ref, what=f"causal Nq={Nq} Nk={Nk}")
 
 
+def test_calls_without_queries_return_empty_results(S):
+    """No queries (Nq == 0 or B == 0): empty out and LSE from every
+    whole-path call, nothing launched, the device status untouched."""
+    g = torch.Generator().manual_seed(39)
+    k = torch.randn(1, 2, 256, 128, generator=g).to(torch.bfloat16)
+    v = torch.randn(1, 2, 256, 128, generator=g).to(torch.bfloat16)
+    q = torch.empty(1, 4, 0, 128, dtype=torch.bfloat16)
+    out, lse = S.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True, return_lse=True)
+    assert out.shape == (1, 4, 0, 128) and lse.shape == (1, 4, 0)
+    out, lse = S.sage_attn_fwd_host(q, k, v, causal=True, return_lse=True)
+    assert out.shape == (1, 4, 0, 128) and lse.shape == (1, 4, 0)
+    out, lse = S.sage_attn_fwd_nvfp4_host(q, k, v, return_lse=True)
+    assert out.shape == (1, 4, 0, 128) and lse.shape == (1, 4, 0)
+    q0, k0 = torch.empty(0, 4, 256, 128, dtype=torch.bfloat16), torch.empty(0, 2, 256, 128, dtype=torch.bfloat16)
+    out = S.sage_attn_fwd(q0.cuda(), k0.cuda(), k0.cuda())
+    assert out.shape == q0.shape
+    torch.cuda.synchronize()
+    st, site = S.sage_get_device_status()
+    assert st == S.SAGE_OK, site
+
+
 def test_lossless_case_matches_exact_attention(S):
     """On the oracle's lossless inputs the GPU must also land on exact
     attention (up to its fp32 exp2 and bf16 output rounding)."""
