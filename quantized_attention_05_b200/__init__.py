@@ -5,9 +5,14 @@ stream, and every step of the computation runs in the library's CUDA
 kernels.  There is no fallback: if the library cannot be loaded, every call
 raises.
 
-Functions keep the C names: ``sage_quantize_qkv``, ``sage_attn_fwd_quantized``,
-``sage_attn_fwd``, ``sage_debug_qk_int32``, ``sage_debug_pv_fp32``,
-``sage_debug_wait_timeout``, ``sage_get_device_status``.
+Functions keep the C names: ``sage_quantize_qkv`` (and ``_noalloc``),
+``sage_attn_fwd_quantized``, ``sage_attn_fwd``, ``sage_attn_fwd_host``,
+``sage_quantize_qkv_nvfp4``, ``sage_attn_fwd_nvfp4``,
+``sage_attn_fwd_nvfp4_host``, ``sage_attn_fwd_varlen``, ``sage_lse_merge``,
+``sage_lse_merge_finalize``, ``sage_debug_qk_int32``, ``sage_debug_pv_fp32``,
+``sage_debug_wait_timeout``, ``sage_get_device_status``.  The device calls
+take CUDA tensors on one GPU and run with that GPU current; the ``*_host``
+calls take host tensors.
 """
 from __future__ import annotations
 
@@ -152,6 +157,24 @@ def _dtype_code(t):
     raise TypeError(f"q/k/v must be bf16 or fp16, got {t.dtype}")
 
 
+def _cuda_device(*tensors):
+    """The one CUDA device that all the given tensors (None entries skipped)
+    live on.  The device calls take device pointers, so a host tensor, or
+    tensors spread over several GPUs, is refused here, before any pointer
+    reaches the library; the call then runs with that device current."""
+    dev = None
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("expected CUDA tensors (the *_host calls take host memory)")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors on {dev} and {t.device}: all must be on one CUDA device")
+    return dev
+
+
 def _as_tensor(t: torch.Tensor, layout: str = "HND") -> SageTensor:
     """Describe a 4-D tensor.  layout "HND": logical (B, H, N, D);
     "NHD": logical (B, N, H, D).  Strides are passed as they are."""
@@ -221,6 +244,10 @@ class QuantizedQKV:
                    torch.empty(B, Hq, Nq, dtype=torch.float32, **kw) if with_qdk else None,
                    B, Hq, Hkv, Nq, Nk, D)
 
+    def tensors(self):
+        return (self.q, self.q_scale, self.k, self.k_scale, self.k_mean, self.v, self.v_scale,
+                self.q_dot_kmean)
+
     def struct(self) -> SageQkvI8F8:
         p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
         return SageQkvI8F8(p(self.q), p(self.q_scale), p(self.k), p(self.k_scale), p(self.k_mean),
@@ -237,6 +264,7 @@ def sage_quantize_qkv(q, k, v, smooth_k=True, layout="HND", with_qdk=True,
                       out: Optional[QuantizedQKV] = None, ws: Optional[torch.Tensor] = None):
     """smooth_k + per-block INT8 Q/K + per-channel FP8 V (sage_quantize_qkv)."""
     L = lib()
+    dev = _cuda_device(q, k, v, ws, *(out.tensors() if out is not None else ()))
     tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
     if out is None:
         out = QuantizedQKV.empty(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D, q.device, with_qdk)
@@ -244,9 +272,10 @@ def sage_quantize_qkv(q, k, v, smooth_k=True, layout="HND", with_qdk=True,
     if ws is None:
         ws = _ws(nbytes, q.device)
     s = out.struct()
-    _check(L.sage_quantize_qkv(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
-                               int(bool(smooth_k)), ctypes.byref(s), ws.data_ptr(), ws.numel(),
-                               _stream(q.device)), "sage_quantize_qkv")
+    with torch.cuda.device(dev):
+        _check(L.sage_quantize_qkv(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                                   int(bool(smooth_k)), ctypes.byref(s), ws.data_ptr(), ws.numel(),
+                                   _stream(dev)), "sage_quantize_qkv")
     return out
 
 
@@ -255,13 +284,15 @@ def sage_quantize_qkv_noalloc(q, k, v, smooth_k=True, layout="HND", with_qdk=Tru
     """sage_quantize_qkv without a caller workspace: the library's own fixed
     device scratch is used instead (for callers that cannot allocate)."""
     L = lib()
+    dev = _cuda_device(q, k, v, *(out.tensors() if out is not None else ()))
     tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
     if out is None:
         out = QuantizedQKV.empty(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D, q.device, with_qdk)
     s = out.struct()
-    _check(L.sage_quantize_qkv_noalloc(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
-                                       int(bool(smooth_k)), ctypes.byref(s), _stream(q.device)),
-           "sage_quantize_qkv_noalloc")
+    with torch.cuda.device(dev):
+        _check(L.sage_quantize_qkv_noalloc(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                                           int(bool(smooth_k)), ctypes.byref(s), _stream(dev)),
+               "sage_quantize_qkv_noalloc")
     return out
 
 
@@ -269,7 +300,7 @@ def sage_attn_fwd_quantized(qkv: QuantizedQKV, causal=False, sm_scale=None, retu
                             mask=None, out=None, out_dtype=torch.bfloat16, lse=None, ws=None):
     """Fused INT8-QK / FP8-PV attention on quantised inputs."""
     L = lib()
-    dev = qkv.q.device
+    dev = _cuda_device(*qkv.tensors(), mask, out, lse if return_lse else None, ws)
     if out is None:
         out = torch.empty(qkv.B, qkv.Hq, qkv.Nq, qkv.D, dtype=out_dtype, device=dev)
     if return_lse and lse is None:
@@ -280,11 +311,12 @@ def sage_attn_fwd_quantized(qkv: QuantizedQKV, causal=False, sm_scale=None, retu
     if ws is None:
         ws = _ws(L.sage_attn_quantized_workspace_bytes(ctypes.byref(s), mstruct), dev)
     sb, sh, sn, _ = out.stride()
-    _check(L.sage_attn_fwd_quantized(ctypes.byref(s), int(bool(causal)),
-                                     float(sm_scale) if sm_scale else 0.0, int(bool(return_lse)),
-                                     mstruct, out.data_ptr(), _dtype_code(out), sb, sh, sn,
-                                     lse.data_ptr() if return_lse else None, ws.data_ptr(),
-                                     ws.numel(), _stream(dev)), "sage_attn_fwd_quantized")
+    with torch.cuda.device(dev):
+        _check(L.sage_attn_fwd_quantized(ctypes.byref(s), int(bool(causal)),
+                                         float(sm_scale) if sm_scale else 0.0, int(bool(return_lse)),
+                                         mstruct, out.data_ptr(), _dtype_code(out), sb, sh, sn,
+                                         lse.data_ptr() if return_lse else None, ws.data_ptr(),
+                                         ws.numel(), _stream(dev)), "sage_attn_fwd_quantized")
     return (out, lse) if return_lse else out
 
 
@@ -303,6 +335,7 @@ def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, num_kv_heads=None, retur
     Returns out (same shape/layout/dtype as q) and, with return_lse, lse
     [B, Hq, Nq] fp32."""
     L = lib()
+    dev = _cuda_device(q, k, v, mask, out, lse if return_lse else None, ws)
     tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
     if num_kv_heads is None:
         num_kv_heads = tk.H
@@ -316,11 +349,13 @@ def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, num_kv_heads=None, retur
     nbytes = L.sage_attn_fwd_workspace_bytes(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D, mstruct)
     if ws is None or ws.numel() < nbytes:
         ws = _ws(nbytes, q.device)
-    _check(L.sage_attn_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), int(bool(causal)),
-                           float(sm_scale) if sm_scale else 0.0, int(num_kv_heads),
-                           int(bool(return_lse)), int(bool(smooth_k)), mstruct, to.ptr, to.sb,
-                           to.sh, to.sn, lse.data_ptr() if return_lse else None, ws.data_ptr(),
-                           ws.numel(), _stream(q.device)), "sage_attn_fwd")
+    with torch.cuda.device(dev):
+        _check(L.sage_attn_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                               int(bool(causal)), float(sm_scale) if sm_scale else 0.0,
+                               int(num_kv_heads), int(bool(return_lse)), int(bool(smooth_k)),
+                               mstruct, to.ptr, to.sb, to.sh, to.sn,
+                               lse.data_ptr() if return_lse else None, ws.data_ptr(), ws.numel(),
+                               _stream(dev)), "sage_attn_fwd")
     return (out, lse) if return_lse else out
 
 
@@ -350,14 +385,12 @@ def sage_attn_fwd_host(q, k, v, causal=False, sm_scale=None, num_kv_heads=None, 
     for t in (q, k, v):
         if t.is_cuda:
             raise ValueError("sage_attn_fwd_host takes host tensors (use sage_attn_fwd for CUDA tensors)")
-    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    device = _host_call_device(device, mask, ws)
     tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
     if num_kv_heads is None:
         num_kv_heads = tk.H
     out, to, lse = _host_outputs(q, tq, layout, out, lse, return_lse)
     mk = _as_mask(mask, tq.B, tq.H, tq.N, tk.N)
-    if mk is not None and not mask.is_cuda:
-        raise ValueError("mask must be a CUDA tensor")
     mstruct = ctypes.byref(mk[0]) if mk else None
     nbytes = L.sage_attn_fwd_host_workspace_bytes(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D, mstruct,
                                                   int(chunk_groups))
@@ -374,6 +407,21 @@ def sage_attn_fwd_host(q, k, v, causal=False, sm_scale=None, num_kv_heads=None, 
                                     ws.data_ptr(), ws.numel(), _stream(device)),
                "sage_attn_fwd_host")
     return (out, lse) if return_lse else out
+
+
+def _host_call_device(device, *device_tensors):
+    """The GPU a host-memory call runs on (``device``, default the current
+    one), after checking that its device-side tensors (mask, workspace) are
+    CUDA tensors on it."""
+    device = torch.device("cuda" if device is None else device)
+    if device.type != "cuda":
+        raise ValueError(f"device must be a CUDA device, got {device}")
+    if device.index is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    dev = _cuda_device(*device_tensors)
+    if dev is not None and dev != device:
+        raise ValueError(f"mask and ws must be CUDA tensors on {device}, got {dev}")
+    return device
 
 
 def _host_outputs(q, tq, layout, out, lse, return_lse):
@@ -408,7 +456,7 @@ def sage_attn_fwd_nvfp4_host(q, k, v, sm_scale=None, causal=False, per_block_mea
     for t in (q, k, v):
         if t.is_cuda:
             raise ValueError("sage_attn_fwd_nvfp4_host takes host tensors")
-    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    device = _host_call_device(device, ws)
     tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
     out, to, lse = _host_outputs(q, tq, layout, out, lse, return_lse)
     nbytes = L.sage_attn_fwd_nvfp4_host_workspace_bytes(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D,
@@ -450,6 +498,7 @@ def sage_attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_
     [total_q, Hq, D] and, with return_lse, lse (fp32, one [Hq, len_s] block
     per sequence, flat)."""
     L = lib()
+    dev = _cuda_device(q, k, v, cu_seqlens_q, cu_seqlens_k, out, lse if return_lse else None, ws)
     tq, tk, tv = _packed(q), _packed(k), _packed(v)
     if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
         raise TypeError("cu_seqlens must be int32")
@@ -468,13 +517,14 @@ def sage_attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_
                                                     int(max_seqlen_k), tq.D, int(bool(return_lse)))
     if ws is None or ws.numel() < nbytes:
         ws = _ws(nbytes, q.device)
-    _check(L.sage_attn_fwd_varlen(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
-                                  cq.data_ptr(), ck.data_ptr(), nseq, int(max_seqlen_q),
-                                  int(max_seqlen_k), int(bool(causal)),
-                                  float(sm_scale) if sm_scale else 0.0, int(bool(smooth_k)),
-                                  int(bool(return_lse)), out.data_ptr(), sn, sh,
-                                  lse.data_ptr() if return_lse else None, ws.data_ptr(),
-                                  ws.numel(), _stream(q.device)), "sage_attn_fwd_varlen")
+    with torch.cuda.device(dev):
+        _check(L.sage_attn_fwd_varlen(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                                      cq.data_ptr(), ck.data_ptr(), nseq, int(max_seqlen_q),
+                                      int(max_seqlen_k), int(bool(causal)),
+                                      float(sm_scale) if sm_scale else 0.0, int(bool(smooth_k)),
+                                      int(bool(return_lse)), out.data_ptr(), sn, sh,
+                                      lse.data_ptr() if return_lse else None, ws.data_ptr(),
+                                      ws.numel(), _stream(dev)), "sage_attn_fwd_varlen")
     return (out, lse) if return_lse else out
 
 
@@ -482,42 +532,50 @@ def sage_lse_merge(acc, acc_lse, part, part_lse, init=False):
     """Merge a partial attention result (part [B, H, N, D] bf16/fp16 in any
     layout with channel stride 1, part_lse [B, H, N]) into the running fp32
     (acc [B, H, N, D] contiguous, acc_lse [B, H, N]) in place."""
+    dev = _cuda_device(acc, acc_lse, part, part_lse)
     B, H, N, D = part.shape
     sb, sh, sn, sd = part.stride()
     if sd != 1 or not acc.is_contiguous() or acc.dtype != torch.float32 or acc_lse.dtype != torch.float32:
         raise ValueError("acc must be contiguous fp32 and part must have channel stride 1")
     if part_lse.dtype != torch.float32 or not part_lse.is_contiguous() or not acc_lse.is_contiguous():
         raise ValueError("the LSE tensors must be contiguous fp32")
-    _check(lib().sage_lse_merge(acc.data_ptr(), acc_lse.data_ptr(), part.data_ptr(), _dtype_code(part),
-                                sb, sh, sn, part_lse.data_ptr(), B, H, N, D, int(bool(init)),
-                                _stream(part.device)), "sage_lse_merge")
+    with torch.cuda.device(dev):
+        _check(lib().sage_lse_merge(acc.data_ptr(), acc_lse.data_ptr(), part.data_ptr(),
+                                    _dtype_code(part), sb, sh, sn, part_lse.data_ptr(), B, H, N, D,
+                                    int(bool(init)), _stream(dev)), "sage_lse_merge")
 
 
 def sage_lse_merge_finalize(acc, out):
     """Write the merged fp32 result into ``out`` (bf16/fp16 [B, H, N, D])."""
+    dev = _cuda_device(acc, out)
     B, H, N, D = out.shape
     sb, sh, sn, sd = out.stride()
     if sd != 1 or not acc.is_contiguous():
         raise ValueError("out must have channel stride 1 and acc be contiguous")
-    _check(lib().sage_lse_merge_finalize(acc.data_ptr(), out.data_ptr(), _dtype_code(out), sb, sh, sn,
-                                         B, H, N, D, _stream(out.device)), "sage_lse_merge_finalize")
+    with torch.cuda.device(dev):
+        _check(lib().sage_lse_merge_finalize(acc.data_ptr(), out.data_ptr(), _dtype_code(out), sb, sh,
+                                             sn, B, H, N, D, _stream(dev)), "sage_lse_merge_finalize")
     return out
 
 
 def sage_debug_qk_int32(qkv: QuantizedQKV, b, h, qblk, kblk):
-    tile = torch.empty(128, 128, dtype=torch.int32, device=qkv.q.device)
+    dev = _cuda_device(*qkv.tensors())
+    tile = torch.empty(128, 128, dtype=torch.int32, device=dev)
     s = qkv.struct()
-    _check(lib().sage_debug_qk_int32(ctypes.byref(s), b, h, qblk, kblk, tile.data_ptr(),
-                                     _stream(qkv.q.device)), "sage_debug_qk_int32")
+    with torch.cuda.device(dev):
+        _check(lib().sage_debug_qk_int32(ctypes.byref(s), b, h, qblk, kblk, tile.data_ptr(),
+                                         _stream(dev)), "sage_debug_qk_int32")
     return tile
 
 
 def sage_debug_pv_fp32(qkv: QuantizedQKV, p_e4m3: torch.Tensor, b, h_kv, kblk):
+    dev = _cuda_device(*qkv.tensors(), p_e4m3)
     p = p_e4m3.contiguous().view(torch.uint8)
-    acc = torch.empty(128, qkv.D, dtype=torch.float32, device=qkv.q.device)
+    acc = torch.empty(128, qkv.D, dtype=torch.float32, device=dev)
     s = qkv.struct()
-    _check(lib().sage_debug_pv_fp32(ctypes.byref(s), p.data_ptr(), b, h_kv, kblk, acc.data_ptr(),
-                                    _stream(qkv.q.device)), "sage_debug_pv_fp32")
+    with torch.cuda.device(dev):
+        _check(lib().sage_debug_pv_fp32(ctypes.byref(s), p.data_ptr(), b, h_kv, kblk, acc.data_ptr(),
+                                        _stream(dev)), "sage_debug_pv_fp32")
     return acc
 
 
@@ -571,6 +629,10 @@ class QuantizedNvfp4:
                    torch.empty(B, Hq, Nq, **f32) if with_qdk else None,
                    B, Hq, Hkv, Nq, Nk, D, unpadded_k_len, bool(per_block_mean))
 
+    def tensors(self):
+        return (self.q, self.q_sf, self.k, self.k_sf, self.v_t, self.v_sf_t, self.qk_correction,
+                self.q_mean, self.k_mean, self.q_dot_kmean)
+
     def struct(self) -> SageQkvNvfp4:
         p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
         return SageQkvNvfp4(p(self.q), p(self.q_sf), p(self.k), p(self.k_sf), p(self.v_t),
@@ -584,6 +646,7 @@ def sage_quantize_qkv_nvfp4(q, k, v, per_block_mean=True, unpadded_k_len=None, l
                             ws: Optional[torch.Tensor] = None):
     """NVFP4 quantisation (sage_quantize_qkv_nvfp4)."""
     L = lib()
+    dev = _cuda_device(q, k, v, ws, *(out.tensors() if out is not None else ()))
     tq, tk, tv = _as_tensor(q, layout), _as_tensor(k, layout), _as_tensor(v, layout)
     ukl = tk.N if unpadded_k_len is None else int(unpadded_k_len)
     if out is None:
@@ -592,9 +655,11 @@ def sage_quantize_qkv_nvfp4(q, k, v, per_block_mean=True, unpadded_k_len=None, l
     if ws is None:
         ws = _ws(L.sage_quantize_nvfp4_workspace_bytes(tq.B, tq.H, tk.H, tq.N, tk.N, tq.D), q.device)
     s = out.struct()
-    _check(L.sage_quantize_qkv_nvfp4(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
-                                     int(bool(per_block_mean)), ukl, ctypes.byref(s), ws.data_ptr(),
-                                     ws.numel(), _stream(q.device)), "sage_quantize_qkv_nvfp4")
+    with torch.cuda.device(dev):
+        _check(L.sage_quantize_qkv_nvfp4(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                                         int(bool(per_block_mean)), ukl, ctypes.byref(s),
+                                         ws.data_ptr(), ws.numel(), _stream(dev)),
+               "sage_quantize_qkv_nvfp4")
     return out
 
 
@@ -602,7 +667,7 @@ def sage_attn_fwd_nvfp4(qkv: QuantizedNvfp4, sm_scale=None, causal=False, per_bl
                         return_lse=True, out=None, out_dtype=torch.bfloat16, lse=None):
     """NVFP4 attention on pre-quantised inputs (sage_attn_fwd_nvfp4)."""
     L = lib()
-    dev = qkv.q.device
+    dev = _cuda_device(*qkv.tensors(), out, lse if return_lse else None)
     pbm = qkv.per_block_mean if per_block_mean is None else bool(per_block_mean)
     if out is None:
         out = torch.empty(qkv.B, qkv.Hq, qkv.Nq, qkv.D, dtype=out_dtype, device=dev)
@@ -610,8 +675,10 @@ def sage_attn_fwd_nvfp4(qkv: QuantizedNvfp4, sm_scale=None, causal=False, per_bl
         lse = torch.empty(qkv.B, qkv.Hq, qkv.Nq, dtype=torch.float32, device=dev)
     sb, sh, sn, _ = out.stride()
     s = qkv.struct()
-    _check(L.sage_attn_fwd_nvfp4(ctypes.byref(s), float(sm_scale) if sm_scale else 0.0,
-                                 int(bool(causal)), int(pbm), int(bool(return_lse)), out.data_ptr(),
-                                 _dtype_code(out), sb, sh, sn, lse.data_ptr() if return_lse else None,
-                                 _stream(dev)), "sage_attn_fwd_nvfp4")
+    with torch.cuda.device(dev):
+        _check(L.sage_attn_fwd_nvfp4(ctypes.byref(s), float(sm_scale) if sm_scale else 0.0,
+                                     int(bool(causal)), int(pbm), int(bool(return_lse)),
+                                     out.data_ptr(), _dtype_code(out), sb, sh, sn,
+                                     lse.data_ptr() if return_lse else None, _stream(dev)),
+               "sage_attn_fwd_nvfp4")
     return (out, lse) if return_lse else out
