@@ -40,9 +40,13 @@
  *     stream); the call returns after enqueueing.  Argument errors are
  *     detected on the host before anything is enqueued.
  *   - Errors: SAGE_ERR_INVALID_ARG (malformed argument), SAGE_ERR_UNSUPPORTED
- *     (valid but outside what the kernels handle, e.g. head_dim not in
- *     {64,128}), SAGE_ERR_WORKSPACE (workspace too small), SAGE_ERR_CUDA (a
- *     CUDA call failed at launch).  Device-side failures (a bounded wait that
+ *     (valid but outside what the kernels handle: head_dim not in {64,128},
+ *     more than 262144 tokens in a sequence, more than 65535 (batch entry, Q
+ *     head) pairs in one device call -- (sequence, KV head) pairs for
+ *     sage_attn_fwd_varlen; the *_host calls work a chunk at a time and are
+ *     not bound by this -- or 2^31 or more padded rows in one tensor),
+ *     SAGE_ERR_WORKSPACE (workspace too small), SAGE_ERR_CUDA (a CUDA call
+ *     failed at launch).  Device-side failures (a bounded wait that
  *     ran out) set a device status word read by sage_get_device_status.
  *   - The calls are thread-safe.  Calls that share a workspace or outputs
  *     must be ordered by the caller (same stream or events).  Library state:

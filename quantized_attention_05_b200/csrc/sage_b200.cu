@@ -71,10 +71,15 @@ sage_status check_qkv_shapes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int
   return SAGE_OK;
 }
 
+// The (batch entry, head) pairs of one launch form a grid's y or z extent,
+// which is at most 65535.
+constexpr int64_t kMaxGridYZ = 65535;
+
 sage_status check_qkv(const sage_qkv_i8f8* z, bool need_qdk) {
   if (!z) return SAGE_ERR_INVALID_ARG;
   sage_status st = check_qkv_shapes(z->B, z->Hq, z->Hkv, z->Nq, z->Nk, z->D);
   if (st != SAGE_OK) return st;
+  if (z->B * z->Hq > kMaxGridYZ) return SAGE_ERR_UNSUPPORTED;
   if (!z->q || !z->q_scale || !z->k || !z->k_scale || !z->k_mean || !z->v || !z->v_scale)
     return SAGE_ERR_INVALID_ARG;
   if (need_qdk && !z->q_dot_kmean) return SAGE_ERR_INVALID_ARG;
@@ -374,6 +379,7 @@ sage_status check_nvfp4(const sage_qkv_nvfp4* z, bool need_qdk) {
   if (!z) return SAGE_ERR_INVALID_ARG;
   sage_status st = check_qkv_shapes(z->B, z->Hq, z->Hkv, z->Nq, z->Nk, z->D);
   if (st != SAGE_OK) return st;
+  if (z->B * z->Hq > kMaxGridYZ) return SAGE_ERR_UNSUPPORTED;
   if (!z->q || !z->q_sf || !z->k || !z->k_sf || !z->v_t || !z->v_sf_t || !z->qk_correction ||
       !z->q_mean || !z->k_mean)
     return SAGE_ERR_INVALID_ARG;
@@ -961,6 +967,7 @@ sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage
   if ((st = check_tensor(q)) || (st = check_tensor(k)) || (st = check_tensor(v))) return st;
   if (num_kv_heads != k->H) return SAGE_ERR_INVALID_ARG;
   if ((st = check_qkv_shapes(q->B, q->H, k->H, q->N, k->N, q->D))) return st;
+  if (q->B * q->H > kMaxGridYZ) return SAGE_ERR_UNSUPPORTED;
   if ((st = check_mask(mask, q->B, q->H, q->N, k->N))) return st;
   const FusedLayout f = fused_layout(q->B, q->H, k->H, q->N, k->N, q->D, mask);
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SAGE_ERR_INVALID_ARG;
@@ -1176,6 +1183,7 @@ sage_status sage_attn_fwd_varlen(const sage_tensor* q, const sage_tensor* k, con
   if (max_seqlen_q < 1 || max_seqlen_k < 1) return SAGE_ERR_INVALID_ARG;
   if (max_seqlen_q > 128 * ATT_MAX_NKT || max_seqlen_k > 128 * ATT_MAX_NKT)
     return SAGE_ERR_UNSUPPORTED;
+  if (nseq * k->H > kMaxGridYZ) return SAGE_ERR_UNSUPPORTED;
   if (!out || !aligned16(out) || out_sn < q->D || out_sn % 8 || out_sh % 8 || out_sh < 0)
     return SAGE_ERR_INVALID_ARG;
   if ((return_lse != 0) != (lse != nullptr)) return SAGE_ERR_INVALID_ARG;

@@ -297,3 +297,29 @@ def test_calls_without_queries_return_ok_without_touching_the_device(L):
     assert fused(_t(ptr=0, H=4, N=0), _t(ptr=0), _t(ptr=0), nkv=1) == S.SAGE_ERR_INVALID_ARG
     assert host(_t(ptr=0, H=4, N=0), _t(ptr=0), _t(ptr=0), nkv=1) == S.SAGE_ERR_INVALID_ARG
     assert nvfp4(_t(ptr=0, H=4, N=0), _t(ptr=0), _t(ptr=0), ukl=257) == S.SAGE_ERR_INVALID_ARG
+
+
+def test_device_calls_refuse_more_head_pairs_than_a_grid_holds(L):
+    """More than 65535 (batch entry, Q head) pairs in one device call --
+    (sequence, KV head) pairs in a varlen call -- is SAGE_ERR_UNSUPPORTED,
+    found on the host before anything is enqueued; the host-buffer call,
+    which works one chunk of heads at a time, is not bound by it."""
+    byref = ctypes.byref
+    q, k = _t(B=64, H=1025, N=128), _t(B=64, H=1, N=128)          # 65600 pairs
+    assert L.sage_attn_fwd(byref(q), byref(k), byref(k), 0, 0.0, 1, 0, 1, None, 256, 0, 0, 64,
+                           None, 256, 1 << 40, None) == S.SAGE_ERR_UNSUPPORTED
+    z = _q(B=64, Hq=1025, Hkv=1, Nq=128, Nk=128)
+    assert L.sage_quantize_qkv(byref(q), byref(k), byref(k), 1, byref(z), 256, 1 << 40,
+                               None) == S.SAGE_ERR_UNSUPPORTED
+    assert L.sage_attn_fwd_quantized(byref(z), 0, 0.0, 0, None, 256, 0, 0, 128 * 64, 64, None, 256,
+                                     1 << 40, None) == S.SAGE_ERR_UNSUPPORTED
+    # 65472 pairs pass the size checks: the next check (a mask of the wrong
+    # key length) is the one that answers
+    zz = _q(B=64, Hq=1023, Hkv=1, Nq=128, Nk=128)
+    bad_mask = S.SageMask(256, 1, 1, 128, 64, 0, 0, 128)
+    assert L.sage_attn_fwd_quantized(byref(zz), 0, 0.0, 0, byref(bad_mask), 256, 0, 0, 128 * 64, 64,
+                                     None, 256, 1 << 40, None) == S.SAGE_ERR_INVALID_ARG
+    assert L.sage_attn_fwd_host_workspace_bytes(64, 1025, 1, 128, 128, 64, None, 0) > 0
+    pq, pk = _t(H=4, N=1 << 20), _t(H=1, N=1 << 20)                # packed: 65600 sequences x 1 KV head
+    assert L.sage_attn_fwd_varlen(byref(pq), byref(pk), byref(pk), 256, 256, 65600, 16, 16, 0, 0.0,
+                                  1, 0, 256, 64, 64, None, 256, 1 << 40, None) == S.SAGE_ERR_UNSUPPORTED
