@@ -20,6 +20,7 @@ import ctypes
 import dataclasses
 import math
 import os
+import threading
 from typing import Optional
 
 import torch
@@ -69,6 +70,7 @@ class SageQkvNvfp4(ctypes.Structure):
 
 
 _lib = None
+_lib_lock = threading.Lock()
 
 
 def lib():
@@ -76,6 +78,13 @@ def lib():
     global _lib
     if _lib is not None:
         return _lib
+    with _lib_lock:
+        if _lib is None:
+            _lib = _load()
+    return _lib
+
+
+def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing; build it with "
                           "`python -m quantized_attention_05_b200.build`")
@@ -135,7 +144,6 @@ def lib():
         fn = getattr(L, name)
         fn.restype = res
         fn.argtypes = args
-    _lib = L
     return L
 
 
