@@ -47,6 +47,38 @@ FP8_PER_BF16 = 2.0
 # dense FP4 : BF16 (9 vs 2.25 PFLOP/s nominal)
 FP4_PER_BF16 = 4.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Two more denominators reported beside the measured-bf16 one: NVIDIA's dense
+# datasheet peaks per B200 (TFLOP/s), and the tcgen05 MMA rate measured on
+# this part (a 128x128x32 kind::i8 or kind::f8f6f4 MMA every 64 clocks per
+# SM: 8192 MACs per clock per SM) at the SM clock sampled during the run.
+DATASHEET_TFLOPS = {"int8/fp8": 4500.0, "fp4": 9000.0}
+MMA_MACS_PER_CLK_SM = {"int8/fp8": 8192}
+N_SMS = 148
+
+
+def extra_denominators(achieved, sm_mhz, nvfp4):
+    """frac of `achieved` TFLOP/s against the datasheet dense peak and, where
+    measured, against the MMA issue rate at the sampled SM clock."""
+    kind = "fp4" if nvfp4 else "int8/fp8"
+    d = {"peak_datasheet": DATASHEET_TFLOPS[kind],
+         "frac_datasheet": round(achieved / DATASHEET_TFLOPS[kind], 4)}
+    macs = MMA_MACS_PER_CLK_SM.get(kind)
+    if macs and sm_mhz:
+        rate = 2.0 * macs * N_SMS * sm_mhz * 1e6 / 1e12
+        d.update(peak_mma_rate=round(rate, 1), frac_mma_rate=round(achieved / rate, 4),
+                 mma_rate_source=f"measured tcgen05 {kind} MMA rate x {N_SMS} SMs at {sm_mhz:g} MHz")
+    return d
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 # ------------------------------------------------------------------ ranks
@@ -170,13 +202,18 @@ def oracle_sample(w: W.Workload, tokens: int):
     Returns (ops, seconds)."""
     import oracle as O
     G = w.Hq // w.Hkv
-    ws = w.scaled(B=1, Hq=G, Hkv=1, N=tokens)
+    ukl = w.unpadded_k_len if w.unpadded_k_len and w.unpadded_k_len < tokens else None
+    ws = w.scaled(B=1, Hq=G, Hkv=1, N=tokens, unpadded_k_len=ukl)
     q, k, v = W.make_qkv(ws)
     mask = W.make_mask(ws)
     t0 = time.perf_counter()
-    oz = O.quantize_qkv_i8f8(q, k, v)
-    O.attention_i8f8(oz, causal=ws.causal, sm_scale=ws.sm_scale,
-                     mask=None if mask is None else mask.numpy())
+    if ws.nvfp4:
+        oz = O.quantize_qkv_nvfp4(q, k, v, per_block_mean=ws.per_block_mean, unpadded_k_len=ukl)
+        O.attention_nvfp4(oz, causal=ws.causal, sm_scale=ws.sm_scale)
+    else:
+        oz = O.quantize_qkv_i8f8(q, k, v)
+        O.attention_i8f8(oz, causal=ws.causal, sm_scale=ws.sm_scale,
+                         mask=None if mask is None else mask.numpy())
     dt = time.perf_counter() - t0
     return ws.ops, dt
 
@@ -200,8 +237,18 @@ def cpu_baseline(w: W.Workload, budget_s=15.0):
         tot_ops += o
         tot_t += t
     return {"value": tot_ops / tot_t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{reps} x (first KV-head group of batch 0, {w.Hq // w.Hkv} Q heads, first "
+            "cpu": cpu_model(), "sample": f"{reps} x (first KV-head group of batch 0, {w.Hq // w.Hkv} Q heads, first "
                       f"{tokens} tokens: oracle quantise + attend in full); {tot_t:.1f} s of CPU work"}
+
+
+def workload_config(w: W.Workload, ranks: int):
+    """The `config` object of both arms' JSON lines."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "D": w.D,
+            "causal": w.causal, "return_lse": True, "mask": w.mask, "input_dtype": "bf16",
+            "nvfp4": w.nvfp4, "unpadded_k_len": w.unpadded_k_len,
+            "l2": f"inputs larger than L2 (q/k/v bf16 "
+                  f"{(w.B * (w.Hq + 2 * w.Hkv) * w.N * w.D * 2) >> 20} MiB per step, not flushed)",
+            "parallelism": f"replicas x{ranks}"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -361,12 +408,7 @@ def run_ours(args, w):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": ("nvfp4 (e2m1 x e2m1, e4m3 block-16 scales) -> f32" if w.nvfp4 else
                   "i8xi8->i32 (QK), e4m3xe4m3->f32 (PV)"), "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "D": w.D,
-                   "causal": w.causal, "return_lse": True, "mask": w.mask, "input_dtype": "bf16",
-                   "nvfp4": w.nvfp4, "unpadded_k_len": w.unpadded_k_len,
-                   "l2": f"inputs larger than L2 (q/k/v bf16 "
-                         f"{(w.B * (w.Hq + 2 * w.Hkv) * w.N * w.D * 2) >> 20} MiB per step, not flushed)",
-                   "parallelism": f"replicas x{ranks}"},
+        "config": workload_config(w, ranks),
         "roofline": {"bound": "tensor",
                      "kernel": "attn_fwd_nvfp4_kernel<128>" if w.nvfp4 else "attn_fwd_i8f8_kernel<128>",
                      "achieved": round(achieved, 1), "peak": round(peak_sus, 1), "unit": "TFLOP/s",
@@ -386,6 +428,7 @@ def run_ours(args, w):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    line["roofline"].update(extra_denominators(achieved, (clocks or {}).get("sm_mhz"), w.nvfp4))
     if rank == 0 and ranks == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
@@ -427,11 +470,9 @@ def run_reference(args, w):
         "warmup": args.warmup, "ms_per_step": round(1e3 * tot_t / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 (oracle)", "data": "synthetic", "impl": "reference",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "D": w.D,
-                   "causal": w.causal, "return_lse": True, "mask": w.mask, "input_dtype": "bf16",
-                   "parallelism": "cpu oracle, rank 0"},
+        "config": workload_config(w, ws_),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                         "sample": sample},
+                         "cpu": cpu_model(), "sample": sample + "; rank 0 only, on the host cores"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -68,3 +68,30 @@ def test_reference_arm_line_on_cpu(capsys):
 def test_warmup_below_three_is_rejected():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])
+
+
+def test_extra_denominators():
+    d = bench.extra_denominators(1225.1, 1965.0, nvfp4=False)
+    # 2 ops x 8192 MACs x 148 SMs x 1.965 GHz = 4765 TOPS
+    assert d["peak_mma_rate"] == pytest.approx(4765.0, abs=1.0)
+    assert d["frac_mma_rate"] == pytest.approx(1225.1 / 4765.0, abs=1e-4)
+    assert d["peak_datasheet"] == 4500.0 and d["frac_datasheet"] == pytest.approx(0.2722, abs=1e-4)
+    nv = bench.extra_denominators(830.0, 1965.0, nvfp4=True)
+    assert nv["peak_datasheet"] == 9000.0 and "peak_mma_rate" not in nv
+    assert "peak_mma_rate" not in bench.extra_denominators(1000.0, None, nvfp4=False)
+
+
+def test_both_arms_share_the_config():
+    assert bench.workload_config(W.CAUSAL_GQA, 1)["l2"].startswith("inputs larger than L2")
+    assert bench.workload_config(W.NVFP4, 2)["parallelism"] == "replicas x2"
+
+
+def test_oracle_sample_times_the_nvfp4_oracle_for_the_nvfp4_workload(monkeypatch):
+    import oracle as O
+    seen = []
+    real_q, real_a = O.quantize_qkv_nvfp4, O.attention_nvfp4
+    monkeypatch.setattr(O, "quantize_qkv_nvfp4", lambda *a, **k: seen.append("q") or real_q(*a, **k))
+    monkeypatch.setattr(O, "attention_nvfp4", lambda *a, **k: seen.append("a") or real_a(*a, **k))
+    ops, dt = bench.oracle_sample(W.NVFP4, 256)
+    assert seen == ["q", "a"] and dt > 0
+    assert ops == W.NVFP4.scaled(B=1, Hq=1, Hkv=1, N=256).ops
