@@ -429,6 +429,8 @@ def run_ours(args, w):
         "clocks": clocks,
     }
     line["roofline"].update(extra_denominators(achieved, (clocks or {}).get("sm_mhz"), w.nvfp4))
+    if w.visible_ops != w.ops:      # a mask hides pairs: the step's TOPS over the visible ones too
+        line["value_visible_pairs"] = round(ranks * w.visible_ops / (ms_step * 1e-3) / 1e12, 2)
     if rank == 0 and ranks == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
