@@ -172,7 +172,10 @@ typedef struct {
 } sage_qkv_nvfp4;
 
 /* ------------------------------------------------------------------ info */
+/* A static, human-readable name of a status code ("unknown status" for a
+ * value outside the enum).  Never NULL; the caller does not free it. */
 const char* sage_status_str(sage_status status);
+/* A static string naming the library and its target (sm_100a).  Never NULL. */
 const char* sage_version(void);
 
 /* Device status word: synchronises `stream`, returns SAGE_ERR_TIMEOUT if a
