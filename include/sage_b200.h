@@ -244,7 +244,9 @@ sage_status sage_attn_fwd(const sage_tensor* q, const sage_tensor* k, const sage
 
 /* ------------------------------------------------------- host-resident inputs */
 /* Workspace bytes of sage_attn_fwd_host for chunks of `chunk_groups` (batch
- * entry, KV head) groups (0 = automatic, about 100 MB of inputs per chunk):
+ * entry, KV head) groups (0 = automatic: about 100 MB of inputs per chunk,
+ * with a single group in the call's first and last chunks, which shortens
+ * the copy before the first kernel and the work after the last copy):
  * three staging slots, each holding one chunk's Q/K/V, output and LSE, plus
  * the quantise + attend workspace of one chunk.  mask as for the call (only
  * its B and H matter).  0 for invalid sizes. */
@@ -285,10 +287,10 @@ sage_status sage_attn_fwd_host(const sage_tensor* q, const sage_tensor* k, const
                                void* ws, size_t ws_bytes, sage_stream_t stream);
 
 /* Workspace bytes of sage_attn_fwd_nvfp4_host for chunks of `chunk_groups`
- * (batch entry, KV head) groups (0 = automatic, about 25 MB of inputs per
- * chunk): three staging slots plus
- * one chunk's quantised NVFP4 arrays and quantiser sums.  0 for invalid
- * sizes. */
+ * (batch entry, KV head) groups (0 = automatic: about 25 MB of inputs per
+ * chunk, single-group first and last chunks as for sage_attn_fwd_host):
+ * three staging slots plus the largest chunk's quantised NVFP4 arrays and
+ * quantiser sums.  0 for invalid sizes. */
 size_t sage_attn_fwd_nvfp4_host_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
                                                 int64_t Nk, int64_t D, int64_t chunk_groups);
 

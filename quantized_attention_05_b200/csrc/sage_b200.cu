@@ -22,6 +22,7 @@
 #include "quantize_nvfp4.cuh"
 #include "attn_fwd_nvfp4.cuh"
 #include "merge.cuh"
+#include "pipe_schedule.h"
 
 using namespace sage;
 
@@ -687,17 +688,18 @@ sage_mask chunk_mask(const sage_mask& m, int64_t b, int64_t h0, int64_t nh) {
 }
 
 struct PipeLayout {
-  int64_t gpc;                 // KV-head groups per chunk
+  int64_t gpc;                 // KV-head groups per chunk (at most)
+  bool edge;                   // one-group first and last chunks (pipe_chunk_groups)
   size_t q, k, v, o, l, slot;  // offsets in a slot, slot bytes
   size_t fused, total;         // one chunk's quantise + attend workspace
 };
 
-// Staging slots for chunks of `chunk_groups` KV-head groups (0: automatic)
-// and, after them, the largest per-chunk quantise + attend workspace that
-// `chunk_ws(ng)` reports for ng groups (full chunks and the last, smaller
-// chunk of a batch entry).
+// Staging slots for chunks of `chunk_groups` KV-head groups (0: automatic,
+// with one-group first and last chunks) and, after them, the largest
+// per-chunk quantise + attend workspace that `chunk_ws(ng)` reports for the
+// chunk sizes the schedule uses.
 template <typename ChunkWs>
-PipeLayout pipe_layout(int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
+PipeLayout pipe_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D,
                        int64_t chunk_groups, size_t auto_bytes, ChunkWs chunk_ws) {
   const int64_t G = Hq / Hkv;
   const size_t per_group = (size_t)(G * Nq + 2 * Nk) * D * 2;
@@ -707,6 +709,7 @@ PipeLayout pipe_layout(int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t 
   gpc = std::min(gpc, Hkv);
   PipeLayout p{};
   p.gpc = gpc;
+  p.edge = chunk_groups == 0 && gpc > 1 && B * Hkv > 2;
   size_t o = 0;
   p.q = o; o += align256((size_t)gpc * G * Nq * D * 2);
   p.k = o; o += align256((size_t)gpc * Nk * D * 2);
@@ -715,9 +718,14 @@ PipeLayout pipe_layout(int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t 
   p.l = o; o += align256((size_t)gpc * G * Nq * 4);
   p.slot = o;
   p.fused = kPipeSlots * p.slot;
+  // every chunk size of the schedule: the first, a middle and the last batch
+  // entry cover every case pipe_chunk_groups distinguishes
   size_t fw = 0;
-  for (const int64_t ng : {gpc, Hkv % gpc})
-    if (ng > 0) fw = std::max(fw, chunk_ws(ng));
+  for (const int64_t b : {int64_t(0), std::min<int64_t>(1, B - 1), B - 1})
+    for (int64_t g0 = 0, ng = 0; g0 < Hkv; g0 += ng) {
+      ng = pipe_chunk_groups(b, g0, B, Hkv, gpc, p.edge);
+      fw = std::max(fw, chunk_ws(ng));
+    }
   p.total = p.fused + fw;
   return p;
 }
@@ -814,8 +822,9 @@ sage_status run_host_pipeline(const sage_tensor* q, const sage_tensor* k, const 
             cudaStreamWaitEvent(ps->out, ps->start, 0) == cudaSuccess;
   int64_t c = 0;
   for (int64_t b = 0; ok && b < B; ++b) {
-    for (int64_t g0 = 0; ok && g0 < Hkv; g0 += p.gpc, ++c) {
-      const int64_t ng = std::min(p.gpc, Hkv - g0), nh = ng * G, h0 = g0 * G;
+    for (int64_t g0 = 0, ng = 0; ok && g0 < Hkv; g0 += ng, ++c) {
+      ng = pipe_chunk_groups(b, g0, B, Hkv, p.gpc, p.edge);
+      const int64_t nh = ng * G, h0 = g0 * G;
       const int r = (int)(c % kPipeRing);
       char* sl = w + (c % kPipeSlots) * p.slot;
       // copy in, once the chunk that last used this slot has been computed
@@ -982,7 +991,7 @@ size_t sage_attn_fwd_host_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, in
   if (!valid_dims(B, Hq, Nq, D) || !valid_dims(B, Hkv, Nk, D) || Hq % Hkv || chunk_groups < 0)
     return 0;
   const int64_t G = Hq / Hkv;
-  return pipe_layout(Hq, Hkv, Nq, Nk, D, chunk_groups, kPipeChunkI8,
+  return pipe_layout(B, Hq, Hkv, Nq, Nk, D, chunk_groups, kPipeChunkI8,
                      [&](int64_t ng) { return i8_chunk_ws(G, Nq, Nk, D, mask, ng); })
       .total;
 }
@@ -1004,7 +1013,7 @@ sage_status sage_attn_fwd_host(const sage_tensor* q, const sage_tensor* k, const
   if ((st = check_mask(mask, q->B, q->H, q->N, k->N))) return st;
   if ((st = check_host_out(q, out, out_sb, out_sh, out_sn, return_lse, lse, chunk_groups))) return st;
   const int64_t Nq = q->N, Nk = k->N, D = q->D, G = q->H / k->H;
-  const PipeLayout p = pipe_layout(q->H, k->H, Nq, Nk, D, chunk_groups, kPipeChunkI8,
+  const PipeLayout p = pipe_layout(q->B, q->H, k->H, Nq, Nk, D, chunk_groups, kPipeChunkI8,
                                    [&](int64_t ng) { return i8_chunk_ws(G, Nq, Nk, D, mask, ng); });
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SAGE_ERR_INVALID_ARG;
   if (ws_bytes < p.total) return SAGE_ERR_WORKSPACE;
@@ -1026,7 +1035,7 @@ size_t sage_attn_fwd_nvfp4_host_workspace_bytes(int64_t B, int64_t Hq, int64_t H
   if (!valid_dims(B, Hq, Nq, D) || !valid_dims(B, Hkv, Nk, D) || Hq % Hkv || chunk_groups < 0)
     return 0;
   const int64_t G = Hq / Hkv;
-  return pipe_layout(Hq, Hkv, Nq, Nk, D, chunk_groups, kPipeChunkNv,
+  return pipe_layout(B, Hq, Hkv, Nq, Nk, D, chunk_groups, kPipeChunkNv,
                      [&](int64_t ng) { return nv_chunk_layout(ng * G, ng, Nq, Nk, D).total; })
       .total;
 }
@@ -1049,7 +1058,7 @@ sage_status sage_attn_fwd_nvfp4_host(const sage_tensor* q, const sage_tensor* k,
   if (L > k->N) return SAGE_ERR_INVALID_ARG;
   if ((st = check_host_out(q, out, out_sb, out_sh, out_sn, return_lse, lse, chunk_groups))) return st;
   const int64_t Nq = q->N, Nk = k->N, D = q->D, G = q->H / k->H;
-  const PipeLayout p = pipe_layout(q->H, k->H, Nq, Nk, D, chunk_groups, kPipeChunkNv,
+  const PipeLayout p = pipe_layout(q->B, q->H, k->H, Nq, Nk, D, chunk_groups, kPipeChunkNv,
                                    [&](int64_t ng) { return nv_chunk_layout(ng * G, ng, Nq, Nk, D).total; });
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SAGE_ERR_INVALID_ARG;
   if (ws_bytes < p.total) return SAGE_ERR_WORKSPACE;

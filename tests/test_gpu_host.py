@@ -38,6 +38,7 @@ CASES = [
     (W.TINY.scaled(B=2, Hq=6, Hkv=3, N=300, D=128, seed=71), True, 2),    # ragged last chunk
     (W.TINY.scaled(B=1, Hq=8, Hkv=2, N=640, D=128, seed=72), False, 0),   # automatic: one chunk
     (W.TINY.scaled(B=3, Hq=4, Hkv=4, N=200, D=64, seed=73), True, 1),     # a chunk per head
+    (W.TINY.scaled(B=2, Hq=8, Hkv=4, N=384, D=128, seed=70), True, 0),    # automatic: chunks 1, 3, 3, 1
 ]
 
 
@@ -125,6 +126,7 @@ NV_CASES = [
     (W.NVFP4.scaled(B=2, Hq=4, Hkv=2, N=300, D=128, unpadded_k_len=260, seed=81), True, False, 1, "HND"),
     (W.NVFP4.scaled(B=1, Hq=6, Hkv=3, N=384, D=64, unpadded_k_len=384, seed=82), False, True, 2, "NHD"),
     (W.NVFP4.scaled(B=1, Hq=2, Hkv=2, N=256, D=128, unpadded_k_len=200, seed=83), True, True, 0, "HND"),
+    (W.NVFP4.scaled(B=2, Hq=6, Hkv=3, N=256, D=128, unpadded_k_len=250, seed=84), True, False, 0, "NHD"),
 ]
 
 
