@@ -24,8 +24,12 @@ readings are listed in the repository's design notes.
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 against closed forms, brute force on tiny inputs, lossless special cases,
-library conversions and invariants.  The P-quantisation step of the NVFP4
-attention is pinned only through its lossless special case.
+library conversions and invariants.  The NVFP4 means (per 128-token Q block
+over its valid rows, or global; K over the first ``unpadded_k_len`` keys)
+are pinned against exact rational sums, and the NVFP4 quantisation of P
+against vectors worked out by hand from the E2M1 and E4M3 grids.  The NVFP4
+attention's tie bound (``attention_nvfp4(tie_band=...)``) is checked to hold
+every output a perturbation of P' within the band produces.
 """
 from .formats import (bf16_round, e2m1_decode, e2m1_encode, e2m1_round, e4m3_decode,  # noqa: F401
                       e4m3_encode, e4m3_round, exact_mean_f32, f32, fraction_to_f32,

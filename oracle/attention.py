@@ -105,19 +105,23 @@ def exact_attention(q, k, v, causal=False, sm_scale=None, mask=None, rows=None,
     return out, lse
 
 
-def _online_softmax_rows(s, vis, vdec, quantise_p, p_gain):
+def _online_softmax_rows(s, vis, vdec, quantise_p, p_gain, p_delta=None):
     """Tile-ordered online softmax for a block of rows of one (b, h).
 
     s: [R, Nk] float64 scores; vis: visibility; vdec: [Nk, D] decoded V;
     quantise_p(P') maps the pre-scaled probabilities of a tile [R, 128] to
-    their decoded quantised values.  Returns (acc, l, m) where
-    out = acc / (p_gain * l).
+    their decoded quantised values.  Returns (acc, l, m, bnd) where
+    out = acc / (p_gain * l).  With ``p_delta`` (P' -> the largest change of
+    each decoded value under a small relative perturbation of P'), ``bnd``
+    [R, D] bounds how far acc can move by such perturbations:
+    sum over keys of |change| * |V|, rescaled like acc; otherwise None.
     """
     R, Nk = s.shape
     D = vdec.shape[1]
     m = np.full(R, -np.inf)
     l = np.zeros(R)
     acc = np.zeros((R, D))
+    bnd = None if p_delta is None else np.zeros((R, D))
     for t0 in range(0, Nk, BLOCK):
         t1 = min(Nk, t0 + BLOCK)
         st = np.where(vis[:, t0:t1], s[:, t0:t1], -np.inf)
@@ -129,8 +133,10 @@ def _online_softmax_rows(s, vis, vdec, quantise_p, p_gain):
         l = l * alpha + p.sum(axis=1)
         pq = quantise_p(p_gain * p)
         acc = acc * alpha[:, None] + pq @ vdec[t0:t1]
+        if bnd is not None:
+            bnd = bnd * alpha[:, None] + p_delta(p_gain * p) @ np.abs(vdec[t0:t1])
         m = m_new
-    return acc, l, m
+    return acc, l, m, bnd
 
 
 def _bf16_keep_nan(x):
@@ -158,6 +164,57 @@ def _p_nvfp4(pp):
     y = (xv * inv[..., None]).astype(np.float64)
     dec = F.e2m1_round(y) * s.astype(np.float64)[..., None]
     return dec.reshape(R, Tp)[:, :T]
+
+
+def _nearby_grid_values(x, grid, band):
+    """For values x >= 0 and a sorted grid of non-negative representable
+    values with round-to-nearest: the representable value x rounds to, and
+    the one it would round to instead if it moved by a relative amount of
+    at most ``band`` across a midpoint (the same value when no midpoint is
+    that close).  Values above the grid's top saturate to it."""
+    x = np.asarray(x, np.float64)
+    mids = (grid[1:] + grid[:-1]) / 2
+    i = np.searchsorted(mids, x, side="left")           # x <= mids[i]: rounds down to grid[i]
+    i = np.minimum(i, len(grid) - 1)
+    # nearest midpoint below / above x
+    lo_mid = np.where(i > 0, mids[np.maximum(i - 1, 0)], -np.inf)
+    hi_mid = np.where(i < len(mids), mids[np.minimum(i, len(mids) - 1)], np.inf)
+    near_lo = x - lo_mid <= band * x
+    near_hi = hi_mid - x <= band * x
+    alt = np.where(near_hi, np.minimum(i + 1, len(grid) - 1), np.where(near_lo, np.maximum(i - 1, 0), i))
+    return grid[i], grid[alt]
+
+
+def _p_nvfp4_delta(pp, band):
+    """The largest change of each decoded NVFP4 P' value (rows x keys of one
+    tile) that a relative perturbation of P' of at most ``band`` can cause.
+
+    Such a perturbation (the GPU's fp32 exponentials and score arithmetic
+    differ from this oracle's float64 ones by a few 1e-6 relative) can move
+    an element across an E2M1 rounding midpoint (one grid step times the
+    vector's scale) or move the vector's amax/6 across an E4M3 midpoint, in
+    which case the whole vector is quantised with the neighbouring scale.
+    Every such alternative is enumerated; the result is elementwise
+    max |alternative - nominal| (0 where no midpoint is within reach)."""
+    R, T = pp.shape
+    Tp = (T + NVFP4_VEC - 1) // NVFP4_VEC * NVFP4_VEC
+    x = np.zeros((R, Tp), dtype=np.float32)
+    x[:, :T] = pp
+    xv = x.reshape(R, Tp // NVFP4_VEC, NVFP4_VEC).astype(np.float32)
+    e4 = np.unique(F.e4m3_decode(np.arange(0x7F, dtype=np.uint8)))      # 0 .. 448
+    a = np.max(np.abs(xv), axis=-1)
+    r = (a / np.float32(6.0)).astype(np.float64)
+    s_nom, s_alt = _nearby_grid_values(r, e4, band)
+    nominal = _p_nvfp4(pp).reshape(R, -1)
+    nominal = np.pad(nominal, ((0, 0), (0, Tp - T))).reshape(xv.shape)
+    delta = np.zeros(xv.shape)
+    for sc in (s_nom, s_alt):
+        scf = sc.astype(np.float32)
+        inv = np.where(scf > 0, np.float32(1.0) / np.where(scf > 0, scf, 1), np.float32(0))
+        y = (xv * inv.astype(np.float32)[..., None]).astype(np.float64)
+        for g in _nearby_grid_values(np.abs(y), F.E2M1_GRID, band):
+            delta = np.maximum(delta, np.abs(g * sc[..., None] - nominal))
+    return delta.reshape(R, Tp)[:, :T]
 
 
 def attention_i8f8(qz, causal=False, sm_scale=None, mask=None, rows=None, heads=None,
@@ -196,7 +253,7 @@ def attention_i8f8(qz, causal=False, sm_scale=None, mask=None, rows=None, heads=
         vis = _visible(rows, keys, Nq, Nk, causal, None if m4 is None else m4[b, h][rows])
         vis &= s > -np.inf
         vdec = F.e4m3_decode(qz["v_t"][b, g, :, :Nk]).T          # [Nk, D]
-        acc, l, m = _online_softmax_rows(s, vis, vdec, _p_e4m3, 448.0)
+        acc, l, m, _ = _online_softmax_rows(s, vis, vdec, _p_e4m3, 448.0)
         vs = qz["v_scale"][b, g].astype(np.float64)
         ok = l > 0
         o = np.where(ok[:, None], acc * vs[None, :] / (448.0 * np.where(ok, l, 1))[:, None], 0.0)
@@ -206,8 +263,15 @@ def attention_i8f8(qz, causal=False, sm_scale=None, mask=None, rows=None, heads=
     return dict(out=_bf16_keep_nan(out), out_f64=out, lse=lse, rows=rows)
 
 
-def attention_nvfp4(qz, causal=False, sm_scale=None, rows=None, heads=None):
-    """Oracle of the NVFP4 attention on the output of ``quantize_qkv_nvfp4``."""
+def attention_nvfp4(qz, causal=False, sm_scale=None, rows=None, heads=None, tie_band=None):
+    """Oracle of the NVFP4 attention on the output of ``quantize_qkv_nvfp4``.
+
+    With ``tie_band`` (a relative width, e.g. 1e-5) the result also holds
+    ``out_tie_bound`` [B, Hq, R, D]: how far the output can move when P' is
+    perturbed by at most that relative amount before its NVFP4 quantisation
+    (``_p_nvfp4_delta``).  A row that sees few keys hinges on single E2M1
+    roundings of P', so every output in out +- out_tie_bound is as correct as
+    the oracle's own for an implementation whose P' differs by rounding."""
     B, Hq, Hkv, Nq, Nk, D = (qz[x] for x in ("B", "Hq", "Hkv", "Nq", "Nk", "D"))
     L = qz["unpadded_k_len"]
     G = Hq // Hkv
@@ -217,6 +281,8 @@ def attention_nvfp4(qz, causal=False, sm_scale=None, rows=None, heads=None):
     heads = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else list(heads)
     out = np.full((B, Hq, len(rows), D), np.nan)
     lse = np.full((B, Hq, len(rows)), np.nan)
+    tie = None if tie_band is None else np.full((B, Hq, len(rows), D), np.nan)
+    p_delta = None if tie_band is None else (lambda pp: _p_nvfp4_delta(pp, tie_band))
 
     def deq(code, sf, lead):
         vals = F.e2m1_decode(code).reshape(lead + (-1, NVFP4_VEC))
@@ -230,12 +296,17 @@ def attention_nvfp4(qz, causal=False, sm_scale=None, rows=None, heads=None):
         s = sm_scale * (qd @ kd.T + corr)
         vis = _visible(rows, keys, Nq, Nk, causal, None, kv_limit=L)
         vdec = deq(qz["v_t"][b, g], qz["v_sf_t"][b, g], (D,))[:, :Nk].T     # [Nk, D]
-        acc, l, m = _online_softmax_rows(s, vis, vdec, _p_nvfp4, 448.0 * 6.0)
+        acc, l, m, bnd = _online_softmax_rows(s, vis, vdec, _p_nvfp4, 448.0 * 6.0, p_delta)
         ok = l > 0
         out[b, h] = np.where(ok[:, None], acc / (2688.0 * np.where(ok, l, 1))[:, None], 0.0)
+        if tie is not None:
+            tie[b, h] = np.where(ok[:, None], bnd / (2688.0 * np.where(ok, l, 1))[:, None], 0.0)
         lse[b, h] = np.where(ok, m + np.log(np.where(ok, l, 1)) + sm_scale * qz["q_dot_kmean"][b, h, rows],
                              -np.inf)
-    return dict(out=_bf16_keep_nan(out), out_f64=out, lse=lse, rows=rows)
+    res = dict(out=_bf16_keep_nan(out), out_f64=out, lse=lse, rows=rows)
+    if tie is not None:
+        res["out_tie_bound"] = tie
+    return res
 
 
 def cosine(a, b):

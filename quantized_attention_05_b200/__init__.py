@@ -18,7 +18,6 @@ from __future__ import annotations
 
 import ctypes
 import dataclasses
-import math
 import os
 import threading
 from typing import Optional
@@ -596,10 +595,6 @@ def sage_get_device_status():
     site = ctypes.c_uint32(0)
     st = lib().sage_get_device_status(_stream(), ctypes.byref(site))
     return st, site.value
-
-
-def default_sm_scale(D):
-    return 1.0 / math.sqrt(D)
 
 
 @dataclasses.dataclass

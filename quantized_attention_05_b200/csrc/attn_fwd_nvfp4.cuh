@@ -59,7 +59,9 @@ struct NvAttnArgs {
 // x / 6 rounded to nearest even, for every fp32 x whose quotient is normal
 // (checked exhaustively against the IEEE division by tests/test_div6.py):
 // the product with RN(1/6), then one correction with the exact residual
-// fma(-q0, 6, x).  Smaller quotients can be one unit off, which no E4M3 code
+// fma(-q0, 6, x) -- Markstein's residual correction of a reciprocal product
+// (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Dev. 34(1), 1990).  Smaller quotients can be one unit off, which no E4M3 code
 // sees (they are below half its smallest subnormal, 2^-10).
 __device__ __forceinline__ float div6_rn(float x) {
   const float c = 0.16666667f;   // RN(1/6) = 0x1.555556p-3

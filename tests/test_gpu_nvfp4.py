@@ -90,22 +90,25 @@ ACASES = [
 def test_nvfp4_attention_on_oracle_codes(S, w, causal):
     q, k, v = W.make_qkv(w)
     oz = O.quantize_qkv_nvfp4(q, k, v, per_block_mean=True, unpadded_k_len=w.unpadded_k_len)
-    ref = O.attention_nvfp4(oz, causal=causal)
+    ref = O.attention_nvfp4(oz, causal=causal, tie_band=TIE_BAND)
     out, lse = S.sage_attn_fwd_nvfp4(nvfp4_from_oracle(S, oz), causal=causal)
     if not causal:
         assert_attention_close(out, lse, ref, what=f"nvfp4 {w.N}")
-        return
-    # Causal rows that see few keys hinge on single E2M1 roundings of P: the
-    # oracle itself moves by up to 1/16 there when P changes by 2e-6 relative
-    # (tests/test_oracle_attention.py, test_nvfp4_short_causal_rows_are_tie_sensitive).  Rows seeing >= 128
-    # keys get the parity bound; the others a bound of one E2M1 step of one
-    # key's weight, and the cosine over all rows.
-    long_rows = np.arange(127, w.N)
-    ref_long = dict(ref, out=ref["out"][:, :, long_rows], lse=ref["lse"][:, :, long_rows])
-    assert_attention_close(out, lse, ref_long, rows=long_rows, what=f"nvfp4 causal {w.N}, long rows")
+    # Rows that see few keys (causal) hinge on single E2M1 roundings of P':
+    # the oracle enumerates every rounding a relative change of P' below
+    # TIE_BAND can flip and bounds the output move per element
+    # (out_tie_bound); every row is held to that bound plus the parity bound,
+    # the LSE (which uses the unquantised P) to the parity bound alone.
     o = out.float().cpu().numpy()
+    excess = np.abs(o - ref["out"]) - ref["out_tie_bound"]
+    assert excess.max() <= 2e-2, f"max excess {excess.max():.3g} over the tie bound"
     assert O.cosine(o, ref["out"]) >= 0.9995
-    assert np.abs(o - ref["out"]).max() <= 0.25
+    np.testing.assert_allclose(lse.cpu().numpy(), ref["lse"], rtol=0, atol=2e-2)
+
+
+# The GPU's P' differs from the oracle's float64 one by its fp32 score
+# arithmetic and MUFU exponentials: a few 1e-6 relative.
+TIE_BAND = 1e-5
 
 
 def test_nvfp4_whole_path_global_mean(S):

@@ -287,3 +287,79 @@ def test_float_mask_row_constant_shifts_only_the_lse():
     np.testing.assert_allclose(b["out_f64"], a["out_f64"], rtol=0, atol=1e-12)
     np.testing.assert_allclose(b["lse"] - a["lse"], np.broadcast_to(shift[..., 0], a["lse"].shape),
                                rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------ NVFP4 P quantisation, by hand
+# ("flashinfer.nvfp4_attention_sm120_fwd": P is quantised to NVFP4 for the PV
+# product -- per 16 keys an E4M3 scale factor E4M3(amax / 6) and E2M1 codes of
+# P' / scale, round to nearest with ties to the even code, saturating at 6.)
+# Each vector's decoded values are worked out by hand from the E2M1 grid
+# {0, .5, 1, 1.5, 2, 3, 4, 6} and the E4M3 grid, not by the oracle's code.
+P_HAND = [
+    # amax 1536: scale E4M3(256) = 256 exactly, so P'/256 is exact and every
+    # tie lands on a midpoint: 2.5 -> 2, 1.75 -> 2, 1.25 -> 1, 0.75 -> 1, 0.25 -> 0
+    ([1536, 1024, 768, 640, 512, 448, 384, 320, 256, 192, 128, 64, 100, 50, 1300, 1270],
+     [1536, 1024, 768, 512, 512, 512, 384, 256, 256, 256, 128, 0, 128, 0, 1536, 1024]),
+    # amax 2688 (the largest P' = 448 * 6): scale 448; no value near a midpoint
+    ([2688, 2000, 1400, 1000, 700, 500, 300, 150, 90, 2300, 1600, 1200, 800, 550, 400, 0],
+     [2688, 1792, 1344, 896, 672, 448, 224, 224, 0, 2688, 1792, 1344, 896, 448, 448, 0]),
+    # amax 1000: amax/6 = 166.7 rounds to the E4M3 value 160 (grid step 16 in
+    # [128, 256)); 1000/160 = 6.25 saturates to 6
+    ([1000, 880, 720, 600, 520, 410, 300, 210, 130, 60, 30, 960, 640, 480, 320, 240],
+     [960, 960, 640, 640, 480, 480, 320, 240, 160, 80, 0, 960, 640, 480, 320, 240]),
+    # amax 0.05: amax/6 = 0.00833 is an E4M3 subnormal, 4 * 2^-9 = 2^-7
+    ([0.05, 0.03, 0.01, 0.004, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0],
+     [6 / 128, 4 / 128, 1.5 / 128, 0.5 / 128] + [0] * 12),
+    # an all-zero vector (a key range the row does not see): scale 0, codes 0
+    ([0] * 16, [0] * 16),
+]
+
+
+def test_p_nvfp4_hand_computed_vectors():
+    from oracle import attention as A
+    pp = np.array([v for v, _ in P_HAND], dtype=np.float64)          # 5 rows x 16 keys
+    want = np.array([d for _, d in P_HAND], dtype=np.float64)
+    np.testing.assert_array_equal(A._p_nvfp4(pp), want)
+    # a 128-key tile is eight independent vectors: rotate the rows through it
+    tile = np.concatenate([np.roll(pp, s, axis=0) for s in range(8)], axis=1)
+    wtile = np.concatenate([np.roll(want, s, axis=0) for s in range(8)], axis=1)
+    np.testing.assert_array_equal(A._p_nvfp4(tile), wtile)
+
+
+def test_p_nvfp4_tie_bound_covers_every_small_perturbation():
+    """The oracle's tie bound (``attention_nvfp4(tie_band=...)``) must hold
+    every output that P' perturbed by less than the band produces: a
+    perturbed run stays inside out +- out_tie_bound on every row, and the
+    bound is non-trivial exactly on the rows that see few keys."""
+    from oracle import attention as A
+    w = W.NVFP4.scaled(B=1, Hq=4, Hkv=2, N=640, D=128, unpadded_k_len=600, seed=5)
+    q, k, v = W.make_qkv(w)
+    oz = O.quantize_qkv_nvfp4(q, k, v, per_block_mean=True, unpadded_k_len=600)
+    band = 1e-5
+    ref = O.attention_nvfp4(oz, causal=True, tie_band=band)
+    bound = ref["out_tie_bound"]
+    orig = A._p_nvfp4
+    worst = 0.0
+    try:
+        for seed in range(3):
+            rng = np.random.default_rng(seed)
+            A._p_nvfp4 = lambda pp: orig(pp * (1 + rng.uniform(-0.9 * band, 0.9 * band, pp.shape)))
+            alt = O.attention_nvfp4(oz, causal=True)
+            d = np.abs(alt["out_f64"] - ref["out_f64"])
+            assert np.all(d <= bound + 1e-12)
+            worst = max(worst, d.max())
+    finally:
+        A._p_nvfp4 = orig
+    assert worst > 2e-2                                  # the flips do happen here
+    short = bound[:, :, :127].max()
+    assert short > 2e-2 and bound[:, :, 256:].max() < 2e-2
+
+
+def test_p_nvfp4_tie_bound_is_zero_without_nearby_midpoints():
+    """Lossless NVFP4 inputs put every P' on a representable value (never
+    within 1e-5 of a midpoint), so the tie bound vanishes."""
+    from lossless_cases import LN2, nvfp4_case
+    q, k, v = nvfp4_case(B=1, Hq=2, Hkv=1, N=256, D=64, L=256, seed=3)
+    oz = O.quantize_qkv_nvfp4(q, k, v, per_block_mean=True, unpadded_k_len=256)
+    r = O.attention_nvfp4(oz, causal=True, sm_scale=LN2, tie_band=1e-5)
+    assert np.all(r["out_tie_bound"] == 0)

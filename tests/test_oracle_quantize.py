@@ -131,3 +131,85 @@ def test_nvfp4_global_mean_is_shared_by_blocks():
     np.testing.assert_array_equal(qz["q_mean"][:, :, 0], qz["q_mean"][:, :, 1])
     qzb = O.quantize_qkv_nvfp4(q, k, v, per_block_mean=True)
     assert not np.array_equal(qzb["q_mean"][:, :, 0], qzb["q_mean"][:, :, 1])
+
+
+# ------------------------------------------------------------ NVFP4 means, pinned by exact sums
+# ("flashinfer.nvfp4_attention_sm120_fwd": ``per_block_mean`` -- one Q mean per
+# 128-token Q block, qk_correction "one row per 128-token Q block";
+# ``unpadded_k_len`` -- keys at and beyond it are padding; thu-ml/sageattention
+# llms.txt, "FP4 Attention for Blackwell GPUs": per_block_mean off uses one
+# global mean instead)
+def _offset_blocks(q, offsets):
+    """Q with a constant added to every row of each 128-token block, so that
+    block means differ by far more than the FP4 quantisation error."""
+    q = q.clone().double()
+    for blk, off in enumerate(offsets):
+        q[:, :, blk * 128:(blk + 1) * 128] += off
+    return q.to(torch.bfloat16)
+
+
+def _frac_mean(x, lo, hi):
+    return O.fraction_to_f32(sum((Fraction(float(t)) for t in x[lo:hi]), Fraction(0)) / (hi - lo))
+
+
+@pytest.mark.parametrize("per_block_mean", [True, False])
+def test_nvfp4_q_means_are_exact_means_of_the_valid_rows(per_block_mean):
+    """N = 300: blocks of 128, 128 and 44 valid rows.  Each q_mean entry is
+    the exact mean of exactly the valid rows of its block (or of all 300
+    rows), rounded once to fp32: a divisor of 128 for the ragged block, rows
+    assigned to the wrong block or padding rows in the sum all fail."""
+    q, k, v = _qkv(N=300, D=64, Hq=2, Hkv=1, seed=21)
+    q = _offset_blocks(q, [5.0, -3.0, 8.0])
+    qz = O.quantize_qkv_nvfp4(q, k, v, per_block_mean=per_block_mean, unpadded_k_len=300)
+    qq = q.double().numpy()
+    assert qz["q_mean"].shape == (1, 2, 3, 64)
+    for h in range(2):
+        for c in (0, 17, 63):
+            col = qq[0, h, :, c]
+            for qb, (lo, hi) in enumerate([(0, 128), (128, 256), (256, 300)]):
+                want = _frac_mean(col, lo, hi) if per_block_mean else _frac_mean(col, 0, 300)
+                assert qz["q_mean"][0, h, qb, c] == np.float32(want), (h, c, qb)
+
+
+def test_nvfp4_k_mean_is_over_the_unpadded_keys_only():
+    """unpadded_k_len = 250 of N = 300, with the 50 padding rows far from the
+    others (+10): the K mean is the exact mean of rows 0..249 alone, and the
+    smoothed K reconstructed from its codes tracks K - that mean."""
+    q, k, v = _qkv(N=300, D=64, Hq=2, Hkv=1, seed=22)
+    k = k.clone().double()
+    k[:, :, 250:] += 10.0
+    k = k.to(torch.bfloat16)
+    qz = O.quantize_qkv_nvfp4(q, k, v, per_block_mean=True, unpadded_k_len=250)
+    kk = k.double().numpy()
+    for c in range(64):
+        assert qz["k_mean"][0, 0, c] == np.float32(_frac_mean(kk[0, 0, :, c], 0, 250)), c
+    # deq(K codes) stays within the E2M1 half-step bound of K - kmean on the
+    # valid rows; a mean over all 300 rows would be off by ~1.7 everywhere
+    s = O.e4m3_decode(qz["k_sf"][0, 0, :250]).astype(np.float64)           # [250, 4]
+    dec = (O.e2m1_decode(qz["k"][0, 0, :250]).reshape(250, 4, 16) * s[..., None]).reshape(250, 64)
+    want = kk[0, 0, :250] - qz["k_mean"][0, 0].astype(np.float64)
+    y = np.abs(want) / np.repeat(np.where(s > 0, s, 1), 16, axis=-1)
+    half = np.where(y < 2, 0.25, np.where(y < 4, 0.5, 1.0)) * np.repeat(s, 16, axis=-1)
+    assert np.all(np.abs(dec - want) <= half * (1 + 1e-5) + 1e-6)
+
+
+@pytest.mark.parametrize("per_block_mean", [True, False])
+def test_nvfp4_q_codes_follow_their_own_block_mean(per_block_mean):
+    """With block offsets +5 / -3 / +8, deq(Q codes) must equal Q minus the
+    exact mean of the row's own block (or the global mean) within the E2M1
+    half-step bound: a row smoothed by another block's mean is off by >= 3."""
+    q, k, v = _qkv(N=300, D=64, Hq=2, Hkv=1, seed=23)
+    q = _offset_blocks(q, [5.0, -3.0, 8.0])
+    qz = O.quantize_qkv_nvfp4(q, k, v, per_block_mean=per_block_mean, unpadded_k_len=300)
+    qq = q.double().numpy()
+    for h in range(2):
+        for i in (0, 127, 128, 255, 256, 299):
+            blk = i // 128 if per_block_mean else None
+            lo, hi = ((blk * 128, min(300, blk * 128 + 128)) if per_block_mean else (0, 300))
+            mean = np.array([_frac_mean(qq[0, h, :, c], lo, hi) for c in range(64)])
+            s = O.e4m3_decode(qz["q_sf"][0, h, i]).astype(np.float64)          # [4]
+            dec = (O.e2m1_decode(qz["q"][0, h, i]).reshape(4, 16) * s[:, None]).ravel()
+            want = qq[0, h, i] - mean
+            y = np.abs(want) / np.repeat(np.where(s > 0, s, 1), 16)
+            half = np.where(y < 2, 0.25, np.where(y < 4, 0.5, 1.0)) * np.repeat(s, 16)
+            assert np.all(np.abs(dec - want) <= half * (1 + 1e-5) + 1e-6), (h, i)
