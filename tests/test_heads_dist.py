@@ -1,5 +1,6 @@
 """Head parallelism (quantized_attention_05_b200.heads) on CPU ranks (gloo,
-world size 2, 3 and 5, with an uneven split and a rank without heads).
+world size 2, 3 and 5, with an uneven split and a rank without heads), with
+full tensors on every rank and with each rank holding only its own slice.
 
 Every KV-head group is a problem of its own, so:
 * the gathered result equals, bit for bit, the per-slice results of the same
@@ -44,12 +45,18 @@ def _worker(rank, world, port, causal, q_out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        from quantized_attention_05_b200.heads import head_parallel_attention
+        from quantized_attention_05_b200.heads import head_parallel_attention, shard_heads
         q, k, v = (t.double() for t in W.make_qkv(WORK))     # bf16 values, fp64 outputs
         out, lse = head_parallel_attention(q, k, v, causal=causal, attn=_oracle_attn)
         part, plse, (h0, h1) = head_parallel_attention(q, k, v, causal=causal, gather=False,
                                                        attn=_oracle_attn)
-        q_out.put((rank, out.numpy(), lse.numpy(), part.numpy(), plse.numpy(), h0, h1))
+        # sliced inputs: this rank holds only its own heads (copies, so no
+        # view of the full tensors reaches the call)
+        qs, ks, vs = (t.clone() for t in shard_heads(q, k, v, rank, world))
+        sout, slse = head_parallel_attention(qs, ks, vs, causal=causal, attn=_oracle_attn,
+                                             heads=(WORK.Hq, WORK.Hkv))
+        q_out.put((rank, out.numpy(), lse.numpy(), part.numpy(), plse.numpy(), h0, h1,
+                   sout.numpy(), slse.numpy(), tuple(qs.shape), tuple(ks.shape)))
         dist.barrier()
     finally:
         dist.destroy_process_group()
@@ -92,7 +99,11 @@ def test_gathered_heads_equal_one_call_over_all_heads(world, causal):
             side_o[:, g0 * G:g1 * G], side_l[:, g0 * G:g1 * G] = o.numpy(), l.numpy()
     full = O.attention_i8f8(O.quantize_qkv_i8f8(q, k, v), causal=causal)
     for r in range(world):
-        out, lse, part, plse, h0, h1 = res[r]
+        out, lse, part, plse, h0, h1, sout, slse, qshape, kshape = res[r]
+        np.testing.assert_array_equal(sout, side_o)
+        np.testing.assert_array_equal(slse, side_l)
+        g0, g1 = kv_head_range(WORK.Hkv, r, world)
+        assert qshape[1] == (g1 - g0) * G and kshape[1] == g1 - g0
         np.testing.assert_array_equal(out, side_o)
         np.testing.assert_array_equal(lse, side_l)
         np.testing.assert_allclose(out, full["out_f64"], rtol=2.0 ** -22, atol=1e-12)
@@ -101,3 +112,16 @@ def test_gathered_heads_equal_one_call_over_all_heads(world, causal):
         assert (h0, h1) == (g0 * G, g1 * G)
         np.testing.assert_array_equal(part, side_o[:, h0:h1])
         np.testing.assert_array_equal(plse, side_l[:, h0:h1])
+
+
+def test_sliced_call_rejects_a_wrong_slice():
+    """With heads=(Hq, Hkv) every rank must pass exactly its own slice."""
+    import quantized_attention_05_b200.heads as Hm
+    orig = (Hm.dist.get_world_size, Hm.dist.get_rank)
+    Hm.dist.get_world_size, Hm.dist.get_rank = (lambda g=None: 2), (lambda g=None: 1)
+    try:
+        q, k, v = W.make_qkv(WORK)
+        with pytest.raises(ValueError, match="expected the slices"):
+            Hm.head_parallel_attention(q, k, v, heads=(WORK.Hq, WORK.Hkv), attn=lambda *a: None)
+    finally:
+        Hm.dist.get_world_size, Hm.dist.get_rank = orig
