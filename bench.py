@@ -252,6 +252,156 @@ def workload_config(w: W.Workload, ranks: int):
 
 
 # ------------------------------------------------------------------ our arm
+def quantiser_bytes(w: W.Workload) -> int:
+    """The quantiser's algorithmic bytes: bf16 Q/K/V read once, codes,
+    scales, means, q.kmean and (NVFP4) qk_correction written once."""
+    eq, ekv = w.B * w.Hq * w.N * w.D, w.B * w.Hkv * w.N * w.D
+    nqb = (w.N + 127) // 128
+    if w.nvfp4:
+        return (2 * (eq + 2 * ekv) + (eq + 2 * ekv) // 2 + (eq + 2 * ekv) // 16
+                + w.B * w.Hq * nqb * (nqb * 128) * 4 + w.B * w.Hq * nqb * w.D * 4
+                + w.B * w.Hkv * w.D * 4 + w.B * w.Hq * w.N * 4)
+    return (3 * (eq + 2 * ekv) + (w.B * w.Hq + w.B * w.Hkv) * nqb * 4
+            + 2 * w.B * w.Hkv * w.D * 4 + w.B * w.Hq * w.N * 4)
+
+
+class StepRunner:
+    """Device buffers and one step (quantise + attend) of workload ``w``."""
+
+    def __init__(self, S, w: W.Workload, device, rank: int = 0):
+        self.S, self.w, self.device = S, w, device
+        wr = rank_workload(w, rank)
+        self.q, self.k, self.v = W.make_qkv(wr, device=device)
+        self.mask = W.make_mask(wr, device=device)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=device)
+        self.stream = torch.cuda.current_stream(device)
+        if w.nvfp4:
+            ukl = w.unpadded_k_len or w.N
+            self.z = S.QuantizedNvfp4.empty(w.B, w.Hq, w.Hkv, w.N, w.N, w.D, ukl, w.per_block_mean,
+                                            device)
+            nbytes = S.lib().sage_quantize_nvfp4_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.N, w.D)
+            self.launches = 6       # column sums x2, means, codes, correction; attention
+        else:
+            self.z = S.QuantizedQKV.empty(w.B, w.Hq, w.Hkv, w.N, w.N, w.D, device, with_qdk=True)
+            nbytes = S.lib().sage_quantize_workspace_bytes(w.B, w.Hkv, w.N, w.D)
+            # K-mean/V-amax partials, their combination, block codes; attention
+            # (+ the mask's tile classification)
+            self.launches = 4 + (1 if self.mask is not None else 0)
+        self.qws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+    def step(self, ev_q=None, ev_a=None, ev_b=None):
+        S, w, z = self.S, self.w, self.z
+        if ev_q is not None:
+            ev_q.record(self.stream)
+        if w.nvfp4:
+            S.sage_quantize_qkv_nvfp4(self.q, self.k, self.v, per_block_mean=w.per_block_mean,
+                                      unpadded_k_len=w.unpadded_k_len, out=z, ws=self.qws)
+        else:
+            S.sage_quantize_qkv(self.q, self.k, self.v, out=z, ws=self.qws)
+        if ev_a is not None:
+            ev_a.record(self.stream)
+        if w.nvfp4:
+            S.sage_attn_fwd_nvfp4(z, sm_scale=w.sm_scale, causal=w.causal, return_lse=True,
+                                  out=self.out, lse=self.lse)
+        else:
+            S.sage_attn_fwd_quantized(z, causal=w.causal, sm_scale=w.sm_scale, return_lse=True,
+                                      mask=self.mask, out=self.out, lse=self.lse)
+        if ev_b is not None:
+            ev_b.record(self.stream)
+
+    def timed(self, steps):
+        """Run ``steps`` steps with CUDA events on the launching stream:
+        (whole-region ms, mean attention ms, mean quantiser ms)."""
+        evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(self.device)
+        e0.record(self.stream)
+        for i in range(steps):
+            self.step(*evs[i])
+        e1.record(self.stream)
+        torch.cuda.synchronize(self.device)
+        return (e0.elapsed_time(e1), sum(a.elapsed_time(b) for _, a, b in evs) / steps,
+                sum(q.elapsed_time(a) for q, a, _ in evs) / steps)
+
+
+def peak_for(w: W.Workload, timed_s: float):
+    """Denominator of roofline.frac: the measured bf16 GEMM rate times the
+    dense INT8/FP8 (x2) or FP4 (x4) ratio; the burst figure for a timed region
+    shorter than 2 s, the sustained one (measured over seconds, under the
+    power cap) for a longer one."""
+    peaks, src = load_peaks()
+    ratio = FP4_PER_BF16 if w.nvfp4 else FP8_PER_BF16
+    sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * ratio
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * ratio
+    kind = "FP4" if w.nvfp4 else "INT8/FP8"
+    if timed_s >= 2.0:
+        return sus, burst, sus, f"{src} bf16 sustained x{ratio:g} (dense {kind}:BF16; timed region {timed_s:.2f} s >= 2 s)"
+    return burst, burst, sus, f"{src} bf16 burst x{ratio:g} (dense {kind}:BF16; timed region {timed_s:.2f} s < 2 s)"
+
+
+def roofline_of(w: W.Workload, attn_ms: float, timed_s: float, sm_mhz):
+    """roofline object for the attention kernel of workload ``w``."""
+    peak, burst, sus, src = peak_for(w, timed_s)
+    achieved = w.visible_ops / (attn_ms * 1e-3) / 1e12
+    r = {"bound": "tensor",
+         "kernel": "attn_fwd_nvfp4_kernel<128>" if w.nvfp4 else "attn_fwd_i8f8_kernel<128>",
+         "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+         "frac": round(achieved / peak, 4), "traffic": None, "peak_source": src,
+         "peak_burst": round(burst, 1), "frac_burst": round(achieved / burst, 4),
+         "peak_sustained": round(sus, 1), "frac_sustained": round(achieved / sus, 4),
+         "attn_ms": round(attn_ms, 4)}
+    r.update(extra_denominators(achieved, sm_mhz, w.nvfp4))
+    return r
+
+
+def quantize_of(w: W.Workload, quant_ms: float):
+    peaks, src = load_peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    qbytes = quantiser_bytes(w)
+    gbs = qbytes / (quant_ms * 1e-3) / 1e9
+    return {"kernels": "all quantiser kernels of the step", "ms": round(quant_ms, 4),
+            "algorithmic_bytes": qbytes, "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(gbs / hbm, 4), "peak_source": f"{src} HBM copy bandwidth"}
+
+
+EXTRA_WORKLOADS = [W.TINY, W.LLM_MASK, W.VIDEO_DIT, W.NVFP4]
+
+
+def extra_configs(S, device, main: W.Workload, warmup=3, min_s=0.25):
+    """The other workloads' figures, each timed in this run after the main
+    timed region: per workload a few warm-up steps, then enough timed steps
+    for about ``min_s`` seconds (at least 10), with the SM clock sampled."""
+    res = {}
+    for w in EXTRA_WORKLOADS:
+        if w.name == main.name:
+            continue
+        r = StepRunner(S, w, device)
+        for _ in range(warmup):
+            r.step()
+        t_ms, _, _ = r.timed(3)
+        steps = max(10, int(min_s * 1e3 / max(t_ms / 3, 1e-3)))
+        sampler = ClockSampler(device.index or 0)
+        time.sleep(0.3)
+        ms, attn_ms, quant_ms = r.timed(steps)
+        clocks = sampler.stop()
+        st, site = S.sage_get_device_status()
+        if st != S.SAGE_OK:
+            raise RuntimeError(f"device wait timed out at site {site} ({w.name})")
+        ms_step = ms / steps
+        e = {"config": workload_config(w, 1), "steps": steps, "warmup": warmup,
+             "ms_per_step": round(ms_step, 4),
+             "value": round(w.ops / (ms_step * 1e-3) / 1e12, 2), "unit": UNIT,
+             "roofline": roofline_of(w, attn_ms, ms * 1e-3, (clocks or {}).get("sm_mhz")),
+             "quantize": quantize_of(w, quant_ms), "clocks": clocks}
+        if w.visible_ops != w.ops:
+            e["value_visible_pairs"] = round(w.visible_ops / (ms_step * 1e-3) / 1e12, 2)
+        res[w.name] = e
+        del r
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, w):
     import quantized_attention_05_b200 as S
     ws_, rank, local = dist_env()
@@ -260,68 +410,24 @@ def run_ours(args, w):
     if ws_ > 1:
         init_dist("nccl")
     S.lib()
-    wr = rank_workload(w, rank)
-    q, k, v = W.make_qkv(wr, device=device)
-    mask = W.make_mask(wr, device=device)
-    out = torch.empty_like(q)
-    lse = torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=device)
-    stream = torch.cuda.current_stream(device)
-    if w.nvfp4:
-        ukl = w.unpadded_k_len or w.N
-        z = S.QuantizedNvfp4.empty(w.B, w.Hq, w.Hkv, w.N, w.N, w.D, ukl, w.per_block_mean, device)
-        qws = torch.empty(S.lib().sage_quantize_nvfp4_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.N, w.D),
-                          dtype=torch.uint8, device=device)
-        launches_per_step = 6       # column sums x2, means, codes, correction; attention
-    else:
-        z = S.QuantizedQKV.empty(w.B, w.Hq, w.Hkv, w.N, w.N, w.D, device, with_qdk=True)
-        qws = torch.empty(S.lib().sage_quantize_workspace_bytes(w.B, w.Hkv, w.N, w.D),
-                          dtype=torch.uint8, device=device)
-        # K-mean/V-amax partials, their combination, block codes; attention
-        # (+ the mask's tile classification)
-        launches_per_step = 4 + (1 if mask is not None else 0)
-
-    def step(ev_q=None, ev_a=None, ev_b=None):
-        if ev_q is not None:
-            ev_q.record(stream)
-        if w.nvfp4:
-            S.sage_quantize_qkv_nvfp4(q, k, v, per_block_mean=w.per_block_mean,
-                                      unpadded_k_len=w.unpadded_k_len, out=z, ws=qws)
-        else:
-            S.sage_quantize_qkv(q, k, v, out=z, ws=qws)
-        if ev_a is not None:
-            ev_a.record(stream)
-        if w.nvfp4:
-            S.sage_attn_fwd_nvfp4(z, sm_scale=w.sm_scale, causal=w.causal, return_lse=True,
-                                  out=out, lse=lse)
-        else:
-            S.sage_attn_fwd_quantized(z, causal=w.causal, sm_scale=w.sm_scale, return_lse=True,
-                                      mask=mask, out=out, lse=lse)
-        if ev_b is not None:
-            ev_b.record(stream)
+    runner = StepRunner(S, w, device, rank)
+    q, k, v, mask, out, lse = runner.q, runner.k, runner.v, runner.mask, runner.out, runner.lse
+    stream = runner.stream
+    launches_per_step = runner.launches
 
     for _ in range(args.warmup):
-        step()
+        runner.step()
     torch.cuda.synchronize(device)
     st, site = S.sage_get_device_status()
     if st != S.SAGE_OK:
         raise RuntimeError(f"device wait timed out at site {site}")
 
-    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local) if rank == 0 else None
     time.sleep(0.3 if sampler else 0)
     barrier(device)
-    torch.cuda.synchronize(device)
-    e0.record(stream)
-    for i in range(args.steps):
-        step(*evs[i])
-    e1.record(stream)
-    torch.cuda.synchronize(device)
+    ms_local, attn_ms_local, quant_ms_local = runner.timed(args.steps)
     barrier(device)
     clocks = sampler.stop() if sampler else None
-    ms_local = e0.elapsed_time(e1)
-    attn_ms_local = sum(a.elapsed_time(b) for _, a, b in evs) / args.steps
-    quant_ms_local = sum(q.elapsed_time(a) for q, a, _ in evs) / args.steps
     ms = max_over_ranks(ms_local, device)
     attn_ms = max_over_ranks(attn_ms_local, device)
     quant_ms = max_over_ranks(quant_ms_local, device)
@@ -376,32 +482,15 @@ def run_ours(args, w):
     ranks = ws_
     ms_step = ms / args.steps
     value = ranks * w.ops / (ms_step * 1e-3) / 1e12
-    peaks, src = load_peaks()
-    ratio = FP4_PER_BF16 if w.nvfp4 else FP8_PER_BF16
-    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * ratio
-    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * ratio
-    achieved = w.visible_ops / (attn_ms * 1e-3) / 1e12
-    traffic = None
+    roof = roofline_of(w, attn_ms, ms * 1e-3, (clocks or {}).get("sm_mhz"))
     tr_path = os.path.join(ROOT, "profiles", "attn_traffic.json")
     if os.path.exists(tr_path):
         try:
             tr = json.load(open(tr_path))
             if tr.get("workload") == w.name and tr.get("kernel_hash") == kernel_hash():
-                traffic = tr.get("bytes_per_launch")
+                roof["traffic"] = tr.get("bytes_per_launch")
         except (OSError, ValueError):
-            traffic = None
-    # the quantiser's algorithmic bytes: bf16 Q/K/V read once, codes, scales,
-    # means, q.kmean and (NVFP4) qk_correction written once
-    eq, ekv = w.B * w.Hq * w.N * w.D, w.B * w.Hkv * w.N * w.D
-    nqb = (w.N + 127) // 128
-    if w.nvfp4:
-        qbytes = (2 * (eq + 2 * ekv) + (eq + 2 * ekv) // 2 + (eq + 2 * ekv) // 16
-                  + w.B * w.Hq * nqb * (nqb * 128) * 4 + w.B * w.Hq * nqb * w.D * 4
-                  + w.B * w.Hkv * w.D * 4 + w.B * w.Hq * w.N * 4)
-    else:
-        qbytes = (3 * (eq + 2 * ekv) + (w.B * w.Hq + w.B * w.Hkv) * nqb * 4
-                  + 2 * w.B * w.Hkv * w.D * 4 + w.B * w.Hq * w.N * 4)
-    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+            pass
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ranks,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -409,28 +498,22 @@ def run_ours(args, w):
         "dtype": ("nvfp4 (e2m1 x e2m1, e4m3 block-16 scales) -> f32" if w.nvfp4 else
                   "i8xi8->i32 (QK), e4m3xe4m3->f32 (PV)"), "data": "synthetic",
         "config": workload_config(w, ranks),
-        "roofline": {"bound": "tensor",
-                     "kernel": "attn_fwd_nvfp4_kernel<128>" if w.nvfp4 else "attn_fwd_i8f8_kernel<128>",
-                     "achieved": round(achieved, 1), "peak": round(peak_sus, 1), "unit": "TFLOP/s",
-                     "frac": round(achieved / peak_sus, 4), "traffic": traffic,
-                     "peak_source": f"{src} bf16 sustained x{ratio:g} (dense "
-                                    f"{'FP4' if w.nvfp4 else 'INT8/FP8'}:BF16)",
-                     "peak_burst": round(peak_burst, 1), "frac_burst": round(achieved / peak_burst, 4),
-                     "attn_ms": round(attn_ms, 4)},
+        "roofline": roof,
         "e2e": {"value": round(ranks * w.ops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 3), "api": e2e_api},
-        "quantize": {"kernels": "all quantiser kernels of the step", "ms": round(quant_ms, 4),
-                     "algorithmic_bytes": qbytes, "achieved": round(qbytes / (quant_ms * 1e-3) / 1e9, 1),
-                     "peak": hbm, "unit": "GB/s",
-                     "frac": round(qbytes / (quant_ms * 1e-3) / 1e9 / hbm, 4),
-                     "peak_source": f"{src} HBM copy bandwidth"},
+        "quantize": quantize_of(w, quant_ms),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
-    line["roofline"].update(extra_denominators(achieved, (clocks or {}).get("sm_mhz"), w.nvfp4))
     if w.visible_ops != w.ops:      # a mask hides pairs: the step's TOPS over the visible ones too
         line["value_visible_pairs"] = round(ranks * w.visible_ops / (ms_step * 1e-3) / 1e12, 2)
+    if ranks == 1 and not args.no_extra:
+        del runner, q, k, v, mask, qh, kh, vh, outh, lseh, ws_host
+        torch.cuda.empty_cache()
+        line["extra"] = {"configs": extra_configs(S, device, w),
+                         "note": "the other workloads, each timed in this run after the main timed "
+                                 "region (same step, metric and roofline rules)"}
     if rank == 0 and ranks == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
@@ -488,14 +571,22 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.CAUSAL_GQA.name, choices=sorted(W.BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads' figures (extra.configs)")
     ap.add_argument("--B", type=int, default=None,
                     help="override the batch size (smaller cases for profiling)")
+    ap.add_argument("--N", type=int, default=None,
+                    help="override the sequence length (smaller cases for profiling; an "
+                         "unpadded key length scales with it)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = W.BY_NAME[args.workload]
     if args.B is not None:
         w = w.scaled(B=args.B, name=w.name.replace(f"_b{w.B}_", f"_b{args.B}_"))
+    if args.N is not None:
+        ukl = None if w.unpadded_k_len is None else w.unpadded_k_len * args.N // w.N
+        w = w.scaled(N=args.N, unpadded_k_len=ukl, name=w.name.replace(f"_n{w.N}_", f"_n{args.N}_"))
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -95,3 +95,27 @@ def test_oracle_sample_times_the_nvfp4_oracle_for_the_nvfp4_workload(monkeypatch
     ops, dt = bench.oracle_sample(W.NVFP4, 256)
     assert seen == ["q", "a"] and dt > 0
     assert ops == W.NVFP4.scaled(B=1, Hq=1, Hkv=1, N=256).ops
+
+
+def test_roofline_peak_is_burst_for_short_timed_regions():
+    """roofline.frac divides by the measured bf16 burst rate (x2 INT8/FP8,
+    x4 FP4) unless the timed region lasts at least 2 s (then the sustained
+    rate, measured over seconds under the power cap)."""
+    peaks, _ = bench.load_peaks()
+    burst = peaks.get("bf16_tflops", bench.FALLBACK_PEAKS["bf16_tflops"])
+    sus = peaks.get("bf16_tflops_sustained", bench.FALLBACK_PEAKS["bf16_tflops_sustained"])
+    p, b, s, src = bench.peak_for(W.CAUSAL_GQA, 0.15)
+    assert p == b == 2 * burst and s == 2 * sus and "burst" in src
+    p, b, s, src = bench.peak_for(W.CAUSAL_GQA, 2.5)
+    assert p == 2 * sus and "sustained" in src
+    p, _, _, src = bench.peak_for(W.NVFP4, 0.3)
+    assert p == 4 * burst and "FP4" in src
+    r = bench.roofline_of(W.CAUSAL_GQA, 7.0, 0.15, 1965.0)
+    assert r["frac"] == r["frac_burst"] and r["frac_sustained"] > r["frac"]
+
+
+def test_quantiser_bytes_of_the_workloads():
+    # causal GQA: bf16 read + int8/e4m3 written per element, plus scales,
+    # means and q.kmean
+    assert bench.quantiser_bytes(W.CAUSAL_GQA) == 1216462848
+    assert bench.quantiser_bytes(W.NVFP4) > 3 * W.NVFP4.B * W.NVFP4.Hq * W.NVFP4.N * W.NVFP4.D * 2
