@@ -223,19 +223,43 @@ __device__ __forceinline__ float block_max(float v, float* s_red) {
   return r;
 }
 
-// Four INT8 codes rint(fp32(x[i] * inv)) (round half to even) packed into a
-// word, x[0] in the low byte.  |x * inv| <= 127 by construction (inv =
+// Eight INT8 codes rint(fp32(x[i] * inv)) (round half to even) packed into
+// two words, x[0] in the low byte.  |x * inv| <= 127 by construction (inv =
 // 127/amax of the block), so adding 1.5*2^23 to the fp32 product leaves the
 // integer in the low mantissa bits and their low byte is the two's-complement
 // code: FMA-pipe arithmetic and byte permutes instead of float-to-int
-// conversions.
-__device__ __forceinline__ uint32_t int8x4_codes(float x0, float x1, float x2, float x3,
-                                                 float inv) {
-  const uint32_t t0 = __float_as_uint(__fadd_rn(__fmul_rn(x0, inv), 12582912.f));
-  const uint32_t t1 = __float_as_uint(__fadd_rn(__fmul_rn(x1, inv), 12582912.f));
-  const uint32_t t2 = __float_as_uint(__fadd_rn(__fmul_rn(x2, inv), 12582912.f));
-  const uint32_t t3 = __float_as_uint(__fadd_rn(__fmul_rn(x3, inv), 12582912.f));
-  return __byte_perm(__byte_perm(t0, t1, 0x0040), __byte_perm(t2, t3, 0x0040), 0x5410);
+// conversions.  The product and the sum are scalar IEEE-rounded operations
+// (__fmul_rn, __fadd_rn): the codes must be those of the two roundings, bit
+// for bit.
+__device__ __forceinline__ uint2 int8x8_codes(const float* x, float inv) {
+  uint32_t t[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t[i] = __float_as_uint(__fadd_rn(__fmul_rn(x[i], inv), 12582912.f));
+  return make_uint2(
+      __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410),
+      __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410));
+}
+
+// Row sums over the TPR threads of each row, for the ITERS = TPR/2 rows a
+// thread holds: a transposed butterfly (each level hands half of the
+// remaining partial sums to the partner lane and keeps the other half), so
+// ITERS rows cost ITERS shuffles instead of ITERS * log2(TPR).  Returns the
+// full sum of row (cg >> 1) of the thread's rows; lanes cg and cg ^ 1 hold
+// the same row.
+template <int TPR>
+__device__ __forceinline__ float rows_sum_transposed(float* v, int cg) {
+  constexpr int ITERS = TPR / 2;
+#pragma unroll
+  for (int half = ITERS / 2; half >= 1; half >>= 1) {
+    const bool up = (cg & (2 * half)) != 0;    // this lane keeps the upper half
+#pragma unroll
+    for (int j = 0; j < half; ++j) {
+      const float keep = up ? v[j + half] : v[j];
+      const float give = up ? v[j] : v[j + half];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, give, 2 * half);
+    }
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
 // ------------------------------------------------------------ pass B
@@ -285,22 +309,28 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
     }
     const float amax = block_max(am, s_red);  // also orders s_c
     const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+    float dsum[ITERS];
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
       const int n = qt * QB + rs + it * RPP;
       float f[8];
       unpack8<T>(raw[it], f);
-      const uint32_t w0 = int8x4_codes(f[0], f[1], f[2], f[3], inv);
-      const uint32_t w1 = int8x4_codes(f[4], f[5], f[6], f[7], inv);
-      *reinterpret_cast<uint2*>(a.q8 + (row0 + n) * D + cg * 8) = make_uint2(w0, w1);
+      *reinterpret_cast<uint2*>(a.q8 + (row0 + n) * D + cg * 8) = int8x8_codes(f, inv);
       if (a.qdk) {
-        float d = 0.f;
+        uint64_t d2 = f2_pack(0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) d = fmaf(f[i], s_c[cg * 8 + i], d);
-#pragma unroll
-        for (int o = TPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-        if (cg == 0 && n < sq.nq) a.qdk[(int64_t)a.Hq * sq.cq + (int64_t)h * sq.nq + n] = d;
+        for (int i = 0; i < 8; i += 2)
+          d2 = f2_fma(f2_pack(f[i], f[i + 1]), f2_pack(s_c[cg * 8 + i], s_c[cg * 8 + i + 1]), d2);
+        float d0, d1;
+        f2_unpack(d2, d0, d1);
+        dsum[it] = d0 + d1;
       }
+    }
+    if (a.qdk) {
+      // row (cg >> 1) of this thread's rows, complete in lanes cg and cg ^ 1
+      const float d = rows_sum_transposed<TPR>(dsum, cg);
+      const int n = qt * QB + rs + (cg >> 1) * RPP;
+      if ((cg & 1) == 0 && n < sq.nq) a.qdk[(int64_t)a.Hq * sq.cq + (int64_t)h * sq.nq + n] = d;
     }
     if (threadIdx.x == 0)
       a.q_scale[(int64_t)a.Hq * (sq.cqp / 128) + (int64_t)h * nqt + qt] = __fdiv_rn(amax, 127.f);
@@ -326,18 +356,24 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
       raw[it] = n < sq.nk ? ldg16(base + (int64_t)n * a.k_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
+    // K - kmean, one IEEE-rounded subtraction per element
     float km[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) km[i] = s_c[cg * 8 + i];
+    auto smooth = [&](const uint4& r, float* f) {
+      unpack8<T>(r, f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] = __fsub_rn(f[i], km[i]);
+    };
     float am = 0.f;
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
       const int n = kt * QB + rs + it * RPP;
       float f[8];
-      unpack8<T>(raw[it], f);
+      smooth(raw[it], f);
       if (n < sq.nk) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(__fsub_rn(f[i], km[i])));
+        for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(f[i]));
       }
     }
     const float amax = block_max(am, s_red);
@@ -346,15 +382,9 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
     for (int it = 0; it < ITERS; ++it) {
       const int n = kt * QB + rs + it * RPP;
       float f[8];
-      unpack8<T>(raw[it], f);
-      uint32_t w0 = 0, w1 = 0;
-      if (n < sq.nk) {
-        w0 = int8x4_codes(__fsub_rn(f[0], km[0]), __fsub_rn(f[1], km[1]), __fsub_rn(f[2], km[2]),
-                          __fsub_rn(f[3], km[3]), inv);
-        w1 = int8x4_codes(__fsub_rn(f[4], km[4]), __fsub_rn(f[5], km[5]), __fsub_rn(f[6], km[6]),
-                          __fsub_rn(f[7], km[7]), inv);
-      }
-      *reinterpret_cast<uint2*>(a.k8 + (row0 + n) * D + cg * 8) = make_uint2(w0, w1);
+      smooth(raw[it], f);
+      const uint2 w = n < sq.nk ? int8x8_codes(f, inv) : make_uint2(0u, 0u);
+      *reinterpret_cast<uint2*>(a.k8 + (row0 + n) * D + cg * 8) = w;
     }
     if (threadIdx.x == 0)
       a.k_scale[(int64_t)a.Hkv * (sq.ckp / 128) + (int64_t)h * nkt + kt] = __fdiv_rn(amax, 127.f);
