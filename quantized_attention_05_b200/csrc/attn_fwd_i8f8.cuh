@@ -9,12 +9,14 @@
 //   warp 8      TMA producer: Q tiles once, then K and V tiles (V in
 //               [token, channel] order, read MN-major by the PV MMA) into a
 //               3-stage ring;
-//   warp 9      MMA issuer (one thread): S_i = 1.5*2^23 (one f16 MMA) +
-//               Q_i K^T with tcgen05 kind::i8 into TMEM (int32, exact, read
-//               back as a float), O_i += P_i V with kind::f8f6f4 (E4M3 x
-//               E4M3 -> FP32 in TMEM); it issues the next tile's QK^T of a
-//               Q tile as soon as that tile's S has been read, so the tensor
-//               pipe runs while softmax works;
+//   warps 9, 10 MMA issuers, one thread each, for Q tile 0 and Q tile 1:
+//               S_i = 1.5*2^23 (one f16 MMA) + Q_i K^T with tcgen05 kind::i8
+//               into TMEM (int32, exact, read back as a float), O_i += P_i V
+//               with kind::f8f6f4 (E4M3 x E4M3 -> FP32 in TMEM); each issues
+//               the next tile's QK^T of its Q tile as soon as that tile's S
+//               has been read, so the tensor pipe runs while softmax works,
+//               and the two threads' waits and commits overlap each other's
+//               MMAs;
 //   warps 0..7  two softmax warpgroups, one per Q tile, one thread per row:
 //               tcgen05.ld of the int32 scores, dequantisation by
 //               q_scale*k_scale*sm_scale*log2(e), masking, online softmax
@@ -36,7 +38,8 @@ namespace sage {
 
 constexpr int ATT_BM = 128, ATT_BN = 128;
 constexpr int ATT_STAGES = 3;
-constexpr int ATT_THREADS = 384;   // 3 warpgroups: 2 softmax, 1 TMA/MMA (+2 idle warps)
+constexpr int ATT_ISSUERS = 2;      // MMA-issuing threads: warps 9 and 10, one per Q tile
+constexpr int ATT_THREADS = 384;   // 3 warpgroups: 2 softmax, 1 TMA/MMA (+1 idle warp)
 // Register split between the warpgroups (setmaxnreg): the TMA/MMA warpgroup
 // keeps ATT_REGS_LOW per thread, the softmax warpgroups grow to
 // ATT_REGS_HIGH.  The sum must not exceed what the block is launched with
@@ -134,10 +137,12 @@ struct AttnLayout {
 static_assert(AttnLayout<128>::bytes(ATT_MAX_NKT) <= 232448, "attention smem");
 static_assert(AttnLayout<64>::bytes(ATT_MAX_NKT) <= 232448, "attention smem");
 
-// Exponentials: every one on MUFU ex2.  Measured on B200 this kernel is
-// not MUFU-throughput bound (MUFU about half busy); FMA-pipe polynomials for
-// a share of them cost more than the MUFU time they saved, and their error
-// moved enough E4M3 roundings of P to break the parity bound on small cases.
+// Exponentials: every one on MUFU ex2.  An FMA-pipe polynomial for one pair
+// in 8 (or 4) gained at most 1 % on B200 and moved enough E4M3 roundings of
+// P to break the parity bound on short rows; a threshold on rescaling O
+// (keeping a stale max until it is exceeded by a margin) gained 7 % but
+// quantises P against another reference than the exact running max, which
+// broke the parity bound on small cases too.
 // int32 score S as the float 1.5*2^23 + S (exact for |S| < 2^22): the QK^T
 // MMA accumulates the int32 S onto the bit pattern of 1.5*2^23 (0x4B400000),
 // which an f16 MMA (512 x 1536 summed over K = 16) writes into S first.
@@ -392,7 +397,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < ATT_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], ATT_ISSUERS);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -402,7 +407,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(&p_full[i], 128);
       mbar_init(&o_ready[i], 1);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, ATT_ISSUERS);
     fence_mbar_init();
   } else if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
@@ -444,14 +449,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ---------------------------------------------------------- MMA issuer
-    // One thread polls the barriers and issues, per Q tile i, the ops
-    // QK(0), QK(1), PV(0), QK(2), PV(1), ... in order, whichever Q tile is
-    // ready first.  A stage of the K/V ring is released once both Q tiles
-    // have issued their PV on it.  Each QK(n) starts with an f16 MMA that
-    // overwrites S with 1.5*2^23 (every operand element equal, so the
-    // operand layout does not matter); the int8 MMAs accumulate onto it.
+  } else if (warp == 9 || warp == 10) {
+    // ---------------------------------------------------------- MMA issuers
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = instr_desc(kDS32, kS8, kS8, ATT_BM, ATT_BN);
       constexpr uint32_t IDESC_INIT = instr_desc(kDF32, 0u, 0u, ATT_BM, ATT_BN);
@@ -459,74 +458,70 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const uint64_t dInitB = smem_desc(smem_u32(sInit) + 4096, 256, 32);
       constexpr uint32_t IDESC_PV = instr_desc(kDF32, kE4M3, kE4M3, ATT_BM, D) | kBMajorMN;
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-      auto next_active = [&](int i, int from) {
-        while (from < ntile && !((s_list[from] >> i) & 1u)) ++from;
-        return from;
+      // One issuing thread per Q tile (warp 9: Q tile 0, warp 10: Q tile 1).
+      // A thread is held by each tcgen05.mma for about its execution time,
+      // so the waits and commits of one thread (~50-100 clocks each) leave
+      // the tensor pipe idle unless the other thread's MMAs fill it.  Per
+      // visible list position e the thread issues QK(e), then PV of its
+      // previous visible position, each gated by one bounded wait; it then
+      // releases, in list order, every K/V stage it is done with by a
+      // commit (which arrives only after its MMAs reading the stage have
+      // completed).  A stage is refilled once both threads have released it
+      // (kv_empty counts 2).  Before releasing position p a thread waits
+      // until p's tile has arrived: otherwise a thread with nothing to read
+      // (a position its Q tile does not see, or no Q tile at all) would
+      // arrive for p and p + 3 before the other thread released p, and the
+      // stage would be refilled while still being read.
+      const int i = warp - 9;
+      uint32_t nqk = 0u, npv = 0u;
+      int rel = 0;   // next list position this thread releases
+      auto release_to = [&](int last) -> bool {
+        for (; rel <= last; ++rel) {
+          if (!mbar_wait(&kv_full[rel % ATT_STAGES], (rel / ATT_STAGES) & 1, SITE_KV_FULL))
+            return false;
+          tc_commit(&kv_empty[rel % ATT_STAGES]);
+        }
+        return true;
+      };
+      auto issue_pv = [&](int ep) -> bool {
+        if (!mbar_wait(&p_full[i * 2 + (npv & 1u)], (npv >> 1) & 1u, SITE_P_FULL)) return false;
+        tc_fence_after();
+        const uint32_t tO = tmem + (uint32_t)(i * 256 + 128);
+        const uint32_t pa = aP + (i * 2 + (npv & 1u)) * L::P_BYTES;
+        const uint32_t va = aV + (ep % ATT_STAGES) * L::V_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < ATT_BN / 32; ++kk)
+          mma_f8f6f4(tO, smem_desc(pa + 32 * kk, 1024, 128),
+                     smem_desc(va + L::V_KSTEP * kk, L::QK_SBO, L::QK_SWIZZLE), IDESC_PV,
+                     (npv > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&o_ready[i * 2 + (npv & 1u)]);
+        ++npv;
+        return release_to(ep);
       };
       bool ok = mbar_wait(q_full, 0, SITE_Q_FULL);
       tc_fence_after();
-      int qk_e[2], pv_e[2];
-      uint32_t qk_k[2] = {0, 0}, pv_k[2] = {0, 0};
-      for (int i = 0; i < 2; ++i) qk_e[i] = pv_e[i] = next_active(i, 0);
-      int rel_e = 0;
-      uint32_t idle = 0;
-      uint64_t idle_t0 = 0;
-      while (ok && rel_e < ntile) {
-        bool prog = false;
+      int ep = -1;   // previous visible position
+      for (int e = 0; ok && e < ntile; ++e) {
+        if (!((s_list[e] >> i) & 1u)) continue;
+        ok = mbar_wait(&kv_full[e % ATT_STAGES], (e / ATT_STAGES) & 1, SITE_KV_FULL) &&
+             mbar_wait(&s_free[i], nqk & 1u, SITE_S_FREE);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tS = tmem + (uint32_t)(i * 256);
+        const uint32_t qa = aQ + i * L::Q_BYTES, ka = aK + (e % ATT_STAGES) * L::K_BYTES;
+        mma_f16(tS, dInitA, dInitB, IDESC_INIT, 0u);
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int e = qk_e[i];
-          if (e < ntile && mbar_test(&kv_full[e % ATT_STAGES], (e / ATT_STAGES) & 1) &&
-              mbar_test(&s_free[i], qk_k[i] & 1)) {
-            tc_fence_after();
-            const uint32_t tS = tmem + (uint32_t)(i * 256);
-            const uint32_t qa = aQ + i * L::Q_BYTES, ka = aK + (e % ATT_STAGES) * L::K_BYTES;
-            mma_f16(tS, dInitA, dInitB, IDESC_INIT, 0u);
-#pragma unroll
-            for (int k = 0; k < D / 32; ++k)
-              mma_i8(tS, smem_desc(qa + 32 * k, L::QK_SBO, L::QK_SWIZZLE),
-                     smem_desc(ka + 32 * k, L::QK_SBO, L::QK_SWIZZLE), IDESC_QK, 1u);
-            tc_commit(&s_full[i]);
-            ++qk_k[i];
-            qk_e[i] = next_active(i, e + 1);
-            prog = true;
-          }
-          const uint32_t k = pv_k[i];
-          if (k < qk_k[i] && mbar_test(&p_full[i * 2 + (k & 1)], (k >> 1) & 1)) {
-            tc_fence_after();
-            const int ep = pv_e[i];
-            const uint32_t tO = tmem + (uint32_t)(i * 256 + 128);
-            const uint32_t pa = aP + (i * 2 + (k & 1)) * L::P_BYTES;
-            const uint32_t va = aV + (ep % ATT_STAGES) * L::V_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < ATT_BN / 32; ++kk)
-              mma_f8f6f4(tO, smem_desc(pa + 32 * kk, 1024, 128),
-                         smem_desc(va + L::V_KSTEP * kk, L::QK_SBO, L::QK_SWIZZLE), IDESC_PV,
-                         (k > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(&o_ready[i * 2 + (k & 1)]);
-            ++pv_k[i];
-            pv_e[i] = next_active(i, ep + 1);
-            prog = true;
-          }
-        }
-        while (rel_e < ntile && rel_e < pv_e[0] && rel_e < pv_e[1]) {
-          tc_commit(&kv_empty[rel_e % ATT_STAGES]);
-          ++rel_e;
-          prog = true;
-        }
-        if (prog) {
-          idle = 0;
-        } else if ((++idle & 255u) == 0) {
-          if (*reinterpret_cast<volatile uint32_t*>(&g_status) != 0u) {
-            ok = false;
-          } else if (idle == 256u) {
-            idle_t0 = globaltimer_ns();
-          } else if (globaltimer_ns() - idle_t0 > 2000000000ull) {
-            report_timeout(SITE_MMA_STALL);
-            ok = false;
-          }
-        }
+        for (int k = 0; k < D / 32; ++k)
+          mma_i8(tS, smem_desc(qa + 32 * k, L::QK_SBO, L::QK_SWIZZLE),
+                 smem_desc(ka + 32 * k, L::QK_SBO, L::QK_SWIZZLE), IDESC_QK, 1u);
+        tc_commit(&s_full[i]);
+        ++nqk;
+        if (ep >= 0) ok = issue_pv(ep);
+        ep = e;
       }
+      if (ok && ep >= 0) ok = issue_pv(ep);
+      // positions after this Q tile's last one (or all, if it has none)
+      if (ok) ok = release_to(ntile - 1);
       // every MMA issued above completes before the CTA tears down TMEM
       tc_commit(mma_done);
       mbar_wait(mma_done, 0, SITE_MMA_DONE);
@@ -641,7 +636,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
       const float m_new = fmaxf(m_ref, mt);
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float alpha = ex2_approx(m_ref - m_use);
+      const float alpha = m_new == m_ref ? 1.f : ex2_approx(m_ref - m_use);
       const float bias = LOG2_448 - m_use;
 
       // the P buffer being overwritten was read by PV(n-2); O is touched only
