@@ -5,17 +5,20 @@
 // microscaling for Q/K and V).
 //
 // One CTA owns one 128-row Q tile of one (batch, Q head):
-//   warp 8   producer: TMA for the packed Q, K and V^T tiles, the tile's
-//            qk_correction row as bf16 hi + lo (the B operand of one bf16
-//            MMA that adds it to S), and the scale factors staged in shared
+//   warp 8   producer: TMA for the packed Q, K and V^T tiles into a
+//            5-stage ring, the tile's qk_correction row as bf16 hi + lo (the
+//            B operand of one bf16 MMA that adds it to S; read from global
+//            memory one tile ahead, like the scale factors), and the scale
+//            factors staged in shared
 //            memory in the layout tcgen05.cp expects (for every 64-element K
 //            block a 512-byte block: row r's four scale factors as one
 //            32-bit word at 16*(r%32) + 4*(r/32));
-//   warp 9   MMA issuer: tcgen05.cp of the scale factors into TMEM and
-//            tcgen05.mma kind::mxf4nvf4 with 16-element E4M3 block scales,
-//            S = Q K^T into a double-buffered TMEM accumulator, then
-//            S += qk_correction (kind::f16 bf16 MMA onto the same fp32
-//            accumulator), and O += P V into TMEM, both fp32;
+//   warps 9, 10  MMA issuers, one thread each: warp 9 the QK^T side
+//            (tcgen05.cp of the K scale factors into TMEM, tcgen05.mma
+//            kind::mxf4nvf4 with 16-element E4M3 block scales, S = Q K^T into
+//            a double-buffered TMEM accumulator, then S += qk_correction by a
+//            kind::f16 bf16 MMA onto the same fp32 accumulator), warp 10 the
+//            PV side (V and P scale factors, O += P V into TMEM, fp32);
 //   warps 0-7  softmax, two threads per row: warps q and q+4 share the
 //            TMEM lane quarter q and take keys 0-63 and 64-127 of each
 //            tile (four 16-key vectors each).  Per tile: the scores (the
@@ -35,9 +38,9 @@
 
 namespace sage {
 
-constexpr int NV_THREADS = 320;
-constexpr int NV_PRODUCER_WARP = 8, NV_MMA_WARP = 9;
-constexpr int NV_STAGES = 3;
+constexpr int NV_THREADS = 352;
+constexpr int NV_PRODUCER_WARP = 8, NV_MMA_WARP = 9, NV_PV_WARP = 10;
+constexpr int NV_STAGES = 5;   // K/V ring depth (5.22 / 5.21 / 5.18 / 5.19 ms for 3 / 4 / 5 / 6)
 constexpr float LOG2_2688 = 11.392317422778761f;   // log2(448 * 6)
 
 struct NvAttnArgs {
@@ -165,6 +168,36 @@ __device__ __forceinline__ void stage_sf(uint8_t* dst, const uint8_t* src, int64
   }
 }
 
+// The same staging in two halves, so that a tile's global loads can be in
+// flight while the producer waits for a free stage: load_sf reads one
+// lane's four rows into registers, store_sf writes them in the layout above.
+template <int NSF>
+struct SfRegs {
+  uint32_t w[4][NSF / 4];
+};
+template <int NSF>
+__device__ __forceinline__ void load_sf(SfRegs<NSF>& r, const uint8_t* src, int64_t row_stride,
+                                        int nrows, int lane) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = lane + 32 * i;
+#pragma unroll
+    for (int b = 0; b < NSF / 4; ++b)
+      r.w[i][b] = row < nrows ? __ldg(reinterpret_cast<const uint32_t*>(src + (int64_t)row * row_stride) + b)
+                              : 0u;
+  }
+}
+template <int NSF>
+__device__ __forceinline__ void store_sf(uint8_t* dst, const SfRegs<NSF>& r, int lane) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = lane + 32 * i;
+#pragma unroll
+    for (int b = 0; b < NSF / 4; ++b)
+      *reinterpret_cast<uint32_t*>(dst + b * 512 + 16 * (row & 31) + 4 * (row >> 5)) = r.w[i][b];
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(NV_THREADS, 1)
     attn_fwd_nvfp4_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -250,7 +283,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
     mbar_init(q_full, 32);
     for (int s = 0; s < NV_STAGES; ++s) {
       mbar_init(&kv_full[s], 32);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], 2);   // released by the QK and the PV issuer
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -258,7 +291,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       mbar_init(&p_full[i], 256);
       mbar_init(&o_ready[i], 1);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);
     for (int i = 0; i < 8; ++i) mbar_init(&pmax_full[i], 64);
     fence_mbar_init();
   } else if (warp == NV_MMA_WARP) {
@@ -290,22 +323,32 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
     } else {
       mbar_arrive(q_full);
     }
+    // Per tile the lane's share of the K and V scale factors and of the
+    // qk_correction row is read into registers one tile ahead: the global
+    // loads of tile idx+1 are in flight while the producer waits for a free
+    // stage and stores tile idx.
+    SfRegs<D / 16> ksf;
+    SfRegs<8> vsf;
+    float4 cv = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto load_tile = [&](int idx) {
+      const int kt = (int)(s_list[idx] >> 8);
+      load_sf<D / 16>(ksf, a.k_sf + ((int64_t)bhk * a.Nkp + kt * 128) * (D / 16), D / 16, 128, lane);
+      load_sf<8>(vsf, a.v_sf_t + (int64_t)bhk * D * (a.Nkp / 16) + kt * 8, a.Nkp / 16, D, lane);
+      cv = __ldg(reinterpret_cast<const float4*>(a.corr + ((int64_t)bhq * a.nqt + qt) * a.Nkp + kt * 128) +
+                 lane);
+    };
+    if (ntile > 0) load_tile(0);
     for (int idx = 0; idx < ntile; ++idx) {
       const int st = idx % NV_STAGES, rd = idx / NV_STAGES;
       if (idx >= NV_STAGES &&
           !__all_sync(0xffffffffu, mbar_wait(&kv_empty[st], (rd - 1) & 1, SITE_KV_EMPTY)))
         break;
       const int kt = (int)(s_list[idx] >> 8);
-      stage_sf<D / 16>(sKsf + st * L::KB_QK * L::SF_BLK,
-                       a.k_sf + ((int64_t)bhk * a.Nkp + kt * 128) * (D / 16), D / 16, 128, lane);
-      stage_sf<8>(sVsf + st * 2 * L::SF_BLK, a.v_sf_t + (int64_t)bhk * D * (a.Nkp / 16) + kt * 8,
-                  a.Nkp / 16, D, lane);
+      store_sf<D / 16>(sKsf + st * L::KB_QK * L::SF_BLK, ksf, lane);
+      store_sf<8>(sVsf + st * 2 * L::SF_BLK, vsf, lane);
       {
         // the correction of keys 4*lane .. 4*lane+3 as bf16 hi + lo
         // (|x - hi - lo| <= 2^-18 |x|), row j of the B tile
-        const float4 cv = __ldg(reinterpret_cast<const float4*>(
-                                    a.corr + ((int64_t)bhq * a.nqt + qt) * a.Nkp + kt * 128) +
-                                lane);
         const float x[4] = {cv.x, cv.y, cv.z, cv.w};
         uint8_t* tile = sCorrB + st * 4096;
 #pragma unroll
@@ -320,6 +363,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
           *reinterpret_cast<uint4*>(tile + j * 32 + ((1 ^ sw) << 4)) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
+      if (idx + 1 < ntile) load_tile(idx + 1);
       fence_proxy_async_smem();
       if (lane == 0) {
         mbar_arrive_expect_tx(&kv_full[st], (uint32_t)(L::K_BYTES + L::V_BYTES));
@@ -331,58 +375,73 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       }
     }
     __syncwarp();
-  } else if (warp == NV_MMA_WARP) {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp == NV_MMA_WARP || warp == NV_PV_WARP) {
+    // ---------------------------------------------------------- MMA issuers
+    // Two issuing threads: warp 9 issues the QK^T side (K scale factors,
+    // QK^T MMAs, the qk_correction MMA), warp 10 the PV side (V and P scale
+    // factors, PV MMAs).  Each tcgen05.mma or tcgen05.cp holds its thread
+    // for about its execution time and each wait or commit costs tens of
+    // clocks, so one thread doing both sides left the tensor pipe idle for
+    // most of a tile; two threads overlap one side's waits with the other's
+    // MMAs.  Their TMEM columns are disjoint (S and the Q/K scale factors,
+    // O and the V/P scale factors), and each side stays in order within its
+    // thread.  A K/V stage is released once both have committed on it.
     if (lane == 0) {
       constexpr uint32_t ID_QK = nv_idesc(128, 128);
       constexpr uint32_t ID_PV = nv_idesc(128, D);
       constexpr int KSTRIDE = (L::OFF_V - L::OFF_K) / NV_STAGES;
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-      bool ok = mbar_wait(q_full, 0, SITE_Q_FULL);
-      tc_fence_after();
-#pragma unroll
-      for (int kb = 0; kb < L::KB_QK; ++kb) sf_copy(tmem + L::T_SFQ + 4 * kb, smem_u32(sQsf) + kb * 512);
-      auto do_pv = [&](int j) {
-        ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, SITE_P_FULL);
-        if (!ok) return;
+      bool ok = true;
+      if (warp == NV_MMA_WARP) {
+        ok = mbar_wait(q_full, 0, SITE_Q_FULL);
         tc_fence_after();
-        const int st = j % NV_STAGES;
 #pragma unroll
-        for (int kb = 0; kb < 2; ++kb) {
-          sf_copy(tmem + L::T_SFV + 4 * kb, smem_u32(sVsf) + (st * 2 + kb) * 512);
-          sf_copy(tmem + L::T_SFP + 4 * kb, smem_u32(sPsf) + ((j & 1) * 2 + kb) * 512);
+        for (int kb = 0; kb < L::KB_QK; ++kb) sf_copy(tmem + L::T_SFQ + 4 * kb, smem_u32(sQsf) + kb * 512);
+        for (int idx = 0; ok && idx < ntile; ++idx) {
+          const int st = idx % NV_STAGES, buf = idx & 1;
+          ok = mbar_wait(&kv_full[st], (idx / NV_STAGES) & 1, SITE_KV_FULL);
+          if (ok && idx >= 2) ok = mbar_wait(&s_free[buf], ((idx - 2) >> 1) & 1, SITE_S_FREE);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kb = 0; kb < L::KB_QK; ++kb)
+            sf_copy(tmem + L::T_SFK + 4 * kb, smem_u32(sKsf) + (st * L::KB_QK + kb) * 512);
+#pragma unroll
+          for (int kb = 0; kb < L::KB_QK; ++kb)
+            mma_nvfp4(tmem + L::T_S + buf * 128,
+                      smem_desc(aQ + 32 * kb, L::QK_SBO, L::QK_SWIZZLE),
+                      smem_desc(aK + st * KSTRIDE + 32 * kb, L::QK_SBO, L::QK_SWIZZLE), ID_QK,
+                      tmem + L::T_SFQ + 4 * kb, tmem + L::T_SFK + 4 * kb, kb > 0 ? 1u : 0u);
+          // S += qk_correction of each key (one bf16 MMA onto the fp32 scores)
+          mma_f16(tmem + L::T_S + buf * 128, smem_desc(smem_u32(sOnes), 256, 32),
+                  smem_desc(smem_u32(sCorrB) + st * 4096, 256, 32), instr_desc(kDF32, 1u, 1u, 128, 128),
+                  1u);
+          tc_commit(&s_full[buf]);
+          tc_commit(&kv_empty[st]);
         }
+      } else {
+        for (int j = 0; ok && j < ntile; ++j) {
+          const int st = j % NV_STAGES;
+          // the V tile and its staged scale factors (kv_full), then P (p_full)
+          ok = mbar_wait(&kv_full[st], (j / NV_STAGES) & 1, SITE_KV_FULL) &&
+               mbar_wait(&p_full[j & 1], (j >> 1) & 1, SITE_P_FULL);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kb = 0; kb < 2; ++kb)
-          mma_nvfp4(tmem + L::T_O, smem_desc(aP + (j & 1) * L::P_BYTES + 32 * kb, 512, 64),
-                    smem_desc(aV + st * L::V_BYTES + 32 * kb, 512, 64), ID_PV,
-                    tmem + L::T_SFP + 4 * kb, tmem + L::T_SFV + 4 * kb, (j > 0 || kb > 0) ? 1u : 0u);
-        tc_commit(&o_ready[j & 1]);
-        tc_commit(&kv_empty[st]);
-      };
-      for (int idx = 0; ok && idx < ntile; ++idx) {
-        const int st = idx % NV_STAGES, buf = idx & 1;
-        ok = mbar_wait(&kv_full[st], (idx / NV_STAGES) & 1, SITE_KV_FULL);
-        if (ok && idx >= 2) ok = mbar_wait(&s_free[buf], ((idx - 2) >> 1) & 1, SITE_S_FREE);
-        if (!ok) break;
-        tc_fence_after();
+          for (int kb = 0; kb < 2; ++kb) {
+            sf_copy(tmem + L::T_SFV + 4 * kb, smem_u32(sVsf) + (st * 2 + kb) * 512);
+            sf_copy(tmem + L::T_SFP + 4 * kb, smem_u32(sPsf) + ((j & 1) * 2 + kb) * 512);
+          }
 #pragma unroll
-        for (int kb = 0; kb < L::KB_QK; ++kb)
-          sf_copy(tmem + L::T_SFK + 4 * kb, smem_u32(sKsf) + (st * L::KB_QK + kb) * 512);
-#pragma unroll
-        for (int kb = 0; kb < L::KB_QK; ++kb)
-          mma_nvfp4(tmem + L::T_S + buf * 128,
-                    smem_desc(aQ + 32 * kb, L::QK_SBO, L::QK_SWIZZLE),
-                    smem_desc(aK + st * KSTRIDE + 32 * kb, L::QK_SBO, L::QK_SWIZZLE), ID_QK,
-                    tmem + L::T_SFQ + 4 * kb, tmem + L::T_SFK + 4 * kb, kb > 0 ? 1u : 0u);
-        // S += qk_correction of each key (one bf16 MMA onto the fp32 scores)
-        mma_f16(tmem + L::T_S + buf * 128, smem_desc(smem_u32(sOnes), 256, 32),
-                smem_desc(smem_u32(sCorrB) + st * 4096, 256, 32), instr_desc(kDF32, 1u, 1u, 128, 128),
-                1u);
-        tc_commit(&s_full[buf]);
-        if (idx >= 1) do_pv(idx - 1);
+          for (int kb = 0; kb < 2; ++kb)
+            mma_nvfp4(tmem + L::T_O, smem_desc(aP + (j & 1) * L::P_BYTES + 32 * kb, 512, 64),
+                      smem_desc(aV + st * L::V_BYTES + 32 * kb, 512, 64), ID_PV,
+                      tmem + L::T_SFP + 4 * kb, tmem + L::T_SFV + 4 * kb, (j > 0 || kb > 0) ? 1u : 0u);
+          tc_commit(&o_ready[j & 1]);
+          tc_commit(&kv_empty[st]);
+        }
       }
-      if (ok && ntile > 0) do_pv(ntile - 1);
+      // every MMA issued above completes before the CTA tears down TMEM
       tc_commit(mma_done);
       mbar_wait(mma_done, 0, SITE_MMA_DONE);
     }
