@@ -504,6 +504,7 @@ sage_status run_attention_nvfp4(const sage_qkv_nvfp4* z, float sm_scale, int cau
   a.Nq = (int)z->Nq; a.Nk = (int)z->Nk;
   a.Nqp = (int)pad128(z->Nq); a.Nkp = (int)pad128(z->Nk);
   a.nqt = a.Nqp / 128; a.nkt = a.Nkp / 128;
+  a.nqp = (a.nqt + 1) / 2;
   a.L = (int)z->unpadded_k_len;
   a.causal = causal ? 1 : 0;
   a.return_lse = return_lse ? 1 : 0;
@@ -519,16 +520,19 @@ sage_status run_attention_nvfp4(const sage_qkv_nvfp4* z, float sm_scale, int cau
       !make_tmap_u8(&tv, z->v_t, a.Nkp / 2, z->B * z->Hkv * D, a.Nkp / 2, 64, (uint32_t)D,
                     CU_TENSOR_MAP_SWIZZLE_64B))
     return SAGE_ERR_CUDA;
-  const int grid = a.B * a.Hq * a.nqt;
-  if (D == 128) {
-    if (!ensure_smem(attn_fwd_nvfp4_kernel<128>, NvLayout<128>::bytes(ATT_MAX_NKT), &g_smem_nv128))
-      return SAGE_ERR_CUDA;
-    attn_fwd_nvfp4_kernel<128><<<grid, NV_THREADS, NvLayout<128>::bytes(a.nkt), stream>>>(tq, tk, tv, a);
-  } else {
-    if (!ensure_smem(attn_fwd_nvfp4_kernel<64>, NvLayout<64>::bytes(ATT_MAX_NKT), &g_smem_nv64))
-      return SAGE_ERR_CUDA;
-    attn_fwd_nvfp4_kernel<64><<<grid, NV_THREADS, NvLayout<64>::bytes(a.nkt), stream>>>(tq, tk, tv, a);
+  const int grid = a.B * a.Hq * a.nqp;
+  auto kernel = D == 128 ? attn_fwd_nvfp4_kernel<128> : attn_fwd_nvfp4_kernel<64>;
+  // the kernel redistributes registers between its warpgroups; that is only
+  // safe if the launch provides at least the sum of their shares
+  {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return SAGE_ERR_CUDA;
+    if (128 * NV_REGS_LOW + 256 * NV_REGS_HIGH > NV_THREADS * fa.numRegs) return SAGE_ERR_UNSUPPORTED;
   }
+  const size_t smem = D == 128 ? NvLayout<128>::bytes(a.nkt) : NvLayout<64>::bytes(a.nkt);
+  const size_t smem_max = D == 128 ? NvLayout<128>::bytes(ATT_MAX_NKT) : NvLayout<64>::bytes(ATT_MAX_NKT);
+  if (!ensure_smem(kernel, smem_max, D == 128 ? &g_smem_nv128 : &g_smem_nv64)) return SAGE_ERR_CUDA;
+  kernel<<<grid, NV_THREADS, smem, stream>>>(tq, tk, tv, a);
   return launch_status();
 }
 
