@@ -201,10 +201,25 @@ __global__ void __launch_bounds__(D) kv_stats_kernel(QuantArgs a) {
   const int nk = seq_view(a.seqs, bh / a.Hkv, a.Nq, a.kv_limit).nk;
   DD s = {0.0, 0.0};
   float m = 0.f;
-  for (int sp = 0; sp < a.splits; ++sp) {
-    const int64_t o = ((int64_t)bh * a.splits + sp) * D + c;
-    dd_add(s, DD{a.part_hi[o], a.part_lo[o]});
-    m = fmaxf(m, a.part_amax[o]);
+  // eight splits' partials loaded before they are combined, in split order
+  constexpr int U = 8;
+  for (int sp0 = 0; sp0 < a.splits; sp0 += U) {
+    double hi[U], lo[U];
+    float am[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t o = ((int64_t)bh * a.splits + sp0 + u) * D + c;
+      const bool live = sp0 + u < a.splits;
+      hi[u] = live ? a.part_hi[o] : 0.0;
+      lo[u] = live ? a.part_lo[o] : 0.0;
+      am[u] = live ? a.part_amax[o] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (sp0 + u >= a.splits) break;
+      dd_add(s, DD{hi[u], lo[u]});
+      m = fmaxf(m, am[u]);
+    }
   }
   a.k_mean[(int64_t)bh * D + c] = a.smooth_k && nk > 0 ? dd_mean_f32(s, (double)nk) : 0.f;
   a.va[(int64_t)bh * D + c] = m;
@@ -263,9 +278,11 @@ __device__ __forceinline__ float rows_sum_transposed(float* v, int cg) {
 }
 
 // ------------------------------------------------------------ pass B
-// One CTA per 128-token block: [0, nQb) Q blocks, [nQb, nQb+nKb) K blocks,
-// then V blocks.  Each thread keeps its 16-byte loads in registers between
-// the amax and the code pass.
+// One CTA per 128-token block: first the K and V blocks, KV heads in
+// descending order (pass A reads the heads in ascending order, so the K and
+// V rows it read last are still in L2 when pass B starts), K and V blocks of
+// a head alternating; then the Q blocks.  Each thread keeps its 16-byte loads
+// in registers between the amax and the code pass.
 template <typename T, int D>
 __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArgs a) {
   constexpr int TPR = D / 8;
@@ -274,14 +291,17 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
   __shared__ float s_c[D];      // k_mean (Q with LSE, K) or 448 / V channel max (V)
   __shared__ float s_red[QUANT_THREADS / 32];
 
-  const int nQb = a.B * a.Hq * a.max_nqt;
   const int nKb = a.B * a.Hkv * a.max_nkt;
-  int job = blockIdx.x;
+  const int job = blockIdx.x;
   const int cg = threadIdx.x % TPR, rs = threadIdx.x / TPR;
+  // K/V job -> (KV head, block, K or V)
+  const int kvh = a.B * a.Hkv - 1 - job / (2 * a.max_nkt);
+  const int kvt = (job % (2 * a.max_nkt)) >> 1;
+  const bool is_v = job & 1;
 
-  if (job < nQb) {
+  if (job >= 2 * nKb) {
     // ---------------- Q block
-    const int bh = job / a.max_nqt, qt = job % a.max_nqt;
+    const int bh = (job - 2 * nKb) / a.max_nqt, qt = (job - 2 * nKb) % a.max_nqt;
     const int b = bh / a.Hq, h = bh % a.Hq;
     const int g = h / a.G;
     const SeqView sq = seq_view(a.seqs, b, a.Nq, a.kv_limit);
@@ -336,10 +356,9 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
       a.q_scale[(int64_t)a.Hq * (sq.cqp / 128) + (int64_t)h * nqt + qt] = __fdiv_rn(amax, 127.f);
     return;
   }
-  job -= nQb;
-  if (job < nKb) {
+  if (!is_v) {
     // ---------------- K block: codes of K - kmean
-    const int bh = job / a.max_nkt, kt = job % a.max_nkt;
+    const int bh = kvh, kt = kvt;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     const SeqView sq = seq_view(a.seqs, b, a.Nq, a.kv_limit);
     const int nkt = (sq.nk + 127) / 128, Nkp = nkt * 128;
@@ -390,10 +409,9 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
       a.k_scale[(int64_t)a.Hkv * (sq.ckp / 128) + (int64_t)h * nkt + kt] = __fdiv_rn(amax, 127.f);
     return;
   }
-  job -= nKb;
   {
     // ---------------- V block: per-channel E4M3 codes, [token, channel] order
-    const int bh = job / a.max_nkt, vt = job % a.max_nkt;
+    const int bh = kvh, vt = kvt;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     const SeqView sq = seq_view(a.seqs, b, a.Nq, a.kv_limit);
     const int nkt = (sq.nk + 127) / 128, Nkp = nkt * 128;

@@ -8,7 +8,7 @@
 //                        sums of K (tokens < unpadded_k_len) or Q;
 //   nv_means_kernel      the K mean and the Q means (per 128-token block or
 //                        global), each rounded once to fp32;
-//   nv_quant_kernel      one CTA per 128-token block of Q, K or V: every
+//   nv_quant_kernel      one CTA per 128-token block of Q, V or K: every
 //                        16-element vector gets sf = e4m3(fp32(amax/6)) and
 //                        codes e2m1(fp32(x * fp32(1/sf))), packed two per byte
 //                        (element 2i in the low nibble); V is transposed so
@@ -116,11 +116,24 @@ __global__ void __launch_bounds__(QUANT_THREADS)
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = {0.0, 0.0};
   const char* base = reinterpret_cast<const char*>(src) + (b * sb + h * sh + cg * 8) * (int64_t)sizeof(T);
-  for (int n = n0 + rs; n < n1; n += RPP) {
-    float f[8];
-    unpack8<T>(ldg16(base + (int64_t)n * sn * sizeof(T)), f);
+  // four rows per iteration, their loads issued before any arithmetic (the
+  // accumulation order per channel is the same fixed row order as one by one)
+  constexpr int UNR = 4;
+  for (int nb = n0 + rs; nb < n1; nb += UNR * RPP) {
+    uint4 r[UNR];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) dd_add(acc[i], (double)f[i]);
+    for (int u = 0; u < UNR; ++u) {
+      const int n = nb + u * RPP;
+      r[u] = n < n1 ? ldg16(base + (int64_t)n * sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      if (nb + u * RPP >= n1) break;
+      float f[8];
+      unpack8<T>(r[u], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dd_add(acc[i], (double)f[i]);
+    }
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -179,14 +192,19 @@ __global__ void __launch_bounds__(D) nv_means_kernel(NvQuantArgs a) {
 }
 
 // ------------------------------------------------------------ block quantiser
-// One CTA per 128-token block: [0, nQb) Q, [nQb, nQb+nKb) K, then V blocks.
-// Q/K: D/16 threads per row, one 16-element vector each.  V: the block is
-// staged in shared memory and every thread quantises 16-token vectors of one
-// channel.
+// One CTA per 128-token block: first the Q blocks, heads in descending order
+// (the Q column sums read the heads in ascending order just before, so the
+// rows they read last are still in L2), then the V blocks, then the K blocks
+// in descending head order (so that the correction kernel, which starts at
+// head 0, finds the K rows read last in L2).
+// Q/K: D/16 threads per row, one 16-element vector each, the block's four
+// rows per thread loaded before any of them is used.  V: the block is staged
+// in shared memory and every thread quantises 16-token vectors of one channel.
 template <typename T, int D>
 __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) {
   constexpr int VPR = D / 16;                 // vectors per row
   constexpr int RPP = QUANT_THREADS / VPR;    // rows per pass
+  constexpr int ITERS = QB / RPP;
   __shared__ float s_m[D];
   __shared__ float s_km[D];
   __shared__ __align__(16) T s_v[QB][D + 8];
@@ -196,24 +214,32 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
   const int vi = threadIdx.x % VPR, rs = threadIdx.x / VPR;
 
   if (job < nQb) {
-    const int bh = job / a.nqt, qt = job % a.nqt;
+    const int bh = a.B * a.Hq - 1 - job / a.nqt, qt = job % a.nqt;
     const int b = bh / a.Hq, h = bh % a.Hq, g = h / a.G;
+    const char* base = reinterpret_cast<const char*>(a.q) +
+                       (b * a.q_sb + h * a.q_sh + vi * 16) * (int64_t)sizeof(T);
+    uint4 raw[ITERS][2];
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int n = qt * QB + rs + it * RPP;
+      const char* p = base + (int64_t)n * a.q_sn * sizeof(T);
+      raw[it][0] = n < a.Nq ? ldg16(p) : make_uint4(0, 0, 0, 0);
+      raw[it][1] = n < a.Nq ? ldg16(p + 8 * sizeof(T)) : make_uint4(0, 0, 0, 0);
+    }
     for (int c = threadIdx.x; c < D; c += blockDim.x) {
       s_m[c] = a.q_mean[((int64_t)bh * a.nqt + qt) * D + c];
       s_km[c] = a.k_mean[((int64_t)b * a.Hkv + g) * D + c];
     }
     __syncthreads();
-    const char* base = reinterpret_cast<const char*>(a.q) +
-                       (b * a.q_sb + h * a.q_sh + vi * 16) * (int64_t)sizeof(T);
-    for (int r = rs; r < QB; r += RPP) {
-      const int n = qt * QB + r;
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int n = qt * QB + rs + it * RPP;
       float x[16];
       float dq = 0.f;
       if (n < a.Nq) {
         float f[16];
-        const char* p = base + (int64_t)n * a.q_sn * sizeof(T);
-        unpack8<T>(ldg16(p), f);
-        unpack8<T>(ldg16(p + 8 * sizeof(T)), f + 8);
+        unpack8<T>(raw[it][0], f);
+        unpack8<T>(raw[it][1], f + 8);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           x[i] = __fsub_rn(f[i], s_m[vi * 16 + i]);
@@ -237,21 +263,30 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
     return;
   }
   job -= nQb;
-  if (job < nKb) {
-    const int bh = job / a.nkt, kt = job % a.nkt;
+  if (job >= nKb) {
+    job -= nKb;
+    const int bh = a.B * a.Hkv - 1 - job / a.nkt, kt = job % a.nkt;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
-    for (int c = threadIdx.x; c < D; c += blockDim.x) s_km[c] = a.k_mean[(int64_t)bh * D + c];
-    __syncthreads();
     const char* base = reinterpret_cast<const char*>(a.k) +
                        (b * a.k_sb + h * a.k_sh + vi * 16) * (int64_t)sizeof(T);
-    for (int r = rs; r < QB; r += RPP) {
-      const int n = kt * QB + r;
+    uint4 raw[ITERS][2];
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int n = kt * QB + rs + it * RPP;
+      const char* p = base + (int64_t)n * a.k_sn * sizeof(T);
+      raw[it][0] = n < a.L ? ldg16(p) : make_uint4(0, 0, 0, 0);
+      raw[it][1] = n < a.L ? ldg16(p + 8 * sizeof(T)) : make_uint4(0, 0, 0, 0);
+    }
+    for (int c = threadIdx.x; c < D; c += blockDim.x) s_km[c] = a.k_mean[(int64_t)bh * D + c];
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int n = kt * QB + rs + it * RPP;
       float x[16];
       if (n < a.L) {
         float f[16];
-        const char* p = base + (int64_t)n * a.k_sn * sizeof(T);
-        unpack8<T>(ldg16(p), f);
-        unpack8<T>(ldg16(p + 8 * sizeof(T)), f + 8);
+        unpack8<T>(raw[it][0], f);
+        unpack8<T>(raw[it][1], f + 8);
 #pragma unroll
         for (int i = 0; i < 16; ++i) x[i] = __fsub_rn(f[i], s_km[vi * 16 + i]);
       } else {
@@ -266,20 +301,23 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
     }
     return;
   }
-  job -= nKb;
   {
     const int bh = job / a.nkt, vt = job % a.nkt;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     constexpr int TPR = D / 8;
+    constexpr int VR = QB / (QUANT_THREADS / TPR);   // staged rows per thread
     const int cg = threadIdx.x % TPR, rr = threadIdx.x / TPR;
     const char* base = reinterpret_cast<const char*>(a.v) +
                        (b * a.v_sb + h * a.v_sh + cg * 8) * (int64_t)sizeof(T);
-    for (int r = rr; r < QB; r += QUANT_THREADS / TPR) {
-      const int n = vt * QB + r;
-      uint4 raw = make_uint4(0, 0, 0, 0);
-      if (n < a.L) raw = ldg16(base + (int64_t)n * a.v_sn * sizeof(T));
-      *reinterpret_cast<uint4*>(&s_v[r][cg * 8]) = raw;
+    uint4 raw[VR];
+#pragma unroll
+    for (int i = 0; i < VR; ++i) {
+      const int n = vt * QB + rr + i * (QUANT_THREADS / TPR);
+      raw[i] = n < a.L ? ldg16(base + (int64_t)n * a.v_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
     }
+#pragma unroll
+    for (int i = 0; i < VR; ++i)
+      *reinterpret_cast<uint4*>(&s_v[rr + i * (QUANT_THREADS / TPR)][cg * 8]) = raw[i];
     __syncthreads();
     // vector (channel c, 16-token group gq): threads cover channels fastest
     for (int idx = threadIdx.x; idx < D * (QB / 16); idx += blockDim.x) {
@@ -303,26 +341,28 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
 // |x - hi - lo| <= 2^-18 |x|, and the MMAs hi.hi + hi.lo + lo.hi accumulate
 // in fp32 in TMEM; the omitted lo.lo and the split leave a relative error of
 // about 2^-16 per product (the fp32 reference sum rounds at 2^-24).
-// grid (nkt, B*Hkv), 256 threads: all threads stage the operands with
-// coalesced 16/32-byte loads; thread 0 issues the MMAs; warps w and w + 4
-// read TMEM lane quarter w%4 back, 64 of the 128 key columns each.
-// Shared memory: B_hi, B_lo (128 keys x D), A_hi, A_lo (128 vectors x D),
-// bf16, K-major with the 128-byte swizzle in 64-channel atoms of 16 KB: row r
-// at r * 128, 16-byte chunk c at (c ^ (r % 8)) * 16; then the fp32 output
-// tile, staged so that the correction rows are written coalesced.
+// grid (nkt, B*Hkv), 256 threads, three CTAs per SM.  Per chunk of 128 Q-mean
+// vectors the D channels are taken 64 at a time: all threads stage that half
+// of the 128 keys (the MMA's M side) and of the 128 vectors (its N side) with
+// coalesced 16/32-byte loads, thread 0 issues the MMAs, and the next half
+// overwrites the tiles once they have completed.  The scores land in TMEM as
+// [key][vector], so for each vector the 32 lanes of a warp store 32
+// consecutive keys: every store instruction writes 128 contiguous bytes of a
+// correction row, with no staging.
+// Shared memory: A_hi, A_lo (128 keys x 64 channels), B_hi, B_lo (128
+// vectors x 64 channels), bf16, K-major with the 128-byte swizzle: row r at
+// r * 128, 16-byte chunk c at (c ^ (r % 8)) * 16.
 constexpr int NVC_THREADS = 256;
 template <int D>
 struct NvCorrLayout {
-  static constexpr int TILE = 128 * D * 2;   // one operand: 128 rows x D bf16
-  static constexpr int OFF_BHI = 0, OFF_BLO = TILE, OFF_AHI = 2 * TILE, OFF_ALO = 3 * TILE;
-  static constexpr int OFF_OUT = 4 * TILE;        // 128 rows x 132 fp32 (output staging)
-  static constexpr int BYTES = OFF_OUT + 128 * 132 * 4 + 1024;   // + alignment slack
+  static constexpr int TILE = 128 * 64 * 2;   // one operand half: 128 rows x 64 bf16
+  static constexpr int OFF_AHI = 0, OFF_ALO = TILE, OFF_BHI = 2 * TILE, OFF_BLO = 3 * TILE;
+  static constexpr int BYTES = 4 * TILE + 1024;   // + alignment slack
 };
 
-// Channels 8*cg .. 8*cg+7 of row r into a swizzled operand tile.
-__device__ __forceinline__ void nvc_put(uint8_t* tile, int r, int cg, const uint4& v) {
-  const int atom = cg >> 3, c = cg & 7;
-  *reinterpret_cast<uint4*>(tile + atom * 16384 + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+// Channels 8*c .. 8*c+7 (c < 8) of row r into a swizzled 64-channel tile.
+__device__ __forceinline__ void nvc_put(uint8_t* tile, int r, int c, const uint4& v) {
+  *reinterpret_cast<uint4*>(tile + r * 128 + ((c ^ (r & 7)) << 4)) = v;
 }
 
 // bf16 hi / lo parts of 8 floats, two per word (lower channel in the low half).
@@ -342,7 +382,7 @@ __device__ __forceinline__ void nvc_split8(const float* x, uint4& hi, uint4& lo)
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(NVC_THREADS, 1) nv_corr_kernel(NvQuantArgs a) {
+__global__ void __launch_bounds__(NVC_THREADS, 3) nv_corr_kernel(NvQuantArgs a) {
   using L = NvCorrLayout<D>;
   extern __shared__ uint8_t nvc_raw[];
   uint8_t* sm = nvc_raw + ((1024u - (smem_u32(nvc_raw) & 1023u)) & 1023u);
@@ -351,9 +391,8 @@ __global__ void __launch_bounds__(NVC_THREADS, 1) nv_corr_kernel(NvQuantArgs a) 
   __shared__ float s_km[D];
   const int kt = blockIdx.x, bg = blockIdx.y;
   const int b = bg / a.Hkv, g = bg % a.Hkv;
-  const int t = threadIdx.x, warp = t >> 5;
-  constexpr int CG = D / 8;                          // 16-byte bf16 chunks per row
-  constexpr int PER = 128 * CG / NVC_THREADS;        // chunks per thread per operand
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  constexpr int PER = 128 * 8 / NVC_THREADS;   // 16-byte chunks per thread per operand half
   for (int c = t; c < D; c += NVC_THREADS) s_km[c] = a.k_mean[(int64_t)bg * D + c];
   if (t == 0) {
     mbar_init(&mma_bar, 1);
@@ -363,96 +402,83 @@ __global__ void __launch_bounds__(NVC_THREADS, 1) nv_corr_kernel(NvQuantArgs a) 
     tmem_alloc(&tmem_slot, 128);
     tmem_relinquish();
   }
+  tc_fence_before();
   __syncthreads();
-  // B: Ks = fp32(K - kmean) for keys < L, 0 beyond.  Chunk q = t + 256 i is
-  // channels 8*(q % CG).. of key q / CG: consecutive threads read consecutive
-  // 16 bytes of a key row, and every load is in flight before the first use.
-  {
-    uint4 raw[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int q = t + NVC_THREADS * i, key = q / CG, cg = q % CG;
-      const int n = kt * 128 + key;
-      raw[i] = n < a.L ? ldg16(reinterpret_cast<const char*>(a.k) +
-                               (b * a.k_sb + g * a.k_sh + (int64_t)n * a.k_sn + cg * 8) *
-                                   (int64_t)sizeof(T))
-                       : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int q = t + NVC_THREADS * i, key = q / CG, cg = q % CG;
-      const bool live = kt * 128 + key < a.L;
-      float f[8];
-      unpack8<T>(raw[i], f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = live ? __fsub_rn(f[e], s_km[cg * 8 + e]) : 0.f;
-      uint4 hi, lo;
-      nvc_split8(f, hi, lo);
-      nvc_put(sm + L::OFF_BHI, key, cg, hi);
-      nvc_put(sm + L::OFF_BLO, key, cg, lo);
-    }
-  }
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
   // the Q means of a chunk are 128 consecutive rows of q_mean: vector v of
   // KV head g is row (b*Hq + g*G)*nqt + v
   const int nvec = a.G * a.nqt;
   const float* qm_base = a.q_mean + ((int64_t)b * a.Hq + (int64_t)g * a.G) * a.nqt * D;
   float* corr_base = a.corr + ((int64_t)b * a.Hq + (int64_t)g * a.G) * a.nqt * a.Nkp + kt * 128;
-  // output staging: 128 rows of 128 fp32, rows 132 floats apart (conflict-free
-  // 16-byte stores)
-  float* s_out = reinterpret_cast<float*>(sm + L::OFF_OUT);
+  const char* kbase = reinterpret_cast<const char*>(a.k) + (b * a.k_sb + g * a.k_sh) * (int64_t)sizeof(T);
   uint32_t phase = 0;
   bool ok = true;
   for (int v0 = 0; ok && v0 < nvec; v0 += 128) {
-    {
-      float4 raw[2 * PER];
+    for (int hf = 0; ok && hf < D / 64; ++hf) {
+      // chunk q = t + 256 i: channels hf*64 + 8*(q % 8) .. of row q / 8;
+      // every load is in flight before the first use
+      uint4 kraw[PER];
+      float4 qraw[2 * PER];
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
-        const int q = t + NVC_THREADS * i, row = q / CG, cg = q % CG;
+        const int q = t + NVC_THREADS * i, row = q >> 3, c = q & 7;
+        const int n = kt * 128 + row;
+        kraw[i] = n < a.L ? ldg16(kbase + ((int64_t)n * a.k_sn + hf * 64 + c * 8) * (int64_t)sizeof(T))
+                          : make_uint4(0, 0, 0, 0);
         const bool live = v0 + row < nvec;
-        const float4* src = reinterpret_cast<const float4*>(qm_base + (int64_t)(v0 + row) * D + cg * 8);
-        raw[2 * i] = live ? __ldg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
-        raw[2 * i + 1] = live ? __ldg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4* src =
+            reinterpret_cast<const float4*>(qm_base + (int64_t)(v0 + row) * D + hf * 64 + c * 8);
+        qraw[2 * i] = live ? __ldg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+        qraw[2 * i + 1] = live ? __ldg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
-        const int q = t + NVC_THREADS * i, row = q / CG, cg = q % CG;
-        const float f[8] = {raw[2 * i].x, raw[2 * i].y, raw[2 * i].z, raw[2 * i].w,
-                            raw[2 * i + 1].x, raw[2 * i + 1].y, raw[2 * i + 1].z, raw[2 * i + 1].w};
+        const int q = t + NVC_THREADS * i, row = q >> 3, c = q & 7;
+        // A: Ks = fp32(K - kmean) for keys < L, 0 beyond
+        const bool live = kt * 128 + row < a.L;
+        float f[8];
+        unpack8<T>(kraw[i], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = live ? __fsub_rn(f[e], s_km[hf * 64 + c * 8 + e]) : 0.f;
         uint4 hi, lo;
         nvc_split8(f, hi, lo);
-        nvc_put(sm + L::OFF_AHI, row, cg, hi);
-        nvc_put(sm + L::OFF_ALO, row, cg, lo);
+        nvc_put(sm + L::OFF_AHI, row, c, hi);
+        nvc_put(sm + L::OFF_ALO, row, c, lo);
+        // B: the Q means
+        const float qf[8] = {qraw[2 * i].x, qraw[2 * i].y, qraw[2 * i].z, qraw[2 * i].w,
+                             qraw[2 * i + 1].x, qraw[2 * i + 1].y, qraw[2 * i + 1].z, qraw[2 * i + 1].w};
+        nvc_split8(qf, hi, lo);
+        nvc_put(sm + L::OFF_BHI, row, c, hi);
+        nvc_put(sm + L::OFF_BLO, row, c, lo);
       }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = tmem_slot;
-    if (t == 0) {
-      constexpr uint32_t ID = instr_desc(kDF32, 1u, 1u, 128, 128);   // bf16 x bf16 -> fp32
-      const uint32_t ah = smem_u32(sm + L::OFF_AHI), al = smem_u32(sm + L::OFF_ALO);
-      const uint32_t bh = smem_u32(sm + L::OFF_BHI), bl = smem_u32(sm + L::OFF_BLO);
-      const uint32_t pa[3] = {ah, ah, al}, pb[3] = {bh, bl, bh};
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (t == 0) {
+        constexpr uint32_t ID = instr_desc(kDF32, 1u, 1u, 128, 128);   // bf16 x bf16 -> fp32
+        const uint32_t ah = smem_u32(sm + L::OFF_AHI), al = smem_u32(sm + L::OFF_ALO);
+        const uint32_t bh = smem_u32(sm + L::OFF_BHI), bl = smem_u32(sm + L::OFF_BLO);
+        const uint32_t pa[3] = {ah, ah, al}, pb[3] = {bh, bl, bh};
 #pragma unroll
-      for (int pass = 0; pass < 3; ++pass)
-#pragma unroll
-        for (int atom = 0; atom < D / 64; ++atom)
+        for (int pass = 0; pass < 3; ++pass)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_f16(tmem, smem_desc(pa[pass] + atom * 16384 + 32 * k, 1024, 128),
-                    smem_desc(pb[pass] + atom * 16384 + 32 * k, 1024, 128), ID,
-                    (pass | atom | k) ? 1u : 0u);
-      tc_commit(&mma_bar);
+            mma_f16(tmem, smem_desc(pa[pass] + 32 * k, 1024, 128), smem_desc(pb[pass] + 32 * k, 1024, 128),
+                    ID, (hf | pass | k) ? 1u : 0u);
+        tc_commit(&mma_bar);
+      }
+      __syncwarp();
+      // the tiles are rewritten by the next half only after the MMAs are done
+      ok = __all_sync(0xffffffffu, mbar_wait(&mma_bar, phase & 1, SITE_MMA_DONE));
+      ++phase;
+      tc_fence_after();
     }
-    __syncwarp();
-    ok = __all_sync(0xffffffffu, mbar_wait(&mma_bar, phase & 1, SITE_MMA_DONE));
-    ++phase;
-    tc_fence_after();
-    // the MMAs are done with the operand tiles: TMEM rows -> s_out
-    // (warps w and w + 4 share lane quarter w % 4, 64 key columns each)
+    // TMEM [key][vector] -> correction rows: warp w holds keys 32*(w%4) ..
+    // and vectors 64*(w/4) .. of the chunk
     if (ok) {
-      const int rr = (warp & 3) * 32 + (t & 31);
+      const int key = (warp & 3) * 32 + lane;
       const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 #pragma unroll
       for (int cb = (warp >> 2) * 64; cb < (warp >> 2) * 64 + 64; cb += 32) {
@@ -460,31 +486,17 @@ __global__ void __launch_bounds__(NVC_THREADS, 1) nv_corr_kernel(NvQuantArgs a) 
         SAGE_TMEM_LD32(tl + cb, o);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          *reinterpret_cast<float4*>(s_out + rr * 132 + cb + 4 * e) =
-              make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
-                          __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+        for (int e = 0; e < 32; ++e)
+          if (v0 + cb + e < nvec) corr_base[(int64_t)(v0 + cb + e) * a.Nkp + key] = __uint_as_float(o[e]);
       }
     }
-    __syncthreads();
-    // coalesced rows of the correction: 32 threads write one 512-byte row
-    if (ok) {
-      for (int q = t; q < 128 * 32; q += NVC_THREADS) {
-        const int row = q >> 5, c4 = q & 31;
-        if (v0 + row < nvec)
-          *reinterpret_cast<float4*>(corr_base + (int64_t)(v0 + row) * a.Nkp + 4 * c4) =
-              *reinterpret_cast<const float4*>(s_out + row * 132 + 4 * c4);
-      }
-    }
-    // TMEM, s_out and the A tiles are rewritten by the next chunk
+    // TMEM is rewritten by the next chunk
     tc_fence_before();
     __syncthreads();
-  }
-  // every MMA issued above has completed (each chunk waited for its commit)
-  if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem_slot, 128);
   }
+  // every MMA issued above has completed (each half waited for its commit)
+  if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
 }  // namespace sage
