@@ -5,9 +5,11 @@
 // microscaling with per-block mean smoothing).
 //
 //   nv_colsum_kernel     per (batch, head, token split) double-double column
-//                        sums of K (tokens < unpadded_k_len) or Q;
-//   nv_means_kernel      the K mean and the Q means (per 128-token block or
-//                        global), each rounded once to fp32;
+//                        sums of K (tokens < unpadded_k_len), and of Q when
+//                        one global Q mean is asked for;
+//   nv_means_kernel      the K mean and the global Q mean, each rounded once
+//                        to fp32 (a per-block Q mean is formed by the block's
+//                        quantiser CTA from the rows it has loaded);
 //   nv_quant_kernel      one CTA per 128-token block of Q, V or K: every
 //                        16-element vector gets sf = e4m3(fp32(amax/6)) and
 //                        codes e2m1(fp32(x * fp32(1/sf))), packed two per byte
@@ -151,9 +153,9 @@ __global__ void __launch_bounds__(QUANT_THREADS)
   }
 }
 
-// grid (B*Hkv + B*Hq*ceil(nqt/NVM_QBLOCKS)): the K mean of each KV head, then
-// the Q means of NVM_QBLOCKS consecutive 128-token blocks of one Q head per
-// CTA (the global mean, when asked for, is formed by each of the head's CTAs).
+// grid (B*Hkv [+ B*Hq*ceil(nqt/NVM_QBLOCKS) for a global Q mean]): the K mean
+// of each KV head, then the global Q mean written to NVM_QBLOCKS consecutive
+// 128-token blocks of one Q head per CTA (each of the head's CTAs forms it).
 constexpr int NVM_QBLOCKS = 8;
 template <int D>
 __global__ void __launch_bounds__(D) nv_means_kernel(NvQuantArgs a) {
@@ -174,21 +176,14 @@ __global__ void __launch_bounds__(D) nv_means_kernel(NvQuantArgs a) {
   id /= ngrp;
   const int qb0 = grp * NVM_QBLOCKS, qb1 = min(a.nqt, qb0 + NVM_QBLOCKS);
   float* qm = a.q_mean + (int64_t)id * a.nqt * D;
-  if (a.per_block_mean) {  // q splits are exactly the 128-token blocks
-    for (int qb = qb0; qb < qb1; ++qb) {
-      const int64_t o = ((int64_t)id * a.q_splits + qb) * D + c;
-      const int cnt = min(a.Nq, (qb + 1) * QB) - qb * QB;
-      qm[qb * D + c] = dd_mean_f32(DD{a.q_hi[o], a.q_lo[o]}, (double)cnt);
-    }
-  } else {
-    DD s = {0.0, 0.0};
-    for (int sp = 0; sp < a.q_splits; ++sp) {
-      const int64_t o = ((int64_t)id * a.q_splits + sp) * D + c;
-      dd_add(s, DD{a.q_hi[o], a.q_lo[o]});
-    }
-    const float m = dd_mean_f32(s, (double)a.Nq);
-    for (int qb = qb0; qb < qb1; ++qb) qm[qb * D + c] = m;
+  // the global Q mean (per-block means are formed by the quantiser CTAs)
+  DD s = {0.0, 0.0};
+  for (int sp = 0; sp < a.q_splits; ++sp) {
+    const int64_t o = ((int64_t)id * a.q_splits + sp) * D + c;
+    dd_add(s, DD{a.q_hi[o], a.q_lo[o]});
   }
+  const float m = dd_mean_f32(s, (double)a.Nq);
+  for (int qb = qb0; qb < qb1; ++qb) qm[qb * D + c] = m;
 }
 
 // ------------------------------------------------------------ block quantiser
@@ -208,6 +203,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
   __shared__ float s_m[D];
   __shared__ float s_km[D];
   __shared__ __align__(16) T s_v[QB][D + 8];
+  __shared__ DD s_dd[QUANT_THREADS / D][D];
   const int nQb = a.B * a.Hq * a.nqt;
   const int nKb = a.B * a.Hkv * a.nkt;
   int job = blockIdx.x;
@@ -226,9 +222,43 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
       raw[it][0] = n < a.Nq ? ldg16(p) : make_uint4(0, 0, 0, 0);
       raw[it][1] = n < a.Nq ? ldg16(p + 8 * sizeof(T)) : make_uint4(0, 0, 0, 0);
     }
-    for (int c = threadIdx.x; c < D; c += blockDim.x) {
-      s_m[c] = a.q_mean[((int64_t)bh * a.nqt + qt) * D + c];
-      s_km[c] = a.k_mean[((int64_t)b * a.Hkv + g) * D + c];
+    for (int c = threadIdx.x; c < D; c += blockDim.x) s_km[c] = a.k_mean[((int64_t)b * a.Hkv + g) * D + c];
+    if (a.per_block_mean) {
+      // the block's mean, from the rows already loaded: staged in shared
+      // memory, double-double column sums of the valid rows (TPC threads
+      // per channel, combined in a fixed order), rounded once to fp32
+      constexpr int TPC = QUANT_THREADS / D;
+      constexpr int RPT = QB / TPC;
+#pragma unroll
+      for (int it = 0; it < ITERS; ++it) {
+        *reinterpret_cast<uint4*>(&s_v[rs + it * RPP][vi * 16]) = raw[it][0];
+        *reinterpret_cast<uint4*>(&s_v[rs + it * RPP][vi * 16 + 8]) = raw[it][1];
+      }
+      __syncthreads();
+      const int c = threadIdx.x % D, part = threadIdx.x / D;
+      const int cnt = min(a.Nq, (qt + 1) * QB) - qt * QB;
+      // four interleaved accumulators (shorter dependency chains), combined in order
+      DD acc[4] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
+      const int r1 = min(cnt, (part + 1) * RPT);
+      for (int r = part * RPT; r < r1; r += 4)
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (r + u < r1) dd_add(acc[u], (double)to_f32<T>(s_v[r + u][c]));
+      dd_add(acc[0], acc[1]);
+      dd_add(acc[2], acc[3]);
+      dd_add(acc[0], acc[2]);
+      s_dd[part][c] = acc[0];
+      __syncthreads();
+      if (threadIdx.x < D) {
+        DD sum = s_dd[0][c];
+#pragma unroll
+        for (int pp = 1; pp < TPC; ++pp) dd_add(sum, s_dd[pp][c]);
+        const float m = dd_mean_f32(sum, (double)cnt);
+        s_m[c] = m;
+        a.q_mean[((int64_t)bh * a.nqt + qt) * D + c] = m;
+      }
+    } else {
+      for (int c = threadIdx.x; c < D; c += blockDim.x) s_m[c] = a.q_mean[((int64_t)bh * a.nqt + qt) * D + c];
     }
     __syncthreads();
 #pragma unroll

@@ -459,11 +459,12 @@ sage_status run_quantize_nvfp4(const sage_tensor* q, const sage_tensor* k, const
     nv_colsum_kernel<T, D><<<gk, QUANT_THREADS, 0, stream>>>(a.k, a.k_sb, a.k_sh, a.k_sn, a.Hkv, \
                                                              a.L, a.k_splits, a.k_split_tokens,  \
                                                              a.k_hi, a.k_lo);                    \
-    nv_colsum_kernel<T, D><<<gq, QUANT_THREADS, 0, stream>>>(a.q, a.q_sb, a.q_sh, a.q_sn, a.Hq,  \
-                                                             a.Nq, a.q_splits, a.q_split_tokens, \
-                                                             a.q_hi, a.q_lo);                    \
-    nv_means_kernel<D><<<a.B * a.Hkv + a.B * a.Hq * ((a.nqt + NVM_QBLOCKS - 1) / NVM_QBLOCKS), D, \
-                         0, stream>>>(a);                                                        \
+    if (!a.per_block_mean)                                                                       \
+      nv_colsum_kernel<T, D><<<gq, QUANT_THREADS, 0, stream>>>(a.q, a.q_sb, a.q_sh, a.q_sn, a.Hq, \
+                                                               a.Nq, a.q_splits, a.q_split_tokens, \
+                                                               a.q_hi, a.q_lo);                  \
+    nv_means_kernel<D><<<a.B * a.Hkv + (a.per_block_mean ? 0 : a.B * a.Hq * ((a.nqt + NVM_QBLOCKS - 1) / NVM_QBLOCKS)), \
+                         D, 0, stream>>>(a);                                                     \
     nv_quant_kernel<T, D><<<nblocks, QUANT_THREADS, 0, stream>>>(a);                             \
     if (!ensure_smem(nv_corr_kernel<T, D>, corr_smem, &corr_smem_flag<T, D>()))                  \
       return SAGE_ERR_CUDA;                                                                      \
