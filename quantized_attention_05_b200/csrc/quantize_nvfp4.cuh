@@ -200,8 +200,10 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
   constexpr int VPR = D / 16;                 // vectors per row
   constexpr int RPP = QUANT_THREADS / VPR;    // rows per pass
   constexpr int ITERS = QB / RPP;
-  __shared__ float s_m[D];
-  __shared__ float s_km[D];
+  // the means, one padding word per 16 channels: the eight threads of a row
+  // read channels vi*16 + i in eight different banks
+  __shared__ float s_m[D + D / 16];
+  __shared__ float s_km[D + D / 16];
   __shared__ __align__(16) T s_v[QB][D + 8];
   __shared__ DD s_dd[QUANT_THREADS / D][D];
   const int nQb = a.B * a.Hq * a.nqt;
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
       raw[it][0] = n < a.Nq ? ldg16(p) : make_uint4(0, 0, 0, 0);
       raw[it][1] = n < a.Nq ? ldg16(p + 8 * sizeof(T)) : make_uint4(0, 0, 0, 0);
     }
-    for (int c = threadIdx.x; c < D; c += blockDim.x) s_km[c] = a.k_mean[((int64_t)b * a.Hkv + g) * D + c];
+    for (int c = threadIdx.x; c < D; c += blockDim.x) s_km[c + (c >> 4)] = a.k_mean[((int64_t)b * a.Hkv + g) * D + c];
     if (a.per_block_mean) {
       // the block's mean, from the rows already loaded: staged in shared
       // memory, double-double column sums of the valid rows (TPC threads
@@ -254,11 +256,11 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
 #pragma unroll
         for (int pp = 1; pp < TPC; ++pp) dd_add(sum, s_dd[pp][c]);
         const float m = dd_mean_f32(sum, (double)cnt);
-        s_m[c] = m;
+        s_m[c + (c >> 4)] = m;
         a.q_mean[((int64_t)bh * a.nqt + qt) * D + c] = m;
       }
     } else {
-      for (int c = threadIdx.x; c < D; c += blockDim.x) s_m[c] = a.q_mean[((int64_t)bh * a.nqt + qt) * D + c];
+      for (int c = threadIdx.x; c < D; c += blockDim.x) s_m[c + (c >> 4)] = a.q_mean[((int64_t)bh * a.nqt + qt) * D + c];
     }
     __syncthreads();
 #pragma unroll
@@ -272,8 +274,8 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
         unpack8<T>(raw[it][1], f + 8);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          x[i] = __fsub_rn(f[i], s_m[vi * 16 + i]);
-          dq = fmaf(f[i], s_km[vi * 16 + i], dq);
+          x[i] = __fsub_rn(f[i], s_m[vi * 17 + i]);
+          dq = fmaf(f[i], s_km[vi * 17 + i], dq);
         }
       } else {
 #pragma unroll
@@ -307,7 +309,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
       raw[it][0] = n < a.L ? ldg16(p) : make_uint4(0, 0, 0, 0);
       raw[it][1] = n < a.L ? ldg16(p + 8 * sizeof(T)) : make_uint4(0, 0, 0, 0);
     }
-    for (int c = threadIdx.x; c < D; c += blockDim.x) s_km[c] = a.k_mean[(int64_t)bh * D + c];
+    for (int c = threadIdx.x; c < D; c += blockDim.x) s_km[c + (c >> 4)] = a.k_mean[(int64_t)bh * D + c];
     __syncthreads();
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
@@ -318,7 +320,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
         unpack8<T>(raw[it][0], f);
         unpack8<T>(raw[it][1], f + 8);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = __fsub_rn(f[i], s_km[vi * 16 + i]);
+        for (int i = 0; i < 16; ++i) x[i] = __fsub_rn(f[i], s_km[vi * 17 + i]);
       } else {
 #pragma unroll
         for (int i = 0; i < 16; ++i) x[i] = 0.f;
@@ -396,16 +398,17 @@ __device__ __forceinline__ void nvc_put(uint8_t* tile, int r, int c, const uint4
 }
 
 // bf16 hi / lo parts of 8 floats, two per word (lower channel in the low half).
-// x - hi is exact in fp32, so lo = bf16(x - hi) is x's next 8 bits.
+// x - hi is exact in fp32, so lo = bf16(x - hi) is x's next 8 bits.  Pairs
+// are converted by one packed round-to-nearest conversion each.
 __device__ __forceinline__ void nvc_split8(const float* x, uint4& hi, uint4& lo) {
   uint32_t h[4], l[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * i]), h1 = __float2bfloat16_rn(x[2 * i + 1]);
-    const __nv_bfloat16 l0 = __float2bfloat16_rn(__fsub_rn(x[2 * i], __bfloat162float(h0)));
-    const __nv_bfloat16 l1 = __float2bfloat16_rn(__fsub_rn(x[2 * i + 1], __bfloat162float(h1)));
-    h[i] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-    l[i] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+    const __nv_bfloat162 hp = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    const float2 hf = __bfloat1622float2(hp);
+    const __nv_bfloat162 lp = __floats2bfloat162_rn(__fsub_rn(x[2 * i], hf.x), __fsub_rn(x[2 * i + 1], hf.y));
+    h[i] = *reinterpret_cast<const uint32_t*>(&hp);
+    l[i] = *reinterpret_cast<const uint32_t*>(&lp);
   }
   hi = make_uint4(h[0], h[1], h[2], h[3]);
   lo = make_uint4(l[0], l[1], l[2], l[3]);
@@ -418,12 +421,12 @@ __global__ void __launch_bounds__(NVC_THREADS, 3) nv_corr_kernel(NvQuantArgs a) 
   uint8_t* sm = nvc_raw + ((1024u - (smem_u32(nvc_raw) & 1023u)) & 1023u);
   __shared__ uint64_t mma_bar;
   __shared__ uint32_t tmem_slot;
-  __shared__ float s_km[D];
+  __shared__ float s_km[D + D / 8];   // one padding word per 8 channels (no bank conflicts)
   const int kt = blockIdx.x, bg = blockIdx.y;
   const int b = bg / a.Hkv, g = bg % a.Hkv;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   constexpr int PER = 128 * 8 / NVC_THREADS;   // 16-byte chunks per thread per operand half
-  for (int c = t; c < D; c += NVC_THREADS) s_km[c] = a.k_mean[(int64_t)bg * D + c];
+  for (int c = t; c < D; c += NVC_THREADS) s_km[c + (c >> 3)] = a.k_mean[(int64_t)bg * D + c];
   if (t == 0) {
     mbar_init(&mma_bar, 1);
     fence_mbar_init();
@@ -470,7 +473,7 @@ __global__ void __launch_bounds__(NVC_THREADS, 3) nv_corr_kernel(NvQuantArgs a) 
         float f[8];
         unpack8<T>(kraw[i], f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = live ? __fsub_rn(f[e], s_km[hf * 64 + c * 8 + e]) : 0.f;
+        for (int e = 0; e < 8; ++e) f[e] = live ? __fsub_rn(f[e], s_km[hf * 72 + c * 9 + e]) : 0.f;
         uint4 hi, lo;
         nvc_split8(f, hi, lo);
         nvc_put(sm + L::OFF_AHI, row, c, hi);
