@@ -383,7 +383,8 @@ sage_status sage_lse_merge_finalize(const float* acc, void* out, int32_t out_dty
                                     int64_t D, sage_stream_t stream);
 
 /* ------------------------------------------------------------------ NVFP4 */
-/* Workspace bytes of sage_quantize_qkv_nvfp4 (per-split K and Q sums). */
+/* Workspace bytes of sage_quantize_qkv_nvfp4 (per-split K and Q sums, and the
+ * Q means split into bf16 hi and lo parts for the correction MMA). */
 size_t sage_quantize_nvfp4_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
                                            int64_t Nk, int64_t D);
 

@@ -47,6 +47,8 @@ struct NvQuantArgs {
   uint8_t* v_sf_t;
   float* corr;
   float* q_mean;              // [B*Hq, nqt, D]
+  uint16_t* qm_bhi;           // [B*Hq, nqt, D] bf16 bits: q_mean = hi + lo (+ 2^-18 relative)
+  uint16_t* qm_blo;
   float* k_mean;              // [B*Hkv, D]
   float* qdk;                 // may be null
 };
@@ -97,6 +99,14 @@ __device__ __forceinline__ uint32_t nvfp4_vector(const float* x, uint32_t* w0, u
     *w1 = 0u;
   }
   return sf;
+}
+
+// bf16 hi / lo parts of x (round to nearest): x - hi is exact in fp32 and lo
+// = bf16(x - hi) holds its next 8 bits, |x - hi - lo| <= 2^-18 |x|.
+__device__ __forceinline__ void bf16_split(float x, uint16_t& hi, uint16_t& lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  hi = __bfloat16_as_ushort(h);
+  lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fsub_rn(x, __bfloat162float(h))));
 }
 
 // ------------------------------------------------------------ column sums
@@ -183,7 +193,13 @@ __global__ void __launch_bounds__(D) nv_means_kernel(NvQuantArgs a) {
     dd_add(s, DD{a.q_hi[o], a.q_lo[o]});
   }
   const float m = dd_mean_f32(s, (double)a.Nq);
-  for (int qb = qb0; qb < qb1; ++qb) qm[qb * D + c] = m;
+  uint16_t mh, ml;
+  bf16_split(m, mh, ml);
+  for (int qb = qb0; qb < qb1; ++qb) {
+    qm[qb * D + c] = m;
+    a.qm_bhi[((int64_t)id * a.nqt + qb) * D + c] = mh;
+    a.qm_blo[((int64_t)id * a.nqt + qb) * D + c] = ml;
+  }
 }
 
 // ------------------------------------------------------------ block quantiser
@@ -257,7 +273,12 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
         for (int pp = 1; pp < TPC; ++pp) dd_add(sum, s_dd[pp][c]);
         const float m = dd_mean_f32(sum, (double)cnt);
         s_m[c + (c >> 4)] = m;
-        a.q_mean[((int64_t)bh * a.nqt + qt) * D + c] = m;
+        const int64_t o = ((int64_t)bh * a.nqt + qt) * D + c;
+        a.q_mean[o] = m;
+        uint16_t mh, ml;
+        bf16_split(m, mh, ml);
+        a.qm_bhi[o] = mh;
+        a.qm_blo[o] = ml;
       }
     } else {
       for (int c = threadIdx.x; c < D; c += blockDim.x) s_m[c + (c >> 4)] = a.q_mean[((int64_t)bh * a.nqt + qt) * D + c];
@@ -375,8 +396,8 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
 // about 2^-16 per product (the fp32 reference sum rounds at 2^-24).
 // grid (nkt, B*Hkv), 256 threads, three CTAs per SM.  Per chunk of 128 Q-mean
 // vectors the D channels are taken 64 at a time: all threads stage that half
-// of the 128 keys (the MMA's M side) and of the 128 vectors (its N side) with
-// coalesced 16/32-byte loads, thread 0 issues the MMAs, and the next half
+// of the 128 keys (the MMA's M side, split here) and of the 128 vectors (its N
+// side, split once where the means are formed) with coalesced 16-byte loads, thread 0 issues the MMAs, and the next half
 // overwrites the tiles once they have completed.  The scores land in TMEM as
 // [key][vector], so for each vector the 32 lanes of a warp store 32
 // consecutive keys: every store instruction writes 128 contiguous bytes of a
@@ -442,7 +463,8 @@ __global__ void __launch_bounds__(NVC_THREADS, 3) nv_corr_kernel(NvQuantArgs a) 
   // the Q means of a chunk are 128 consecutive rows of q_mean: vector v of
   // KV head g is row (b*Hq + g*G)*nqt + v
   const int nvec = a.G * a.nqt;
-  const float* qm_base = a.q_mean + ((int64_t)b * a.Hq + (int64_t)g * a.G) * a.nqt * D;
+  const uint16_t* qmh_base = a.qm_bhi + ((int64_t)b * a.Hq + (int64_t)g * a.G) * a.nqt * D;
+  const uint16_t* qml_base = a.qm_blo + ((int64_t)b * a.Hq + (int64_t)g * a.G) * a.nqt * D;
   float* corr_base = a.corr + ((int64_t)b * a.Hq + (int64_t)g * a.G) * a.nqt * a.Nkp + kt * 128;
   const char* kbase = reinterpret_cast<const char*>(a.k) + (b * a.k_sb + g * a.k_sh) * (int64_t)sizeof(T);
   uint32_t phase = 0;
@@ -451,8 +473,7 @@ __global__ void __launch_bounds__(NVC_THREADS, 3) nv_corr_kernel(NvQuantArgs a) 
     for (int hf = 0; ok && hf < D / 64; ++hf) {
       // chunk q = t + 256 i: channels hf*64 + 8*(q % 8) .. of row q / 8;
       // every load is in flight before the first use
-      uint4 kraw[PER];
-      float4 qraw[2 * PER];
+      uint4 kraw[PER], qh[PER], ql[PER];
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
         const int q = t + NVC_THREADS * i, row = q >> 3, c = q & 7;
@@ -460,10 +481,9 @@ __global__ void __launch_bounds__(NVC_THREADS, 3) nv_corr_kernel(NvQuantArgs a) 
         kraw[i] = n < a.L ? ldg16(kbase + ((int64_t)n * a.k_sn + hf * 64 + c * 8) * (int64_t)sizeof(T))
                           : make_uint4(0, 0, 0, 0);
         const bool live = v0 + row < nvec;
-        const float4* src =
-            reinterpret_cast<const float4*>(qm_base + (int64_t)(v0 + row) * D + hf * 64 + c * 8);
-        qraw[2 * i] = live ? __ldg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
-        qraw[2 * i + 1] = live ? __ldg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int64_t o = (int64_t)(v0 + row) * D + hf * 64 + c * 8;
+        qh[i] = live ? ldg16(qmh_base + o) : make_uint4(0, 0, 0, 0);
+        ql[i] = live ? ldg16(qml_base + o) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
@@ -478,12 +498,9 @@ __global__ void __launch_bounds__(NVC_THREADS, 3) nv_corr_kernel(NvQuantArgs a) 
         nvc_split8(f, hi, lo);
         nvc_put(sm + L::OFF_AHI, row, c, hi);
         nvc_put(sm + L::OFF_ALO, row, c, lo);
-        // B: the Q means
-        const float qf[8] = {qraw[2 * i].x, qraw[2 * i].y, qraw[2 * i].z, qraw[2 * i].w,
-                             qraw[2 * i + 1].x, qraw[2 * i + 1].y, qraw[2 * i + 1].z, qraw[2 * i + 1].w};
-        nvc_split8(qf, hi, lo);
-        nvc_put(sm + L::OFF_BHI, row, c, hi);
-        nvc_put(sm + L::OFF_BLO, row, c, lo);
+        // B: the Q means, split where they were formed
+        nvc_put(sm + L::OFF_BHI, row, c, qh[i]);
+        nvc_put(sm + L::OFF_BLO, row, c, ql[i]);
       }
       fence_proxy_async_smem();
       tc_fence_before();

@@ -360,7 +360,7 @@ sage_status run_attention(const sage_qkv_i8f8* z, int causal, float sm_scale, in
 // ---------------------------------------------------------------- NVFP4 quantise
 struct NvPlan {
   QuantPlan k, q;
-  size_t k_bytes, q_bytes, total;
+  size_t k_bytes, q_bytes, qm_bytes, total;
 };
 NvPlan nv_plan(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64_t D) {
   NvPlan p;
@@ -372,7 +372,9 @@ NvPlan nv_plan(int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq, int64_t Nk, int64
   const int64_t qs = std::max<int64_t>(p.q.splits, nqt);
   p.k_bytes = 2 * align256((size_t)B * Hkv * p.k.splits * D * 8);
   p.q_bytes = 2 * align256((size_t)B * Hq * qs * D * 8);
-  p.total = p.k_bytes + p.q_bytes;
+  // the Q means as bf16 hi and lo parts, the correction MMA's B operand
+  p.qm_bytes = 2 * align256((size_t)B * Hq * nqt * D * 2);
+  p.total = p.k_bytes + p.q_bytes + p.qm_bytes;
   return p;
 }
 
@@ -446,6 +448,9 @@ sage_status run_quantize_nvfp4(const sage_tensor* q, const sage_tensor* k, const
   a.k_lo = reinterpret_cast<double*>(w + align256(kn * 8));
   a.q_hi = reinterpret_cast<double*>(w + plan.k_bytes);
   a.q_lo = reinterpret_cast<double*>(w + plan.k_bytes + align256(qn * 8));
+  const size_t qmn = (size_t)a.B * a.Hq * a.nqt * q->D;
+  a.qm_bhi = reinterpret_cast<uint16_t*>(w + plan.k_bytes + plan.q_bytes);
+  a.qm_blo = reinterpret_cast<uint16_t*>(w + plan.k_bytes + plan.q_bytes + align256(qmn * 2));
   a.q4 = out->q; a.q_sf = out->q_sf; a.k4 = out->k; a.k_sf = out->k_sf;
   a.v4t = out->v_t; a.v_sf_t = out->v_sf_t; a.corr = out->qk_correction;
   a.q_mean = out->q_mean; a.k_mean = out->k_mean; a.qdk = out->q_dot_kmean;
