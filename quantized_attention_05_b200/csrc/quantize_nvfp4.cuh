@@ -396,12 +396,13 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
 // about 2^-16 per product (the fp32 reference sum rounds at 2^-24).
 // grid (nkt, B*Hkv), 256 threads, three CTAs per SM.  Per chunk of 128 Q-mean
 // vectors the D channels are taken 64 at a time: all threads stage that half
-// of the 128 keys (the MMA's M side, split here) and of the 128 vectors (its N
-// side, split once where the means are formed) with coalesced 16-byte loads, thread 0 issues the MMAs, and the next half
-// overwrites the tiles once they have completed.  The scores land in TMEM as
-// [key][vector], so for each vector the 32 lanes of a warp store 32
-// consecutive keys: every store instruction writes 128 contiguous bytes of a
-// correction row, with no staging.
+// of the 128 keys (the MMA's M side, split here; the next half's rows are
+// loaded while the MMAs of this one run) and of the 128 vectors (its N side,
+// split once where the means are formed, copied by cp.async); thread 0
+// issues the MMAs, and the next half overwrites the tiles once they have
+// completed.  The scores land in TMEM as [key][vector], so for each vector
+// the 32 lanes of a warp store 32 consecutive keys: every store instruction
+// writes 128 contiguous bytes of a correction row, with no staging.
 // Shared memory: A_hi, A_lo (128 keys x 64 channels), B_hi, B_lo (128
 // vectors x 64 channels), bf16, K-major with the 128-byte swizzle: row r at
 // r * 128, 16-byte chunk c at (c ^ (r % 8)) * 16.
@@ -433,6 +434,16 @@ __device__ __forceinline__ void nvc_split8(const float* x, uint4& hi, uint4& lo)
   }
   hi = make_uint4(h[0], h[1], h[2], h[3]);
   lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// 16-byte asynchronous copy global -> shared (L1 bypassed), and the wait
+// for all of this thread's outstanding copies.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 template <typename T, int D>
@@ -469,26 +480,41 @@ __global__ void __launch_bounds__(NVC_THREADS, 3) nv_corr_kernel(NvQuantArgs a) 
   const char* kbase = reinterpret_cast<const char*>(a.k) + (b * a.k_sb + g * a.k_sh) * (int64_t)sizeof(T);
   uint32_t phase = 0;
   bool ok = true;
+  // K rows of one 64-channel half: chunk q = t + 256 i is channels
+  // hf*64 + 8*(q % 8) .. of key q / 8
+  uint4 kraw[PER];
+  auto load_k = [&](int hf) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int q = t + NVC_THREADS * i, row = q >> 3, c = q & 7;
+      const int n = kt * 128 + row;
+      kraw[i] = n < a.L ? ldg16(kbase + ((int64_t)n * a.k_sn + hf * 64 + c * 8) * (int64_t)sizeof(T))
+                        : make_uint4(0, 0, 0, 0);
+    }
+  };
   for (int v0 = 0; ok && v0 < nvec; v0 += 128) {
+    load_k(0);
     for (int hf = 0; ok && hf < D / 64; ++hf) {
-      // chunk q = t + 256 i: channels hf*64 + 8*(q % 8) .. of row q / 8;
-      // every load is in flight before the first use
-      uint4 kraw[PER], qh[PER], ql[PER];
+      // B: the Q means' hi and lo parts (split where the means were formed),
+      // copied straight into the swizzled tiles; zero rows past nvec
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
         const int q = t + NVC_THREADS * i, row = q >> 3, c = q & 7;
-        const int n = kt * 128 + row;
-        kraw[i] = n < a.L ? ldg16(kbase + ((int64_t)n * a.k_sn + hf * 64 + c * 8) * (int64_t)sizeof(T))
-                          : make_uint4(0, 0, 0, 0);
-        const bool live = v0 + row < nvec;
-        const int64_t o = (int64_t)(v0 + row) * D + hf * 64 + c * 8;
-        qh[i] = live ? ldg16(qmh_base + o) : make_uint4(0, 0, 0, 0);
-        ql[i] = live ? ldg16(qml_base + o) : make_uint4(0, 0, 0, 0);
+        uint8_t* dh = sm + L::OFF_BHI + row * 128 + ((c ^ (row & 7)) << 4);
+        uint8_t* dl = sm + L::OFF_BLO + row * 128 + ((c ^ (row & 7)) << 4);
+        if (v0 + row < nvec) {
+          const int64_t o = (int64_t)(v0 + row) * D + hf * 64 + c * 8;
+          cp_async16(dh, qmh_base + o);
+          cp_async16(dl, qml_base + o);
+        } else {
+          *reinterpret_cast<uint4*>(dh) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(dl) = make_uint4(0, 0, 0, 0);
+        }
       }
+      // A: Ks = fp32(K - kmean) for keys < L, 0 beyond, split into hi + lo
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
         const int q = t + NVC_THREADS * i, row = q >> 3, c = q & 7;
-        // A: Ks = fp32(K - kmean) for keys < L, 0 beyond
         const bool live = kt * 128 + row < a.L;
         float f[8];
         unpack8<T>(kraw[i], f);
@@ -498,10 +524,8 @@ __global__ void __launch_bounds__(NVC_THREADS, 3) nv_corr_kernel(NvQuantArgs a) 
         nvc_split8(f, hi, lo);
         nvc_put(sm + L::OFF_AHI, row, c, hi);
         nvc_put(sm + L::OFF_ALO, row, c, lo);
-        // B: the Q means, split where they were formed
-        nvc_put(sm + L::OFF_BHI, row, c, qh[i]);
-        nvc_put(sm + L::OFF_BLO, row, c, ql[i]);
       }
+      cp_async_wait_all();
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
@@ -520,6 +544,8 @@ __global__ void __launch_bounds__(NVC_THREADS, 3) nv_corr_kernel(NvQuantArgs a) 
         tc_commit(&mma_bar);
       }
       __syncwarp();
+      // the next half's K rows are in flight while these MMAs run
+      if (hf + 1 < D / 64) load_k(hf + 1);
       // the tiles are rewritten by the next half only after the MMAs are done
       ok = __all_sync(0xffffffffu, mbar_wait(&mma_bar, phase & 1, SITE_MMA_DONE));
       ++phase;
