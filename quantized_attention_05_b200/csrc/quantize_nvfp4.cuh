@@ -109,6 +109,16 @@ __device__ __forceinline__ void bf16_split(float x, uint16_t& hi, uint16_t& lo) 
   lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fsub_rn(x, __bfloat162float(h))));
 }
 
+// 16-byte asynchronous copy global -> shared (L1 bypassed), and the wait
+// for all of this thread's outstanding copies.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // ------------------------------------------------------------ column sums
 // grid (splits, B*H), 256 threads: per split of tokens [s*T, min(limit,(s+1)*T)),
 // double-double sums of every channel.
@@ -204,18 +214,19 @@ __global__ void __launch_bounds__(D) nv_means_kernel(NvQuantArgs a) {
 
 // ------------------------------------------------------------ block quantiser
 // One CTA per 128-token block: first the Q blocks, heads in descending order
-// (the Q column sums read the heads in ascending order just before, so the
-// rows they read last are still in L2), then the V blocks, then the K blocks
-// in descending head order (so that the correction kernel, which starts at
-// head 0, finds the K rows read last in L2).
-// Q/K: D/16 threads per row, one 16-element vector each, the block's four
-// rows per thread loaded before any of them is used.  V: the block is staged
-// in shared memory and every thread quantises 16-token vectors of one channel.
+// (the Q column sums, when there are any, read the heads in ascending order
+// just before), then the V blocks, then the K blocks in descending head order
+// (so that the correction kernel, which starts at head 0, finds the K rows
+// read last in L2).  The block is copied into shared memory by cp.async (no
+// registers hold it in flight, so more CTAs fit per SM).  Q/K: D/16 threads
+// per row, one 16-element vector each.  V: every thread quantises 16-token
+// vectors of one channel.
 template <typename T, int D>
 __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) {
   constexpr int VPR = D / 16;                 // vectors per row
   constexpr int RPP = QUANT_THREADS / VPR;    // rows per pass
   constexpr int ITERS = QB / RPP;
+  constexpr int CPR = D / 8;                  // 16-byte chunks per row
   // the means, one padding word per 16 channels: the eight threads of a row
   // read channels vi*16 + i in eight different banks
   __shared__ float s_m[D + D / 16];
@@ -226,33 +237,38 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
   const int nKb = a.B * a.Hkv * a.nkt;
   int job = blockIdx.x;
   const int vi = threadIdx.x % VPR, rs = threadIdx.x / VPR;
+  // rows row0 .. row0+127 of one head into s_v (rows at and past `limit`
+  // become zero); coalesced: consecutive threads copy consecutive 16 bytes
+  auto stage = [&](const void* src, int64_t sb, int64_t sh, int64_t sn, int b, int h, int row0,
+                   int limit) {
+    const char* base = reinterpret_cast<const char*>(src) + (b * sb + h * sh) * (int64_t)sizeof(T);
+    for (int q = threadIdx.x; q < QB * CPR; q += QUANT_THREADS) {
+      const int r = q / CPR, c = q % CPR;
+      T* dst = &s_v[r][c * 8];
+      if (row0 + r < limit)
+        cp_async16(dst, base + ((int64_t)(row0 + r) * sn + c * 8) * (int64_t)sizeof(T));
+      else
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    }
+    cp_async_wait_all();
+  };
+  // the thread's 16 elements of block row r
+  auto row16 = [&](int r, float* f) {
+    unpack8<T>(*reinterpret_cast<const uint4*>(&s_v[r][vi * 16]), f);
+    unpack8<T>(*reinterpret_cast<const uint4*>(&s_v[r][vi * 16 + 8]), f + 8);
+  };
 
   if (job < nQb) {
     const int bh = a.B * a.Hq - 1 - job / a.nqt, qt = job % a.nqt;
     const int b = bh / a.Hq, h = bh % a.Hq, g = h / a.G;
-    const char* base = reinterpret_cast<const char*>(a.q) +
-                       (b * a.q_sb + h * a.q_sh + vi * 16) * (int64_t)sizeof(T);
-    uint4 raw[ITERS][2];
-#pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-      const int n = qt * QB + rs + it * RPP;
-      const char* p = base + (int64_t)n * a.q_sn * sizeof(T);
-      raw[it][0] = n < a.Nq ? ldg16(p) : make_uint4(0, 0, 0, 0);
-      raw[it][1] = n < a.Nq ? ldg16(p + 8 * sizeof(T)) : make_uint4(0, 0, 0, 0);
-    }
+    stage(a.q, a.q_sb, a.q_sh, a.q_sn, b, h, qt * QB, a.Nq);
     for (int c = threadIdx.x; c < D; c += blockDim.x) s_km[c + (c >> 4)] = a.k_mean[((int64_t)b * a.Hkv + g) * D + c];
+    __syncthreads();
     if (a.per_block_mean) {
-      // the block's mean, from the rows already loaded: staged in shared
-      // memory, double-double column sums of the valid rows (TPC threads
-      // per channel, combined in a fixed order), rounded once to fp32
+      // the block's mean: double-double column sums of the valid rows (TPC
+      // threads per channel, combined in a fixed order), rounded once to fp32
       constexpr int TPC = QUANT_THREADS / D;
       constexpr int RPT = QB / TPC;
-#pragma unroll
-      for (int it = 0; it < ITERS; ++it) {
-        *reinterpret_cast<uint4*>(&s_v[rs + it * RPP][vi * 16]) = raw[it][0];
-        *reinterpret_cast<uint4*>(&s_v[rs + it * RPP][vi * 16 + 8]) = raw[it][1];
-      }
-      __syncthreads();
       const int c = threadIdx.x % D, part = threadIdx.x / D;
       const int cnt = min(a.Nq, (qt + 1) * QB) - qt * QB;
       // four interleaved accumulators (shorter dependency chains), combined in order
@@ -286,13 +302,12 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
     __syncthreads();
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
-      const int n = qt * QB + rs + it * RPP;
+      const int r = rs + it * RPP, n = qt * QB + r;
       float x[16];
       float dq = 0.f;
       if (n < a.Nq) {
         float f[16];
-        unpack8<T>(raw[it][0], f);
-        unpack8<T>(raw[it][1], f + 8);
+        row16(r, f);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           x[i] = __fsub_rn(f[i], s_m[vi * 17 + i]);
@@ -320,26 +335,16 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
     job -= nKb;
     const int bh = a.B * a.Hkv - 1 - job / a.nkt, kt = job % a.nkt;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
-    const char* base = reinterpret_cast<const char*>(a.k) +
-                       (b * a.k_sb + h * a.k_sh + vi * 16) * (int64_t)sizeof(T);
-    uint4 raw[ITERS][2];
-#pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-      const int n = kt * QB + rs + it * RPP;
-      const char* p = base + (int64_t)n * a.k_sn * sizeof(T);
-      raw[it][0] = n < a.L ? ldg16(p) : make_uint4(0, 0, 0, 0);
-      raw[it][1] = n < a.L ? ldg16(p + 8 * sizeof(T)) : make_uint4(0, 0, 0, 0);
-    }
+    stage(a.k, a.k_sb, a.k_sh, a.k_sn, b, h, kt * QB, a.L);
     for (int c = threadIdx.x; c < D; c += blockDim.x) s_km[c + (c >> 4)] = a.k_mean[(int64_t)bh * D + c];
     __syncthreads();
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
-      const int n = kt * QB + rs + it * RPP;
+      const int r = rs + it * RPP, n = kt * QB + r;
       float x[16];
       if (n < a.L) {
         float f[16];
-        unpack8<T>(raw[it][0], f);
-        unpack8<T>(raw[it][1], f + 8);
+        row16(r, f);
 #pragma unroll
         for (int i = 0; i < 16; ++i) x[i] = __fsub_rn(f[i], s_km[vi * 17 + i]);
       } else {
@@ -357,20 +362,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
   {
     const int bh = job / a.nkt, vt = job % a.nkt;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
-    constexpr int TPR = D / 8;
-    constexpr int VR = QB / (QUANT_THREADS / TPR);   // staged rows per thread
-    const int cg = threadIdx.x % TPR, rr = threadIdx.x / TPR;
-    const char* base = reinterpret_cast<const char*>(a.v) +
-                       (b * a.v_sb + h * a.v_sh + cg * 8) * (int64_t)sizeof(T);
-    uint4 raw[VR];
-#pragma unroll
-    for (int i = 0; i < VR; ++i) {
-      const int n = vt * QB + rr + i * (QUANT_THREADS / TPR);
-      raw[i] = n < a.L ? ldg16(base + (int64_t)n * a.v_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int i = 0; i < VR; ++i)
-      *reinterpret_cast<uint4*>(&s_v[rr + i * (QUANT_THREADS / TPR)][cg * 8]) = raw[i];
+    stage(a.v, a.v_sb, a.v_sh, a.v_sn, b, h, vt * QB, a.L);
     __syncthreads();
     // vector (channel c, 16-token group gq): threads cover channels fastest
     for (int idx = threadIdx.x; idx < D * (QB / 16); idx += blockDim.x) {
@@ -434,16 +426,6 @@ __device__ __forceinline__ void nvc_split8(const float* x, uint4& hi, uint4& lo)
   }
   hi = make_uint4(h[0], h[1], h[2], h[3]);
   lo = make_uint4(l[0], l[1], l[2], l[3]);
-}
-
-// 16-byte asynchronous copy global -> shared (L1 bypassed), and the wait
-// for all of this thread's outstanding copies.
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 template <typename T, int D>
