@@ -63,20 +63,6 @@ struct NvAttnArgs {
   float sm_scale;
 };
 
-// x / 6 rounded to nearest even, for every fp32 x whose quotient is normal
-// (checked exhaustively against the IEEE division by tests/test_div6.py):
-// the product with RN(1/6), then one correction with the exact residual
-// fma(-q0, 6, x) -- Markstein's residual correction of a reciprocal product
-// (P. Markstein, "Computation of elementary functions on the IBM RISC
-// System/6000 processor", IBM J. Res. Dev. 34(1), 1990).  Smaller quotients can be one unit off, which no E4M3 code
-// sees (they are below half its smallest subnormal, 2^-10).
-__device__ __forceinline__ float div6_rn(float x) {
-  const float c = 0.16666667f;   // RN(1/6) = 0x1.555556p-3
-  const float q0 = __fmul_rn(x, c);
-  const float r = __fmaf_rn(-q0, 6.f, x);
-  return __fmaf_rn(r, c, q0);
-}
-
 template <int D>
 struct NvLayout {
   static constexpr int ROWB = D / 2;            // bytes per packed Q/K row
@@ -298,10 +284,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ float s_inv[256];   // 1 / value(E4M3 code), 0 for code 0
   __shared__ float s_one[D];     // unit value scales of the shared epilogue
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) {
-    const float v = i < 128 ? e4m3_value((uint32_t)i) : 0.f;
-    s_inv[i] = v > 0.f ? __frcp_rn(v) : 0.f;
-  }
+  fill_e4m3_inverse(s_inv);
   for (int i = threadIdx.x; i < D; i += blockDim.x) s_one[i] = 1.f;
   // work: (b, h, pair of Q tiles); causal -> longest rows first
   int b, h, qp;

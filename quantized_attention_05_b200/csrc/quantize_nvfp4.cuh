@@ -79,16 +79,41 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
+// x / 6 rounded to nearest even, for every fp32 x whose quotient is normal
+// (checked exhaustively against the IEEE division by tests/test_div6.py):
+// the product with RN(1/6), then one correction with the exact residual
+// fma(-q0, 6, x) -- Markstein's residual correction of a reciprocal product
+// (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Dev. 34(1), 1990).  Smaller quotients can be one unit off, which no E4M3 code
+// sees (they are below half its smallest subnormal, 2^-10).
+__device__ __forceinline__ float div6_rn(float x) {
+  const float c = 0.16666667f;   // RN(1/6) = 0x1.555556p-3
+  const float q0 = __fmul_rn(x, c);
+  const float r = __fmaf_rn(-q0, 6.f, x);
+  return __fmaf_rn(r, c, q0);
+}
+
+// 1 / value(E4M3 code) for the 128 non-negative codes (0 for code 0), the
+// table nvfp4_vector reads; filled by a CTA's threads before first use.
+__device__ __forceinline__ void fill_e4m3_inverse(float* s_inv) {
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+    const float v = i < 128 ? e4m3_value((uint32_t)i) : 0.f;
+    s_inv[i] = v > 0.f ? __frcp_rn(v) : 0.f;
+  }
+}
+
 // NVFP4 quantisation of one 16-element vector: returns the scale-factor
-// code; writes the 8 packed bytes (two words) of codes.
-__device__ __forceinline__ uint32_t nvfp4_vector(const float* x, uint32_t* w0, uint32_t* w1) {
+// code; writes the 8 packed bytes (two words) of codes.  sf = e4m3(amax / 6)
+// with the quotient of div6_rn (the IEEE one wherever an E4M3 code can tell),
+// 1 / value(sf) from the table of fill_e4m3_inverse (the IEEE reciprocal).
+__device__ __forceinline__ uint32_t nvfp4_vector(const float* x, const float* s_inv, uint32_t* w0,
+                                                 uint32_t* w1) {
   float a = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
-  const uint32_t sf = e4m3_code(__fdiv_rn(a, 6.f));
-  const float s = e4m3_value(sf);
-  if (s > 0.f) {
-    const float inv = __frcp_rn(s);
+  const uint32_t sf = e4m3_code(div6_rn(a));
+  const float inv = s_inv[sf];
+  if (inv > 0.f) {
     float y[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(x[i], inv);
@@ -233,6 +258,8 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
   __shared__ float s_km[D + D / 16];
   __shared__ __align__(16) T s_v[QB][D + 8];
   __shared__ DD s_dd[QUANT_THREADS / D][D];
+  __shared__ float s_inv[256];
+  fill_e4m3_inverse(s_inv);   // ordered before its first use by the __syncthreads below
   const int nQb = a.B * a.Hq * a.nqt;
   const int nKb = a.B * a.Hkv * a.nkt;
   int job = blockIdx.x;
@@ -318,7 +345,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
         for (int i = 0; i < 16; ++i) x[i] = 0.f;
       }
       uint32_t w0, w1;
-      const uint32_t sf = nvfp4_vector(x, &w0, &w1);
+      const uint32_t sf = nvfp4_vector(x, s_inv, &w0, &w1);
       const int64_t row = (int64_t)bh * a.Nqp + n;
       *reinterpret_cast<uint2*>(a.q4 + row * (D / 2) + vi * 8) = make_uint2(w0, w1);
       a.q_sf[row * (D / 16) + vi] = (uint8_t)sf;
@@ -352,7 +379,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
         for (int i = 0; i < 16; ++i) x[i] = 0.f;
       }
       uint32_t w0, w1;
-      const uint32_t sf = nvfp4_vector(x, &w0, &w1);
+      const uint32_t sf = nvfp4_vector(x, s_inv, &w0, &w1);
       const int64_t row = (int64_t)bh * a.Nkp + n;
       *reinterpret_cast<uint2*>(a.k4 + row * (D / 2) + vi * 8) = make_uint2(w0, w1);
       a.k_sf[row * (D / 16) + vi] = (uint8_t)sf;
@@ -371,7 +398,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) nv_quant_kernel(NvQuantArgs a) 
 #pragma unroll
       for (int i = 0; i < 16; ++i) x[i] = to_f32<T>(s_v[gq * 16 + i][c]);
       uint32_t w0, w1;
-      const uint32_t sf = nvfp4_vector(x, &w0, &w1);
+      const uint32_t sf = nvfp4_vector(x, s_inv, &w0, &w1);
       const int64_t row = (int64_t)bh * D + c;
       *reinterpret_cast<uint2*>(a.v4t + row * (a.Nkp / 2) + vt * (QB / 2) + gq * 8) =
           make_uint2(w0, w1);

@@ -1,7 +1,8 @@
-"""The NVFP4 attention kernel forms each P' vector's scale code from
-amax / 6 with one multiply by RN(1/6) and one fma correction with the exact
-residual (div6_rn in attn_fwd_nvfp4.cuh; Markstein's residual correction of a
-reciprocal product, IBM J. Res. Dev. 34(1), 1990).  The scale codes must be those of
+"""The NVFP4 attention kernel (each P' vector's scale code) and the NVFP4
+quantiser (each Q/K/V vector's scale code) form amax / 6 with one multiply by
+RN(1/6) and one fma correction with the exact residual (div6_rn in
+quantize_nvfp4.cuh; Markstein's residual correction of a reciprocal product,
+IBM J. Res. Dev. 34(1), 1990).  The scale codes must be those of
 the IEEE-rounded quotient, so the identity is checked here for EVERY finite
 non-negative fp32 x whose quotient is normal (smaller quotients are below half
 the smallest E4M3 subnormal and give code 0 either way), with the C library's
