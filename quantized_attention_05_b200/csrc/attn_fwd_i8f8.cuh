@@ -126,8 +126,8 @@ struct AttnLayout {
   static constexpr int OFF_INIT = OFF_P + 4 * P_BYTES;   // f16 A (4 KB) and B (4 KB) of the S init
   static constexpr int OFF_BAR = OFF_INIT + 8192;
   // q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2][2],
-  // o_ready[2][2], mma_done
-  static constexpr int NBAR = 1 + 2 * ATT_STAGES + 2 + 2 + 4 + 4 + 1;
+  // o_ready[2][2], mma_done, wg0_started
+  static constexpr int NBAR = 1 + 2 * ATT_STAGES + 2 + 2 + 4 + 4 + 1 + 1;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_VS = (OFF_TMEM + 16 + 15) / 16 * 16;
   static constexpr int OFF_NLIST = OFF_VS + D * 4;
@@ -348,6 +348,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint64_t* p_full = s_free + 2;              // [wg * 2 + buffer]
   uint64_t* o_ready = p_full + 4;             // [wg * 2 + buffer]
   uint64_t* mma_done = o_ready + 4;
+  uint64_t* wg0_started = mma_done + 1;    // Q tile 0's first P tile is published
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   float* s_vs = reinterpret_cast<float*>(smem + L::OFF_VS);
   int* s_nlist = reinterpret_cast<int*>(smem + L::OFF_NLIST);
@@ -410,6 +411,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(&o_ready[i], 1);
     }
     mbar_init(mma_done, ATT_ISSUERS);
+    mbar_init(wg0_started, 128);
     fence_mbar_init();
   } else if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
@@ -552,10 +554,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // S starts free; each QK^T is preceded by an f16 MMA that sets S to
     // 1.5*2^23, so the int32 sum on top reads as the float 1.5*2^23 + S.
     mbar_arrive(&s_free[wg]);
+    // Q tile 1's warpgroup starts once Q tile 0's has published its first P
+    // tile (when it has one; a barrier of its own, completed once): the two
+    // warpgroups' exponential phases then start half a tile apart instead of
+    // contending for MUFU from the first tile on (causal GQA workload at B=4:
+    // 7.18 -> 7.09 ms; the masked LLM workload 1.14 -> 1.10 ms).
+    bool ok = true;
+    if (wg == 1 && (orf & 1u))
+      ok = __all_sync(0xffffffffu, mbar_wait(wg0_started, 0, SITE_P_FULL));
     float m_ref = -INFINITY, l = 0.f;
     uint32_t n = 0;
-    bool ok = true;
-    for (int idx = 0; idx < ntile; ++idx) {
+    for (int idx = 0; ok && idx < ntile; ++idx) {
       const uint32_t e = s_list[idx];
       if (!((e >> wg) & 1u)) continue;
       const int kt = (int)(e >> 8);
@@ -683,6 +692,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[wg * 2 + buf]);
+      if (wg == 0 && n == 0) mbar_arrive(wg0_started);
       l = l * alpha + rs;
       m_ref = m_new;
       ++n;
