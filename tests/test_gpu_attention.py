@@ -85,6 +85,27 @@ def test_mask_second_half_and_random_mask(S):
     assert torch.all(out[:, :, 7] == 0) and torch.all(torch.isneginf(l[:, :, 7]))
 
 
+def test_mask_hides_every_key_from_one_q_tile_of_a_pair(S):
+    """A CTA works on a pair of 128-row Q tiles, and the second tile's
+    softmax starts after the first tile's first P tile.  With the first tile
+    (or the second) seeing no key at all, nothing may wait for it: rows 0..127
+    (then 128..255) are fully masked, the other tile of the pair sees a random
+    half of the keys."""
+    w = W.TINY.scaled(B=1, Hq=2, Hkv=2, N=512, D=128, seed=37)
+    q, k, v = W.make_qkv(w)
+    oz = O.quantize_qkv_i8f8(q, k, v)
+    z = qkv_from_oracle(S, oz)
+    g = torch.Generator().manual_seed(5)
+    for hidden in (slice(0, 128), slice(128, 256)):
+        rm = torch.rand(1, 1, 512, 512, generator=g) < 0.5
+        rm[:, :, hidden, :] = False
+        ref = O.attention_i8f8(oz, mask=rm.numpy())
+        out, l = S.sage_attn_fwd_quantized(z, return_lse=True, mask=rm.cuda())
+        assert S.sage_get_device_status()[0] == S.SAGE_OK
+        assert_attention_close(out, l, ref, what=f"rows {hidden.start}.. hidden")
+        assert torch.all(out[:, :, hidden] == 0) and torch.all(torch.isneginf(l[:, :, hidden]))
+
+
 def test_mask_unaligned_key_length(S):
     w = W.TINY.scaled(B=1, Hq=2, Hkv=2, N=200, D=64, seed=36)
     q, k, v = W.make_qkv(w)
