@@ -114,15 +114,36 @@ __device__ __forceinline__ float dd_mean_f32(const DD& s, double n) {
 }
 
 // ------------------------------------------------------------ pass A
+// 16-byte asynchronous copy global -> shared (L1 bypassed), one commit group
+// per call of cp_async_commit, and the waits.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // grid (splits, B*Hkv), 256 threads.  Thread layout: D/8 threads per token
-// row (one 16-byte load each), 256/(D/8) rows per step.
+// row (16 bytes each), 256/(D/8) rows per pass.  Each thread copies its own
+// 16 bytes of K and V of the next passes into shared memory by cp.async, a
+// ring of PA_SLOTS passes (PA_SLOTS - 1 in flight: no registers hold them,
+// so four CTAs fit per SM), and accumulates its channels in row order.
+constexpr int PA_SLOTS = 6;
 template <typename T, int D>
 __global__ void __launch_bounds__(QUANT_THREADS) kmean_vamax_partial_kernel(QuantArgs a) {
   constexpr int TPR = D / 8;
   constexpr int RPP = QUANT_THREADS / TPR;
-  __shared__ double s_hi[RPP][D];
-  __shared__ double s_lo[RPP][D];
-  __shared__ float s_am[RPP][D];
+  constexpr int ROWB = D * (int)sizeof(T);
+  constexpr int SLOT = 2 * RPP * ROWB;            // K rows, then V rows, of one pass
+  constexpr int RED = RPP * D * (8 + 8 + 4);      // the per-row-group partials
+  constexpr int BUF = PA_SLOTS * SLOT > RED ? PA_SLOTS * SLOT : RED;
+  __shared__ __align__(16) uint8_t s_buf[BUF];
 
   const int split = blockIdx.x;
   const int bh = blockIdx.y;
@@ -145,36 +166,45 @@ __global__ void __launch_bounds__(QUANT_THREADS) kmean_vamax_partial_kernel(Quan
   const char* vb = reinterpret_cast<const char*>(a.v) +
                    (seq_in_offset(a, sq.ck, b, a.v_sn, a.v_sb) + h * a.v_sh + cg * 8) *
                        (int64_t)sizeof(T);
-  // four rows per iteration, their loads issued before any arithmetic (the
-  // accumulation order per channel is the same fixed row order as one by one)
-  constexpr int UNR = 4;
-  for (int nb = n0 + rs; nb < n1; nb += UNR * RPP) {
-    uint4 kr[UNR], vr[UNR];
-#pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const int n = nb + u * RPP;
-      kr[u] = (a.smooth_k && n < n1) ? ldg16(kb + (int64_t)n * a.k_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
-      vr[u] = n < n1 ? ldg16(vb + (int64_t)n * a.v_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
+  // pass p covers rows n0 + p*RPP + rs; every call commits one group (empty
+  // past the split), so the group count stays uniform
+  auto issue = [&](int p) {
+    const int n = n0 + p * RPP + rs;
+    uint8_t* slot = s_buf + (p % PA_SLOTS) * SLOT + rs * ROWB + cg * 16;
+    if (n < n1) {
+      if (a.smooth_k) cp_async16(slot, kb + (int64_t)n * a.k_sn * sizeof(T));
+      cp_async16(slot + RPP * ROWB, vb + (int64_t)n * a.v_sn * sizeof(T));
     }
+    cp_async_commit();
+  };
+  const int npass = n1 > n0 ? (n1 - n0 + RPP - 1) / RPP : 0;
 #pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      if (nb + u * RPP >= n1) break;
-      float f[8];
-      if (a.smooth_k) {
-        unpack8<T>(kr[u], f);
+  for (int p = 0; p < PA_SLOTS - 1; ++p) issue(p);
+  for (int p = 0; p < npass; ++p) {
+    issue(p + PA_SLOTS - 1);         // into the slot this thread read at pass p - 1
+    cp_async_wait<PA_SLOTS - 1>();   // pass p's copies (this thread's own) are done
+    if (n0 + p * RPP + rs >= n1) break;
+    const uint8_t* slot = s_buf + (p % PA_SLOTS) * SLOT + rs * ROWB + cg * 16;
+    float f[8];
+    if (a.smooth_k) {
+      unpack8<T>(*reinterpret_cast<const uint4*>(slot), f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dd_add(acc[i], (double)f[i]);
-      }
-      unpack8<T>(vr[u], f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) am[i] = fmaxf(am[i], fabsf(f[i]));
+      for (int i = 0; i < 8; ++i) dd_add(acc[i], (double)f[i]);
     }
+    unpack8<T>(*reinterpret_cast<const uint4*>(slot + RPP * ROWB), f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) am[i] = fmaxf(am[i], fabsf(f[i]));
   }
+  cp_async_wait_all();
+  __syncthreads();   // the ring is reused for the partials below
+  double* s_hi = reinterpret_cast<double*>(s_buf);
+  double* s_lo = s_hi + RPP * D;
+  float* s_am = reinterpret_cast<float*>(s_lo + RPP * D);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    s_hi[rs][cg * 8 + i] = acc[i].hi;
-    s_lo[rs][cg * 8 + i] = acc[i].lo;
-    s_am[rs][cg * 8 + i] = am[i];
+    s_hi[rs * D + cg * 8 + i] = acc[i].hi;
+    s_lo[rs * D + cg * 8 + i] = acc[i].lo;
+    s_am[rs * D + cg * 8 + i] = am[i];
   }
   __syncthreads();
   if (threadIdx.x < D) {
@@ -182,8 +212,8 @@ __global__ void __launch_bounds__(QUANT_THREADS) kmean_vamax_partial_kernel(Quan
     DD s = {0.0, 0.0};
     float m = 0.f;
     for (int r = 0; r < RPP; ++r) {  // fixed order: deterministic
-      dd_add(s, DD{s_hi[r][c], s_lo[r][c]});
-      m = fmaxf(m, s_am[r][c]);
+      dd_add(s, DD{s_hi[r * D + c], s_lo[r * D + c]});
+      m = fmaxf(m, s_am[r * D + c]);
     }
     const int64_t o = ((int64_t)bh * a.splits + split) * D + c;
     a.part_hi[o] = s.hi;

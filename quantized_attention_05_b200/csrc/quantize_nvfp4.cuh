@@ -134,27 +134,24 @@ __device__ __forceinline__ void bf16_split(float x, uint16_t& hi, uint16_t& lo) 
   lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fsub_rn(x, __bfloat162float(h))));
 }
 
-// 16-byte asynchronous copy global -> shared (L1 bypassed), and the wait
-// for all of this thread's outstanding copies.
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-
 // ------------------------------------------------------------ column sums
 // grid (splits, B*H), 256 threads: per split of tokens [s*T, min(limit,(s+1)*T)),
-// double-double sums of every channel.
+// double-double sums of every channel.  D/8 threads per row (16 bytes each);
+// each thread copies its own 16 bytes of the next passes into shared memory
+// by cp.async (a ring of CS_SLOTS passes, CS_SLOTS - 1 in flight) and adds
+// its channels in row order.
+constexpr int CS_SLOTS = 8;
 template <typename T, int D>
 __global__ void __launch_bounds__(QUANT_THREADS)
     nv_colsum_kernel(const void* src, int64_t sb, int64_t sh, int64_t sn, int H, int limit,
                      int splits, int split_tokens, double* part_hi, double* part_lo) {
   constexpr int TPR = D / 8;
   constexpr int RPP = QUANT_THREADS / TPR;
-  __shared__ double s_hi[RPP][D];
-  __shared__ double s_lo[RPP][D];
+  constexpr int ROWB = D * (int)sizeof(T);
+  constexpr int SLOT = RPP * ROWB;
+  constexpr int RED = RPP * D * 16;
+  constexpr int BUF = CS_SLOTS * SLOT > RED ? CS_SLOTS * SLOT : RED;
+  __shared__ __align__(16) uint8_t s_buf[BUF];
   const int split = blockIdx.x, bh = blockIdx.y;
   const int b = bh / H, h = bh % H;
   const int cg = threadIdx.x % TPR, rs = threadIdx.x / TPR;
@@ -163,35 +160,38 @@ __global__ void __launch_bounds__(QUANT_THREADS)
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = {0.0, 0.0};
   const char* base = reinterpret_cast<const char*>(src) + (b * sb + h * sh + cg * 8) * (int64_t)sizeof(T);
-  // four rows per iteration, their loads issued before any arithmetic (the
-  // accumulation order per channel is the same fixed row order as one by one)
-  constexpr int UNR = 4;
-  for (int nb = n0 + rs; nb < n1; nb += UNR * RPP) {
-    uint4 r[UNR];
+  auto issue = [&](int p) {
+    const int n = n0 + p * RPP + rs;
+    if (n < n1)
+      cp_async16(s_buf + (p % CS_SLOTS) * SLOT + rs * ROWB + cg * 16, base + (int64_t)n * sn * sizeof(T));
+    cp_async_commit();
+  };
+  const int npass = n1 > n0 ? (n1 - n0 + RPP - 1) / RPP : 0;
 #pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const int n = nb + u * RPP;
-      r[u] = n < n1 ? ldg16(base + (int64_t)n * sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
-    }
+  for (int p = 0; p < CS_SLOTS - 1; ++p) issue(p);
+  for (int p = 0; p < npass; ++p) {
+    issue(p + CS_SLOTS - 1);         // into the slot this thread read at pass p - 1
+    cp_async_wait<CS_SLOTS - 1>();   // pass p's copy (this thread's own) is done
+    if (n0 + p * RPP + rs >= n1) break;
+    float f[8];
+    unpack8<T>(*reinterpret_cast<const uint4*>(s_buf + (p % CS_SLOTS) * SLOT + rs * ROWB + cg * 16), f);
 #pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      if (nb + u * RPP >= n1) break;
-      float f[8];
-      unpack8<T>(r[u], f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) dd_add(acc[i], (double)f[i]);
-    }
+    for (int i = 0; i < 8; ++i) dd_add(acc[i], (double)f[i]);
   }
+  cp_async_wait_all();
+  __syncthreads();   // the ring is reused for the partials below
+  double* s_hi = reinterpret_cast<double*>(s_buf);
+  double* s_lo = s_hi + RPP * D;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    s_hi[rs][cg * 8 + i] = acc[i].hi;
-    s_lo[rs][cg * 8 + i] = acc[i].lo;
+    s_hi[rs * D + cg * 8 + i] = acc[i].hi;
+    s_lo[rs * D + cg * 8 + i] = acc[i].lo;
   }
   __syncthreads();
   if (threadIdx.x < D) {
     const int c = threadIdx.x;
     DD s = {0.0, 0.0};
-    for (int r = 0; r < RPP; ++r) dd_add(s, DD{s_hi[r][c], s_lo[r][c]});
+    for (int r = 0; r < RPP; ++r) dd_add(s, DD{s_hi[r * D + c], s_lo[r * D + c]});
     const int64_t o = ((int64_t)bh * splits + split) * D + c;
     part_hi[o] = s.hi;
     part_lo[o] = s.lo;
