@@ -311,10 +311,11 @@ __device__ __forceinline__ float rows_sum_transposed(float* v, int cg) {
 // One CTA per 128-token block: first the K and V blocks, KV heads in
 // descending order (pass A reads the heads in ascending order, so the K and
 // V rows it read last are still in L2 when pass B starts), K and V blocks of
-// a head alternating; then the Q blocks.  Each thread keeps its 16-byte loads
-// in registers between the amax and the code pass.
+// a head alternating; then the Q blocks.  Each thread copies its 16-byte
+// pieces of the block into shared memory by cp.async and reads them for the
+// amax and again for the codes.
 template <typename T, int D>
-__global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(QUANT_THREADS, 6) quant_blocks_kernel(QuantArgs a) {
   constexpr int TPR = D / 8;
   constexpr int RPP = QUANT_THREADS / TPR;
   constexpr int ITERS = QB / RPP;
@@ -324,6 +325,25 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
   const int nKb = a.B * a.Hkv * a.max_nkt;
   const int job = blockIdx.x;
   const int cg = threadIdx.x % TPR, rs = threadIdx.x / TPR;
+  // the block's rows in shared memory: each thread copies its own 16 bytes
+  // of its ITERS rows by cp.async (no registers hold them in flight) and
+  // reads them back for the amax and for the codes; rows past `limit` are 0
+  __shared__ __align__(16) uint8_t s_blk[QB * D * sizeof(T)];
+  auto stage = [&](const char* base, int64_t sn, int row0, int limit) {
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int r = rs + it * RPP;
+      uint8_t* dst = s_blk + (r * D + cg * 8) * sizeof(T);
+      if (row0 + r < limit)
+        cp_async16(dst, base + (int64_t)(row0 + r) * sn * sizeof(T));
+      else
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    }
+    cp_async_wait_all();
+  };
+  auto raw = [&](int it) -> uint4 {
+    return *reinterpret_cast<const uint4*>(s_blk + ((rs + it * RPP) * D + cg * 8) * sizeof(T));
+  };
   // K/V job -> (KV head, block, K or V)
   const int kvh = a.B * a.Hkv - 1 - job / (2 * a.max_nkt);
   const int kvt = (job % (2 * a.max_nkt)) >> 1;
@@ -343,17 +363,12 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
     const char* base = reinterpret_cast<const char*>(a.q) +
                        (seq_in_offset(a, sq.cq, b, a.q_sn, a.q_sb) + h * a.q_sh + cg * 8) *
                            (int64_t)sizeof(T);
-    uint4 raw[ITERS];
+    stage(base, a.q_sn, qt * QB, sq.nq);
     float am = 0.f;
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
-      const int n = qt * QB + rs + it * RPP;
-      raw[it] = n < sq.nq ? ldg16(base + (int64_t)n * a.q_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
       float f[8];
-      unpack8<T>(raw[it], f);
+      unpack8<T>(raw(it), f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(f[i]));
     }
@@ -364,7 +379,7 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
     for (int it = 0; it < ITERS; ++it) {
       const int n = qt * QB + rs + it * RPP;
       float f[8];
-      unpack8<T>(raw[it], f);
+      unpack8<T>(raw(it), f);
       *reinterpret_cast<uint2*>(a.q8 + (row0 + n) * D + cg * 8) = int8x8_codes(f, inv);
       if (a.qdk) {
         uint64_t d2 = f2_pack(0.f, 0.f);
@@ -398,12 +413,7 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
     const char* base = reinterpret_cast<const char*>(a.k) +
                        (seq_in_offset(a, sq.ck, b, a.k_sn, a.k_sb) + h * a.k_sh + cg * 8) *
                            (int64_t)sizeof(T);
-    uint4 raw[ITERS];
-#pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-      const int n = kt * QB + rs + it * RPP;
-      raw[it] = n < sq.nk ? ldg16(base + (int64_t)n * a.k_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
-    }
+    stage(base, a.k_sn, kt * QB, sq.nk);
     __syncthreads();
     // K - kmean, one IEEE-rounded subtraction per element
     float km[8];
@@ -419,7 +429,7 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
     for (int it = 0; it < ITERS; ++it) {
       const int n = kt * QB + rs + it * RPP;
       float f[8];
-      smooth(raw[it], f);
+      smooth(raw(it), f);
       if (n < sq.nk) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(f[i]));
@@ -431,7 +441,7 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
     for (int it = 0; it < ITERS; ++it) {
       const int n = kt * QB + rs + it * RPP;
       float f[8];
-      smooth(raw[it], f);
+      smooth(raw(it), f);
       const uint2 w = n < sq.nk ? int8x8_codes(f, inv) : make_uint2(0u, 0u);
       *reinterpret_cast<uint2*>(a.k8 + (row0 + n) * D + cg * 8) = w;
     }
@@ -454,12 +464,7 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
     const char* base = reinterpret_cast<const char*>(a.v) +
                        (seq_in_offset(a, sq.ck, b, a.v_sn, a.v_sb) + h * a.v_sh + cg * 8) *
                            (int64_t)sizeof(T);
-    uint4 raw[ITERS];
-#pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-      const int n = vt * QB + rs + it * RPP;
-      raw[it] = n < sq.nk ? ldg16(base + (int64_t)n * a.v_sn * sizeof(T)) : make_uint4(0, 0, 0, 0);
-    }
+    stage(base, a.v_sn, vt * QB, sq.nk);
     __syncthreads();
     float inv[8];
 #pragma unroll
@@ -468,7 +473,7 @@ __global__ void __launch_bounds__(QUANT_THREADS, 3) quant_blocks_kernel(QuantArg
     for (int it = 0; it < ITERS; ++it) {
       const int n = vt * QB + rs + it * RPP;
       float f[8];
-      unpack8<T>(raw[it], f);
+      unpack8<T>(raw(it), f);
       uint32_t w[2] = {0u, 0u};
       if (n < sq.nk) {
 #pragma unroll
