@@ -592,10 +592,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[128];
-      SAGE_TMEM_LD32(tS + 0, (sr + 0));
-      SAGE_TMEM_LD32(tS + 32, (sr + 32));
-      SAGE_TMEM_LD32(tS + 64, (sr + 64));
-      SAGE_TMEM_LD32(tS + 96, (sr + 96));
+      SAGE_TMEM_LD128(tS, sr);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&s_free[t]);
