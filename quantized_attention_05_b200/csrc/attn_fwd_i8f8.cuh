@@ -288,7 +288,7 @@ __device__ __forceinline__ float exp_tile(const uint32_t* sr, const uint32_t* vi
     uint32_t pw[8];
 #pragma unroll
     for (int i = 0; i < 16; i += 2) {
-      uint32_t half[2];
+      float pp[4];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int j = ch * 32 + 2 * (i + u);
@@ -307,11 +307,9 @@ __device__ __forceinline__ float exp_tile(const uint32_t* sr, const uint32_t* vi
           p = f2_pack(p0, p1);
         }
         acc = f2_add(acc, p);
-        float p0, p1;
-        f2_unpack(p, p0, p1);
-        half[u] = cvt_e4m3x2(p0, p1);
+        f2_unpack(p, pp[2 * u], pp[2 * u + 1]);
       }
-      pw[i >> 1] = half[0] | (half[1] << 16);
+      pw[i >> 1] = cvt_e4m3x4(pp[0], pp[1], pp[2], pp[3]);
     }
     // 16-byte chunks 2ch and 2ch+1 of the row, 128-byte swizzle
     *reinterpret_cast<uint4*>(prow + (((2 * ch) ^ (rt & 7)) << 4)) =

@@ -372,6 +372,19 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 // Two fp32 values to two E4M3 bytes, round to nearest even, saturating;
 // `lo` lands in the low byte.
+// Four fp32 values to four E4M3 codes (rn, satfinite) in one word, a in the
+// lowest byte: two paired conversions and one register pack, no 16-bit
+// shifts in between.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
