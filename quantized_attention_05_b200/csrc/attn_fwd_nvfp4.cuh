@@ -204,15 +204,15 @@ __device__ __forceinline__ float nv_exp_tile(const uint32_t* sr, const uint32_t*
                                              const float* s_inv, uint8_t* prow, int rt,
                                              uint32_t* sfw) {
   const uint64_t c2 = f2_pack(c, c), b2 = f2_pack(bias, bias);
-  float inv[8];
-  sfw[0] = sfw[1] = 0u;
+  float inv[8], q[8];
 #pragma unroll
-  for (int vv = 0; vv < 8; ++vv) {
-    const float pmax = ex2_approx(fmaf(vmax[vv], c, bias));
-    const uint32_t sf = e4m3_code(div6_rn(pmax));
-    inv[vv] = s_inv[sf];
-    sfw[vv >> 2] |= sf << (8 * (vv & 3));
-  }
+  for (int vv = 0; vv < 8; ++vv) q[vv] = div6_rn(ex2_approx(fmaf(vmax[vv], c, bias)));
+  // the eight scale codes, four per conversion statement, already in the
+  // byte order of the scale-factor words
+  sfw[0] = cvt_e4m3x4(q[0], q[1], q[2], q[3]);
+  sfw[1] = cvt_e4m3x4(q[4], q[5], q[6], q[7]);
+#pragma unroll
+  for (int vv = 0; vv < 8; ++vv) inv[vv] = s_inv[(sfw[vv >> 2] >> (8 * (vv & 3))) & 0xFFu];
   uint64_t acc = f2_pack(0.f, 0.f);
 #pragma unroll
   for (int ch = 0; ch < 4; ++ch) {
