@@ -82,6 +82,31 @@ __device__ __forceinline__ void unpack8(const uint4& raw, float* f) {
   for (int i = 0; i < 8; ++i) f[i] = to_f32<T>(e[i]);
 }
 
+// max(|a|, |b|) of two packed pairs of T (elementwise), and the fp32 value of
+// the low / high element of a pair.
+template <typename T>
+__device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b);
+template <>
+__device__ __forceinline__ uint32_t absmax2<__nv_bfloat16>(uint32_t a, uint32_t b) {
+  const __nv_bfloat162 r = __hmax2(__habs2(*reinterpret_cast<const __nv_bfloat162*>(&a)),
+                                   __habs2(*reinterpret_cast<const __nv_bfloat162*>(&b)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+template <>
+__device__ __forceinline__ uint32_t absmax2<__half>(uint32_t a, uint32_t b) {
+  const __half2 r = __hmax2(__habs2(*reinterpret_cast<const __half2*>(&a)),
+                            __habs2(*reinterpret_cast<const __half2*>(&b)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+template <typename T>
+__device__ __forceinline__ float lo_f32(uint32_t w) {
+  return to_f32<T>(*reinterpret_cast<const T*>(&w));
+}
+template <typename T>
+__device__ __forceinline__ float hi_f32(uint32_t w) {
+  return to_f32<T>(*(reinterpret_cast<const T*>(&w) + 1));
+}
+
 __device__ __forceinline__ uint4 ldg16(const void* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
 }
@@ -364,14 +389,15 @@ __global__ void __launch_bounds__(QUANT_THREADS, 6) quant_blocks_kernel(QuantArg
                        (seq_in_offset(a, sq.cq, b, a.q_sn, a.q_sb) + h * a.q_sh + cg * 8) *
                            (int64_t)sizeof(T);
     stage(base, a.q_sn, qt * QB, sq.nq);
-    float am = 0.f;
+    // |x| max on packed pairs of the input type (exact: every bf16/fp16
+    // value is an fp32 value, and the max of magnitudes is one of them)
+    uint32_t m2 = 0u;
 #pragma unroll
     for (int it = 0; it < ITERS; ++it) {
-      float f[8];
-      unpack8<T>(raw(it), f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(f[i]));
+      const uint4 r = raw(it);
+      m2 = absmax2<T>(m2, absmax2<T>(absmax2<T>(r.x, r.y), absmax2<T>(r.z, r.w)));
     }
+    const float am = fmaxf(lo_f32<T>(m2), hi_f32<T>(m2));
     const float amax = block_max(am, s_red);  // also orders s_c
     const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
     float dsum[ITERS];
