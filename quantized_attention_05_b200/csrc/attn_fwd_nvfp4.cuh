@@ -181,13 +181,10 @@ __device__ __forceinline__ void load_sf(SfRegs<NSF>& r, const uint8_t* src, int6
 }
 template <int NSF>
 __device__ __forceinline__ void store_sf(uint8_t* dst, const SfRegs<NSF>& r, int lane) {
+  // the lane's rows lane + 32i are the four words of one 16-byte chunk
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int row = lane + 32 * i;
-#pragma unroll
-    for (int b = 0; b < NSF / 4; ++b)
-      *reinterpret_cast<uint32_t*>(dst + b * 512 + 16 * (row & 31) + 4 * (row >> 5)) = r.w[i][b];
-  }
+  for (int b = 0; b < NSF / 4; ++b)
+    *reinterpret_cast<uint4*>(dst + b * 512 + 16 * lane) = make_uint4(r.w[0][b], r.w[1][b], r.w[2][b], r.w[3][b]);
 }
 
 // The 16-key vectors of one thread's row: P' = 2688 * p quantised to E2M1
@@ -357,9 +354,12 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
     prefetch_tmap(&tmV);
   }
   // A operand of the correction MMA: bf16 1.0 (0x3F80) at k = 0 and 1 of
-  // both 16-byte chunks of every row
+  // both 16-byte chunks of every row; the correction B tiles start zero (only
+  // the first word of each row's data chunk is ever rewritten)
   for (int u = threadIdx.x; u < 256; u += blockDim.x)
     *reinterpret_cast<uint4*>(sOnes + 16 * u) = make_uint4(0x3F803F80u, 0u, 0u, 0u);
+  for (int u = threadIdx.x; u < NV_STAGES * 2 * 4096 / 16; u += blockDim.x)
+    reinterpret_cast<uint4*>(sCorrB)[u] = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -418,17 +418,19 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
       // -------------------------------------------------------- correction rows
       // The qk_correction rows of the stage's key tile for the Q tiles that
       // see it, as the B operand of the correction MMA; read one tile ahead
-      // like the scale factors.
-      float4 cv[2];
+      // like the scale factors.  Lane l handles keys l, l + 32, l + 64,
+      // l + 96 (coalesced loads; its 4-byte stores at 32-byte row strides
+      // hit eight banks per eight rows).
+      float cv[2][4];
       const float* corr0 = a.corr + ((int64_t)bhq * a.nqt + qt0) * a.Nkp;
       auto load_tile = [&](int idx) {
         const uint32_t e = s_list[idx];
         const int kt = (int)(e >> 8);
 #pragma unroll
         for (int t = 0; t < 2; ++t)
-          cv[t] = ((e >> t) & 1u)
-                      ? __ldg(reinterpret_cast<const float4*>(corr0 + (int64_t)t * a.Nkp + kt * 128) + lane)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            cv[t][i] = ((e >> t) & 1u) ? __ldg(corr0 + (int64_t)t * a.Nkp + kt * 128 + lane + 32 * i) : 0.f;
       };
       if (ntile > 0) load_tile(0);
       for (int idx = 0; idx < ntile; ++idx) {
@@ -438,20 +440,20 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
           break;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          // the correction of keys 4*lane .. 4*lane+3 as bf16 hi + lo
-          // (|x - hi - lo| <= 2^-18 |x|), row j of the B tile
-          const float x[4] = {cv[t].x, cv[t].y, cv[t].z, cv[t].w};
+          // the correction of key j as bf16 hi + lo (|x - hi - lo| <= 2^-18 |x|),
+          // the first word of row j's data chunk in the B tile (the rest of
+          // the tile stays zero from the setup)
           uint8_t* tile = sCorrB + (st * 2 + t) * 4096;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int j = 4 * lane + i;
-            const __nv_bfloat16 hi = __float2bfloat16_rn(x[i]);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(x[i], __bfloat162float(hi)));
+            const int j = lane + 32 * i;
+            const float x = cv[t][i];
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
             const uint32_t w =
                 (uint32_t)__bfloat16_as_ushort(hi) | ((uint32_t)__bfloat16_as_ushort(lo) << 16);
             const int sw = (j >> 2) & 1;   // 32-byte swizzle: chunk c of row j at (c ^ sw) * 16
-            *reinterpret_cast<uint4*>(tile + j * 32 + (sw << 4)) = make_uint4(w, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(tile + j * 32 + ((1 ^ sw) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint32_t*>(tile + j * 32 + (sw << 4)) = w;
           }
         }
         if (idx + 1 < ntile) load_tile(idx + 1);
