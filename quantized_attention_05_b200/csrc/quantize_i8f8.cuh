@@ -503,9 +503,9 @@ __global__ void __launch_bounds__(QUANT_THREADS, 6) quant_blocks_kernel(QuantArg
       uint32_t w[2] = {0u, 0u};
       if (n < sq.nk) {
 #pragma unroll
-        for (int i = 0; i < 8; i += 2)
-          w[i >> 2] |= (uint32_t)cvt_e4m3x2(__fmul_rn(f[i], inv[i]), __fmul_rn(f[i + 1], inv[i + 1]))
-                       << (8 * (i & 3));
+        for (int i = 0; i < 8; i += 4)
+          w[i >> 2] = cvt_e4m3x4(__fmul_rn(f[i], inv[i]), __fmul_rn(f[i + 1], inv[i + 1]),
+                                 __fmul_rn(f[i + 2], inv[i + 2]), __fmul_rn(f[i + 3], inv[i + 3]));
       }
       *reinterpret_cast<uint2*>(a.v8 + (row0 + n) * D + cg * 8) = make_uint2(w[0], w[1]);
     }
