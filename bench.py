@@ -19,7 +19,7 @@ Multi-GPU (torchrun, one process per GPU): every rank runs its own replica
 of the workload (seeded by rank; the path has no exchange step), so the
 scaling is weak and the value is the ops of all ranks over the max time.
 
---impl reference times the CPU oracle (the reference arm of this build) on
+--impl reference times the CPU oracle (the reference arm) on
 rank 0: every step quantises and attends a bounded sample of the workload.
 """
 from __future__ import annotations
