@@ -441,6 +441,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_arrive_expect_tx(q_full, (uint32_t)((act0 ? L::Q_BYTES : 0) + (act1 ? L::Q_BYTES : 0)));
       if (act0) tma_load_2d(sQ, &tmQ, q_full, 0, (int)(cs.qrow0 + qt0 * ATT_BM));
       if (act1) tma_load_2d(sQ + L::Q_BYTES, &tmQ, q_full, 0, (int)(cs.qrow0 + (qt0 + 1) * ATT_BM));
+      int issued = 0;
       for (int idx = 0; idx < ntile; ++idx) {
         const int st = idx % ATT_STAGES, rd = idx / ATT_STAGES;
         if (idx >= ATT_STAGES && !mbar_wait(&kv_empty[st], (rd - 1) & 1, SITE_KV_EMPTY)) break;
@@ -448,6 +449,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         mbar_arrive_expect_tx(&kv_full[st], (uint32_t)(L::K_BYTES + L::V_BYTES));
         tma_load_2d(sK + st * L::K_BYTES, &tmK, &kv_full[st], 0, (int)(cs.krow0 + kt * ATT_BN));
         tma_load_2d(sV + st * L::V_BYTES, &tmV, &kv_full[st], 0, (int)(cs.krow0 + kt * ATT_BN));
+        ++issued;
+      }
+      // every copy issued above lands before the CTA's shared memory is
+      // released, also when a wait gave up (otherwise already the case: the
+      // issuers wait for every tile)
+      mbar_drain(q_full, 0);
+      for (int st = 0; st < ATT_STAGES && st < issued; ++st) {
+        const int last = st + (issued - 1 - st) / ATT_STAGES * ATT_STAGES;
+        mbar_drain(&kv_full[st], (last / ATT_STAGES) & 1);
       }
     }
     __syncwarp();

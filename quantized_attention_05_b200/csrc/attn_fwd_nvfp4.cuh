@@ -395,6 +395,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
         load_sf<8>(vsf, a.v_sf_t + (int64_t)bhk * D * (a.Nkp / 16) + kt * 8, a.Nkp / 16, D, lane);
       };
       if (ntile > 0) load_tile(0);
+      int issued = 0;
       for (int idx = 0; idx < ntile; ++idx) {
         const int st = idx % NV_STAGES, rd = idx / NV_STAGES;
         if (idx >= NV_STAGES &&
@@ -411,6 +412,17 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
           tma_load_2d(sV + st * L::V_BYTES, &tmV, &kv_full[st], kt * 64, bhk * D);
         } else {
           mbar_arrive(&kv_full[st]);
+        }
+        ++issued;
+      }
+      // every copy issued above lands before the CTA's shared memory is
+      // released, also when a wait gave up (otherwise already the case: the
+      // issuers wait for every tile)
+      if (lane == 0) {
+        mbar_drain(q_full, 0);
+        for (int st = 0; st < NV_STAGES && st < issued; ++st) {
+          const int last = st + (issued - 1 - st) / NV_STAGES * NV_STAGES;
+          mbar_drain(&kv_full[st], (last / NV_STAGES) & 1);
         }
       }
       __syncwarp();

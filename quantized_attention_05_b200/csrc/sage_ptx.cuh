@@ -113,6 +113,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
 }
 
+// The wait of a thread on its way out: until the phase of `parity` has
+// completed (the thread's own bulk copies into shared memory have landed,
+// so none is still writing when the CTA's shared memory is released), for at
+// most `limit_ns`.  Unlike mbar_wait it does not give up because another wait
+// has failed, and it records nothing: in a launch without failures the phase
+// is complete or about to be.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity,
+                                           uint64_t limit_ns = 10000000ull) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((it & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
