@@ -536,7 +536,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       if (ok) ok = release_to(ntile - 1);
       // every MMA issued above completes before the CTA tears down TMEM
       tc_commit(mma_done);
-      mbar_wait(mma_done, 0, SITE_MMA_DONE);
+      // (a wait that gives up because another one failed is followed by the
+      // drain: the MMAs still finish before TMEM is freed)
+      if (!mbar_wait(mma_done, 0, SITE_MMA_DONE)) mbar_drain(mma_done, 0);
     }
     __syncwarp();
     }
@@ -820,6 +822,8 @@ __global__ void __launch_bounds__(128, 1)
       for (int k = 0; k < D / 32; ++k)
         mma_i8(tmem, smem_desc(smem_u32(sQ) + 32 * k, L::QK_SBO, L::QK_SWIZZLE),
                smem_desc(smem_u32(sK) + 32 * k, L::QK_SBO, L::QK_SWIZZLE), IDESC, k > 0 ? 1u : 0u);
+    } else {
+      mbar_drain(&bar[0], 0);   // the copies land before shared memory is released
     }
     tc_commit(&bar[1]);
   }
@@ -839,6 +843,7 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
+    if (!ok) mbar_drain(&bar[1], 0);   // the MMAs finish before TMEM is freed
     tc_fence_after();
     tmem_dealloc(tmem, 128);
   }
@@ -886,6 +891,8 @@ __global__ void __launch_bounds__(128, 1)
         mma_f8f6f4(tmem, smem_desc(smem_u32(sP) + 32 * k, 1024, 128),
                    smem_desc(smem_u32(sV) + L::V_KSTEP * k, L::QK_SBO, L::QK_SWIZZLE), IDESC,
                    k > 0 ? 1u : 0u);
+    } else {
+      mbar_drain(&bar[0], 0);   // the copy lands before shared memory is released
     }
     tc_commit(&bar[1]);
   }
@@ -904,6 +911,7 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
+    if (!ok) mbar_drain(&bar[1], 0);   // the MMAs finish before TMEM is freed
     tc_fence_after();
     tmem_dealloc(tmem, 128);
   }

@@ -578,7 +578,9 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
         }
         // every MMA issued above completes before the CTA tears down TMEM
         tc_commit(mma_done);
-        mbar_wait(mma_done, 0, SITE_MMA_DONE);
+        // (a wait that gives up because another one failed is followed by the
+        // drain: the MMAs still finish before TMEM is freed)
+        if (!mbar_wait(mma_done, 0, SITE_MMA_DONE)) mbar_drain(mma_done, 0);
       }
       __syncwarp();
     }

@@ -580,8 +580,12 @@ __global__ void __launch_bounds__(NVC_THREADS, 3) nv_corr_kernel(NvQuantArgs a) 
     __syncthreads();
     tc_fence_after();
   }
-  // every MMA issued above has completed (each half waited for its commit)
-  if (warp == 0) tmem_dealloc(tmem, 128);
+  // every MMA issued above has completed (each half waited for its commit);
+  // after a wait that gave up, warp 0 first lets the last MMAs finish
+  if (warp == 0) {
+    if (!ok && phase > 0) mbar_drain(&mma_bar, (phase - 1) & 1);
+    tmem_dealloc(tmem, 128);
+  }
 }
 
 }  // namespace sage
