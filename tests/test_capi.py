@@ -97,6 +97,8 @@ def test_quantize_rejects_bad_arguments_on_host(L):
     assert call(_t(), _t(), _t(), _q(Nk=300)) == S.SAGE_ERR_INVALID_ARG   # out shape mismatch
     assert call(_t(), _t(), _t(), ws=0) == S.SAGE_ERR_INVALID_ARG         # no workspace
     assert call(_t(), _t(), _t(), nb=16) == S.SAGE_ERR_WORKSPACE          # workspace too small
+    n1 = 128 * 2048 + 1                                                   # one key past the longest
+    assert call(_t(), _t(N=n1), _t(N=n1), _q(Nk=n1)) == S.SAGE_ERR_UNSUPPORTED
 
 
 def test_attention_rejects_bad_arguments_on_host(L):
@@ -123,6 +125,9 @@ def test_attention_rejects_bad_arguments_on_host(L):
         == S.SAGE_ERR_WORKSPACE
     zbig = _q(Nq=128 * 4096, Nk=128 * 4096)
     assert f(byref(zbig), 0, 0.0, 0, None, 256, 0, 0, 256 * 64, 64, None, None, 0, None) \
+        == S.SAGE_ERR_UNSUPPORTED
+    zlong = _q(Nk=128 * 2048 + 1)                                   # one key past the longest
+    assert f(byref(zlong), 0, 0.0, 0, None, 256, 0, 0, 256 * 64, 64, None, None, 0, None) \
         == S.SAGE_ERR_UNSUPPORTED
 
 

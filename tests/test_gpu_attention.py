@@ -168,6 +168,23 @@ def test_causal_bottom_right_when_lengths_differ(S):
         assert_attention_close(out, l, ref, what=f"causal Nq={Nq} Nk={Nk}")
 
 
+def test_longest_supported_key_length(S):
+    """The longest key sequence the kernels accept: 2048 key tiles (262144
+    keys), the most the per-CTA list of visible key tiles holds in shared
+    memory.  256 queries, non-causal and causal (bottom-right aligned),
+    through the whole path (the quantiser included) against the oracle."""
+    wq = W.TINY.scaled(B=1, Hq=2, Hkv=1, N=256, D=128, seed=41)
+    wk = W.TINY.scaled(B=1, Hq=2, Hkv=1, N=128 * 2048, D=128, seed=42)
+    q = W.make_qkv(wq)[0]
+    _, k, v = W.make_qkv(wk)
+    oz = O.quantize_qkv_i8f8(q, k, v)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    for causal in (False, True):
+        ref = O.attention_i8f8(oz, causal=causal, sm_scale=wq.sm_scale)
+        out, l = S.sage_attn_fwd(qd, kd, vd, causal=causal, sm_scale=wq.sm_scale, return_lse=True)
+        assert_attention_close(out, l, ref, what=f"Nk=262144 causal={causal}")
+
+
 def test_calls_without_queries_return_empty_results(S):
     """No queries (Nq == 0 or B == 0): empty out and LSE from every
     whole-path call, nothing launched, the device status untouched."""

@@ -111,6 +111,21 @@ def test_nvfp4_attention_on_oracle_codes(S, w, causal):
 TIE_BAND = 1e-5
 
 
+def test_nvfp4_longest_supported_key_length(S):
+    """The longest key sequence the NVFP4 kernels accept (2048 key tiles),
+    with the last 100 keys past unpadded_k_len: 256 queries, non-causal,
+    through the whole path against the oracle."""
+    wq = W.NVFP4.scaled(B=1, Hq=2, Hkv=1, N=256, D=128, unpadded_k_len=None, seed=43)
+    wk = W.NVFP4.scaled(B=1, Hq=2, Hkv=1, N=128 * 2048, D=128, unpadded_k_len=None, seed=44)
+    q = W.make_qkv(wq)[0]
+    _, k, v = W.make_qkv(wk)
+    L = 128 * 2048 - 100
+    ref = O.attention_nvfp4(O.quantize_qkv_nvfp4(q, k, v, per_block_mean=True, unpadded_k_len=L))
+    z = S.sage_quantize_qkv_nvfp4(q.cuda(), k.cuda(), v.cuda(), per_block_mean=True, unpadded_k_len=L)
+    out, lse = S.sage_attn_fwd_nvfp4(z)
+    assert_attention_close(out, lse, ref, what="nvfp4 Nk=262144")
+
+
 def test_nvfp4_whole_path_global_mean(S):
     w = W.NVFP4.scaled(B=1, Hq=4, Hkv=4, N=512, D=128, unpadded_k_len=480, seed=11)
     q, k, v = W.make_qkv(w)
