@@ -30,14 +30,12 @@ def qkv_from_oracle(S, oz, device="cuda", with_qdk=True):
         B=oz["B"], Hq=oz["Hq"], Hkv=oz["Hkv"], Nq=oz["Nq"], Nk=oz["Nk"], D=oz["D"])
 
 
-def assert_attention_close(out_gpu, lse_gpu, ref, rows=None, heads=None, what=""):
+def assert_attention_close(out_gpu, lse_gpu, ref, rows=None, what=""):
     """Compare device outputs with the oracle's (bf16-rounded out, lse)."""
     rows = ref["rows"] if rows is None else rows
     o = out_gpu.float().cpu().numpy().astype(np.float64)[:, :, rows]
     r = ref["out"]
     sel = ~np.isnan(r[..., 0])                        # heads the oracle computed
-    if heads is not None:
-        pass
     og, rg = o[sel], r[sel]
     err = np.abs(og - rg).max()
     cos = O.cosine(og, rg)

@@ -185,6 +185,41 @@ def test_longest_supported_key_length(S):
         assert_attention_close(out, l, ref, what=f"Nk=262144 causal={causal}")
 
 
+def test_single_tokens_and_decode_shape(S):
+    """One query and one key per head (a tile with one live row and one
+    live key), causal and not; then one query against 300 keys, causal
+    (bottom-right aligned, so the query sees every key: the decode shape)."""
+    w = W.TINY.scaled(B=2, Hq=4, Hkv=2, N=1, D=128, seed=46)
+    q, k, v = W.make_qkv(w)
+    oz = O.quantize_qkv_i8f8(q, k, v)
+    for causal in (False, True):
+        ref = O.attention_i8f8(oz, causal=causal, sm_scale=w.sm_scale)
+        out, l = S.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, sm_scale=w.sm_scale,
+                                 return_lse=True)
+        assert_attention_close(out, l, ref, what=f"N=1 causal={causal}")
+    _, k, v = W.make_qkv(W.TINY.scaled(B=2, Hq=4, Hkv=2, N=300, D=128, seed=47))
+    ref = O.attention_i8f8(O.quantize_qkv_i8f8(q, k, v), causal=True, sm_scale=w.sm_scale)
+    out, l = S.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True, sm_scale=w.sm_scale,
+                             return_lse=True)
+    assert_attention_close(out, l, ref, what="Nq=1 Nk=300 causal")
+
+
+def test_most_query_heads_one_call_takes(S):
+    """B * Hq = 17 * 3855 = 65535, the most (batch entry, Q head) pairs one
+    call takes (at most 4096 heads per entry), one token each and every Q
+    head on its entry's one KV head.  Heads are independent given the shared
+    K and V, so the oracle runs on a sample of them (first, last and 61
+    random)."""
+    w = W.TINY.scaled(B=17, Hq=3855, Hkv=1, N=1, D=64, seed=45)
+    q, k, v = W.make_qkv(w)
+    out, l = S.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), sm_scale=w.sm_scale, return_lse=True)
+    rng = np.random.default_rng(45)
+    idx = torch.from_numpy(np.unique(np.concatenate([[0, 1, w.Hq - 1],
+                                                     rng.choice(w.Hq, 61, replace=False)])))
+    ref = O.attention_i8f8(O.quantize_qkv_i8f8(q[:, idx], k, v), sm_scale=w.sm_scale)
+    assert_attention_close(out[:, idx.cuda()], l[:, idx.cuda()], ref, what="B*Hq=65535")
+
+
 def test_calls_without_queries_return_empty_results(S):
     """No queries (Nq == 0 or B == 0): empty out and LSE from every
     whole-path call, nothing launched, the device status untouched."""
