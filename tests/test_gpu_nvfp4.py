@@ -126,6 +126,24 @@ def test_nvfp4_longest_supported_key_length(S):
     assert_attention_close(out, lse, ref, what="nvfp4 Nk=262144")
 
 
+@pytest.mark.parametrize("N,L,causal", [(1, 1, False), (1, 1, True), (256, 1, False), (256, 1, True)])
+def test_nvfp4_degenerate_shapes(S, N, L, causal):
+    """One token per head, and 256 queries that all see only the first key
+    (unpadded_k_len = 1): P' of a row is then one vector holding a single
+    non-zero entry.  Whole path against the oracle, with the tie bound."""
+    w = W.NVFP4.scaled(B=2, Hq=4, Hkv=2, N=N, D=128, unpadded_k_len=L, seed=48 + N)
+    q, k, v = W.make_qkv(w)
+    ref = O.attention_nvfp4(O.quantize_qkv_nvfp4(q, k, v, per_block_mean=True, unpadded_k_len=L),
+                            causal=causal, tie_band=TIE_BAND)
+    z = S.sage_quantize_qkv_nvfp4(q.cuda(), k.cuda(), v.cuda(), per_block_mean=True, unpadded_k_len=L)
+    out, lse = S.sage_attn_fwd_nvfp4(z, causal=causal)
+    o = out.float().cpu().numpy()
+    excess = np.abs(o - ref["out"]) - ref["out_tie_bound"]
+    assert excess.max() <= 2e-2, f"max excess {excess.max():.3g} over the tie bound"
+    assert O.cosine(o, ref["out"]) >= 0.9995
+    np.testing.assert_allclose(lse.cpu().numpy(), ref["lse"], rtol=0, atol=2e-2)
+
+
 def test_nvfp4_whole_path_global_mean(S):
     w = W.NVFP4.scaled(B=1, Hq=4, Hkv=4, N=512, D=128, unpadded_k_len=480, seed=11)
     q, k, v = W.make_qkv(w)
