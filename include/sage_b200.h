@@ -39,7 +39,8 @@
  *   - Work is enqueued asynchronously on `stream` (NULL = legacy default
  *     stream); the call returns after enqueueing.  Argument errors are
  *     detected on the host before anything is enqueued.
- *   - Errors: SAGE_ERR_INVALID_ARG (malformed argument), SAGE_ERR_UNSUPPORTED
+ *   - Errors: SAGE_ERR_INVALID_ARG (malformed argument, including a tensor
+ *     with more than 65536 batch entries or 4096 heads), SAGE_ERR_UNSUPPORTED
  *     (valid but outside what the kernels handle: head_dim not in {64,128},
  *     more than 262144 tokens in a sequence, more than 65535 (batch entry, Q
  *     head) pairs in one device call -- (sequence, KV head) pairs for

@@ -97,6 +97,7 @@ def test_quantize_rejects_bad_arguments_on_host(L):
     assert call(_t(), _t(), _t(), _q(Nk=300)) == S.SAGE_ERR_INVALID_ARG   # out shape mismatch
     assert call(_t(), _t(), _t(), ws=0) == S.SAGE_ERR_INVALID_ARG         # no workspace
     assert call(_t(), _t(), _t(), nb=16) == S.SAGE_ERR_WORKSPACE          # workspace too small
+    assert call(_t(H=4097), _t(H=1), _t(H=1), _q(Hq=4097, Hkv=1)) == S.SAGE_ERR_INVALID_ARG  # heads
     n1 = 128 * 2048 + 1                                                   # one key past the longest
     assert call(_t(), _t(N=n1), _t(N=n1), _q(Nk=n1)) == S.SAGE_ERR_UNSUPPORTED
 
